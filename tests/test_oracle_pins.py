@@ -1,0 +1,440 @@
+"""Pins of the float64 oracle to things other than itself: library routines
+(torch scaled_dot_product_attention in float64), closed forms, invariants,
+brute force on tiny inputs and hand-worked examples under tests/golden/.
+
+Each test is chosen so that a plausible slip in the oracle (a dropped term, a
+wrong sign, index or axis, a transposed operand, '>' for '>=') fails it."""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import svg_inputs as si
+from oracle import svg_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def sdpa64(q, k, v, mask=None, scale=None):
+    """torch's own attention in float64 (library cross-check)."""
+    t = lambda a: torch.from_numpy(np.asarray(a, np.float64))[None, None]
+    m = None if mask is None else torch.from_numpy(np.asarray(mask, bool))[None, None]
+    o = torch.nn.functional.scaled_dot_product_attention(t(q), t(k), t(v), attn_mask=m,
+                                                         scale=scale)
+    return o[0, 0].numpy()
+
+
+def rand(shape, seed=0, scale=1.0):
+    return np.random.default_rng(seed).standard_normal(shape) * scale
+
+
+# ---------------------------------------------------------------- O1 / O2
+
+class TestDenseAttention:
+    def test_matches_torch_sdpa(self):
+        q, k, v = rand((37, 64), 1, 2.0), rand((91, 64), 2, 2.0), rand((91, 64), 3)
+        np.testing.assert_allclose(O.dense_attention(q, k, v), sdpa64(q, k, v), atol=1e-12)
+
+    def test_non_square_head_dim_and_scale(self):
+        q, k, v = rand((5, 128), 4), rand((300, 128), 5), rand((300, 128), 6)
+        np.testing.assert_allclose(O.dense_attention(q, k, v, scale=0.3),
+                                   sdpa64(q, k, v, scale=0.3), atol=1e-12)
+
+    def test_default_scale_is_inverse_sqrt_d(self):
+        assert O.softmax_scale(64) == 0.125
+        q, k, v = rand((3, 16), 7), rand((20, 16), 8), rand((20, 16), 9)
+        np.testing.assert_allclose(O.dense_attention(q, k, v),
+                                   O.dense_attention(q, k, v, scale=0.25), atol=0)
+
+    def test_zero_query_gives_mean_of_values(self):
+        k, v = rand((50, 32), 10), rand((50, 32), 11)
+        o = O.dense_attention(np.zeros((4, 32)), k, v)
+        np.testing.assert_allclose(o, np.broadcast_to(v.mean(0), o.shape), atol=1e-13)
+
+    def test_constant_values_pass_through(self):
+        q, k = rand((6, 32), 12, 3.0), rand((40, 32), 13, 3.0)
+        v = np.tile(rand((1, 32), 14), (40, 1))
+        np.testing.assert_allclose(O.dense_attention(q, k, v), np.tile(v[:1], (6, 1)), atol=1e-12)
+
+    def test_two_key_closed_form(self):
+        q = np.array([[1.0, 0.0]])
+        k = np.array([[1.0, 0.0], [0.0, 1.0]])
+        v = np.array([[2.0, -1.0], [4.0, 3.0]])
+        p0 = math.e / (math.e + 1.0)
+        want = p0 * v[0] + (1 - p0) * v[1]
+        np.testing.assert_allclose(O.dense_attention(q, k, v, scale=1.0)[0], want, atol=1e-15)
+
+    def test_probabilities_rows_sum_to_one_and_large_logits(self):
+        q, k = rand((8, 64), 15, 30.0), rand((70, 64), 16, 30.0)
+        p = O.attention_probs(q, k, 0.125)
+        assert np.isfinite(p).all()
+        np.testing.assert_allclose(p.sum(1), 1.0, atol=1e-13)
+
+
+class TestMaskedAttention:
+    def test_all_true_equals_dense(self):
+        q, k, v = rand((9, 64), 20), rand((33, 64), 21), rand((33, 64), 22)
+        np.testing.assert_allclose(O.masked_attention(q, k, v, np.ones((9, 33), bool)),
+                                   O.dense_attention(q, k, v), atol=1e-13)
+
+    def test_matches_torch_sdpa_bool_mask(self):
+        q, k, v = rand((16, 64), 23, 2), rand((64, 64), 24, 2), rand((64, 64), 25)
+        mask = np.random.default_rng(26).random((16, 64)) < 0.3
+        mask[:, 0] = True
+        np.testing.assert_allclose(O.masked_attention(q, k, v, mask), sdpa64(q, k, v, mask),
+                                   atol=1e-12)
+
+    def test_single_key_returns_that_value(self):
+        q, k, v = rand((3, 8), 27), rand((10, 8), 28), rand((10, 8), 29)
+        mask = np.zeros((3, 10), bool)
+        mask[0, 4] = mask[1, 7] = mask[2, 0] = True
+        o = O.masked_attention(q, k, v, mask)
+        np.testing.assert_allclose(o, v[[4, 7, 0]], atol=0)
+
+    def test_empty_row_is_zero(self):
+        q, k, v = rand((2, 8), 30), rand((5, 8), 31), rand((5, 8), 32)
+        mask = np.zeros((2, 5), bool)
+        mask[1, 2] = True
+        o = O.masked_attention(q, k, v, mask)
+        assert (o[0] == 0).all()
+        np.testing.assert_allclose(o[1], v[2], atol=0)
+
+
+# ---------------------------------------------------------------- O3
+
+class TestTokenMasks:
+    def test_golden_F3_P2(self):
+        g = golden("token_masks_F3_P2.json")
+        n = np.arange(g["F"] * g["P"])
+        np.testing.assert_array_equal(O.spatial_mask(n, n, g["P"], g["width"]),
+                                      np.array(g["spatial"], bool))
+        np.testing.assert_array_equal(O.temporal_mask_frame_major(n, n, g["P"]),
+                                      np.array(g["temporal_frame_major"], bool))
+
+    @pytest.mark.parametrize("F,P", [(4, 3), (5, 7), (1, 6), (6, 1)])
+    def test_temporal_mask_commutes_with_permutation(self, F, P):
+        # the token-major temporal mask is the frame-major one read through the map
+        src = O.token_major_source(F, P)
+        m = np.arange(F * P)
+        np.testing.assert_array_equal(O.temporal_mask_token_major(m, m, F),
+                                      O.temporal_mask_frame_major(src, src, P))
+
+    def test_spatial_width_covers_everything(self):
+        n = np.arange(4 * 5)
+        assert O.spatial_mask(n, n, 5, 3).all()
+        assert not O.spatial_mask(n, n, 5, 2).all()
+
+
+# ---------------------------------------------------------------- O5
+
+class TestPermutation:
+    def test_golden_F3_P4(self):
+        g = golden("permutation_F3_P4.json")
+        np.testing.assert_array_equal(O.token_major_source(g["F"], g["P"]),
+                                      g["token_major_source"])
+        x = np.arange(12, dtype=np.float64).reshape(12, 1)
+        np.testing.assert_array_equal(O.permute_token_major(x, 3, 4)[:, 0],
+                                      g["token_major_source"])
+
+    @pytest.mark.parametrize("F,P", [(13, 7), (4, 64), (1, 9), (9, 1), (21, 5)])
+    def test_bijection_inverse_and_closed_form(self, F, P):
+        N = F * P
+        src = O.token_major_source(F, P)
+        np.testing.assert_array_equal(np.sort(src), np.arange(N))
+        m = np.arange(N)
+        np.testing.assert_array_equal(src, (m % F) * P + m // F)
+        x = np.random.default_rng(F * 100 + P).standard_normal((2, 3, N, 4))
+        y = O.permute_token_major(x, F, P)
+        np.testing.assert_array_equal(y, x[..., src, :])
+        np.testing.assert_array_equal(O.permute_frame_major(y, F, P), x)
+        np.testing.assert_array_equal(O.permute_token_major(O.permute_frame_major(x, F, P), F, P), x)
+
+    def test_identity_cases(self):
+        x = rand((10, 3), 40)
+        np.testing.assert_array_equal(O.permute_token_major(x, 1, 10), x)
+        np.testing.assert_array_equal(O.permute_token_major(x, 10, 1), x)
+
+    def test_temporal_stripes_become_contiguous(self):
+        # after the transform, the keys a temporal row sees are one contiguous run
+        F, P = 6, 11
+        src = O.token_major_source(F, P)
+        for m in range(F * P):
+            cols = np.nonzero(O.temporal_mask_frame_major(src[m:m + 1], src, P)[0])[0]
+            assert cols[-1] - cols[0] + 1 == len(cols) == F
+
+
+# ---------------------------------------------------------------- O7
+
+def brute_lists(mask, N, T):
+    nb = (N + T - 1) // T
+    indptr, indices = [0], []
+    for i in range(nb):
+        for j in range(nb):
+            if mask[i * T:(i + 1) * T, j * T:(j + 1) * T].any():
+                indices.append(j)
+        indptr.append(len(indices))
+    return np.array(indptr), np.array(indices)
+
+
+def closed_form_lists(kind, F, P, w, N, T):
+    """Interval overlap: rows of tile i span frames (or positions) [a_i, b_i]."""
+    nb = (N + T - 1) // T
+    div = P if kind == O.MODE_SPATIAL else F
+    lo = [i * T // div for i in range(nb)]
+    hi = [(min(N, (i + 1) * T) - 1) // div for i in range(nb)]
+    ww = w if kind == O.MODE_SPATIAL else 0
+    indptr, indices = [0], []
+    for i in range(nb):
+        for j in range(nb):
+            if kind == O.MODE_DENSE or (lo[j] <= hi[i] + ww and hi[j] >= lo[i] - ww):
+                indices.append(j)
+        indptr.append(len(indices))
+    return np.array(indptr), np.array(indices)
+
+
+class TestGeometricLists:
+    def test_golden_small_tile(self):
+        g = golden("block_lists_F3_P5_T4.json")
+        F, P, N, T = g["F"], g["P"], g["N"], g["T"]
+        for key, kind, w in [("spatial_w0", O.MODE_SPATIAL, 0), ("spatial_w1", O.MODE_SPATIAL, 1),
+                             ("temporal", O.MODE_TEMPORAL, 0)]:
+            ip, ix = O.geometric_block_lists(kind, F, P, w, N, T)
+            np.testing.assert_array_equal(ip, g[key]["indptr"])
+            np.testing.assert_array_equal(ix, g[key]["indices"])
+
+    @pytest.mark.parametrize("F,P,w,T", [(3, 5, 1, 4), (4, 7, 1, 8), (5, 9, 2, 16), (7, 3, 0, 5),
+                                         (2, 40, 1, 32), (13, 11, 1, 128), (6, 50, 1, 128)])
+    def test_brute_force_and_closed_form(self, F, P, w, T):
+        N = F * P
+        n = np.arange(N)
+        src = O.token_major_source(F, P)
+        masks = {O.MODE_SPATIAL: O.spatial_mask(n, n, P, w),
+                 O.MODE_TEMPORAL: O.temporal_mask_frame_major(src, src, P),
+                 O.MODE_DENSE: np.ones((N, N), bool)}
+        for kind, M in masks.items():
+            ip, ix = O.geometric_block_lists(kind, F, P, w, N, T)
+            bp, bx = brute_lists(M, N, T)
+            np.testing.assert_array_equal(ip, bp)
+            np.testing.assert_array_equal(ix, bx)
+            cp, cx = closed_form_lists(kind, F, P, w, N, T)
+            np.testing.assert_array_equal(ip, cp)
+            np.testing.assert_array_equal(ix, cx)
+
+    @pytest.mark.parametrize("F,P,w", [(13, 1350, 1), (21, 1560, 1), (33, 3600, 2)])
+    def test_closed_form_at_workload_shapes(self, F, P, w):
+        N = F * P
+        for kind in (O.MODE_SPATIAL, O.MODE_TEMPORAL):
+            ip, ix = O.geometric_block_lists(kind, F, P, w, N)
+            cp, cx = closed_form_lists(kind, F, P, w, N, 128)
+            np.testing.assert_array_equal(ip, cp)
+            np.testing.assert_array_equal(ix, cx)
+
+    def test_wide_band_keeps_everything_and_diagonal_always_kept(self):
+        F, P = 5, 33
+        N = F * P
+        ip, ix = O.geometric_block_lists(O.MODE_SPATIAL, F, P, F - 1, N, 16)
+        dp, dx = O.geometric_block_lists(O.MODE_DENSE, F, P, 0, N, 16)
+        np.testing.assert_array_equal(ip, dp)
+        np.testing.assert_array_equal(ix, dx)
+        for kind in (O.MODE_SPATIAL, O.MODE_TEMPORAL):
+            ip, ix = O.geometric_block_lists(kind, F, P, 0, N, 16)
+            for i in range(len(ip) - 1):
+                assert i in ix[ip[i]:ip[i + 1]]
+                assert (np.diff(ix[ip[i]:ip[i + 1]]) > 0).all()
+
+    def test_block_mask_contains_token_mask(self):
+        F, P, w, T = 4, 37, 1, 32
+        N = F * P
+        n = np.arange(N)
+        ip, ix = O.geometric_block_lists(O.MODE_SPATIAL, F, P, w, N, T)
+        MB = O.block_mask_from_lists(ip, ix, N, T)
+        assert (MB | ~O.spatial_mask(n, n, P, w)).all()
+
+
+# ---------------------------------------------------------------- O8
+
+def kron_mask(indptr, indices, N, T):
+    nb = len(indptr) - 1
+    tiles = np.zeros((nb, nb), bool)
+    for i in range(nb):
+        tiles[i, indices[indptr[i]:indptr[i + 1]]] = True
+    return np.kron(tiles, np.ones((T, T), bool))[:N, :N]
+
+
+class TestBlockSparseAttention:
+    def test_all_kept_equals_dense(self):
+        N, T = 300, 64
+        q, k, v = rand((N, 64), 50, 2), rand((N, 64), 51, 2), rand((N, 64), 52)
+        ip, ix = O.geometric_block_lists(O.MODE_DENSE, 1, N, 0, N, T)
+        np.testing.assert_allclose(O.block_sparse_attention(q, k, v, ip, ix, T), sdpa64(q, k, v),
+                                   atol=1e-12)
+
+    def test_geometric_lists_match_sdpa_with_tile_mask(self):
+        F, P, w, T = 5, 41, 1, 32
+        N = F * P
+        q, k, v = rand((N, 32), 53, 2), rand((N, 32), 54, 2), rand((N, 32), 55)
+        ip, ix = O.geometric_block_lists(O.MODE_SPATIAL, F, P, w, N, T)
+        np.testing.assert_allclose(O.block_sparse_attention(q, k, v, ip, ix, T),
+                                   sdpa64(q, k, v, kron_mask(ip, ix, N, T)), atol=1e-12)
+        rows = np.array([0, 31, 32, 150, N - 1])
+        np.testing.assert_allclose(O.block_sparse_rows(q, k, v, rows, ip, ix, T),
+                                   sdpa64(q, k, v, kron_mask(ip, ix, N, T))[rows], atol=1e-12)
+
+    def test_empty_list_gives_zero_rows_and_ragged_tail(self):
+        N, T = 70, 32                       # tiles of 32, 32, 6 rows
+        q, k, v = rand((N, 16), 56), rand((N, 16), 57), rand((N, 16), 58)
+        ip = np.array([0, 1, 1, 3])
+        ix = np.array([2, 0, 2])
+        o = O.block_sparse_attention(q, k, v, ip, ix, T)
+        assert (o[32:64] == 0).all()
+        # tile 0 sees only the 6 keys of the ragged last tile
+        np.testing.assert_allclose(o[:32], O.dense_attention(q[:32], k[64:], v[64:]), atol=1e-13)
+        keys = np.r_[0:32, 64:70]
+        np.testing.assert_allclose(o[64:], O.dense_attention(q[64:], k[keys], v[keys]), atol=1e-13)
+
+
+# ---------------------------------------------------------------- O4
+
+def brute_profile(q, k, v, idx, P, w):
+    """Full N x N attention for each mask through torch, then the sampled rows."""
+    N = q.shape[0]
+    sp = np.zeros((N, N), bool)
+    tp = np.zeros((N, N), bool)
+    for i in range(N):
+        for j in range(N):
+            sp[i, j] = abs(i // P - j // P) <= w
+            tp[i, j] = (i % P) == (j % P)
+    od = sdpa64(q, k, v)[idx]
+    os_ = sdpa64(q, k, v, sp)[idx]
+    ot = sdpa64(q, k, v, tp)[idx]
+    return ((os_ - od) ** 2).mean(), ((ot - od) ** 2).mean()
+
+
+class TestProfiling:
+    def test_brute_force_on_tiny_workload(self):
+        wl = si.WORKLOADS["tiny"]
+        q, k, v, types = si.generate(wl)
+        idx = si.sample_queries(wl)
+        for h in range(wl.H):
+            qh, kh, vh = (si.as_float64(t[0, h]) for t in (q, k, v))
+            ms, mt, mode = O.profile_head(qh, kh, vh, idx, wl.F, wl.P, wl.width)
+            bs, bt = brute_profile(qh, kh, vh, idx, wl.P, wl.width)
+            assert ms == pytest.approx(bs, rel=1e-10, abs=1e-15)
+            assert mt == pytest.approx(bt, rel=1e-10, abs=1e-15)
+
+    def test_designed_labels_with_margin(self):
+        wl = si.WORKLOADS["tiny"]
+        q, k, v, types = si.generate(wl)
+        idx = si.sample_queries(wl)
+        mse, mode = O.profile_heads(*(si.as_float64(t) for t in (q, k, v)), idx, wl.F, wl.P,
+                                    wl.width)
+        assert list(types) == [si.SPATIAL_TYPE, si.TEMPORAL_TYPE]
+        assert list(mode) == [O.MODE_SPATIAL, O.MODE_TEMPORAL]
+        assert mse[0, 1] > 10 * mse[0, 0]
+        assert mse[1, 0] > 10 * mse[1, 1]
+
+    def test_tie_goes_to_spatial_and_constant_v(self):
+        N, P, F = 24, 6, 4
+        q, k = rand((N, 8), 60), rand((N, 8), 61)
+        ms, mt, mode = O.profile_head(q, k, np.zeros((N, 8)), np.array([0, 5, 13]), F, P, 1)
+        assert ms == 0 and mt == 0 and mode == O.MODE_SPATIAL
+        ms, mt, mode = O.profile_head(q, k, np.ones((N, 8)), np.array([0, 5, 13]), F, P, 1)
+        assert ms < 1e-28 and mt < 1e-28
+
+    def test_designed_labels_small_workloads(self):
+        for name in ("cogvideox", "wan480", "hunyuan720"):
+            wl = si.small(name)
+            q, k, v, types = si.generate(wl)
+            idx = si.sample_queries(wl)
+            mse, mode = O.profile_heads(*(si.as_float64(t) for t in (q, k, v)), idx, wl.F,
+                                        wl.P, wl.width)
+            np.testing.assert_array_equal(mode, types)
+
+
+# ---------------------------------------------------------------- O9
+
+class TestCalibration:
+    def test_golden_minimal_sets(self):
+        for case in golden("calibration_examples.json")["minimal_set"]:
+            assert O.minimal_energy_set(case["energy"], case["eps"]) == case["kept"]
+
+    def test_golden_votes(self):
+        for case in golden("calibration_examples.json")["vote"]:
+            E = [np.array([row]) for row in case["energies"]]
+            ip, ix = O.calibrate_lists(E, case["eps"], case["rho"])
+            np.testing.assert_array_equal(ip, [0, len(case["kept"])])
+            np.testing.assert_array_equal(ix, case["kept"])
+
+    def test_minimality_against_exhaustive_search(self):
+        rng = np.random.default_rng(70)
+        for trial in range(60):
+            nb = int(rng.integers(1, 9))
+            e = rng.dirichlet(np.ones(nb) * 0.5)
+            eps = float(rng.uniform(0.3, 0.99))
+            kept = O.minimal_energy_set(e, eps)
+            assert e[kept].sum() >= eps or len(kept) == nb
+            best = min(len(s) for r in range(1, nb + 1)
+                       for s in itertools.combinations(range(nb), r) if e[list(s)].sum() >= eps)
+            assert len(kept) == best
+            # dropping the smallest kept block falls below eps
+            if len(kept) > 1:
+                assert e[kept].sum() - e[kept].min() < eps
+
+    def test_single_input_returns_its_sets_and_eps_one_keeps_all_nonzero(self):
+        rng = np.random.default_rng(71)
+        E = rng.dirichlet(np.ones(7), size=5)
+        ip, ix = O.calibrate_lists([E], 0.8, 0.5)
+        for r in range(5):
+            assert list(ix[ip[r]:ip[r + 1]]) == O.minimal_energy_set(E[r], 0.8)
+        E[:, 3] = 0.0
+        E = E / E.sum(1, keepdims=True)
+        ip, ix = O.calibrate_lists([E], 1.0 - 1e-12, 0.5)
+        for r in range(5):
+            assert list(ix[ip[r]:ip[r + 1]]) == [0, 1, 2, 4, 5, 6]
+
+    def test_energy_matches_torch_softmax_and_rows_sum_to_one(self):
+        N, T, d = 200, 64, 32
+        q, k = rand((N, d), 72, 2), rand((N, d), 73, 2)
+        E = O.block_energy(q, k, T)
+        p = torch.softmax(torch.from_numpy(q @ k.T) / math.sqrt(d), dim=-1).numpy()
+        nb = 4
+        pad = np.zeros((nb * T, nb * T))
+        pad[:N, :N] = p
+        sums = pad.reshape(nb, T, nb, T).sum(axis=(1, 3))
+        counts = np.array([64, 64, 64, 8])[:, None]
+        np.testing.assert_allclose(E, sums / counts, atol=1e-13)
+        np.testing.assert_allclose(E.sum(1), 1.0, atol=1e-13)
+
+    def test_energy_uniform_for_zero_queries(self):
+        N, T = 150, 64
+        E = O.block_energy(np.zeros((N, 8)), rand((N, 8), 74), T)
+        np.testing.assert_allclose(E, np.tile(np.array([64, 64, 22]) / N, (3, 1)), atol=1e-14)
+
+
+# ---------------------------------------------------------------- whole layer
+
+def test_layer_composes_steps_on_tiny():
+    wl = si.WORKLOADS["tiny"]
+    q, k, v, _ = (si.generate(wl)[i] for i in range(4))
+    q64, k64, v64 = (si.as_float64(t) for t in (q, k, v))
+    idx = si.sample_queries(wl)
+    o, mode, mse = O.svg_layer(q64, k64, v64, idx, wl.F, wl.P, wl.width)
+    # head 0 is spatial: N = 256 is two tiles spanning frames {0,1} and {2,3},
+    # so the band |f - f'| <= 1 touches both tiles and the head is dense
+    np.testing.assert_allclose(o[0, 0], sdpa64(q64[0, 0], k64[0, 0], v64[0, 0]), atol=1e-12)
+    # head 1 is temporal: token-major tiles of 128 rows hold positions 0-31 and
+    # 32-63, each tile sees only itself, i.e. keys of the same half of positions
+    P = wl.P
+    n = np.arange(wl.N)
+    half = (n % P) // 32
+    M = half[:, None] == half[None, :]
+    np.testing.assert_allclose(o[0, 1], sdpa64(q64[0, 1], k64[0, 1], v64[0, 1], M), atol=1e-12)
