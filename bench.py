@@ -1,0 +1,377 @@
+"""Benchmark of one sparse spatial/temporal attention layer on B200.
+
+A step is one pass of the whole hot path over one layer's inputs:
+    profile heads -> permute q, k, v (temporal heads) -> block-sparse attention
+    -> permute the output back.
+Workload (default): the CogVideoX-shaped layer, B=1 H=48 N=17550 (13 frames x
+30x45 tokens) d=64 bf16, synthetic biased-Gaussian q/k/v, 64 sampled queries.
+
+Metric: effective TFLOPS of the layer = sum over heads of 4 * d * (query-key
+pairs inside kept 128x128 tiles, ragged tiles counted by their valid rows and
+columns) / step time.  tokens/s = B * N / step time is reported beside it.
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
+        python bench.py --impl reference ...    (the float64 CPU oracle)
+Multi-GPU (torchrun): every rank runs its own independent layer (a different
+input seed); no collective touches the data path (weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import svg_inputs as si  # noqa: E402
+
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+METRIC = "effective TFLOPS and tokens/s of sparse 3D attention per layer; % of bf16 TC peak"
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kept_pairs(indptr, indices, N, T=128):
+    """Query-key pairs inside the kept tiles of one list (ragged tiles count
+    their valid rows and columns)."""
+    nb = len(indptr) - 1
+    sizes = np.minimum(T, N - np.arange(nb) * T).astype(np.int64)
+    total = 0
+    for i in range(nb):
+        total += int(sizes[i]) * int(sizes[indices[indptr[i]:indptr[i + 1]]].sum())
+    return total
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"svg_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import sparse_attention_video_svg_b200 as svg
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = si.WORKLOADS[args.config]
+    if wl.kind != "profiled":
+        raise SystemExit(f"bench runs profiled layers; {wl.name} is {wl.kind}")
+    seed = wl.seed + rank
+    q, k, v, types = si.generate(wl, seed=seed)
+    idx = si.sample_queries(wl, seed=wl.seed)
+    host = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in (q, k, v)]
+    del q, k, v
+    qd, kd, vd = (h.to(dev) for h in host)
+    idx_d = torch.from_numpy(idx).to(dev)
+    F, P, w, N, d = wl.F, wl.P, wl.width, wl.N, wl.d
+    lists = svg.geometric_lists(F, P, w, N, device=dev)
+    bufs = svg.LayerBuffers(qd, wl.S)
+    stream = torch.cuda.current_stream()
+
+    # effective work from the modes the layer picks (deterministic for the input)
+    _, mode, _ = svg.svg_layer(qd, kd, vd, F, P, w, idx_d, lists, bufs)
+    torch.cuda.synchronize()
+    modes = mode.cpu().numpy()
+    nb = svg.n_tiles(N)
+    ip = lists.indptr.cpu().numpy().reshape(3, nb + 1)
+    ix = lists.indices.cpu().numpy()
+    pairs = {kind: kept_pairs(ip[kind] - ip[kind][0], ix[ip[kind][0]:ip[kind][-1]], N)
+             for kind in (0, 1)}
+    flops = float(sum(4 * d * pairs[int(m)] for m in modes))   # per layer, this rank
+    kept_frac = {kind: pairs[kind] / float(N * N) for kind in pairs}
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # > 126 MB L2
+    K, W = args.steps, args.warmup
+
+    def step():
+        return svg.svg_layer(qd, kd, vd, F, P, w, idx_d, lists, bufs)
+
+    for _ in range(W):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    for i in range(K):
+        flush.fill_(i & 0xff)
+        s0, a0, a1, s1 = ev[i]
+        s0.record(stream)
+        svg.svg_profile_heads(qd, kd, vd, F, P, w, idx_d, mse_out=bufs.mse, mode_out=bufs.mode,
+                              workspace=bufs.ws)
+        for x, y in ((qd, bufs.qp), (kd, bufs.kp), (vd, bufs.vp)):
+            svg.svg_permute_token_major(x, F, P, bufs.mode, out=y)
+        a0.record(stream)
+        svg.svg_sparse_attn(bufs.qp, bufs.kp, bufs.vp, bufs.mode, lists, out=bufs.op)
+        a1.record(stream)
+        svg.svg_permute_frame_major(bufs.op, F, P, bufs.mode, out=bufs.o)
+        s1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    step_ms = [e[0].elapsed_time(e[3]) for e in ev]
+    attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    total_ms = float(sum(step_ms))
+    attn_avg = float(sum(attn_ms) / K)
+
+    # end to end through the public API with host buffers
+    out_host = torch.empty(qd.shape, dtype=torch.bfloat16).pin_memory()
+    mode_host = torch.empty(modes.shape, dtype=torch.int32).pin_memory()
+    for _ in range(2):
+        dq, dk, dv = (h.to(dev, non_blocking=True) for h in host)
+        o, m, _ = svg.svg_layer(dq, dk, dv, F, P, w, idx_d, lists, bufs)
+        out_host.copy_(o, non_blocking=True)
+        mode_host.copy_(m, non_blocking=True)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        qd.copy_(host[0], non_blocking=True)
+        kd.copy_(host[1], non_blocking=True)
+        vd.copy_(host[2], non_blocking=True)
+        o, m, _ = svg.svg_layer(qd, kd, vd, F, P, w, idx_d, lists, bufs)
+        out_host.copy_(o, non_blocking=True)
+        mode_host.copy_(m, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+
+    if world > 1:
+        t = torch.tensor([total_ms, e2e_ms, attn_avg], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, e2e_ms, attn_avg = (float(x) for x in t.tolist())
+    if rank != 0:
+        return None
+
+    peaks, src = load_peaks()
+    peak_tf = float(peaks["bf16_tflops"])
+    all_flops = flops * world
+    value = all_flops / (total_ms / K * 1e-3) / 1e12
+    tokens_s = wl.B * N * world / (total_ms / K * 1e-3)
+    attn_tf = flops / (attn_avg * 1e-3) / 1e12
+    h2d = sum(h.numel() * 2 for h in host)
+    d2h = out_host.numel() * 2 + mode_host.numel() * 4
+    launches_per_step = 2 + 3 + 1 + 1   # profile partial+combine, 3 permutes, attention, permute back
+    line = {
+        "metric": METRIC,
+        "value": round(value, 3),
+        "unit": "TFLOPS",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": W,
+        "ms_per_step": round(total_ms / K, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded biased-Gaussian q/k/v, no model weights)",
+        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "frames": F, "tokens_per_frame": P,
+                   "N": N, "d": d, "sampled_queries": wl.S, "spatial_width": w,
+                   "modes": {"spatial": int((modes == 0).sum()), "temporal": int((modes == 1).sum())},
+                   "kept_fraction": {"spatial": round(kept_frac[0], 5),
+                                     "temporal": round(kept_frac[1], 5)},
+                   "l2": "flushed (256 MB write) before every timed step",
+                   "parallelism": f"independent layer per GPU x{world}"},
+        "tokens_per_s": round(tokens_s, 1),
+        "pct_of_bf16_peak": round(100 * value / world / peak_tf, 2),
+        "attention_only": {"ms": round(attn_avg, 5), "effective_tflops": round(attn_tf, 3)},
+        "roofline": {"kernel": "svg_sparse_attn", "bound": "tensor", "achieved": round(attn_tf, 3),
+                     "peak": peak_tf, "unit": "TFLOP/s", "frac": round(attn_tf / peak_tf, 4),
+                     "peak_source": f"{src} bf16 burst", "traffic": None},
+        "e2e": {"value": round(all_flops / (e2e_ms / K * 1e-3) / 1e12, 3), "unit": "TFLOPS",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(e2e_ms / K, 5)},
+        "gpu_launches": launches_per_step * K,
+        "clocks": clk,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_budget)
+    return line
+
+
+# ------------------------------------------------------------- oracle timing
+
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:  # noqa: BLE001
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(wl, budget_s=15.0, seed=None):
+    """The float64 oracle on a bounded sample of the same layer: profiling and
+    block-sparse attention for as many (head, query tile) units as fit the
+    budget, converted to the same effective-TFLOPS unit."""
+    from oracle import svg_oracle as O
+
+    seed = wl.seed if seed is None else seed
+    one = wl.scaled(wl.name, H=2)
+    q, k, v, types = si.generate(one, seed=seed)
+    idx = si.sample_queries(wl)
+    F, P, w, N = wl.F, wl.P, wl.width, wl.N
+    lists = {kind: O.geometric_block_lists(kind, F, P, w, N) for kind in (0, 1)}
+    t0 = time.perf_counter()
+    flops = 0.0
+    units = 0
+    heads_profiled = 0
+    for h in range(one.H):
+        qh, kh, vh = (si.as_float64(t[0, h]) for t in (q, k, v))
+        ms, mt, md = O.profile_head(qh, kh, vh, idx, F, P, w)
+        heads_profiled += 1
+        ip, ix = lists[md]
+        if md == O.MODE_TEMPORAL:
+            qh, kh, vh = (O.permute_token_major(t, F, P) for t in (qh, kh, vh))
+        nb = len(ip) - 1
+        for i in range(nb):
+            rows = O.tile_rows(i, N)
+            O.block_sparse_rows(qh, kh, vh, rows, ip, ix)
+            cols = sum(min(128, N - j * 128) for j in ix[ip[i]:ip[i + 1]])
+            flops += 4.0 * wl.d * len(rows) * cols
+            units += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": flops / dt / 1e12, "unit": "TFLOPS", "cores": oracle_threads(),
+            "kind": "oracle",
+            "sample": f"{wl.name}: {heads_profiled} head(s) profiled, {units} query tiles of "
+                      f"block-sparse attention (float64 NumPy), {dt:.1f} s"}
+
+
+def run_reference(args):
+    wl = si.WORKLOADS[args.config]
+    K, W = args.steps, args.warmup
+    budget = max(1.0, args.cpu_budget / max(1, K + W))
+    for _ in range(W):
+        cpu_baseline(wl, budget_s=budget)
+    vals = [cpu_baseline(wl, budget_s=budget) for _ in range(K)]
+    value = statistics.mean(v["value"] for v in vals)
+    return {
+        "impl": "reference",
+        "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": 1, "steps": K, "warmup": W,
+        "ms_per_step": None, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic (seeded biased-Gaussian q/k/v, no model weights)",
+        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "N": wl.N, "d": wl.d},
+        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": vals[-1]["cores"],
+                         "kind": "oracle", "sample": vals[-1]["sample"]},
+        "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="cogvideox", choices=[n for n in si.ORDER if n != "tiny"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    line = run_ours(args, rank, world, local_rank)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

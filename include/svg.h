@@ -1,0 +1,251 @@
+/*
+ * svg.h -- C ABI of the B200 (sm_100a) sparse spatial/temporal video attention
+ * library.
+ *
+ * The library implements one attention layer of Sparse VideoGen-style sparse
+ * 3D attention for video diffusion transformers:
+ *
+ *   1. svg_profile_heads        online profiling: per head, pick the spatial or
+ *                               the temporal mask from a few sampled queries;
+ *   2. svg_permute_token_major  frame-major -> token-major reordering of the
+ *                               heads that run temporal;
+ *   3. svg_build_block_mask     per-query-block key-block lists (CSR) from the
+ *                               spatial / temporal geometry, or
+ *      svg_block_energy +
+ *      svg_build_block_mask_calibrated   lists from cumulative-energy calibration;
+ *   4. svg_sparse_attn          block-sparse attention over 128x128 tiles that
+ *                               walks only the kept key blocks;
+ *   5. svg_permute_frame_major  the inverse reordering of the output.
+ *
+ * Sources (cited by page title and section):
+ *   [SVG]  Sparse VideoGen article, m.jxzklqfsx.com/article/815093.html
+ *   [CAL]  CalibAtt article, lpnh.cn/news/568491
+ *   [SURV] video-diffusion acceleration survey, wmrh.cn/news/48564
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  * Tensors q, k, v, o, x, y are caller-owned DEVICE memory, contiguous
+ *    row-major [B, H, N, d] with d in {64, 128}; element type per `dtype`
+ *    (SVG_BF16 or SVG_FP32).  Base pointers must be 16-byte aligned.
+ *  * Tokens are frame-major unless stated: n = f * P + s, where f < F is the
+ *    frame, s < P the spatial position and P = tokens_per_frame, N = F * P.
+ *    Token-major order is m = s * F + f.
+ *  * Tiles are T = 128 tokens; tile i holds tokens [128 i, min(N, 128 i + 128)).
+ *    nB = ceil(N / 128).
+ *  * The library allocates no device memory.  Scratch it needs is passed in
+ *    as `workspace` (device, 256-byte aligned, size from the matching
+ *    *_workspace_size call).
+ *  * `stream` is a cudaStream_t cast to void*; NULL means the legacy default
+ *    stream.  Every call is asynchronous on that stream.  Arguments are
+ *    validated on the host before anything is launched; on a non-SVG_OK
+ *    return nothing was launched (except SVG_ERR_CUDA, which reports a launch
+ *    failure) and svg_last_error() describes the problem.
+ *  * Device-side index checks never fault: out-of-range list entries are
+ *    skipped and recorded in the optional `device_status` word.
+ *  * No call blocks the host, throws, or traps on the device.
+ */
+#ifndef SVG_B200_H_
+#define SVG_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SVG_OK = 0,
+  SVG_ERR_INVALID_ARG = 1, /* bad shape, pointer, alignment or enum value */
+  SVG_ERR_UNSUPPORTED = 2, /* valid request this build does not implement */
+  SVG_ERR_CUDA = 3,        /* a CUDA launch or query failed */
+  SVG_ERR_TIMEOUT = 4      /* device status: a bounded wait gave up */
+} svg_status;
+
+typedef enum { SVG_BF16 = 0, SVG_FP32 = 1 } svg_dtype;
+
+/* Per-head attention mode.  Also the list id svg_sparse_attn uses when the
+ * lists are the three geometric ones concatenated in this order. */
+typedef enum {
+  SVG_MODE_SPATIAL = 0,  /* [SVG] "Spatial Head": same and adjacent frames */
+  SVG_MODE_TEMPORAL = 1, /* [SVG] "Temporal Head": same position, all frames */
+  SVG_MODE_DENSE = 2     /* every key (only by explicit caller choice) */
+} svg_mode;
+
+/* Bits of the optional device status word (int32, device memory, OR-ed). */
+#define SVG_DEVICE_BAD_LIST_ID 0x1   /* a list id outside [0, n_lists)      */
+#define SVG_DEVICE_BAD_INDEX 0x2     /* a key-block index outside [0, nB)   */
+#define SVG_DEVICE_TIMEOUT 0x4       /* a bounded pipeline wait gave up      */
+#define SVG_DEVICE_CAPACITY 0x8      /* a list did not fit the given buffer */
+
+#define SVG_TILE 128
+
+/* Library identification, e.g. "svg_b200 0.1 sm_100a". */
+const char* svg_version(void);
+
+/* Text of the last error returned on the calling host thread ("" if none). */
+const char* svg_last_error(void);
+
+/* --------------------------------------------------------------------------
+ * 1. Online head profiling
+ *    [SVG] section "動態自適應的稀疏策略", steps 1-3: sample a few query
+ *    tokens, compute their attention under the spatial and the temporal
+ *    masks, compare each with dense attention, and give every head the mask
+ *    of smaller error.
+ *
+ *  q, k, v       device [B, H, N, d], frame-major.
+ *  sample_idx    device int32 [S], frame-major token indices in [0, N),
+ *                shared by every (b, h).  1 <= S <= 64.  Values outside
+ *                [0, N) are clamped into range on the device.
+ *  frames, tokens_per_frame   F and P with F * P == N.
+ *  spatial_width w: the spatial mask keeps keys with |f - f'| <= w.
+ *                The temporal mask keeps keys with the same position s.
+ *  mse_out       device float [B*H][2] or NULL: mean over the S x d sampled
+ *                outputs of (o_spatial - o_dense)^2 and (o_temporal - o_dense)^2.
+ *  mode_out      device int32 [B*H]: SVG_MODE_TEMPORAL if the temporal error
+ *                is strictly smaller, else SVG_MODE_SPATIAL.
+ *  workspace     device scratch of svg_profile_workspace_size(...) bytes.
+ * Arithmetic: bf16 inputs use bf16 tensor-core products with fp32
+ * accumulation; fp32 inputs use fp32 arithmetic throughout.  Error sums and
+ * the mode decision are fp32.
+ * ------------------------------------------------------------------------ */
+size_t svg_profile_workspace_size(int B, int H, int N, int d, int S);
+
+svg_status svg_profile_heads(const void* q, const void* k, const void* v, int dtype,
+                             int B, int H, int N, int d,
+                             int frames, int tokens_per_frame, int spatial_width,
+                             const int32_t* sample_idx, int S,
+                             float* mse_out, int32_t* mode_out,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* --------------------------------------------------------------------------
+ * 2. / 5. Frame-major <-> token-major permutation
+ *    [SVG] section "Layout Transformation + Kernel 加速": reorder so that the
+ *    tokens a temporal head needs (one position in every frame) are
+ *    contiguous.
+ *
+ *  svg_permute_token_major:  y[b,h, s*F + f, :] = x[b,h, f*P + s, :]
+ *  svg_permute_frame_major:  y[b,h, f*P + s, :] = x[b,h, s*F + f, :]
+ *  for every head whose mode[b*H + h] == SVG_MODE_TEMPORAL; every other head
+ *  is copied unchanged, so y is always a complete tensor.  mode == NULL
+ *  permutes every head.  x and y are device [B, H, N, d] and must not
+ *  overlap (out of place).  Bit-exact: pure data movement.
+ * ------------------------------------------------------------------------ */
+svg_status svg_permute_token_major(const void* x, void* y, int dtype,
+                                   int B, int H, int N, int d,
+                                   int frames, int tokens_per_frame,
+                                   const int32_t* mode, void* stream);
+
+svg_status svg_permute_frame_major(const void* x, void* y, int dtype,
+                                   int B, int H, int N, int d,
+                                   int frames, int tokens_per_frame,
+                                   const int32_t* mode, void* stream);
+
+/* --------------------------------------------------------------------------
+ * 3a. Geometric key-block lists
+ *    [CAL] section 2.2 (keep/skip decisions on 128x128 tiles) applied to the
+ *    [SVG] head masks.  Tile pair (i, j) is kept iff some token of query tile
+ *    i and some token of key tile j satisfy the token mask:
+ *      SVG_MODE_SPATIAL   frame-major tokens, |f - f'| <= spatial_width;
+ *      SVG_MODE_TEMPORAL  token-major tokens (the order temporal heads run
+ *                         in), same position s;
+ *      SVG_MODE_DENSE     every pair.
+ *
+ *  indptr    device int32 [nB + 1]: row i is indices[indptr[i] - index_base ..
+ *            indptr[i+1] - index_base), i.e. every indptr value is offset by
+ *            `index_base` (>= 0) so that several lists can share one indices
+ *            buffer: pass indices + index_base for a list stored there.
+ *  indices   device int32 [capacity], ascending within a row.
+ *  nnz_out   device int64 [1]: number of entries.  If it exceeds `capacity`
+ *            the indices are not written (indptr and nnz still are) and
+ *            SVG_DEVICE_CAPACITY is set in *device_status (if non-NULL).
+ *            capacity = nB * nB always suffices.
+ * ------------------------------------------------------------------------ */
+svg_status svg_build_block_mask(int kind, int frames, int tokens_per_frame,
+                                int spatial_width, int N,
+                                int32_t* indptr, int32_t* indices, int64_t capacity,
+                                int64_t index_base, int64_t* nnz_out,
+                                int32_t* device_status, void* stream);
+
+/* --------------------------------------------------------------------------
+ * 3b. Block energy for calibration
+ *    [CAL] section 3.1: the attention energy E(r, c) of query block r on key
+ *    block c.  E[b,h,r,c] = sum over rows i of block r and keys j of block c
+ *    of softmax_j(q_i . k_j / sqrt(d)), divided by the row count of block r,
+ *    so every row of E sums to 1.
+ *
+ *  q, k      device [B, H, N, d].
+ *  energy    device float [B*H][nB][nB].
+ *  workspace device scratch of svg_block_energy_workspace_size(...) bytes.
+ * ------------------------------------------------------------------------ */
+size_t svg_block_energy_workspace_size(int B, int H, int N);
+
+svg_status svg_block_energy(const void* q, const void* k, int dtype,
+                            int B, int H, int N, int d, float* energy,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/* --------------------------------------------------------------------------
+ * 3c. Calibrated key-block lists
+ *    [CAL] section 3.1: for every list l, input r and query block i, sort the
+ *    key blocks by descending energy (ties: smaller index first) and keep the
+ *    shortest prefix whose running sum (float64, in that order) reaches eps;
+ *    over the R inputs keep block c iff (#inputs keeping c) / R >= rho
+ *    (float64); a row left empty keeps the block of largest summed energy
+ *    (float64 sum over inputs in order; smallest index on ties).
+ *
+ *  energy    device float [R][L][nQB][nKB] (e.g. svg_block_energy outputs for
+ *            R inputs, with L = B*H lists).  1 <= R <= 16, nKB <= 4096.
+ *  indptr    device int32 [L][nQB + 1], offsets into the shared `indices`
+ *            (list l row i: indices[indptr[l*(nQB+1)+i] .. indptr[l*(nQB+1)+i+1])).
+ *  indices   device int32 [capacity]; nnz_out, device_status as in 3a.
+ *            capacity = L * nQB * nKB always suffices.
+ *  workspace device scratch of svg_calibrated_workspace_size(...) bytes.
+ * Given the same energies, the lists are bit-identical to a float64
+ * evaluation of the rule above (the running sums use the same order).
+ * ------------------------------------------------------------------------ */
+size_t svg_calibrated_workspace_size(int L, int nQB, int nKB);
+
+svg_status svg_build_block_mask_calibrated(const float* energy, int R, int L,
+                                           int nQB, int nKB, double eps, double rho,
+                                           int32_t* indptr, int32_t* indices,
+                                           int64_t capacity, int64_t* nnz_out,
+                                           int32_t* device_status,
+                                           void* workspace, size_t workspace_bytes,
+                                           void* stream);
+
+/* --------------------------------------------------------------------------
+ * 4. Block-sparse attention
+ *    [SURV] section 2.1 (softmax(Q K^T / sqrt(d)) V), [CAL] sections 2.2 and
+ *    3.3 (128x128 tiles, per-query-block list of kept key blocks).  For every
+ *    (b, h) and query tile i, with l = list_id[b*H + h]:
+ *        o[rows of tile i] = softmax over every key j < N of every kept tile
+ *                            (scale * q . k_j) . v_j
+ *    A kept tile is attended in full; a query tile with an empty list gets
+ *    o = 0.  Heads that run temporal pass token-major q/k/v and get
+ *    token-major o (see svg_permute_*).
+ *
+ *  q, k, v, o   device [B, H, N, d]; o may not alias q, k or v.
+ *  list_id      device int32 [B*H] in [0, n_lists).  With the three
+ *               geometric lists concatenated as (spatial, temporal, dense),
+ *               the profiling output mode_out is a valid list_id.
+ *  indptr       device int32 [n_lists][n_qblocks + 1], absolute offsets into
+ *               `indices`; n_qblocks must equal nB.
+ *  indices      device int32, key-block indices in [0, nB), ascending per row.
+ *  scale        softmax scale; 0 selects 1/sqrt(d).
+ *  device_status  optional device int32 (may be NULL), see SVG_DEVICE_*.
+ * Arithmetic (bf16): bf16 tensor-core products with fp32 accumulation, fp32
+ * online softmax; the probabilities enter P.V as two bf16 terms (P_hi + P_lo,
+ * about 16 significant bits); output rounded to nearest bf16.  fp32 inputs
+ * use fp32 arithmetic throughout.
+ * ------------------------------------------------------------------------ */
+svg_status svg_sparse_attn(const void* q, const void* k, const void* v, void* o, int dtype,
+                           int B, int H, int N, int d,
+                           const int32_t* list_id, int n_lists, int n_qblocks,
+                           const int32_t* indptr, const int32_t* indices,
+                           float scale, int32_t* device_status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SVG_B200_H_ */

@@ -1,0 +1,245 @@
+"""B200 (sm_100a) sparse spatial/temporal 3D attention for video DiTs.
+
+Thin Python binding of the C ABI in include/svg.h (libsvg_b200.so).  Each
+function below marshals torch tensors into pointers, sizes and the current
+CUDA stream and calls the entry point of the same name; every step of the
+computation runs in the library's CUDA kernels.  torch is used only to
+allocate device memory (outputs and scratch the caller did not pass) and to
+name the stream.
+
+The layer the library implements (Sparse VideoGen article,
+m.jxzklqfsx.com/article/815093.html; CalibAtt article, lpnh.cn/news/568491):
+
+    mse, mode = svg_profile_heads(q, k, v, F, P, w, sample_idx)
+    lists     = geometric_lists(F, P, w, N)            # spatial, temporal, dense
+    q', k', v' = svg_permute_token_major(x, F, P, mode)  for x in (q, k, v)
+    o'        = svg_sparse_attn(q', k', v', mode, *lists)
+    o         = svg_permute_frame_major(o', F, P, mode)
+
+``svg_layer`` runs exactly that sequence.
+"""
+from __future__ import annotations
+
+from typing import NamedTuple, Optional, Sequence
+
+import torch
+
+from . import _lib
+from ._lib import (SVG_BF16, SVG_FP32, SVG_MODE_DENSE, SVG_MODE_SPATIAL, SVG_MODE_TEMPORAL,
+                   SVG_TILE, SvgError)
+
+__all__ = [
+    "SVG_MODE_SPATIAL", "SVG_MODE_TEMPORAL", "SVG_MODE_DENSE", "SVG_TILE", "SvgError",
+    "BlockLists", "svg_version", "svg_profile_heads", "svg_permute_token_major",
+    "svg_permute_frame_major", "svg_build_block_mask", "svg_block_energy",
+    "svg_build_block_mask_calibrated", "svg_sparse_attn", "geometric_lists", "svg_layer",
+    "n_tiles",
+]
+
+
+def n_tiles(N: int) -> int:
+    return (N + SVG_TILE - 1) // SVG_TILE
+
+
+def svg_version() -> str:
+    return _lib.lib.svg_version().decode()
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return SVG_BF16
+    if t.dtype == torch.float32:
+        return SVG_FP32
+    raise TypeError(f"unsupported dtype {t.dtype} (bf16 or float32)")
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _check_qkv(*ts: torch.Tensor):
+    t0 = ts[0]
+    for t in ts:
+        if t.dim() != 4 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("tensors must be contiguous CUDA [B, H, N, d]")
+        if t.shape != t0.shape or t.dtype != t0.dtype:
+            raise ValueError("q, k, v must share shape and dtype")
+    return t0.shape
+
+
+def _scratch(nbytes: int, device) -> torch.Tensor:
+    # torch's caching allocator hands out 512-byte aligned blocks
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+class BlockLists(NamedTuple):
+    """Several CSR key-block lists sharing one indices buffer.
+    indptr: int32 [n_lists * (n_qblocks + 1)], absolute offsets into indices."""
+    indptr: torch.Tensor
+    indices: torch.Tensor
+    n_lists: int
+    n_qblocks: int
+
+
+# --------------------------------------------------------------------- steps
+
+def svg_profile_heads(q, k, v, frames: int, tokens_per_frame: int, spatial_width: int,
+                      sample_idx: torch.Tensor, *, mse_out=None, mode_out=None, workspace=None,
+                      stream=None):
+    """Online profiling; returns (mse [B*H, 2] float32, mode [B*H] int32)."""
+    B, H, N, d = _check_qkv(q, k, v)
+    S = sample_idx.numel()
+    dev = q.device
+    if mse_out is None:
+        mse_out = torch.empty(B * H, 2, dtype=torch.float32, device=dev)
+    if mode_out is None:
+        mode_out = torch.empty(B * H, dtype=torch.int32, device=dev)
+    need = _lib.lib.svg_profile_workspace_size(B, H, N, d, S)
+    if workspace is None:
+        workspace = _scratch(need, dev)
+    _lib.call("svg_profile_heads", q.data_ptr(), k.data_ptr(), v.data_ptr(), _dt(q), B, H, N, d,
+              frames, tokens_per_frame, spatial_width, sample_idx.data_ptr(), S,
+              mse_out.data_ptr(), mode_out.data_ptr(), workspace.data_ptr(), workspace.numel(),
+              _stream(stream))
+    return mse_out, mode_out
+
+
+def _permute(name, x, frames, tokens_per_frame, mode, out, stream):
+    B, H, N, d = _check_qkv(x)
+    if out is None:
+        out = torch.empty_like(x)
+    _lib.call(name, x.data_ptr(), out.data_ptr(), _dt(x), B, H, N, d, frames, tokens_per_frame,
+              _ptr(mode), _stream(stream))
+    return out
+
+
+def svg_permute_token_major(x, frames: int, tokens_per_frame: int, mode=None, out=None,
+                            stream=None):
+    """y[b,h,s*F+f] = x[b,h,f*P+s] for TEMPORAL heads (all heads if mode is None)."""
+    return _permute("svg_permute_token_major", x, frames, tokens_per_frame, mode, out, stream)
+
+
+def svg_permute_frame_major(x, frames: int, tokens_per_frame: int, mode=None, out=None,
+                            stream=None):
+    """The inverse of svg_permute_token_major."""
+    return _permute("svg_permute_frame_major", x, frames, tokens_per_frame, mode, out, stream)
+
+
+def svg_build_block_mask(kind: int, frames: int, tokens_per_frame: int, spatial_width: int,
+                         N: int, *, indptr=None, indices=None, index_base: int = 0, nnz=None,
+                         status=None, device=None, stream=None):
+    """Geometric key-block list of one kind; returns (indptr, indices, nnz).
+    indices has capacity nB*nB unless given; nnz is a device int64 [1]."""
+    nb = n_tiles(N)
+    device = device or torch.device("cuda")
+    if indptr is None:
+        indptr = torch.empty(nb + 1, dtype=torch.int32, device=device)
+    if indices is None:
+        indices = torch.empty(nb * nb, dtype=torch.int32, device=device)
+    if nnz is None:
+        nnz = torch.empty(1, dtype=torch.int64, device=device)
+    _lib.call("svg_build_block_mask", kind, frames, tokens_per_frame, spatial_width, N,
+              indptr.data_ptr(), indices.data_ptr(), indices.numel(), index_base, nnz.data_ptr(),
+              _ptr(status), _stream(stream))
+    return indptr, indices, nnz
+
+
+def geometric_lists(frames: int, tokens_per_frame: int, spatial_width: int, N: int,
+                    device=None, stream=None) -> BlockLists:
+    """The spatial, temporal and dense lists in one BlockLists (list id = mode)."""
+    nb = n_tiles(N)
+    device = device or torch.device("cuda")
+    indptr = torch.empty(3 * (nb + 1), dtype=torch.int32, device=device)
+    indices = torch.empty(3 * nb * nb, dtype=torch.int32, device=device)
+    for kind in (SVG_MODE_SPATIAL, SVG_MODE_TEMPORAL, SVG_MODE_DENSE):
+        base = kind * nb * nb
+        svg_build_block_mask(kind, frames, tokens_per_frame, spatial_width, N,
+                             indptr=indptr[kind * (nb + 1):(kind + 1) * (nb + 1)],
+                             indices=indices[base:base + nb * nb], index_base=base,
+                             device=device, stream=stream)
+    return BlockLists(indptr, indices, 3, nb)
+
+
+def svg_block_energy(q, k, *, out=None, workspace=None, stream=None):
+    """Dense block energy E [B*H, nB, nB] (float32)."""
+    B, H, N, d = _check_qkv(q, k)
+    nb = n_tiles(N)
+    if out is None:
+        out = torch.empty(B * H, nb, nb, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = _scratch(_lib.lib.svg_block_energy_workspace_size(B, H, N), q.device)
+    _lib.call("svg_block_energy", q.data_ptr(), k.data_ptr(), _dt(q), B, H, N, d, out.data_ptr(),
+              workspace.data_ptr(), workspace.numel(), _stream(stream))
+    return out
+
+
+def svg_build_block_mask_calibrated(energy: torch.Tensor, eps: float, rho: float, *,
+                                    status=None, stream=None) -> BlockLists:
+    """energy [R, L, nQB, nKB] float32 -> one list per L (BlockLists)."""
+    if energy.dim() != 4 or energy.dtype != torch.float32 or not energy.is_contiguous():
+        raise ValueError("energy must be contiguous float32 [R, L, nQB, nKB]")
+    R, L, nq, nk = energy.shape
+    dev = energy.device
+    indptr = torch.empty(L * (nq + 1), dtype=torch.int32, device=dev)
+    indices = torch.empty(L * nq * nk, dtype=torch.int32, device=dev)
+    nnz = torch.empty(1, dtype=torch.int64, device=dev)
+    ws = _scratch(_lib.lib.svg_calibrated_workspace_size(L, nq, nk), dev)
+    _lib.call("svg_build_block_mask_calibrated", energy.data_ptr(), R, L, nq, nk, float(eps),
+              float(rho), indptr.data_ptr(), indices.data_ptr(), indices.numel(), nnz.data_ptr(),
+              _ptr(status), ws.data_ptr(), ws.numel(), _stream(stream))
+    return BlockLists(indptr, indices, L, nq)
+
+
+def svg_sparse_attn(q, k, v, list_id: torch.Tensor, lists: BlockLists, *, scale: float = 0.0,
+                    out=None, status=None, stream=None):
+    """Block-sparse attention over 128x128 tiles; returns o [B, H, N, d]."""
+    B, H, N, d = _check_qkv(q, k, v)
+    if out is None:
+        out = torch.empty_like(q)
+    _lib.call("svg_sparse_attn", q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), _dt(q),
+              B, H, N, d, list_id.data_ptr(), lists.n_lists, lists.n_qblocks,
+              lists.indptr.data_ptr(), lists.indices.data_ptr(), float(scale), _ptr(status),
+              _stream(stream))
+    return out
+
+
+# --------------------------------------------------------------------- layer
+
+class LayerBuffers:
+    """Preallocated buffers for svg_layer at one shape (reused across steps)."""
+
+    def __init__(self, q: torch.Tensor, S: int):
+        B, H, N, d = q.shape
+        dev = q.device
+        self.qp = torch.empty_like(q)
+        self.kp = torch.empty_like(q)
+        self.vp = torch.empty_like(q)
+        self.op = torch.empty_like(q)
+        self.o = torch.empty_like(q)
+        self.mse = torch.empty(B * H, 2, dtype=torch.float32, device=dev)
+        self.mode = torch.empty(B * H, dtype=torch.int32, device=dev)
+        self.ws = _scratch(_lib.lib.svg_profile_workspace_size(B, H, N, d, S), dev)
+
+
+def svg_layer(q, k, v, frames: int, tokens_per_frame: int, spatial_width: int,
+              sample_idx: torch.Tensor, lists: BlockLists, bufs: Optional[LayerBuffers] = None,
+              stream=None):
+    """One attention layer: profile -> permute temporal heads -> block-sparse
+    attention on the list the mode selects -> permute back.
+    Returns (o, mode, mse)."""
+    if bufs is None:
+        bufs = LayerBuffers(q, sample_idx.numel())
+    F, P = frames, tokens_per_frame
+    svg_profile_heads(q, k, v, F, P, spatial_width, sample_idx, mse_out=bufs.mse,
+                      mode_out=bufs.mode, workspace=bufs.ws, stream=stream)
+    for x, y in ((q, bufs.qp), (k, bufs.kp), (v, bufs.vp)):
+        svg_permute_token_major(x, F, P, bufs.mode, out=y, stream=stream)
+    svg_sparse_attn(bufs.qp, bufs.kp, bufs.vp, bufs.mode, lists, out=bufs.op, stream=stream)
+    svg_permute_frame_major(bufs.op, F, P, bufs.mode, out=bufs.o, stream=stream)
+    return bufs.o, bufs.mode, bufs.mse

@@ -1,0 +1,41 @@
+// svg_sparse_attn: argument validation and dispatch.
+#include <math.h>
+
+#include "attn.cuh"
+
+using namespace svg;
+
+extern "C" svg_status svg_sparse_attn(const void* q, const void* k, const void* v, void* o,
+                                      int dtype, int B, int H, int N, int d,
+                                      const int32_t* list_id, int n_lists, int n_qblocks,
+                                      const int32_t* indptr, const int32_t* indices, float scale,
+                                      int32_t* device_status, void* stream) {
+  clear_error();
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || list_id == nullptr ||
+      indptr == nullptr || indices == nullptr)
+    return fail(SVG_ERR_INVALID_ARG, "sparse_attn: null pointer");
+  if (dtype != SVG_BF16 && dtype != SVG_FP32)
+    return fail(SVG_ERR_INVALID_ARG, "sparse_attn: bad dtype %d", dtype);
+  if (B <= 0 || H <= 0 || N <= 0 || B * H > 65535)
+    return fail(SVG_ERR_INVALID_ARG, "sparse_attn: bad shape B=%d H=%d N=%d", B, H, N);
+  if (d != 64 && d != 128) return fail(SVG_ERR_INVALID_ARG, "sparse_attn: d=%d not in {64,128}", d);
+  if (n_lists <= 0) return fail(SVG_ERR_INVALID_ARG, "sparse_attn: n_lists must be positive");
+  if (n_qblocks != n_tiles(N))
+    return fail(SVG_ERR_INVALID_ARG, "sparse_attn: n_qblocks=%d but ceil(N/128)=%d", n_qblocks,
+                n_tiles(N));
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return fail(SVG_ERR_INVALID_ARG, "sparse_attn: tensors must be 16-byte aligned");
+  const long long bytes = static_cast<long long>(B) * H * N * d * elt_bytes(dtype);
+  const char* ob = static_cast<const char*>(o);
+  for (const void* t : {q, k, v}) {
+    const char* tb = static_cast<const char*>(t);
+    if (ob < tb + bytes && tb < ob + bytes)
+      return fail(SVG_ERR_INVALID_ARG, "sparse_attn: o overlaps an input");
+  }
+  if (!(scale >= 0.f) || isinf(scale)) return fail(SVG_ERR_INVALID_ARG, "sparse_attn: bad scale");
+  AttnArgs a{q, k, v, o, dtype, B, H, N, d, list_id, n_lists, n_qblocks, indptr, indices,
+             scale == 0.f ? 1.f / sqrtf(static_cast<float>(d)) : scale, device_status};
+  cudaStream_t s = as_stream(stream);
+  if (dtype == SVG_FP32) return d == 64 ? launch_attn_fp32<64>(a, s) : launch_attn_fp32<128>(a, s);
+  return d == 64 ? launch_attn_sm100<64>(a, s) : launch_attn_sm100<128>(a, s);
+}

@@ -1,0 +1,499 @@
+// Block-sparse attention on the B200 tensor core (tcgen05 + TMEM + TMA).
+//
+// Video-diffusion acceleration survey (wmrh.cn/news/48564), section 2.1:
+// o = softmax(Q K^T / sqrt(d_k)) V; section 5.3: tiled on chip with an online
+// softmax.  CalibAtt article (lpnh.cn/news/568491), sections 2.2 and 3.3:
+// keep/skip decisions on 128 x 128 tiles, walked through a per-query-block
+// list of kept key blocks.
+//
+// Persistent kernel, one CTA per SM, work item = (head, 128-row query tile).
+// Warp roles (256 threads):
+//   warp 0      TMA producer: Q tile (double-buffered across items), then the
+//               K and V tiles of every kept key block into a ring of slots;
+//   warp 1      MMA issuer (one thread): S = Q K^T into TMEM (two S buffers),
+//               O += P_hi V + P_lo V with P read from TMEM and V from shared
+//               memory;
+//   warps 4-7   softmax: one thread per query row; reads S from TMEM, online
+//               softmax in fp32 with lazy rescaling (O is only rescaled when
+//               the running max grows by more than 2^8), writes P into the S
+//               buffer as two bf16 terms (P = P_hi + P_lo), and runs the
+//               epilogue (O / l -> bf16 -> swizzled shared memory -> TMA
+//               store, rows beyond N clipped).
+// Order of MMA issue per item: QK_0, QK_1, PV_0, QK_2, PV_1, ... so that the
+// tensor core computes S_{j+1} while the softmax works on S_j.
+//
+// TMEM columns: S buffer b at [128 b, 128 b + 128), O at [256, 256 + d).
+// Every mbarrier wait is bounded; a wait that gives up sets
+// SVG_DEVICE_TIMEOUT, raises a CTA-wide abort flag and every role drains out.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "attn.cuh"
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace svg {
+namespace {
+
+using namespace sm100;
+
+constexpr int kThreads = 256;
+constexpr int kBox = 16384;             // one 128-row x 128-byte TMA box
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleLog2 = 8.0f;    // lazy-rescale threshold (factor 256)
+constexpr uint32_t kSpinLimit = 1u << 22;
+
+template <int D>
+struct Cfg {
+  static constexpr int kTile = 128 * D * 2;           // bytes of a Q / K / V / O tile
+  static constexpr int kBoxes = D / 64;               // 64-column boxes per tile
+  static constexpr int kSlots = D == 64 ? 8 : 4;      // K/V ring slots
+  static constexpr int kOffQ = 0;                     // 2 Q buffers
+  static constexpr int kOffKV = 2 * kTile;
+  static constexpr int kOffO = kOffKV + kSlots * kTile;
+  static constexpr int kOffBar = kOffO + kTile;
+  static constexpr int kBars = 2 + 2 + 2 * kSlots + 2 + 2 + 2 + 1;
+  static constexpr int kSmem = kOffBar + kBars * 8 + 16 + 1024;  // + alignment slack
+  static constexpr uint32_t kIdescQK = idesc_bf16(128, 128, false);
+  static constexpr uint32_t kIdescPV = idesc_bf16(128, D, true);
+};
+
+struct Maps {
+  CUtensorMap q, k, v, o;
+};
+
+struct Bars {
+  uint64_t* q_full;   // [2]
+  uint64_t* q_empty;  // [2]
+  uint64_t* kv_full;  // [slots]
+  uint64_t* kv_empty; // [slots]
+  uint64_t* s_full;   // [2]
+  uint64_t* p_ready;  // [2]
+  uint64_t* o_done;   // [2]
+  uint64_t* o_free;   // [1]
+};
+
+// The list of (bh, qt): [beg, end) into indices, or empty.
+__device__ __forceinline__ void item_list(const AttnArgs& a, int bh, int qt, int& beg, int& end,
+                                          bool report = false) {
+  beg = end = 0;
+  const int lid = a.list_id[bh];
+  if (lid < 0 || lid >= a.n_lists) {
+    if (report) set_status(a.status, SVG_DEVICE_BAD_LIST_ID);
+    return;
+  }
+  const int32_t* ip = a.indptr + static_cast<long long>(lid) * (a.n_qblocks + 1);
+  const int b = ip[qt], e = ip[qt + 1];
+  if (b < 0 || e < b) return;
+  beg = b;
+  end = e;
+}
+
+__device__ __forceinline__ bool valid_tile(int j, int nb) { return j >= 0 && j < nb; }
+
+// Bounded wait on an mbarrier phase; false if it timed out or another role
+// aborted.
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                         int32_t* status) {
+  const uint32_t addr = smem_u32(bar);
+  for (uint32_t i = 0; i < kSpinLimit; ++i) {
+    if (mbar_try_wait(addr, parity)) return true;
+    if ((i & 255u) == 255u && *abort_flag) return false;
+  }
+  *abort_flag = 1;
+  set_status(status, SVG_DEVICE_TIMEOUT);
+  return false;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_sm100_kernel(const __grid_constant__ Maps maps, const AttnArgs a) {
+  using C = Cfg<D>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* bar_base = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  Bars B;
+  B.q_full = bar_base;
+  B.q_empty = bar_base + 2;
+  B.kv_full = bar_base + 4;
+  B.kv_empty = B.kv_full + C::kSlots;
+  B.s_full = B.kv_empty + C::kSlots;
+  B.p_ready = B.s_full + 2;
+  B.o_done = B.p_ready + 2;
+  B.o_free = B.o_done + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(B.o_free + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int N = a.N, nb = n_tiles(N);
+  const int BH = a.B * a.H;
+  const int n_items = BH * nb;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&B.q_full[i], 1);
+      mbar_init(&B.q_empty[i], 1);
+      mbar_init(&B.s_full[i], 1);
+      mbar_init(&B.p_ready[i], 4);
+      mbar_init(&B.o_done[i], 1);
+    }
+    for (int i = 0; i < C::kSlots; ++i) {
+      mbar_init(&B.kv_full[i], 1);
+      mbar_init(&B.kv_empty[i], 1);
+    }
+    mbar_init(B.o_free, 4);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&maps.q);
+    prefetch_tmap(&maps.k);
+    prefetch_tmap(&maps.v);
+    prefetch_tmap(&maps.o);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem_s0 = tmem, tmem_o = tmem + 256;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t L = 0, c = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+        const int bh = item / nb, qt = item - bh * nb;
+        int beg, end;
+        item_list(a, bh, qt, beg, end, true);
+        int first = beg;
+        while (first < end && !valid_tile(a.indices[first], nb)) {
+          set_status(a.status, SVG_DEVICE_BAD_INDEX);
+          ++first;
+        }
+        if (first == end) continue;
+        const int qb = c & 1;
+        if (!(ok = wait_bar(&B.q_empty[qb], ((c >> 1) & 1) ^ 1, abort_flag, a.status))) break;
+        mbar_arrive_expect_tx(&B.q_full[qb], C::kTile);
+        for (int bx = 0; bx < C::kBoxes; ++bx)
+          tma_load_3d(smem + C::kOffQ + qb * C::kTile + bx * kBox, &maps.q, &B.q_full[qb], 64 * bx,
+                      qt * 128, bh);
+        for (int e = first; e < end && ok; ++e) {
+          const int j = a.indices[e];
+          if (!valid_tile(j, nb)) {
+            set_status(a.status, SVG_DEVICE_BAD_INDEX);
+            continue;
+          }
+          for (int t = 0; t < 2; ++t, ++L) {
+            const int slot = L % C::kSlots;
+            if (!(ok = wait_bar(&B.kv_empty[slot], ((L / C::kSlots) & 1) ^ 1, abort_flag,
+                                a.status)))
+              break;
+            mbar_arrive_expect_tx(&B.kv_full[slot], C::kTile);
+            const CUtensorMap* m = t == 0 ? &maps.k : &maps.v;
+            for (int bx = 0; bx < C::kBoxes; ++bx)
+              tma_load_3d(smem + C::kOffKV + slot * C::kTile + bx * kBox, m, &B.kv_full[slot],
+                          64 * bx, j * 128, bh);
+          }
+        }
+        ++c;
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t L = 0, g = 0, c = 0;
+      bool ok = true;
+      auto issue_pv = [&](uint32_t gp, uint32_t lv, bool first_of_item) -> bool {
+        const int sb = gp & 1;
+        if (!wait_bar(&B.p_ready[sb], (gp >> 1) & 1, abort_flag, a.status)) return false;
+        if (first_of_item && c > 0 && !wait_bar(B.o_free, (c - 1) & 1, abort_flag, a.status))
+          return false;
+        const int slot = lv % C::kSlots;
+        if (!wait_bar(&B.kv_full[slot], (lv / C::kSlots) & 1, abort_flag, a.status)) return false;
+        tc_fence_after();
+        const uint32_t vbase = smem_u32(smem + C::kOffKV + slot * C::kTile);
+        // O (+)= P_hi V + P_lo V; P_hi in columns [0, 64), P_lo in [64, 128)
+#pragma unroll
+        for (int part = 0; part < 2; ++part)
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t bdesc = sdesc_sw128(vbase + kk * 2048, kBox, 1024);
+            mma_ts(tmem_o, tmem_s0 + sb * 128 + part * 64 + kk * 8, bdesc, C::kIdescPV,
+                   (first_of_item && part == 0 && kk == 0) ? 0u : 1u);
+          }
+        tc_commit(&B.kv_empty[slot]);
+        tc_commit(&B.o_done[sb]);
+        return true;
+      };
+      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+        const int bh = item / nb, qt = item - bh * nb;
+        int beg, end;
+        item_list(a, bh, qt, beg, end);
+        bool any = false;
+        for (int e = beg; e < end && !any; ++e) any = valid_tile(a.indices[e], nb);
+        if (!any) continue;
+        const int qb = c & 1;
+        if (!(ok = wait_bar(&B.q_full[qb], (c >> 1) & 1, abort_flag, a.status))) break;
+        const uint32_t qbase = smem_u32(smem + C::kOffQ + qb * C::kTile);
+        bool have_pending = false, pending_first = false;
+        uint32_t pend_g = 0, pend_lv = 0;
+        bool first = true;
+        for (int e = beg; e < end && ok; ++e) {
+          if (!valid_tile(a.indices[e], nb)) continue;
+          const int slot = L % C::kSlots;
+          if (!(ok = wait_bar(&B.kv_full[slot], (L / C::kSlots) & 1, abort_flag, a.status))) break;
+          tc_fence_after();
+          const int sb = g & 1;
+          const uint32_t kbase = smem_u32(smem + C::kOffKV + slot * C::kTile);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
+            mma_ss(tmem_s0 + sb * 128, sdesc_sw128(qbase + off, 16, 1024),
+                   sdesc_sw128(kbase + off, 16, 1024), C::kIdescQK, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(&B.s_full[sb]);
+          tc_commit(&B.kv_empty[slot]);
+          if (have_pending && !(ok = issue_pv(pend_g, pend_lv, pending_first))) break;
+          have_pending = true;
+          pending_first = first;
+          pend_g = g;
+          pend_lv = L + 1;
+          L += 2;
+          ++g;
+          first = false;
+        }
+        if (!ok) break;
+        tc_commit(&B.q_empty[qb]);  // Q buffer free once its last QK^T completes
+        if (!(ok = issue_pv(pend_g, pend_lv, pending_first))) break;
+        ++c;
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax
+    const int q4 = warp - 4;
+    const int row = q4 * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
+    const float sl2 = a.scale * kLog2e;
+    unsigned char* ost = smem + C::kOffO;
+    uint32_t g = 0;
+    bool ok = true;
+    bool store_pending = false;
+    for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+      const int bh = item / nb, qt = item - bh * nb;
+      int beg, end;
+      item_list(a, bh, qt, beg, end);
+      float m_used = -INFINITY, l = 0.f;
+      bool first = true;
+      for (int e = beg; e < end && ok; ++e) {
+        const int j = a.indices[e];
+        if (!valid_tile(j, nb)) continue;
+        const int sb = g & 1;
+        if (!(ok = wait_bar(&B.s_full[sb], (g >> 1) & 1, abort_flag, a.status))) break;
+        tc_fence_after();
+        float s[128];
+        {
+          uint32_t r0[32], r1[32], r2[32], r3[32];
+          const uint32_t sa = tmem_s0 + lane_off + sb * 128;
+          tmem_ld32(sa, r0);
+          tmem_ld32(sa + 32, r1);
+          tmem_ld32(sa + 64, r2);
+          tmem_ld32(sa + 96, r3);
+          tmem_wait_ld();
+          reg_fence32(r0);
+          reg_fence32(r1);
+          reg_fence32(r2);
+          reg_fence32(r3);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            s[i] = __uint_as_float(r0[i]);
+            s[32 + i] = __uint_as_float(r1[i]);
+            s[64 + i] = __uint_as_float(r2[i]);
+            s[96 + i] = __uint_as_float(r3[i]);
+          }
+        }
+        const int valid_cols = min(128, N - j * 128);
+        if (valid_cols < 128) {
+#pragma unroll
+          for (int i = 0; i < 128; ++i)
+            if (i >= valid_cols) s[i] = -INFINITY;
+        }
+        float mx = s[0];
+#pragma unroll
+        for (int i = 1; i < 128; ++i) mx = fmaxf(mx, s[i]);
+        const float tm = mx * sl2;
+        if (first) {
+          m_used = tm;
+        } else {
+          const bool need = tm > m_used + kRescaleLog2;
+          if (__any_sync(0xffffffffu, need)) {
+            // O must hold PV of the previous tile before it is rescaled
+            if (!(ok = wait_bar(&B.o_done[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_flag,
+                                a.status)))
+              break;
+            tc_fence_after();
+            const float m_new = need ? tm : m_used;
+            const float alpha = exp2f(m_used - m_new);
+            uint32_t r[32];
+#pragma unroll
+            for (int ch = 0; ch < D / 32; ++ch) {
+              tmem_ld32(tmem_o + lane_off + ch * 32, r);
+              tmem_wait_ld();
+              reg_fence32(r);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+              tmem_st32(tmem_o + lane_off + ch * 32, r);
+              tmem_wait_st();  // r is reused by the next chunk
+            }
+            l *= alpha;
+            m_used = m_new;
+          }
+        }
+        const float neg = -m_used;
+        {
+          // P = hi + lo, both bf16: hi is the nearest bf16 to p, lo the
+          // nearest bf16 to the remainder.  O accumulates P_hi V + P_lo V, so
+          // the weights carry ~16 bits instead of bf16's 8.
+          const uint32_t sa = tmem_s0 + lane_off + sb * 128;
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            uint32_t hi[32], lo[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float p0 = fast_exp2(fmaf(s[64 * half + 2 * i], sl2, neg));
+              const float p1 = fast_exp2(fmaf(s[64 * half + 2 * i + 1], sl2, neg));
+              hi[i] = pack_bf16x2(p0, p1);
+              lo[i] = pack_bf16x2(p0 - __uint_as_float(hi[i] << 16),
+                                  p1 - __uint_as_float(hi[i] & 0xffff0000u));
+              l += p0 + p1;
+            }
+            tmem_st32(sa + 32 * half, hi);
+            tmem_st32(sa + 64 + 32 * half, lo);
+            tmem_wait_st();  // hi / lo are rewritten by the next half
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&B.p_ready[sb]);
+        first = false;
+        ++g;
+      }
+      if (!ok) break;
+      // ---------------------------------------------------------- epilogue
+      const bool empty = first;
+      if (!empty) {
+        if (!(ok = wait_bar(&B.o_done[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_flag, a.status)))
+          break;
+        tc_fence_after();
+      }
+      if (store_pending && row == 0) bulk_wait_read0();
+      named_bar_sync(1, 128);
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t r[32];
+        if (!empty) {
+          tmem_ld32(tmem_o + lane_off + ch * 32, r);
+          tmem_wait_ld();
+          reg_fence32(r);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) r[i] = 0u;
+        }
+        // 32 fp32 columns -> 64 bytes of bf16 = 4 swizzled 16-byte chunks
+#pragma unroll
+        for (int c16 = 0; c16 < 4; ++c16) {
+          uint4 v;
+          v.x = pack_bf16x2(__uint_as_float(r[8 * c16 + 0]) * inv, __uint_as_float(r[8 * c16 + 1]) * inv);
+          v.y = pack_bf16x2(__uint_as_float(r[8 * c16 + 2]) * inv, __uint_as_float(r[8 * c16 + 3]) * inv);
+          v.z = pack_bf16x2(__uint_as_float(r[8 * c16 + 4]) * inv, __uint_as_float(r[8 * c16 + 5]) * inv);
+          v.w = pack_bf16x2(__uint_as_float(r[8 * c16 + 6]) * inv, __uint_as_float(r[8 * c16 + 7]) * inv);
+          const int col = ch * 32 + c16 * 8;  // first column of this chunk
+          const int box = col >> 6, cc = (col & 63) >> 3;
+          *reinterpret_cast<uint4*>(ost + box * kBox + row * 128 + ((cc ^ (row & 7)) << 4)) = v;
+        }
+      }
+      if (!empty) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(B.o_free);
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(1, 128);
+      if (row == 0) {
+        for (int bx = 0; bx < C::kBoxes; ++bx)
+          tma_store_3d(&maps.o, ost + bx * kBox, 64 * bx, qt * 128, bh);
+        bulk_commit();
+      }
+      store_pending = true;
+    }
+    if (row == 0) bulk_wait0();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// ------------------------------------------------------------ host side
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// [B*H][N][d] bf16 viewed as a 3-D tensor (d, N, B*H); box 64 x 128 x 1,
+// 128-byte swizzle.  Rows beyond N are zero-filled on load, dropped on store.
+bool make_map(CUtensorMap* m, const void* base, int BH, int N, int d) {
+  auto enc = get_encode();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+}  // namespace
+
+template <int D>
+svg_status launch_attn_sm100(const AttnArgs& a, cudaStream_t s) {
+  using C = Cfg<D>;
+  Maps maps;
+  const int BH = a.B * a.H;
+  if (!make_map(&maps.q, a.q, BH, a.N, D) || !make_map(&maps.k, a.k, BH, a.N, D) ||
+      !make_map(&maps.v, a.v, BH, a.N, D) || !make_map(&maps.o, a.o, BH, a.N, D))
+    return fail(SVG_ERR_CUDA, "sparse_attn: cannot encode TMA descriptors");
+  if (cudaFuncSetAttribute(attn_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           C::kSmem) != cudaSuccess)
+    return fail(SVG_ERR_CUDA, "sparse_attn: cannot reserve %d bytes of shared memory", C::kSmem);
+  const long long items = static_cast<long long>(BH) * n_tiles(a.N);
+  const int grid = static_cast<int>(items < sm_count() ? items : sm_count());
+  attn_sm100_kernel<D><<<grid, kThreads, C::kSmem, s>>>(maps, a);
+  return check_launch("sparse_attn sm100");
+}
+
+template svg_status launch_attn_sm100<64>(const AttnArgs&, cudaStream_t);
+template svg_status launch_attn_sm100<128>(const AttnArgs&, cudaStream_t);
+
+}  // namespace svg

@@ -1,0 +1,448 @@
+// Online head profiling.
+//
+// Sparse VideoGen article (m.jxzklqfsx.com/article/815093.html), section
+// "動態自適應的稀疏策略", steps 1-3: at every step a few query tokens (about
+// 64) are sampled; their attention outputs are computed under the spatial and
+// the temporal mask and compared with dense attention; each head takes the
+// mask with the smaller error.  Error = mean over the S x d sampled outputs of
+// the squared difference; an exact tie keeps SPATIAL.
+//
+// Work split (one layer, all heads, one launch each):
+//   partial  grid (chunks, B*H, 2): the keys of a head are cut into `chunks`
+//            contiguous ranges; each CTA streams one range through shared
+//            memory and keeps an online-softmax state (max, sum, o) per
+//            sampled row, for the dense mask (z = 0) or the spatial mask
+//            (z = 1).  bf16: mma.sync tensor-core products; fp32: SIMT.
+//   combine  grid (B*H): merges the chunk states, computes the temporal
+//            output directly (a row sees only the F keys of its position),
+//            the two errors and the mode.
+// The pass reads K and V once per mask variant: it is bound by HBM and the
+// legacy MMA rate, and costs a few percent of the attention it configures.
+#include <float.h>
+
+#include "common.cuh"
+#include "mma_frag.cuh"
+
+namespace svg {
+namespace {
+
+constexpr int kRows = 64;          // sampled rows per head (S padded to 64)
+constexpr int kKeys = 64;          // keys per shared-memory stage
+constexpr int kThreads = 128;      // 4 warps x 16 rows
+constexpr int kTargetCtas = 1024;  // partial-grid size the chunking aims for
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Sampled indices outside [0, N) are clamped into range (never read out of bounds).
+__device__ __forceinline__ int clamp_index(int n, int N) { return n < 0 ? 0 : (n >= N ? N - 1 : n); }
+
+struct ProfileShape {
+  int chunks;     // key ranges per head
+  int chunk_len;  // keys per range (multiple of kKeys)
+};
+
+ProfileShape profile_shape(int B, int H, int N) {
+  const long long bh2 = 2LL * B * H;
+  long long chunks = (kTargetCtas + bh2 - 1) / bh2;
+  const long long max_chunks = (N + 4 * kKeys - 1) / (4 * kKeys);  // >= 4 stages per range
+  if (chunks > max_chunks) chunks = max_chunks;
+  if (chunks < 1) chunks = 1;
+  long long len = (N + chunks - 1) / chunks;
+  len = (len + kKeys - 1) / kKeys * kKeys;
+  chunks = (N + len - 1) / len;
+  return {static_cast<int>(chunks), static_cast<int>(len)};
+}
+
+// floats per partial state row: m, l, o[D]
+template <int D>
+constexpr int state_floats() {
+  return D + 2;
+}
+
+size_t partial_bytes(int B, int H, int N, int d) {
+  ProfileShape ps = profile_shape(B, H, N);
+  return static_cast<size_t>(B) * H * 2 * ps.chunks * kRows * (d + 2) * sizeof(float);
+}
+
+// --------------------------------------------------------------- bf16 partial
+
+template <int D>
+__global__ void __launch_bounds__(kThreads) profile_partial_bf16(
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+    const __nv_bfloat16* __restrict__ v, const int32_t* __restrict__ idx, int S, int N, int P,
+    int width, float scale_log2, int chunks, int chunk_len, float* __restrict__ ws) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  constexpr int TILE = kKeys * D * 2;  // bytes of one K or V stage
+  unsigned char* sQ = smem;
+  unsigned char* sK = smem + kRows * D * 2;
+  unsigned char* sV = sK + 2 * TILE;
+  __shared__ int row_frame[kRows];
+
+  const int chunk = blockIdx.x, bh = blockIdx.y, variant = blockIdx.z;
+  const long long head = static_cast<long long>(bh) * N * D;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int key_begin = chunk * chunk_len;
+  const int key_end = min(N, key_begin + chunk_len);
+
+  // gather the sampled query rows (padding rows are zero)
+  for (int t = threadIdx.x; t < kRows * (D / 8); t += kThreads) {
+    const int r = t / (D / 8), c = t % (D / 8);
+    const bool ok = r < S;
+    const int n = ok ? clamp_index(idx[r], N) : 0;
+    cp_async16(sQ + swz(r, c, 2 * D), q + head + static_cast<long long>(n) * D + c * 8, ok);
+  }
+  if (threadIdx.x < kRows)
+    row_frame[threadIdx.x] = threadIdx.x < S ? clamp_index(idx[threadIdx.x], N) / P : -(1 << 29);
+  const int n_stages = (key_end - key_begin + kKeys - 1) / kKeys;
+  load_tile_async<D, kKeys, kThreads>(sK, k + head, key_begin, key_end);
+  load_tile_async<D, kKeys, kThreads>(sV, v + head, key_begin, key_end);
+  cp_async_commit();
+
+  // warp w owns rows [16 w, 16 w + 16): thread rows g and g + 8
+  const int g = lane >> 2, t4 = lane & 3;
+  float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+  float o[D / 8][4];
+#pragma unroll
+  for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+  uint32_t qa[D / 16][4];
+
+  for (int st = 0; st < n_stages; ++st) {
+    if (st + 1 < n_stages) {
+      const int nb = (st + 1) & 1;
+      load_tile_async<D, kKeys, kThreads>(sK + nb * TILE, k + head, key_begin + (st + 1) * kKeys,
+                                          key_end);
+      load_tile_async<D, kKeys, kThreads>(sV + nb * TILE, v + head, key_begin + (st + 1) * kKeys,
+                                          key_end);
+      cp_async_commit();
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    if (st == 0) load_a_frags<D>(qa, smem_u32(sQ), warp * 16);
+    const int key0 = key_begin + st * kKeys;
+    const int fr0 = row_frame[warp * 16 + g], fr1 = row_frame[warp * 16 + g + 8];
+    bool skip = false;
+    if (variant == 1) {
+      // skip the stage when none of this warp's rows has a spatial key in it
+      const int kf0 = key0 / P, kf1 = (min(key0 + kKeys, key_end) - 1) / P;
+      int lo = min(fr0, fr1), hi = max(fr0, fr1);
+#pragma unroll
+      for (int o2 = 4; o2 < 32; o2 <<= 1) {
+        lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o2));
+        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o2));
+      }
+      skip = (kf1 < lo - width) || (kf0 > hi + width);
+    }
+    if (!skip) {
+      const uint32_t kt = smem_u32(sK + (st & 1) * TILE), vt = smem_u32(sV + (st & 1) * TILE);
+      float s[kKeys / 8][4];
+      qk_frags<D, kKeys>(s, qa, kt, 0);
+      float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+      for (int n = 0; n < kKeys / 8; ++n) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int key = key0 + 8 * n + 2 * t4 + (e & 1);
+          const int fr = (e < 2) ? fr0 : fr1;
+          bool ok = key < key_end;
+          if (variant == 1) ok = ok && abs(key / P - fr) <= width;
+          s[n][e] = ok ? s[n][e] * scale_log2 : -INFINITY;
+          mx[e >> 1] = fmaxf(mx[e >> 1], s[n][e]);
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
+        mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
+        const float mn = fmaxf(m[h], mx[h]);
+        const float base = mn == -INFINITY ? 0.f : mn;
+        const float alpha = fast_exp2(m[h] - base);  // exp2(-inf) = 0 on the first stage
+        m[h] = mn;
+        l[h] *= alpha;
+#pragma unroll
+        for (int n = 0; n < D / 8; ++n) {
+          o[n][2 * h] *= alpha;
+          o[n][2 * h + 1] *= alpha;
+        }
+#pragma unroll
+        for (int n = 0; n < kKeys / 8; ++n) {
+          s[n][2 * h] = round_bf16(fast_exp2(s[n][2 * h] - base));
+          s[n][2 * h + 1] = round_bf16(fast_exp2(s[n][2 * h + 1] - base));
+          l[h] += s[n][2 * h] + s[n][2 * h + 1];
+        }
+      }
+      pv_frags<D, kKeys>(o, s, vt, 0);
+    }
+    __syncthreads();  // stage (st & 1) is refilled next iteration
+  }
+
+  // per-row partial state -> workspace [bh][variant][chunk][row][m, l, o[D]]
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    l[h] += __shfl_xor_sync(0xffffffffu, l[h], 1);
+    l[h] += __shfl_xor_sync(0xffffffffu, l[h], 2);
+  }
+  float* base = ws + ((static_cast<long long>(bh) * 2 + variant) * chunks + chunk) * kRows *
+                         state_floats<D>();
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int r = warp * 16 + g + 8 * h;
+    float* row = base + r * state_floats<D>();
+    if (t4 == 0) {
+      row[0] = m[h];
+      row[1] = l[h];
+    }
+#pragma unroll
+    for (int n = 0; n < D / 8; ++n) {
+      row[2 + 8 * n + 2 * t4] = o[n][2 * h];
+      row[2 + 8 * n + 2 * t4 + 1] = o[n][2 * h + 1];
+    }
+  }
+}
+
+// --------------------------------------------------------------- fp32 partial
+
+// SIMT fp32: warp per sampled row, lanes split the head dimension.
+template <int D>
+__global__ void __launch_bounds__(256) profile_partial_fp32(
+    const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v,
+    const int32_t* __restrict__ idx, int S, int N, int P, int width, float scale_log2, int chunks,
+    int chunk_len, float* __restrict__ ws) {
+  constexpr int E = D / 32;
+  const int chunk = blockIdx.x, bh = blockIdx.y, variant = blockIdx.z;
+  const long long head = static_cast<long long>(bh) * N * D;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int key_begin = chunk * chunk_len;
+  const int key_end = min(N, key_begin + chunk_len);
+  float* base = ws + ((static_cast<long long>(bh) * 2 + variant) * chunks + chunk) * kRows *
+                         state_floats<D>();
+  for (int r = warp; r < kRows; r += 8) {
+    float m = -INFINITY, l = 0.f, acc[E], qv[E];
+    const int n = r < S ? clamp_index(idx[r], N) : 0;
+    const int fr = n / P;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      acc[e] = 0.f;
+      qv[e] = r < S ? q[head + static_cast<long long>(n) * D + lane + 32 * e] : 0.f;
+    }
+    if (r < S) {
+      for (int j = key_begin; j < key_end; ++j) {
+        if (variant == 1 && abs(j / P - fr) > width) continue;
+        float dot = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) dot = fmaf(qv[e], k[head + static_cast<long long>(j) * D + lane + 32 * e], dot);
+#pragma unroll
+        for (int o2 = 16; o2 > 0; o2 >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o2);
+        const float t = dot * scale_log2;
+        const float mn = fmaxf(m, t);
+        const float alpha = exp2f(m - mn);
+        const float p = exp2f(t - mn);
+        l = l * alpha + p;
+#pragma unroll
+        for (int e = 0; e < E; ++e)
+          acc[e] = fmaf(p, v[head + static_cast<long long>(j) * D + lane + 32 * e], acc[e] * alpha);
+        m = mn;
+      }
+    }
+    float* row = base + r * state_floats<D>();
+    if (lane == 0) {
+      row[0] = m;
+      row[1] = l;
+    }
+#pragma unroll
+    for (int e = 0; e < E; ++e) row[2 + lane + 32 * e] = acc[e];
+  }
+}
+
+// --------------------------------------------------------------- combine
+
+template <typename T>
+__device__ __forceinline__ float to_f(T x);
+template <>
+__device__ __forceinline__ float to_f<float>(float x) {
+  return x;
+}
+template <>
+__device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) {
+  return __bfloat162float(x);
+}
+
+template <int D, typename T>
+__global__ void __launch_bounds__(256) profile_combine(
+    const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+    const int32_t* __restrict__ idx, int S, int N, int F, int P, float scale_log2, int chunks,
+    const float* __restrict__ ws, float* __restrict__ mse_out, int32_t* __restrict__ mode_out) {
+  __shared__ float o_t[kRows][D];  // temporal outputs
+  __shared__ float red[2][8];
+  const int bh = blockIdx.x;
+  const long long head = static_cast<long long>(bh) * N * D;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int E = D / 32;
+
+  // temporal mask: the F keys of the row's position, exact online softmax
+  for (int r = warp; r < S; r += 8) {
+    const int n = clamp_index(idx[r], N);
+    const int s = n % P;
+    float qv[E], acc[E], m = -INFINITY, l = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      qv[e] = to_f(q[head + static_cast<long long>(n) * D + lane + 32 * e]);
+      acc[e] = 0.f;
+    }
+    for (int f = 0; f < F; ++f) {
+      const long long j = static_cast<long long>(f) * P + s;
+      float dot = 0.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) dot = fmaf(qv[e], to_f(k[head + j * D + lane + 32 * e]), dot);
+#pragma unroll
+      for (int o2 = 16; o2 > 0; o2 >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o2);
+      const float t = dot * scale_log2;
+      const float mn = fmaxf(m, t);
+      const float alpha = exp2f(m - mn);
+      const float p = exp2f(t - mn);
+      l = l * alpha + p;
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[e] = fmaf(p, to_f(v[head + j * D + lane + 32 * e]), acc[e] * alpha);
+      m = mn;
+    }
+#pragma unroll
+    for (int e = 0; e < E; ++e) o_t[r][lane + 32 * e] = acc[e] / l;
+  }
+  __syncthreads();
+
+  // merge the chunk states of the dense and spatial variants; accumulate errors
+  const float* wd = ws + (static_cast<long long>(bh) * 2 + 0) * chunks * kRows * state_floats<D>();
+  const float* wsp = ws + (static_cast<long long>(bh) * 2 + 1) * chunks * kRows * state_floats<D>();
+  float err_s = 0.f, err_t = 0.f;
+  for (int t = threadIdx.x; t < S * D; t += blockDim.x) {
+    const int r = t / D, c = t % D;
+    float od, os;
+    {
+      float M = -INFINITY;
+      for (int ch = 0; ch < chunks; ++ch) M = fmaxf(M, wd[(ch * kRows + r) * state_floats<D>()]);
+      float L = 0.f, O = 0.f;
+      for (int ch = 0; ch < chunks; ++ch) {
+        const float* st = wd + (ch * kRows + r) * state_floats<D>();
+        const float wgt = exp2f(st[0] - M);
+        L += st[1] * wgt;
+        O += st[2 + c] * wgt;
+      }
+      od = O / L;
+    }
+    {
+      float M = -INFINITY;
+      for (int ch = 0; ch < chunks; ++ch) M = fmaxf(M, wsp[(ch * kRows + r) * state_floats<D>()]);
+      float L = 0.f, O = 0.f;
+      for (int ch = 0; ch < chunks; ++ch) {
+        const float* st = wsp + (ch * kRows + r) * state_floats<D>();
+        const float wgt = st[0] == -INFINITY ? 0.f : exp2f(st[0] - M);
+        L += st[1] * wgt;
+        O += st[2 + c] * wgt;
+      }
+      os = O / L;
+    }
+    const float ds = os - od, dt = o_t[r][c] - od;
+    err_s = fmaf(ds, ds, err_s);
+    err_t = fmaf(dt, dt, err_t);
+  }
+#pragma unroll
+  for (int o2 = 16; o2 > 0; o2 >>= 1) {
+    err_s += __shfl_xor_sync(0xffffffffu, err_s, o2);
+    err_t += __shfl_xor_sync(0xffffffffu, err_t, o2);
+  }
+  if (lane == 0) {
+    red[0][warp] = err_s;
+    red[1][warp] = err_t;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float es = 0.f, et = 0.f;
+    for (int w = 0; w < 8; ++w) {
+      es += red[0][w];
+      et += red[1][w];
+    }
+    const float denom = static_cast<float>(S) * D;
+    es /= denom;
+    et /= denom;
+    if (mse_out != nullptr) {
+      mse_out[2 * bh] = es;
+      mse_out[2 * bh + 1] = et;
+    }
+    mode_out[bh] = et < es ? SVG_MODE_TEMPORAL : SVG_MODE_SPATIAL;
+  }
+}
+
+template <int D>
+svg_status launch_profile(const void* q, const void* k, const void* v, int dtype, int B, int H,
+                          int N, int F, int P, int width, const int32_t* idx, int S,
+                          float* mse_out, int32_t* mode_out, float* ws, cudaStream_t s) {
+  ProfileShape ps = profile_shape(B, H, N);
+  const float scale_log2 = kLog2e / sqrtf(static_cast<float>(D));
+  dim3 grid(ps.chunks, B * H, 2);
+  if (dtype == SVG_BF16) {
+    const size_t smem = static_cast<size_t>(kRows) * D * 2 + 4 * static_cast<size_t>(kKeys) * D * 2;
+    if (cudaFuncSetAttribute(profile_partial_bf16<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return fail(SVG_ERR_CUDA, "profile: cannot reserve shared memory");
+    profile_partial_bf16<D><<<grid, kThreads, smem, s>>>(
+        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+        static_cast<const __nv_bfloat16*>(v), idx, S, N, P, width, scale_log2, ps.chunks,
+        ps.chunk_len, ws);
+    if (svg_status st = check_launch("profile partial")) return st;
+    profile_combine<D, __nv_bfloat16><<<B * H, 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+        static_cast<const __nv_bfloat16*>(v), idx, S, N, F, P, scale_log2, ps.chunks, ws, mse_out,
+        mode_out);
+  } else {
+    profile_partial_fp32<D><<<grid, 256, 0, s>>>(
+        static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
+        idx, S, N, P, width, scale_log2, ps.chunks, ps.chunk_len, ws);
+    if (svg_status st = check_launch("profile partial")) return st;
+    profile_combine<D, float><<<B * H, 256, 0, s>>>(
+        static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
+        idx, S, N, F, P, scale_log2, ps.chunks, ws, mse_out, mode_out);
+  }
+  return check_launch("profile combine");
+}
+
+}  // namespace
+}  // namespace svg
+
+using namespace svg;
+
+extern "C" size_t svg_profile_workspace_size(int B, int H, int N, int d, int S) {
+  if (B <= 0 || H <= 0 || N <= 0 || (d != 64 && d != 128) || S <= 0) return 0;
+  return (partial_bytes(B, H, N, d) + 255) / 256 * 256;
+}
+
+extern "C" svg_status svg_profile_heads(const void* q, const void* k, const void* v, int dtype,
+                                        int B, int H, int N, int d, int frames,
+                                        int tokens_per_frame, int spatial_width,
+                                        const int32_t* sample_idx, int S, float* mse_out,
+                                        int32_t* mode_out, void* workspace, size_t workspace_bytes,
+                                        void* stream) {
+  clear_error();
+  if (q == nullptr || k == nullptr || v == nullptr || sample_idx == nullptr || mode_out == nullptr)
+    return fail(SVG_ERR_INVALID_ARG, "profile: null pointer");
+  if (dtype != SVG_BF16 && dtype != SVG_FP32)
+    return fail(SVG_ERR_INVALID_ARG, "profile: bad dtype %d", dtype);
+  if (B <= 0 || H <= 0 || N <= 0 || B * H > 65535)
+    return fail(SVG_ERR_INVALID_ARG, "profile: bad shape");
+  if (d != 64 && d != 128) return fail(SVG_ERR_INVALID_ARG, "profile: d=%d not in {64,128}", d);
+  if (frames <= 0 || tokens_per_frame <= 0 || static_cast<long long>(frames) * tokens_per_frame != N)
+    return fail(SVG_ERR_INVALID_ARG, "profile: frames*tokens_per_frame != N");
+  if (spatial_width < 0) return fail(SVG_ERR_INVALID_ARG, "profile: spatial_width < 0");
+  if (S < 1 || S > kRows) return fail(SVG_ERR_INVALID_ARG, "profile: S=%d not in [1,%d]", S, kRows);
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v))
+    return fail(SVG_ERR_INVALID_ARG, "profile: tensors must be 16-byte aligned");
+  if (workspace == nullptr || !aligned256(workspace) ||
+      workspace_bytes < svg_profile_workspace_size(B, H, N, d, S))
+    return fail(SVG_ERR_INVALID_ARG, "profile: workspace too small or not 256-byte aligned");
+  auto* ws = static_cast<float*>(workspace);
+  cudaStream_t s = as_stream(stream);
+  if (d == 64)
+    return launch_profile<64>(q, k, v, dtype, B, H, N, frames, tokens_per_frame, spatial_width,
+                              sample_idx, S, mse_out, mode_out, ws, s);
+  return launch_profile<128>(q, k, v, dtype, B, H, N, frames, tokens_per_frame, spatial_width,
+                             sample_idx, S, mse_out, mode_out, ws, s);
+}

@@ -1,0 +1,113 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry point
+include/svg.h declares, sizes its scratch, and rejects bad arguments on the
+host before launching anything (the fake device pointers below are never
+dereferenced)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "svg.h")
+
+from sparse_attention_video_svg_b200 import _lib  # noqa: E402
+
+L = _lib.lib
+FAKE = 1 << 20          # 16-byte aligned, never dereferenced on the host
+FAKE2 = 2 << 20
+FAKE3 = 3 << 20
+FAKE4 = 4 << 20
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(svg_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol():
+    names = declared_functions()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(L, n), n
+        assert n in _lib.SIGNATURES, f"{n} has no ctypes signature"
+    assert set(_lib.SIGNATURES) == set(names)
+
+
+def test_exported_dynamic_symbols_match_header():
+    out = os.popen(f"nm -D --defined-only {_lib.LIB_PATH}").read()
+    exported = set(re.findall(r" T (svg_[a-z_0-9]+)", out))
+    assert exported == set(declared_functions())
+
+
+def test_version():
+    assert L.svg_version().decode().startswith("svg_b200")
+
+
+def test_workspace_sizes():
+    assert L.svg_profile_workspace_size(1, 48, 17550, 64, 64) > 0
+    assert L.svg_profile_workspace_size(1, 48, 17550, 64, 64) % 256 == 0
+    assert L.svg_profile_workspace_size(1, 48, 17550, 96, 64) == 0
+    assert L.svg_block_energy_workspace_size(1, 40, 75600) >= 40 * 75600 * 4
+    assert L.svg_calibrated_workspace_size(40, 591, 591) >= 40 * 591 * 19 * 4
+    assert L.svg_calibrated_workspace_size(0, 1, 1) == 0
+
+
+def expect(status, fn, *args, match=None):
+    st = getattr(L, fn)(*args)
+    assert st == status, (fn, st, L.svg_last_error())
+    if match:
+        assert match in L.svg_last_error().decode()
+
+
+INVALID = _lib.SVG_ERR_INVALID_ARG
+
+
+class TestHostValidation:
+    def test_sparse_attn(self):
+        base = [FAKE, FAKE2, FAKE3, FAKE4 * 4, 0, 1, 2, 256, 64, FAKE, 3, 2, FAKE, FAKE, 0.0, None,
+                None]
+        expect(_lib.SVG_OK if False else INVALID, "svg_sparse_attn",
+               *(base[:8] + [96] + base[9:]), match="d=96")
+        expect(INVALID, "svg_sparse_attn", *(base[:11] + [3] + base[12:]), match="n_qblocks")
+        expect(INVALID, "svg_sparse_attn", *([FAKE + 8] + base[1:]), match="aligned")
+        expect(INVALID, "svg_sparse_attn", *(base[:3] + [FAKE] + base[4:]), match="overlaps")
+        expect(INVALID, "svg_sparse_attn", *(base[:4] + [7] + base[5:]), match="dtype")
+        expect(INVALID, "svg_sparse_attn", *(base[:14] + [-1.0] + base[15:]), match="scale")
+        expect(INVALID, "svg_sparse_attn", *([None] + base[1:]), match="null")
+
+    def test_permute(self):
+        args = [FAKE, FAKE4 * 4, 0, 1, 2, 12, 64, 3, 4, None, None]
+        expect(INVALID, "svg_permute_token_major", *(args[:7] + [5] + args[8:]), match="!= N")
+        expect(INVALID, "svg_permute_frame_major", *([FAKE, FAKE + 64] + args[2:]), match="overlap")
+        expect(INVALID, "svg_permute_token_major", *(args[:6] + [32] + args[7:]), match="d=32")
+
+    def test_profile(self):
+        ws = L.svg_profile_workspace_size(1, 2, 256, 64, 16)
+        args = [FAKE, FAKE2, FAKE3, 1, 1, 2, 256, 64, 4, 64, 1, FAKE, 16, None, FAKE4, FAKE4 * 2,
+                ws, None]
+        expect(INVALID, "svg_profile_heads", *(args[:12] + [65] + args[13:]), match="S=65")
+        expect(INVALID, "svg_profile_heads", *(args[:16] + [ws - 256] + args[17:]),
+               match="workspace")
+        expect(INVALID, "svg_profile_heads", *(args[:10] + [-1] + args[11:]),
+               match="spatial_width")
+
+    def test_block_masks(self):
+        expect(INVALID, "svg_build_block_mask", 7, 3, 4, 1, 12, FAKE, FAKE2, 1, 0, FAKE3, None,
+               None, match="kind")
+        expect(INVALID, "svg_build_block_mask", 0, 3, 4, 1, 13, FAKE, FAKE2, 1, 0, FAKE3, None,
+               None, match="!= N")
+        expect(_lib.SVG_ERR_UNSUPPORTED, "svg_build_block_mask", 0, 3, 4, 1, 12, FAKE, FAKE2, 1,
+               0x7fffffff, FAKE3, None, None)
+        ws = L.svg_calibrated_workspace_size(2, 3, 3)
+        expect(INVALID, "svg_build_block_mask_calibrated", FAKE, 17, 2, 3, 3, C.c_double(0.9),
+               C.c_double(0.5), FAKE2, FAKE3, 18, FAKE4, None, FAKE4 * 2, ws, None, match="R=17")
+        expect(INVALID, "svg_build_block_mask_calibrated", FAKE, 2, 2, 3, 3, C.c_double(0.9),
+               C.c_double(1.5), FAKE2, FAKE3, 18, FAKE4, None, FAKE4 * 2, ws, None, match="rho")
+        expect(INVALID, "svg_build_block_mask_calibrated", FAKE, 2, 2, 3, 5000, C.c_double(0.9),
+               C.c_double(0.5), FAKE2, FAKE3, 18, FAKE4, None, FAKE4 * 2, ws, None, match="nKB")
+
+    def test_block_energy(self):
+        expect(INVALID, "svg_block_energy", FAKE, FAKE2, 0, 1, 2, 256, 64, FAKE3, FAKE4 * 2, 10,
+               None, match="workspace")

@@ -1,0 +1,383 @@
+"""GPU parity: every step of the CUDA path, called through the C ABI, against
+the float64 CPU oracle on the same seeded inputs.
+
+Small workloads (seconds of oracle time, several tiles and a ragged tail) are
+compared element by element; full-size workloads on sampled query tiles, in
+the launch configuration bench.py times.  Integer and data-movement results
+are bit-exact; floating-point outputs meet max-abs 2e-2 and rel-RMS 1e-2."""
+import numpy as np
+import pytest
+import torch
+
+import svg_inputs as si
+from oracle import svg_oracle as O
+from tests.helpers import (MODE_MARGIN, assert_close, bits, to_device, to_float64,
+                           workload_tensors)
+
+pytestmark = pytest.mark.gpu
+
+svg = pytest.importorskip("sparse_attention_video_svg_b200")
+DEV = "cuda"
+
+SMALL = [si.small(n) for n in si.ORDER]
+FULL_BF16 = ["cogvideox", "wan480", "wan720", "hunyuan720"]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    torch.cuda.init()
+
+
+def head64(x, b, h):
+    return si.as_float64(x[b, h])
+
+
+# --------------------------------------------------------------------- lists
+
+def gpu_list(kind, F, P, w, N):
+    ip, ix, nnz = svg.svg_build_block_mask(kind, F, P, w, N)
+    n = int(nnz.item())
+    return ip.cpu().numpy(), ix[:n].cpu().numpy()
+
+
+@pytest.mark.parametrize("F,P,w", [(4, 64, 1), (13, 1350, 1), (21, 1560, 1), (21, 3600, 1),
+                                   (33, 3600, 2), (5, 130, 1), (1, 300, 1), (300, 1, 1),
+                                   (7, 3, 0), (2, 61, 3), (6, 126, 1)])
+def test_geometric_lists_bit_exact(F, P, w):
+    N = F * P
+    for kind in (O.MODE_SPATIAL, O.MODE_TEMPORAL, O.MODE_DENSE):
+        gp, gx = gpu_list(kind, F, P, w, N)
+        op, ox = O.geometric_block_lists(kind, F, P, w, N)
+        np.testing.assert_array_equal(gp, op)
+        np.testing.assert_array_equal(gx, ox)
+
+
+def test_geometric_lists_shared_buffer_offsets():
+    F, P, w = 5, 130, 1
+    N = F * P
+    nb = svg.n_tiles(N)
+    L = svg.geometric_lists(F, P, w, N)
+    ip = L.indptr.cpu().numpy().reshape(3, nb + 1)
+    ix = L.indices.cpu().numpy()
+    for kind in range(3):
+        op, ox = O.geometric_block_lists(kind, F, P, w, N)
+        np.testing.assert_array_equal(ip[kind] - ip[kind][0], op)
+        np.testing.assert_array_equal(ix[ip[kind][0]:ip[kind][-1]], ox)
+
+
+# --------------------------------------------------------------- permutation
+
+@pytest.mark.parametrize("wl", SMALL, ids=lambda w: w.name)
+def test_permute_small_bit_exact(wl):
+    (q, _, _), (qd, _, _), types = workload_tensors(wl)
+    mode = torch.from_numpy(types).to(DEV)
+    F, P = wl.F, wl.P
+    y = svg.svg_permute_token_major(qd, F, P, mode)
+    want = q.copy()
+    for b in range(wl.B):
+        for h in range(wl.H):
+            if types[h] == si.TEMPORAL_TYPE:
+                want[b, h] = O.permute_token_major(q[b, h], F, P)
+    np.testing.assert_array_equal(bits(y), want.view(np.int16 if q.dtype == np.uint16 else np.int32))
+    back = svg.svg_permute_frame_major(y, F, P, mode)
+    assert torch.equal(bits_t(back), bits_t(qd))
+    yall = svg.svg_permute_token_major(qd, F, P, None)
+    np.testing.assert_array_equal(bits(yall), O.permute_token_major(q, F, P).view(bits(yall).dtype))
+
+
+def bits_t(t):
+    return t.view(torch.int16) if t.dtype == torch.bfloat16 else t.view(torch.int32)
+
+
+@pytest.mark.parametrize("F,P,d,dt", [(1, 77, 64, "bf16"), (77, 1, 128, "bf16"), (3, 5, 128, "fp32"),
+                                      (9, 13, 64, "fp32")])
+def test_permute_edge_shapes(F, P, d, dt):
+    rng = np.random.default_rng(F * 1000 + P)
+    N = F * P
+    if dt == "bf16":
+        x = rng.integers(0, 1 << 16, size=(2, 3, N, d), dtype=np.uint16)
+    else:
+        x = rng.standard_normal((2, 3, N, d), dtype=np.float32)
+    xd = to_device(x)
+    y = svg.svg_permute_token_major(xd, F, P)
+    np.testing.assert_array_equal(bits(y), O.permute_token_major(x, F, P).view(bits(y).dtype))
+    z = svg.svg_permute_frame_major(xd, F, P)
+    np.testing.assert_array_equal(bits(z), O.permute_frame_major(x, F, P).view(bits(z).dtype))
+
+
+@pytest.mark.parametrize("name", FULL_BF16)
+def test_permute_full_size_sampled(name):
+    wl = si.WORKLOADS[name]
+    F, P, N, d = wl.F, wl.P, wl.N, wl.d
+    H = 4  # the per-head map is independent of H; 4 heads keep host memory small
+    rng = np.random.default_rng(7)
+    x = rng.integers(0, 1 << 16, size=(1, H, N, d), dtype=np.uint16)
+    xd = to_device(x)
+    mode = torch.tensor([1, 0, 1, 1], dtype=torch.int32, device=DEV)
+    y = svg.svg_permute_token_major(xd, F, P, mode)
+    yb = bits(y)
+    src = O.token_major_source(F, P)
+    rows = rng.choice(N, size=4096, replace=False)
+    for h in range(H):
+        s = src[rows] if h != 1 else rows
+        np.testing.assert_array_equal(yb[0, h, rows], x[0, h, s].view(np.int16))
+    back = svg.svg_permute_frame_major(y, F, P, mode)
+    assert torch.equal(bits_t(back), bits_t(xd))
+
+
+# ------------------------------------------------------------------ profiling
+
+def check_profile(mse_gpu, mode_gpu, mse_ref, mode_ref, what):
+    mse_gpu = np.asarray(mse_gpu, np.float64)
+    for i in range(len(mode_ref)):
+        for c in range(2):
+            r = mse_ref[i, c]
+            assert abs(mse_gpu[i, c] - r) <= 0.02 * r + 2e-5, (what, i, c, mse_gpu[i], mse_ref[i])
+        margin = abs(mse_ref[i, 0] - mse_ref[i, 1]) / max(mse_ref[i].max(), 1e-30)
+        if margin > MODE_MARGIN:
+            assert mode_gpu[i] == mode_ref[i], (what, i, mse_gpu[i], mse_ref[i])
+
+
+@pytest.mark.parametrize("wl", SMALL, ids=lambda w: w.name)
+def test_profile_small(wl):
+    (q, k, v), (qd, kd, vd), types = workload_tensors(wl)
+    idx = si.sample_queries(wl)
+    mse, mode = svg.svg_profile_heads(qd, kd, vd, wl.F, wl.P, wl.width,
+                                      torch.from_numpy(idx).to(DEV))
+    mse_ref, mode_ref = O.profile_heads(si.as_float64(q), si.as_float64(k), si.as_float64(v), idx,
+                                        wl.F, wl.P, wl.width)
+    check_profile(mse.cpu().numpy(), mode.cpu().numpy(), mse_ref, mode_ref, wl.name)
+    np.testing.assert_array_equal(mode.cpu().numpy(), types)
+
+
+@pytest.fixture(scope="module")
+def full_inputs():
+    cache = {}
+
+    def get(name):
+        if name not in cache:
+            cache.clear()
+            wl = si.WORKLOADS[name]
+            cache[name] = workload_tensors(wl)
+        return cache[name]
+    return get
+
+
+@pytest.mark.parametrize("name", ["cogvideox", "hunyuan720"])
+def test_profile_full_size(name, full_inputs):
+    wl = si.WORKLOADS[name]
+    (q, k, v), (qd, kd, vd), types = full_inputs(name)
+    idx = si.sample_queries(wl)
+    mse, mode = svg.svg_profile_heads(qd, kd, vd, wl.F, wl.P, wl.width,
+                                      torch.from_numpy(idx).to(DEV))
+    mse = mse.cpu().numpy()
+    mode = mode.cpu().numpy()
+    heads = range(wl.H) if wl.H <= 24 else range(0, wl.H, 3)
+    for h in heads:
+        ms, mt, md = O.profile_head(head64(q, 0, h), head64(k, 0, h), head64(v, 0, h), idx, wl.F,
+                                    wl.P, wl.width)
+        check_profile(mse[h:h + 1], mode[h:h + 1], np.array([[ms, mt]]), np.array([md]),
+                      f"{name} head {h}")
+
+
+# ---------------------------------------------------------- sparse attention
+
+@pytest.mark.parametrize("wl", SMALL, ids=lambda w: w.name)
+@pytest.mark.parametrize("kind", [O.MODE_SPATIAL, O.MODE_TEMPORAL, O.MODE_DENSE])
+def test_sparse_attn_small(wl, kind):
+    (q, k, v), (qd, kd, vd), _ = workload_tensors(wl)
+    lists = svg.geometric_lists(wl.F, wl.P, wl.width, wl.N)
+    list_id = torch.full((wl.B * wl.H,), kind, dtype=torch.int32, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o = svg.svg_sparse_attn(qd, kd, vd, list_id, lists, status=status)
+    got = to_float64(o)
+    ip, ix = O.geometric_block_lists(kind, wl.F, wl.P, wl.width, wl.N)
+    for b in range(wl.B):
+        for h in range(wl.H):
+            ref = O.block_sparse_attention(head64(q, b, h), head64(k, b, h), head64(v, b, h), ip, ix)
+            assert_close(got[b, h], ref, f"{wl.name} kind {kind} head {h}",
+                         bf16=wl.dtype == "bf16")
+    assert status.item() == 0
+
+
+@pytest.mark.parametrize("name", FULL_BF16[:1] + ["wan480", "hunyuan720"])
+def test_sparse_attn_full_size_sampled(name, full_inputs):
+    wl = si.WORKLOADS[name]
+    (q, k, v), (qd, kd, vd), types = full_inputs(name)
+    lists = svg.geometric_lists(wl.F, wl.P, wl.width, wl.N)
+    # spatial-type heads on the spatial list, temporal-type heads on the
+    # temporal list (run on frame-major data: the list is applied as given)
+    list_id = torch.from_numpy(types).to(DEV)
+    o = svg.svg_sparse_attn(qd, kd, vd, list_id, lists)
+    ob = o.view(torch.int16)
+    rng = np.random.default_rng(11)
+    nb = svg.n_tiles(wl.N)
+    heads = rng.choice(wl.H, size=6, replace=False)
+    for h in heads:
+        kind = int(types[h])
+        ip, ix = O.geometric_block_lists(kind, wl.F, wl.P, wl.width, wl.N)
+        tiles = np.r_[rng.choice(nb - 1, size=3, replace=False), nb - 1]  # incl. ragged tail
+        qh, kh, vh = head64(q, 0, h), head64(k, 0, h), head64(v, 0, h)
+        for t in tiles:
+            rows = O.tile_rows(int(t), wl.N)
+            ref = O.block_sparse_rows(qh, kh, vh, rows, ip, ix)
+            got = to_float64(o[0, h, rows[0]:rows[-1] + 1])
+            assert_close(got, ref, f"{name} head {h} tile {t}")
+
+
+def test_sparse_attn_empty_and_invalid_lists():
+    wl = si.small("wan480")
+    (q, k, v), (qd, kd, vd), _ = workload_tensors(wl)
+    N, nb = wl.N, svg.n_tiles(wl.N)
+    # list 0: row 0 empty, row 1 = [nb-1], row 2 = [-3 (bad), 0], others = [i]
+    rows = [[]] + [[nb - 1]] + [[-3, 0]] + [[i] for i in range(3, nb)]
+    ip = np.cumsum([0] + [len(r) for r in rows]).astype(np.int32)
+    ix = np.array([j for r in rows for j in r], dtype=np.int32)
+    lists = svg.BlockLists(torch.from_numpy(ip).to(DEV), torch.from_numpy(ix).to(DEV), 1, nb)
+    list_id = torch.tensor([0, 0, 5, 0], dtype=torch.int32, device=DEV)  # head 2: bad id
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o = to_float64(svg.svg_sparse_attn(qd, kd, vd, list_id, lists, status=status))
+    st = status.item()
+    assert st & svg._lib.SVG_DEVICE_BAD_LIST_ID and st & svg._lib.SVG_DEVICE_BAD_INDEX
+    assert (o[0, 2] == 0).all()
+    assert (o[0, 0, :128] == 0).all()
+    okp = np.cumsum([0] + [len([j for j in r if 0 <= j < nb]) for r in rows]).astype(np.int32)
+    okx = np.array([j for r in rows for j in r if 0 <= j < nb], dtype=np.int32)
+    for h in (0, 1, 3):
+        ref = O.block_sparse_attention(head64(q, 0, h), head64(k, 0, h), head64(v, 0, h), okp, okx)
+        assert_close(o[0, h], ref, f"head {h}")
+
+
+@pytest.mark.parametrize("N,d", [(100, 64), (128, 128), (129, 64), (383, 128)])
+def test_sparse_attn_ragged_dense(N, d):
+    rng = np.random.default_rng(N + d)
+    x = [si.to_bf16_bits(rng.standard_normal((2, 1, N, d), dtype=np.float32) * 2) for _ in range(3)]
+    qd, kd, vd = (to_device(t) for t in x)
+    lists = svg.geometric_lists(1, N, 0, N)
+    list_id = torch.full((2,), O.MODE_DENSE, dtype=torch.int32, device=DEV)
+    o = to_float64(svg.svg_sparse_attn(qd, kd, vd, list_id, lists))
+    for b in range(2):
+        ref = O.dense_attention(*(si.as_float64(t[b, 0]) for t in x))
+        assert_close(o[b, 0], ref, f"N={N} d={d} b={b}")
+
+
+# ---------------------------------------------------------------- the layer
+
+@pytest.mark.parametrize("wl", SMALL, ids=lambda w: w.name)
+def test_layer_small(wl):
+    (q, k, v), (qd, kd, vd), types = workload_tensors(wl)
+    idx = si.sample_queries(wl)
+    lists = svg.geometric_lists(wl.F, wl.P, wl.width, wl.N)
+    o, mode, mse = svg.svg_layer(qd, kd, vd, wl.F, wl.P, wl.width,
+                                 torch.from_numpy(idx).to(DEV), lists)
+    o_ref, mode_ref, mse_ref = O.svg_layer(si.as_float64(q), si.as_float64(k), si.as_float64(v),
+                                           idx, wl.F, wl.P, wl.width)
+    check_profile(mse.cpu().numpy(), mode.cpu().numpy(), mse_ref, mode_ref, wl.name)
+    np.testing.assert_array_equal(mode.cpu().numpy(), mode_ref)
+    got = to_float64(o)
+    for h in range(wl.H):
+        assert_close(got[0, h], o_ref[0, h], f"{wl.name} head {h}", bf16=wl.dtype == "bf16")
+
+
+def test_layer_full_size_cogvideox_sampled(full_inputs):
+    name = "cogvideox"
+    wl = si.WORKLOADS[name]
+    (q, k, v), (qd, kd, vd), types = full_inputs(name)
+    idx = si.sample_queries(wl)
+    lists = svg.geometric_lists(wl.F, wl.P, wl.width, wl.N)
+    o, mode, mse = svg.svg_layer(qd, kd, vd, wl.F, wl.P, wl.width,
+                                 torch.from_numpy(idx).to(DEV), lists)
+    mode = mode.cpu().numpy()
+    np.testing.assert_array_equal(mode, types)
+    src = O.token_major_source(wl.F, wl.P)
+    rng = np.random.default_rng(5)
+    nb = svg.n_tiles(wl.N)
+    for h in rng.choice(wl.H, size=6, replace=False):
+        md = int(mode[h])
+        ip, ix = O.geometric_block_lists(md, wl.F, wl.P, wl.width, wl.N)
+        qh, kh, vh = head64(q, 0, h), head64(k, 0, h), head64(v, 0, h)
+        if md == O.MODE_TEMPORAL:
+            qh, kh, vh = (O.permute_token_major(t, wl.F, wl.P) for t in (qh, kh, vh))
+        for t in np.r_[rng.choice(nb - 1, size=2, replace=False), nb - 1]:
+            rows = O.tile_rows(int(t), wl.N)
+            ref = O.block_sparse_rows(qh, kh, vh, rows, ip, ix)
+            out_rows = src[rows] if md == O.MODE_TEMPORAL else rows
+            got = to_float64(o[0, h][torch.from_numpy(out_rows).to(DEV)])
+            assert_close(got, ref, f"layer head {h} tile {t}")
+
+
+# ------------------------------------------------------ energy and calibration
+
+@pytest.mark.parametrize("name", ["tiny", "wan720", "cogvideox"])
+def test_block_energy_small(name):
+    wl = si.small(name)
+    (q, k, v), (qd, kd, vd), _ = workload_tensors(wl)
+    E = svg.svg_block_energy(qd, kd).cpu().numpy().astype(np.float64)
+    for h in range(wl.H):
+        ref = O.block_energy(head64(q, 0, h), head64(k, 0, h))
+        np.testing.assert_allclose(E[h], ref, rtol=2e-3, atol=2e-5, err_msg=f"{name} head {h}")
+        np.testing.assert_allclose(E[h].sum(1), 1.0, atol=1e-4)
+
+
+def test_calibrated_lists_bit_exact_given_energies():
+    rng = np.random.default_rng(21)
+    R, L, nq, nk = 4, 3, 9, 37
+    E = rng.dirichlet(np.ones(nk) * 0.3, size=(R, L, nq)).astype(np.float32)
+    E[0, 0, 0] = 0.0
+    E[0, 0, 0, :4] = 0.25                        # exact ties
+    E[:, 1, 2] = np.float32(1.0 / nk)            # all ties, every input
+    E[1, 2, 3] = np.eye(nk, dtype=np.float32)[5]
+    for eps, rho in [(0.9, 0.5), (0.5, 1.0), (0.99, 0.25), (0.3, 0.75)]:
+        lists = svg.svg_build_block_mask_calibrated(torch.from_numpy(E).to(DEV), eps, rho)
+        ip = lists.indptr.cpu().numpy().reshape(L, nq + 1)
+        ix = lists.indices.cpu().numpy()
+        for l in range(L):
+            op, ox = O.calibrate_lists([E[r, l].astype(np.float64) for r in range(R)], eps, rho)
+            np.testing.assert_array_equal(ip[l] - ip[l][0], op, err_msg=f"eps {eps} rho {rho}")
+            np.testing.assert_array_equal(ix[ip[l][0]:ip[l][-1]], ox)
+
+
+def cut_margin(e_row, eps):
+    order = O.energy_order(e_row)
+    cum = np.cumsum(np.asarray(e_row, np.float64)[order])
+    kk = int(np.searchsorted(cum, eps))  # first index with cum >= eps
+    prev = cum[kk - 1] if kk > 0 else 0.0
+    nxt = cum[kk] if kk < len(cum) else 1.0
+    gap = (e_row[order[kk]] - e_row[order[kk + 1]]) if kk + 1 < len(order) else 1.0
+    return min(eps - prev, nxt - eps, gap)
+
+
+def test_calibration_end_to_end_small():
+    wl = si.small("wan720")
+    types_seed = wl.calib_seeds[0]
+    Es_gpu, Es_ref = [], []
+    for s in wl.calib_seeds:
+        (q, k, v), (qd, kd, vd), _ = workload_tensors(wl, seed=s, types_seed=types_seed)
+        Es_gpu.append(svg.svg_block_energy(qd, kd))
+        Es_ref.append([O.block_energy(head64(q, 0, h), head64(k, 0, h)) for h in range(wl.H)])
+    E = torch.stack(Es_gpu)  # [R, L, nq, nk]
+    lists = svg.svg_build_block_mask_calibrated(E.contiguous(), wl.eps, wl.rho)
+    nq = svg.n_tiles(wl.N)
+    ip = lists.indptr.cpu().numpy().reshape(wl.H, nq + 1)
+    ix = lists.indices.cpu().numpy()
+    compared = 0
+    for h in range(wl.H):
+        op, ox = O.calibrate_lists([Es_ref[r][h] for r in range(len(wl.calib_seeds))], wl.eps,
+                                   wl.rho)
+        for r in range(nq):
+            if min(cut_margin(Es_ref[s][h][r], wl.eps) for s in range(len(wl.calib_seeds))) <= 1e-3:
+                continue
+            compared += 1
+            np.testing.assert_array_equal(ix[ip[h][r]:ip[h][r + 1]], ox[op[r]:op[r + 1]])
+    assert compared > 0
+    # and attention on the calibrated lists for the timed input
+    (q, k, v), (qd, kd, vd), _ = workload_tensors(wl, seed=wl.seed, types_seed=types_seed)
+    list_id = torch.arange(wl.H, dtype=torch.int32, device=DEV)
+    o = to_float64(svg.svg_sparse_attn(qd, kd, vd, list_id, lists))
+    for h in range(wl.H):
+        hp = ip[h] - ip[h][0]
+        hx = ix[ip[h][0]:ip[h][-1]]
+        ref = O.block_sparse_attention(head64(q, 0, h), head64(k, 0, h), head64(v, 0, h), hp, hx)
+        assert_close(o[0, h], ref, f"calibrated head {h}")
