@@ -119,6 +119,34 @@ svg_status svg_profile_heads(const void* q, const void* k, const void* v, int dt
                              void* workspace, size_t workspace_bytes, void* stream);
 
 /* --------------------------------------------------------------------------
+ * 1b. Online head profiling without caller-provided scratch
+ *    The pages have no counterpart to this entry point; it exists for callers
+ *    that cannot allocate device memory (a plugin inside an engine that owns
+ *    all device memory and passes no workspace, or a region of a program
+ *    where a cudaMalloc would synchronise the device or is not allowed).
+ *
+ *  Same arguments and results as svg_profile_heads, minus the workspace: the
+ *  scratch is a 16 MiB array in device global memory owned by the library
+ *  (every GPU that loads the library holds it until the process exits).
+ *  The keys of each head are cut into fewer, longer ranges when needed so
+ *  that the states fit; results agree with svg_profile_heads to rounding.
+ *  Limit: B*H*2*64*(d+2)*4 bytes <= 16 MiB, i.e. B*H <= 496 at d = 64 and
+ *  B*H <= 252 at d = 128; larger shapes return SVG_ERR_INVALID_ARG.
+ *  No device memory is allocated or freed by this call.
+ *  The first call on a device looks up the array's device address
+ *  (cudaGetSymbolAddress); make that first call on each device before any
+ *  stream capture.  Every call shares the one array and leaves its contents
+ *  behind; nothing in it needs to start at zero.  Calls whose kernels
+ *  overlap on the GPU (e.g. on two streams) race on the array: serialise
+ *  them.
+ * ------------------------------------------------------------------------ */
+svg_status svg_profile_heads_noalloc(const void* q, const void* k, const void* v, int dtype,
+                                     int B, int H, int N, int d,
+                                     int frames, int tokens_per_frame, int spatial_width,
+                                     const int32_t* sample_idx, int S,
+                                     float* mse_out, int32_t* mode_out, void* stream);
+
+/* --------------------------------------------------------------------------
  * 2. / 5. Frame-major <-> token-major permutation
  *    [SVG] section "Layout Transformation + Kernel 加速": reorder so that the
  *    tokens a temporal head needs (one position in every frame) are

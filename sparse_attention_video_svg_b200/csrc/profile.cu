@@ -446,3 +446,146 @@ extern "C" svg_status svg_profile_heads(const void* q, const void* k, const void
   return launch_profile<128>(q, k, v, dtype, B, H, N, frames, tokens_per_frame, spatial_width,
                              sample_idx, S, mse_out, mode_out, ws, s);
 }
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant: svg_profile_heads_noalloc.
+//
+// Some callers cannot allocate device memory at all: a plugin running inside
+// an engine that owns every byte of device memory and hands out no
+// workspace, or a latency-critical or captured region of a program where a
+// cudaMalloc would synchronise the device or is not permitted.  For them the
+// profiling scratch (the per-chunk online-softmax states) lives in one
+// fixed-size array in device global memory that belongs to this library.
+// Its size is a compile-time constant; every GPU that loads the library
+// holds it until the process exits.
+// ---------------------------------------------------------------------------
+
+#include <mutex>
+
+namespace svg {
+namespace {
+
+constexpr size_t kFixedScratchBytes = size_t(16) << 20;  // 16 MiB
+
+// The library-owned scratch.  Host code must not pass this symbol itself to
+// a kernel (on the host it is only a stand-in); it uses the device address
+// that cudaGetSymbolAddress returns for the current device.
+static __device__ __align__(256) unsigned char g_profile_scratch[kFixedScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices] = {nullptr};
+
+// Device address of g_profile_scratch on the current device, looked up once
+// per device on first use.
+svg_status fixed_scratch(float** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(SVG_ERR_CUDA, "profile_noalloc: cudaGetDevice: %s",
+                                    cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices)
+    return fail(SVG_ERR_UNSUPPORTED, "profile_noalloc: device index %d >= %d", dev, kMaxDevices);
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_profile_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return fail(SVG_ERR_CUDA, "profile_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+    g_scratch_addr[dev] = p;
+  }
+  *out = static_cast<float*>(g_scratch_addr[dev]);
+  return SVG_OK;
+}
+
+// Bytes of scratch one key range (chunk) of every head needs.
+size_t fixed_bytes_per_chunk(int B, int H, int d) {
+  return static_cast<size_t>(B) * H * 2 * kRows * (d + 2) * sizeof(float);
+}
+
+// The chunking of profile_shape, reduced until the states fit the fixed
+// scratch (fewer, longer key ranges per head).
+ProfileShape fixed_shape(int B, int H, int N, int d) {
+  ProfileShape ps = profile_shape(B, H, N);
+  const long long max_chunks =
+      static_cast<long long>(kFixedScratchBytes / fixed_bytes_per_chunk(B, H, d));
+  if (ps.chunks > max_chunks) {
+    long long len = (N + max_chunks - 1) / max_chunks;
+    len = (len + kKeys - 1) / kKeys * kKeys;
+    ps.chunk_len = static_cast<int>(len);
+    ps.chunks = static_cast<int>((N + len - 1) / len);
+  }
+  return ps;
+}
+
+template <int D>
+svg_status launch_profile_fixed(const void* q, const void* k, const void* v, int dtype, int B,
+                                int H, int N, int F, int P, int width, const int32_t* idx, int S,
+                                float* mse_out, int32_t* mode_out, float* ws, cudaStream_t s) {
+  const ProfileShape ps = fixed_shape(B, H, N, D);
+  const float scale_log2 = kLog2e / sqrtf(static_cast<float>(D));
+  dim3 grid(ps.chunks, B * H, 2);
+  if (dtype == SVG_BF16) {
+    const size_t smem = static_cast<size_t>(kRows) * D * 2 + 4 * static_cast<size_t>(kKeys) * D * 2;
+    if (cudaFuncSetAttribute(profile_partial_bf16<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return fail(SVG_ERR_CUDA, "profile_noalloc: cannot reserve shared memory");
+    profile_partial_bf16<D><<<grid, kThreads, smem, s>>>(
+        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+        static_cast<const __nv_bfloat16*>(v), idx, S, N, P, width, scale_log2, ps.chunks,
+        ps.chunk_len, ws);
+    if (svg_status st = check_launch("profile_noalloc partial")) return st;
+    profile_combine<D, __nv_bfloat16><<<B * H, 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+        static_cast<const __nv_bfloat16*>(v), idx, S, N, F, P, scale_log2, ps.chunks, ws, mse_out,
+        mode_out);
+  } else {
+    profile_partial_fp32<D><<<grid, 256, 0, s>>>(
+        static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
+        idx, S, N, P, width, scale_log2, ps.chunks, ps.chunk_len, ws);
+    if (svg_status st = check_launch("profile_noalloc partial")) return st;
+    profile_combine<D, float><<<B * H, 256, 0, s>>>(
+        static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
+        idx, S, N, F, P, scale_log2, ps.chunks, ws, mse_out, mode_out);
+  }
+  return check_launch("profile_noalloc combine");
+}
+
+}  // namespace
+}  // namespace svg
+
+extern "C" svg_status svg_profile_heads_noalloc(const void* q, const void* k, const void* v,
+                                                int dtype, int B, int H, int N, int d, int frames,
+                                                int tokens_per_frame, int spatial_width,
+                                                const int32_t* sample_idx, int S, float* mse_out,
+                                                int32_t* mode_out, void* stream) {
+  clear_error();
+  if (q == nullptr || k == nullptr || v == nullptr || sample_idx == nullptr || mode_out == nullptr)
+    return fail(SVG_ERR_INVALID_ARG, "profile_noalloc: null pointer");
+  if (dtype != SVG_BF16 && dtype != SVG_FP32)
+    return fail(SVG_ERR_INVALID_ARG, "profile_noalloc: bad dtype %d", dtype);
+  if (B <= 0 || H <= 0 || N <= 0 || B * H > 65535)
+    return fail(SVG_ERR_INVALID_ARG, "profile_noalloc: bad shape");
+  if (d != 64 && d != 128)
+    return fail(SVG_ERR_INVALID_ARG, "profile_noalloc: d=%d not in {64,128}", d);
+  if (frames <= 0 || tokens_per_frame <= 0 || static_cast<long long>(frames) * tokens_per_frame != N)
+    return fail(SVG_ERR_INVALID_ARG, "profile_noalloc: frames*tokens_per_frame != N");
+  if (spatial_width < 0) return fail(SVG_ERR_INVALID_ARG, "profile_noalloc: spatial_width < 0");
+  if (S < 1 || S > kRows)
+    return fail(SVG_ERR_INVALID_ARG, "profile_noalloc: S=%d not in [1,%d]", S, kRows);
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v))
+    return fail(SVG_ERR_INVALID_ARG, "profile_noalloc: tensors must be 16-byte aligned");
+  if (fixed_bytes_per_chunk(B, H, d) > kFixedScratchBytes)
+    return fail(SVG_ERR_INVALID_ARG,
+                "profile_noalloc: B*H=%d heads at d=%d need %zu bytes of scratch per key range; the "
+                "fixed scratch holds %zu bytes (at most %zu heads)",
+                B * H, d, fixed_bytes_per_chunk(B, H, d), kFixedScratchBytes,
+                kFixedScratchBytes / fixed_bytes_per_chunk(1, 1, d));
+  float* ws = nullptr;
+  if (svg_status st = fixed_scratch(&ws)) return st;
+  cudaStream_t s = as_stream(stream);
+  if (d == 64)
+    return launch_profile_fixed<64>(q, k, v, dtype, B, H, N, frames, tokens_per_frame,
+                                    spatial_width, sample_idx, S, mse_out, mode_out, ws, s);
+  return launch_profile_fixed<128>(q, k, v, dtype, B, H, N, frames, tokens_per_frame,
+                                   spatial_width, sample_idx, S, mse_out, mode_out, ws, s);
+}
