@@ -77,6 +77,7 @@ typedef enum {
 #define SVG_DEVICE_BAD_INDEX 0x2     /* a key-block index outside [0, nB)   */
 #define SVG_DEVICE_TIMEOUT 0x4       /* a bounded pipeline wait gave up      */
 #define SVG_DEVICE_CAPACITY 0x8      /* a list did not fit the given buffer */
+#define SVG_DEVICE_RANGE 0x10        /* a bf16 V value exceeded the fp16 range */
 
 #define SVG_TILE 128
 
@@ -261,10 +262,12 @@ svg_status svg_build_block_mask_calibrated(const float* energy, int R, int L,
  *  indices      device int32, key-block indices in [0, nB), ascending per row.
  *  scale        softmax scale; 0 selects 1/sqrt(d).
  *  device_status  optional device int32 (may be NULL), see SVG_DEVICE_*.
- * Arithmetic (bf16): bf16 tensor-core products with fp32 accumulation, fp32
- * online softmax; the probabilities enter P.V as two bf16 terms (P_hi + P_lo,
- * about 16 significant bits); output rounded to nearest bf16.  fp32 inputs
- * use fp32 arithmetic throughout.
+ * Arithmetic (bf16): Q.K^T on bf16 tensor cores with fp32 accumulation, fp32
+ * online softmax; P.V on fp16 tensor cores (P in [0, 256] with an 11-bit
+ * significand; V converted from bf16 to fp16 on chip, exact for
+ * |v| <= 65504 -- larger values become inf and set SVG_DEVICE_RANGE) with
+ * fp32 accumulation; output rounded to nearest bf16.  fp32 inputs use fp32
+ * arithmetic throughout.
  * ------------------------------------------------------------------------ */
 svg_status svg_sparse_attn(const void* q, const void* k, const void* v, void* o, int dtype,
                            int B, int H, int N, int d,

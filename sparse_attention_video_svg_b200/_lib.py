@@ -14,6 +14,7 @@ SVG_OK, SVG_ERR_INVALID_ARG, SVG_ERR_UNSUPPORTED, SVG_ERR_CUDA, SVG_ERR_TIMEOUT 
 SVG_BF16, SVG_FP32 = 0, 1
 SVG_MODE_SPATIAL, SVG_MODE_TEMPORAL, SVG_MODE_DENSE = 0, 1, 2
 SVG_DEVICE_BAD_LIST_ID, SVG_DEVICE_BAD_INDEX, SVG_DEVICE_TIMEOUT, SVG_DEVICE_CAPACITY = 1, 2, 4, 8
+SVG_DEVICE_RANGE = 16
 SVG_TILE = 128
 
 _p = C.c_void_p

@@ -7,24 +7,30 @@
 // list of kept key blocks.
 //
 // Persistent kernel, one CTA per SM, work item = (head, 128-row query tile).
-// Warp roles (256 threads):
-//   warp 0      TMA producer: Q tile (double-buffered across items), then the
-//               K and V tiles of every kept key block into a ring of slots;
-//   warp 1      MMA issuer (one thread): S = Q K^T into TMEM (two S buffers),
-//               O += P_hi V + P_lo V with P read from TMEM and V from shared
-//               memory;
-//   warps 4-7   softmax: one thread per query row; reads S from TMEM, online
-//               softmax in fp32 with lazy rescaling (O is only rescaled when
-//               the running max grows by more than 2^8), writes P into the S
-//               buffer as two bf16 terms (P = P_hi + P_lo), and runs the
-//               epilogue (O / l -> bf16 -> swizzled shared memory -> TMA
-//               store, rows beyond N clipped).
-// Order of MMA issue per item: QK_0, QK_1, PV_0, QK_2, PV_1, ... so that the
-// tensor core computes S_{j+1} while the softmax works on S_j.
+// Warp roles (384 threads, three warpgroups):
+//   warp 0      TMA producer: the Q tile of each item (double-buffered across
+//               items), then K and V of every kept key block into a ring;
+//   warp 1      MMA issuer (one thread): S = Q K^T into TMEM (two S buffers,
+//               bf16 operands) and O += P V (fp16 operands), P read from
+//               TMEM, V from smem;
+//   warps 2-3   convert each V tile in shared memory from bf16 to fp16;
+//   warps 4-7   softmax of S columns [0, 64), warps 8-11 of [64, 128): one
+//               thread per (query row, column half).  The two halves swap
+//               their row maxima through shared memory, then each computes
+//               fp32 online-softmax weights for its 64 keys with lazy
+//               rescaling (O is rescaled only when the running max grows by
+//               more than 2^8) and writes them into the S buffer as fp16
+//               (11 significant bits; the row sum uses the same rounded
+//               values).  In the
+//               epilogue each half writes its half of the columns of O / l as
+//               bf16 straight from registers to global memory.
+// MMA order per item: QK_0, QK_1, PV_0, QK_2, PV_1, ... so the tensor core
+// computes S_{j+1} while the softmax works on S_j.
 //
 // TMEM columns: S buffer b at [128 b, 128 b + 128), O at [256, 256 + d).
 // Every mbarrier wait is bounded; a wait that gives up sets
 // SVG_DEVICE_TIMEOUT, raises a CTA-wide abort flag and every role drains out.
+#include <cuda_fp16.h>
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -38,40 +44,43 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 256;
-constexpr int kBox = 16384;             // one 128-row x 128-byte TMA box
+constexpr int kThreads = 384;
+constexpr int kBox = 16384;           // one 128-row x 128-byte TMA box
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kRescaleLog2 = 8.0f;    // lazy-rescale threshold (factor 256)
+constexpr float kRescaleLog2 = 8.0f;  // lazy-rescale threshold (factor 256)
 constexpr uint32_t kSpinLimit = 1u << 22;
+constexpr int kBarMax = 1;            // named barriers of the 256 softmax threads
+constexpr int kBarSum = 2;
 
 template <int D>
 struct Cfg {
-  static constexpr int kTile = 128 * D * 2;           // bytes of a Q / K / V / O tile
-  static constexpr int kBoxes = D / 64;               // 64-column boxes per tile
-  static constexpr int kSlots = D == 64 ? 8 : 4;      // K/V ring slots
-  static constexpr int kOffQ = 0;                     // 2 Q buffers
+  static constexpr int kTile = 128 * D * 2;        // bytes of a Q / K / V tile
+  static constexpr int kBoxes = D / 64;            // 64-column boxes per tile
+  static constexpr int kSlots = D == 64 ? 10 : 4;  // K/V ring entries
+  static constexpr int kOffQ = 0;                  // 2 Q buffers
   static constexpr int kOffKV = 2 * kTile;
-  static constexpr int kOffO = kOffKV + kSlots * kTile;
-  static constexpr int kOffBar = kOffO + kTile;
-  static constexpr int kBars = 2 + 2 + 2 * kSlots + 2 + 2 + 2 + 1;
+  static constexpr int kOffRed = kOffKV + kSlots * kTile;  // float [2][2][128] + [2][128]
+  static constexpr int kOffBar = kOffRed + 6 * 128 * 4;
+  static constexpr int kBars = 2 + 2 + 3 * kSlots + 2 + 2 + 2 + 1;
   static constexpr int kSmem = kOffBar + kBars * 8 + 16 + 1024;  // + alignment slack
   static constexpr uint32_t kIdescQK = idesc_bf16(128, 128, false);
-  static constexpr uint32_t kIdescPV = idesc_bf16(128, D, true);
+  static constexpr uint32_t kIdescPV = idesc_f16(128, D, true);
 };
 
 struct Maps {
-  CUtensorMap q, k, v, o;
+  CUtensorMap q, k, v;
 };
 
 struct Bars {
-  uint64_t* q_full;   // [2]
-  uint64_t* q_empty;  // [2]
-  uint64_t* kv_full;  // [slots]
-  uint64_t* kv_empty; // [slots]
-  uint64_t* s_full;   // [2]
-  uint64_t* p_ready;  // [2]
-  uint64_t* o_done;   // [2]
-  uint64_t* o_free;   // [1]
+  uint64_t* q_full;    // [2]
+  uint64_t* q_empty;   // [2]
+  uint64_t* kv_full;   // [slots]
+  uint64_t* kv_empty;  // [slots]
+  uint64_t* v_ready;   // [slots] V tile converted to fp16
+  uint64_t* s_full;    // [2]
+  uint64_t* p_ready;   // [2]
+  uint64_t* o_done;    // [2]
+  uint64_t* o_free;    // [1]
 };
 
 // The list of (bh, qt): [beg, end) into indices, or empty.
@@ -85,7 +94,10 @@ __device__ __forceinline__ void item_list(const AttnArgs& a, int bh, int qt, int
   }
   const int32_t* ip = a.indptr + static_cast<long long>(lid) * (a.n_qblocks + 1);
   const int b = ip[qt], e = ip[qt + 1];
-  if (b < 0 || e < b) return;
+  if (b < 0 || e < b) {
+    if (report) set_status(a.status, SVG_DEVICE_BAD_INDEX);
+    return;
+  }
   beg = b;
   end = e;
 }
@@ -106,6 +118,171 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
   return false;
 }
 
+// Softmax of one column half (64 keys) of every S tile, and the matching half
+// of the output columns.
+template <int D>
+__device__ __forceinline__ void softmax_half(const AttnArgs& a, const Bars& B,
+                                             volatile int* abort_flag, uint32_t tmem,
+                                             float* red_max, float* red_sum, int n_items,
+                                             int nb) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int half = (warp >> 2) - 1;  // 0: S columns [0, 64), 1: [64, 128)
+  const int quarter = warp & 3;      // TMEM lane quarter this warp may access
+  const int row = quarter * 32 + lane;
+  const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+  const uint32_t t_o = tmem + lane_off + 256 + half * (D / 2);
+  const float sl2 = a.scale * kLog2e;
+  const int N = a.N;
+  uint32_t g = 0;  // tiles so far
+  bool ok = true;
+  for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+    const int bh = item / nb, qt = item - bh * nb;
+    int beg, end;
+    item_list(a, bh, qt, beg, end);
+    float m_used = -INFINITY, l = 0.f;
+    bool first = true;
+    for (int e = beg; e < end && ok; ++e) {
+      const int j = a.indices[e];
+      if (!valid_tile(j, nb)) continue;
+      const int sb = g & 1;
+      if (!(ok = wait_bar(&B.s_full[sb], (g >> 1) & 1, abort_flag, a.status))) break;
+      tc_fence_after();
+      const uint32_t t_s = tmem + lane_off + sb * 128;
+      float s[64];
+      {
+        uint32_t r0[32], r1[32];
+        tmem_ld32(t_s + 64 * half, r0);
+        tmem_ld32(t_s + 64 * half + 32, r1);
+        tmem_wait_ld();
+        reg_fence32(r0);
+        reg_fence32(r1);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          s[i] = __uint_as_float(r0[i]);
+          s[32 + i] = __uint_as_float(r1[i]);
+        }
+      }
+      const int valid_cols = min(128, N - j * 128) - 64 * half;
+      if (valid_cols < 64) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
+          if (i >= valid_cols) s[i] = -INFINITY;
+      }
+      float mx8[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) mx8[t] = s[t];
+#pragma unroll
+      for (int i = 8; i < 64; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], s[i]);
+      float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      // both halves have read all of S once they pass this barrier, so the P
+      // writes below cannot overwrite scores the other half still needs
+      float* rm = red_max + (sb * 2) * 128;
+      rm[half * 128 + row] = mx;
+      named_bar_sync(kBarMax, 256);
+      mx = fmaxf(mx, rm[(half ^ 1) * 128 + row]);
+      const float tm = mx * sl2;
+      if (first) {
+        m_used = tm;
+      } else {
+        const bool need = tm > m_used + kRescaleLog2;
+        if (__any_sync(0xffffffffu, need)) {
+          // O must hold PV of the previous tile before it is rescaled
+          if (!(ok = wait_bar(&B.o_done[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_flag, a.status)))
+            break;
+          tc_fence_after();
+          const float m_new = need ? tm : m_used;
+          const float alpha = exp2f(m_used - m_new);
+          uint32_t r[32];
+#pragma unroll
+          for (int ch = 0; ch < D / 64; ++ch) {
+            tmem_ld32(t_o + ch * 32, r);
+            tmem_wait_ld();
+            reg_fence32(r);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            tmem_st32(t_o + ch * 32, r);
+            tmem_wait_st();  // r is reused by the next chunk
+          }
+          l *= alpha;
+          m_used = m_new;
+        }
+      }
+      const float neg = -m_used;
+#pragma unroll
+      for (int q2 = 0; q2 < 2; ++q2) {
+        uint32_t ph[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = fast_exp2(fmaf(s[32 * q2 + 2 * i], sl2, neg));
+          const float p1 = fast_exp2(fmaf(s[32 * q2 + 2 * i + 1], sl2, neg));
+          const __half2 h = __floats2half2_rn(p0, p1);
+          ph[i] = *reinterpret_cast<const uint32_t*>(&h);
+          // the row sum uses the fp16-rounded weights the MMA sees
+          const float2 r = __half22float2(h);
+          l += r.x + r.y;
+        }
+        // P column c (fp16 pair) holds keys 2c, 2c+1
+        tmem_st16(t_s + 32 * half + 16 * q2, ph);
+        tmem_wait_st();  // ph is rewritten by the next quarter
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&B.p_ready[sb]);
+      first = false;
+      ++g;
+    }
+    if (!ok) break;
+    // -------------------------------------------------------------- epilogue
+    const bool empty = first;
+    float ltot = 0.f;
+    if (!empty) {
+      if (!(ok = wait_bar(&B.o_done[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_flag, a.status)))
+        break;
+      tc_fence_after();
+      red_sum[half * 128 + row] = l;
+      named_bar_sync(kBarSum, 256);
+      ltot = l + red_sum[(half ^ 1) * 128 + row];
+    }
+    const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
+    const int n = qt * 128 + row;
+    __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.o) +
+                          (static_cast<long long>(bh) * N + n) * D + half * (D / 2);
+#pragma unroll
+    for (int ch = 0; ch < D / 64; ++ch) {
+      uint32_t r[32];
+      if (!empty) {
+        tmem_ld32(t_o + ch * 32, r);
+        tmem_wait_ld();
+        reg_fence32(r);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) r[i] = 0u;
+      }
+      if (n < N) {
+#pragma unroll
+        for (int c16 = 0; c16 < 4; ++c16) {
+          uint4 v;
+          v.x = pack_bf16x2(__uint_as_float(r[8 * c16 + 0]) * inv,
+                            __uint_as_float(r[8 * c16 + 1]) * inv);
+          v.y = pack_bf16x2(__uint_as_float(r[8 * c16 + 2]) * inv,
+                            __uint_as_float(r[8 * c16 + 3]) * inv);
+          v.z = pack_bf16x2(__uint_as_float(r[8 * c16 + 4]) * inv,
+                            __uint_as_float(r[8 * c16 + 5]) * inv);
+          v.w = pack_bf16x2(__uint_as_float(r[8 * c16 + 6]) * inv,
+                            __uint_as_float(r[8 * c16 + 7]) * inv);
+          *reinterpret_cast<uint4*>(orow + ch * 32 + c16 * 8) = v;
+        }
+      }
+    }
+    if (!empty) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(B.o_free);
+    }
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_sm100_kernel(const __grid_constant__ Maps maps, const AttnArgs a) {
@@ -119,31 +296,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   B.q_empty = bar_base + 2;
   B.kv_full = bar_base + 4;
   B.kv_empty = B.kv_full + C::kSlots;
-  B.s_full = B.kv_empty + C::kSlots;
+  B.v_ready = B.kv_empty + C::kSlots;
+  B.s_full = B.v_ready + C::kSlots;
   B.p_ready = B.s_full + 2;
   B.o_done = B.p_ready + 2;
   B.o_free = B.o_done + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(B.o_free + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* red_max = reinterpret_cast<float*>(smem + C::kOffRed);  // [S buffer][half][row]
+  float* red_sum = red_max + 4 * 128;                             // [half][row]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int N = a.N, nb = n_tiles(N);
-  const int BH = a.B * a.H;
-  const int n_items = BH * nb;
+  const int n_items = a.B * a.H * nb;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&B.q_full[i], 1);
       mbar_init(&B.q_empty[i], 1);
       mbar_init(&B.s_full[i], 1);
-      mbar_init(&B.p_ready[i], 4);
+      mbar_init(&B.p_ready[i], 8);
       mbar_init(&B.o_done[i], 1);
     }
     for (int i = 0; i < C::kSlots; ++i) {
       mbar_init(&B.kv_full[i], 1);
       mbar_init(&B.kv_empty[i], 1);
+      mbar_init(&B.v_ready[i], 2);
     }
-    mbar_init(B.o_free, 4);
+    mbar_init(B.o_free, 8);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -151,7 +331,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&maps.q);
     prefetch_tmap(&maps.k);
     prefetch_tmap(&maps.v);
-    prefetch_tmap(&maps.o);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
@@ -216,18 +395,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (first_of_item && c > 0 && !wait_bar(B.o_free, (c - 1) & 1, abort_flag, a.status))
           return false;
         const int slot = lv % C::kSlots;
-        if (!wait_bar(&B.kv_full[slot], (lv / C::kSlots) & 1, abort_flag, a.status)) return false;
+        if (!wait_bar(&B.v_ready[slot], (lv / C::kSlots) & 1, abort_flag, a.status)) return false;
         tc_fence_after();
         const uint32_t vbase = smem_u32(smem + C::kOffKV + slot * C::kTile);
-        // O (+)= P_hi V + P_lo V; P_hi in columns [0, 64), P_lo in [64, 128)
+        // O (+)= P V, P (fp16) in S columns [0, 64), V converted to fp16
 #pragma unroll
-        for (int part = 0; part < 2; ++part)
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t bdesc = sdesc_sw128(vbase + kk * 2048, kBox, 1024);
-            mma_ts(tmem_o, tmem_s0 + sb * 128 + part * 64 + kk * 8, bdesc, C::kIdescPV,
-                   (first_of_item && part == 0 && kk == 0) ? 0u : 1u);
-          }
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem_o, tmem_s0 + sb * 128 + kk * 8, sdesc_sw128(vbase + kk * 2048, kBox, 1024),
+                 C::kIdescPV, (first_of_item && kk == 0) ? 0u : 1u);
         tc_commit(&B.kv_empty[slot]);
         tc_commit(&B.o_done[sb]);
         return true;
@@ -275,166 +450,47 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++c;
       }
     }
-  } else if (warp >= 4) {
-    // ------------------------------------------------------------ softmax
-    const int q4 = warp - 4;
-    const int row = q4 * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
-    const float sl2 = a.scale * kLog2e;
-    unsigned char* ost = smem + C::kOffO;
-    uint32_t g = 0;
-    bool ok = true;
-    bool store_pending = false;
+  } else if (warp == 2 || warp == 3) {
+    // ------------------------------------------------------------ V to fp16
+    // Converts every V tile in place, in the order the MMA issuer consumes
+    // them.  bf16 -> fp16 is exact for |v| <= 65504 (fp16 subnormals keep
+    // the absolute error below 2^-25); larger values become inf and are
+    // reported as SVG_DEVICE_RANGE.
+    const int t = threadIdx.x - 64;  // 0..63
+    uint32_t L = 0;
+    bool ok = true, range = false;
     for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
       const int bh = item / nb, qt = item - bh * nb;
       int beg, end;
       item_list(a, bh, qt, beg, end);
-      float m_used = -INFINITY, l = 0.f;
-      bool first = true;
       for (int e = beg; e < end && ok; ++e) {
-        const int j = a.indices[e];
-        if (!valid_tile(j, nb)) continue;
-        const int sb = g & 1;
-        if (!(ok = wait_bar(&B.s_full[sb], (g >> 1) & 1, abort_flag, a.status))) break;
-        tc_fence_after();
-        float s[128];
-        {
-          uint32_t r0[32], r1[32], r2[32], r3[32];
-          const uint32_t sa = tmem_s0 + lane_off + sb * 128;
-          tmem_ld32(sa, r0);
-          tmem_ld32(sa + 32, r1);
-          tmem_ld32(sa + 64, r2);
-          tmem_ld32(sa + 96, r3);
-          tmem_wait_ld();
-          reg_fence32(r0);
-          reg_fence32(r1);
-          reg_fence32(r2);
-          reg_fence32(r3);
+        if (!valid_tile(a.indices[e], nb)) continue;
+        const uint32_t lv = L + 1;
+        const int slot = lv % C::kSlots;
+        if (!(ok = wait_bar(&B.kv_full[slot], (lv / C::kSlots) & 1, abort_flag, a.status))) break;
+        uint4* tile = reinterpret_cast<uint4*>(smem + C::kOffKV + slot * C::kTile);
+#pragma unroll 4
+        for (int c = t; c < C::kTile / 16; c += 64) {
+          uint4 v = tile[c];
+          uint32_t* w = reinterpret_cast<uint32_t*>(&v);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            s[i] = __uint_as_float(r0[i]);
-            s[32 + i] = __uint_as_float(r1[i]);
-            s[64 + i] = __uint_as_float(r2[i]);
-            s[96 + i] = __uint_as_float(r3[i]);
+          for (int i = 0; i < 4; ++i) {
+            const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xffff0000u);
+            range |= fabsf(lo) > 65504.f || fabsf(hi) > 65504.f;
+            const __half2 h = __floats2half2_rn(lo, hi);
+            w[i] = *reinterpret_cast<const uint32_t*>(&h);
           }
+          tile[c] = v;
         }
-        const int valid_cols = min(128, N - j * 128);
-        if (valid_cols < 128) {
-#pragma unroll
-          for (int i = 0; i < 128; ++i)
-            if (i >= valid_cols) s[i] = -INFINITY;
-        }
-        float mx = s[0];
-#pragma unroll
-        for (int i = 1; i < 128; ++i) mx = fmaxf(mx, s[i]);
-        const float tm = mx * sl2;
-        if (first) {
-          m_used = tm;
-        } else {
-          const bool need = tm > m_used + kRescaleLog2;
-          if (__any_sync(0xffffffffu, need)) {
-            // O must hold PV of the previous tile before it is rescaled
-            if (!(ok = wait_bar(&B.o_done[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_flag,
-                                a.status)))
-              break;
-            tc_fence_after();
-            const float m_new = need ? tm : m_used;
-            const float alpha = exp2f(m_used - m_new);
-            uint32_t r[32];
-#pragma unroll
-            for (int ch = 0; ch < D / 32; ++ch) {
-              tmem_ld32(tmem_o + lane_off + ch * 32, r);
-              tmem_wait_ld();
-              reg_fence32(r);
-#pragma unroll
-              for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-              tmem_st32(tmem_o + lane_off + ch * 32, r);
-              tmem_wait_st();  // r is reused by the next chunk
-            }
-            l *= alpha;
-            m_used = m_new;
-          }
-        }
-        const float neg = -m_used;
-        {
-          // P = hi + lo, both bf16: hi is the nearest bf16 to p, lo the
-          // nearest bf16 to the remainder.  O accumulates P_hi V + P_lo V, so
-          // the weights carry ~16 bits instead of bf16's 8.
-          const uint32_t sa = tmem_s0 + lane_off + sb * 128;
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            uint32_t hi[32], lo[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const float p0 = fast_exp2(fmaf(s[64 * half + 2 * i], sl2, neg));
-              const float p1 = fast_exp2(fmaf(s[64 * half + 2 * i + 1], sl2, neg));
-              hi[i] = pack_bf16x2(p0, p1);
-              lo[i] = pack_bf16x2(p0 - __uint_as_float(hi[i] << 16),
-                                  p1 - __uint_as_float(hi[i] & 0xffff0000u));
-              l += p0 + p1;
-            }
-            tmem_st32(sa + 32 * half, hi);
-            tmem_st32(sa + 64 + 32 * half, lo);
-            tmem_wait_st();  // hi / lo are rewritten by the next half
-          }
-        }
-        tmem_wait_st();
-        tc_fence_before();
+        fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
         __syncwarp();
-        if (lane == 0) mbar_arrive(&B.p_ready[sb]);
-        first = false;
-        ++g;
+        if (lane == 0) mbar_arrive(&B.v_ready[slot]);
+        L += 2;
       }
-      if (!ok) break;
-      // ---------------------------------------------------------- epilogue
-      const bool empty = first;
-      if (!empty) {
-        if (!(ok = wait_bar(&B.o_done[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_flag, a.status)))
-          break;
-        tc_fence_after();
-      }
-      if (store_pending && row == 0) bulk_wait_read0();
-      named_bar_sync(1, 128);
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-#pragma unroll
-      for (int ch = 0; ch < D / 32; ++ch) {
-        uint32_t r[32];
-        if (!empty) {
-          tmem_ld32(tmem_o + lane_off + ch * 32, r);
-          tmem_wait_ld();
-          reg_fence32(r);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) r[i] = 0u;
-        }
-        // 32 fp32 columns -> 64 bytes of bf16 = 4 swizzled 16-byte chunks
-#pragma unroll
-        for (int c16 = 0; c16 < 4; ++c16) {
-          uint4 v;
-          v.x = pack_bf16x2(__uint_as_float(r[8 * c16 + 0]) * inv, __uint_as_float(r[8 * c16 + 1]) * inv);
-          v.y = pack_bf16x2(__uint_as_float(r[8 * c16 + 2]) * inv, __uint_as_float(r[8 * c16 + 3]) * inv);
-          v.z = pack_bf16x2(__uint_as_float(r[8 * c16 + 4]) * inv, __uint_as_float(r[8 * c16 + 5]) * inv);
-          v.w = pack_bf16x2(__uint_as_float(r[8 * c16 + 6]) * inv, __uint_as_float(r[8 * c16 + 7]) * inv);
-          const int col = ch * 32 + c16 * 8;  // first column of this chunk
-          const int box = col >> 6, cc = (col & 63) >> 3;
-          *reinterpret_cast<uint4*>(ost + box * kBox + row * 128 + ((cc ^ (row & 7)) << 4)) = v;
-        }
-      }
-      if (!empty) {
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(B.o_free);
-      }
-      fence_proxy_async_smem();
-      named_bar_sync(1, 128);
-      if (row == 0) {
-        for (int bx = 0; bx < C::kBoxes; ++bx)
-          tma_store_3d(&maps.o, ost + bx * kBox, 64 * bx, qt * 128, bh);
-        bulk_commit();
-      }
-      store_pending = true;
     }
-    if (row == 0) bulk_wait0();
+    if (__any_sync(0xffffffffu, range) && lane == 0) set_status(a.status, SVG_DEVICE_RANGE);
+  } else if (warp >= 4) {
+    softmax_half<D>(a, B, abort_flag, tmem, red_max, red_sum, n_items, nb);
   }
   tc_fence_before();
   __syncthreads();
@@ -459,7 +515,7 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 }
 
 // [B*H][N][d] bf16 viewed as a 3-D tensor (d, N, B*H); box 64 x 128 x 1,
-// 128-byte swizzle.  Rows beyond N are zero-filled on load, dropped on store.
+// 128-byte swizzle.  Rows beyond N are zero-filled on load.
 bool make_map(CUtensorMap* m, const void* base, int BH, int N, int d) {
   auto enc = get_encode();
   if (enc == nullptr) return false;
@@ -482,7 +538,7 @@ svg_status launch_attn_sm100(const AttnArgs& a, cudaStream_t s) {
   Maps maps;
   const int BH = a.B * a.H;
   if (!make_map(&maps.q, a.q, BH, a.N, D) || !make_map(&maps.k, a.k, BH, a.N, D) ||
-      !make_map(&maps.v, a.v, BH, a.N, D) || !make_map(&maps.o, a.o, BH, a.N, D))
+      !make_map(&maps.v, a.v, BH, a.N, D))
     return fail(SVG_ERR_CUDA, "sparse_attn: cannot encode TMA descriptors");
   if (cudaFuncSetAttribute(attn_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            C::kSmem) != cudaSuccess)

@@ -8,16 +8,20 @@
 // the squared difference; an exact tie keeps SPATIAL.
 //
 // Work split (one layer, all heads, one launch each):
-//   partial  grid (chunks, B*H, 2): the keys of a head are cut into `chunks`
-//            contiguous ranges; each CTA streams one range through shared
-//            memory and keeps an online-softmax state (max, sum, o) per
-//            sampled row, for the dense mask (z = 0) or the spatial mask
-//            (z = 1).  bf16: mma.sync tensor-core products; fp32: SIMT.
-//   combine  grid (B*H): merges the chunk states, computes the temporal
-//            output directly (a row sees only the F keys of its position),
-//            the two errors and the mode.
-// The pass reads K and V once per mask variant: it is bound by HBM and the
-// legacy MMA rate, and costs a few percent of the attention it configures.
+//   partial  grid (chunks, B*H): the keys of a head are cut into `chunks`
+//            contiguous ranges.  A CTA streams one range through a 3-stage
+//            cp.async ring; warps 0-3 keep the dense online-softmax state
+//            (max, sum, o) of the 64 sampled rows, warps 4-7 the state under
+//            the spatial mask (each row's band of frames is one contiguous
+//            key range, tested with two compares; stages outside a warp's
+//            bands are skipped).  bf16: mma.sync tensor-core products;
+//            fp32: SIMT (one launch per mask, grid z).
+//   combine  grid (B*H): per row, the chunk weights exp2(m_c - M) / L are
+//            computed once; the merged dense and spatial outputs, the
+//            temporal output (a row sees only the F keys of its position,
+//            computed directly), the two errors and the mode follow.
+// The pass reads K and V once per head and costs a few percent of the
+// attention it configures.
 #include <float.h>
 
 #include "common.cuh"
@@ -28,8 +32,10 @@ namespace {
 
 constexpr int kRows = 64;          // sampled rows per head (S padded to 64)
 constexpr int kKeys = 64;          // keys per shared-memory stage
-constexpr int kThreads = 128;      // 4 warps x 16 rows
-constexpr int kTargetCtas = 1024;  // partial-grid size the chunking aims for
+constexpr int kStages = 3;         // cp.async ring depth
+constexpr int kThreads = 256;      // 8 warps: 4 dense + 4 spatial, 16 rows each
+constexpr int kTargetCtas = 592;   // partial-grid size the chunking aims for (4 x 148)
+constexpr int kMaxChunks = 24;     // combine keeps per-row chunk weights in smem
 constexpr float kLog2e = 1.4426950408889634f;
 
 // Sampled indices outside [0, N) are clamped into range (never read out of bounds).
@@ -40,16 +46,20 @@ struct ProfileShape {
   int chunk_len;  // keys per range (multiple of kKeys)
 };
 
-ProfileShape profile_shape(int B, int H, int N) {
-  const long long bh2 = 2LL * B * H;
-  long long chunks = (kTargetCtas + bh2 - 1) / bh2;
+ProfileShape shape_for(int N, long long chunks) {
   const long long max_chunks = (N + 4 * kKeys - 1) / (4 * kKeys);  // >= 4 stages per range
   if (chunks > max_chunks) chunks = max_chunks;
+  if (chunks > kMaxChunks) chunks = kMaxChunks;
   if (chunks < 1) chunks = 1;
   long long len = (N + chunks - 1) / chunks;
   len = (len + kKeys - 1) / kKeys * kKeys;
   chunks = (N + len - 1) / len;
   return {static_cast<int>(chunks), static_cast<int>(len)};
+}
+
+ProfileShape profile_shape(int B, int H, int N) {
+  const long long bh = static_cast<long long>(B) * H;
+  return shape_for(N, (kTargetCtas + bh - 1) / bh);
 }
 
 // floats per partial state row: m, l, o[D]
@@ -66,7 +76,7 @@ size_t partial_bytes(int B, int H, int N, int d) {
 // --------------------------------------------------------------- bf16 partial
 
 template <int D>
-__global__ void __launch_bounds__(kThreads) profile_partial_bf16(
+__global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) profile_partial_bf16(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
     const __nv_bfloat16* __restrict__ v, const int32_t* __restrict__ idx, int S, int N, int P,
     int width, float scale_log2, int chunks, int chunk_len, float* __restrict__ ws) {
@@ -74,14 +84,17 @@ __global__ void __launch_bounds__(kThreads) profile_partial_bf16(
   constexpr int TILE = kKeys * D * 2;  // bytes of one K or V stage
   unsigned char* sQ = smem;
   unsigned char* sK = smem + kRows * D * 2;
-  unsigned char* sV = sK + 2 * TILE;
-  __shared__ int row_frame[kRows];
+  unsigned char* sV = sK + kStages * TILE;
 
-  const int chunk = blockIdx.x, bh = blockIdx.y, variant = blockIdx.z;
+  const int chunk = blockIdx.x, bh = blockIdx.y;
   const long long head = static_cast<long long>(bh) * N * D;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int variant = warp >> 2;  // 0 dense, 1 spatial
+  const int row0 = (warp & 3) * 16;
+  const int g = lane >> 2, t4 = lane & 3;
   const int key_begin = chunk * chunk_len;
   const int key_end = min(N, key_begin + chunk_len);
+  const int n_stages = (key_end - key_begin + kKeys - 1) / kKeys;
 
   // gather the sampled query rows (padding rows are zero)
   for (int t = threadIdx.x; t < kRows * (D / 8); t += kThreads) {
@@ -90,15 +103,38 @@ __global__ void __launch_bounds__(kThreads) profile_partial_bf16(
     const int n = ok ? clamp_index(idx[r], N) : 0;
     cp_async16(sQ + swz(r, c, 2 * D), q + head + static_cast<long long>(n) * D + c * 8, ok);
   }
-  if (threadIdx.x < kRows)
-    row_frame[threadIdx.x] = threadIdx.x < S ? clamp_index(idx[threadIdx.x], N) / P : -(1 << 29);
-  const int n_stages = (key_end - key_begin + kKeys - 1) / kKeys;
-  load_tile_async<D, kKeys, kThreads>(sK, k + head, key_begin, key_end);
-  load_tile_async<D, kKeys, kThreads>(sV, v + head, key_begin, key_end);
-  cp_async_commit();
+  // the keys each of this thread's two rows may see, clipped to the chunk
+  int lo[2], hi[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int r = row0 + g + 8 * h;
+    lo[h] = key_begin;
+    hi[h] = key_end;
+    if (r >= S) {
+      hi[h] = lo[h];  // padding row: no keys
+    } else if (variant == 1) {
+      const int f = clamp_index(idx[r], N) / P;
+      lo[h] = max(key_begin, max(0, f - width) * P);
+      hi[h] = min(key_end, static_cast<int>(min(static_cast<long long>(N),
+                                                static_cast<long long>(f + width + 1) * P)));
+    }
+  }
+  int wlo = min(lo[0], lo[1]), whi = max(hi[0], hi[1]);
+#pragma unroll
+  for (int o2 = 4; o2 < 32; o2 <<= 1) {
+    wlo = min(wlo, __shfl_xor_sync(0xffffffffu, wlo, o2));
+    whi = max(whi, __shfl_xor_sync(0xffffffffu, whi, o2));
+  }
 
-  // warp w owns rows [16 w, 16 w + 16): thread rows g and g + 8
-  const int g = lane >> 2, t4 = lane & 3;
+#pragma unroll
+  for (int st = 0; st < kStages - 1; ++st) {
+    if (st < n_stages) {
+      load_tile_async<D, kKeys, kThreads>(sK + st * TILE, k + head, key_begin + st * kKeys, key_end);
+      load_tile_async<D, kKeys, kThreads>(sV + st * TILE, v + head, key_begin + st * kKeys, key_end);
+    }
+    cp_async_commit();
+  }
+
   float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
   float o[D / 8][4];
 #pragma unroll
@@ -106,74 +142,55 @@ __global__ void __launch_bounds__(kThreads) profile_partial_bf16(
   uint32_t qa[D / 16][4];
 
   for (int st = 0; st < n_stages; ++st) {
-    if (st + 1 < n_stages) {
-      const int nb = (st + 1) & 1;
-      load_tile_async<D, kKeys, kThreads>(sK + nb * TILE, k + head, key_begin + (st + 1) * kKeys,
-                                          key_end);
-      load_tile_async<D, kKeys, kThreads>(sV + nb * TILE, v + head, key_begin + (st + 1) * kKeys,
-                                          key_end);
-      cp_async_commit();
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    if (st == 0) load_a_frags<D>(qa, smem_u32(sQ), warp * 16);
-    const int key0 = key_begin + st * kKeys;
-    const int fr0 = row_frame[warp * 16 + g], fr1 = row_frame[warp * 16 + g + 8];
-    bool skip = false;
-    if (variant == 1) {
-      // skip the stage when none of this warp's rows has a spatial key in it
-      const int kf0 = key0 / P, kf1 = (min(key0 + kKeys, key_end) - 1) / P;
-      int lo = min(fr0, fr1), hi = max(fr0, fr1);
-#pragma unroll
-      for (int o2 = 4; o2 < 32; o2 <<= 1) {
-        lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o2));
-        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o2));
+    cp_async_wait<kStages - 2>();
+    __syncthreads();  // stage st landed; the buffer refilled below is free
+    {
+      const int ns = st + kStages - 1;
+      if (ns < n_stages) {
+        const int b = ns % kStages;
+        load_tile_async<D, kKeys, kThreads>(sK + b * TILE, k + head, key_begin + ns * kKeys, key_end);
+        load_tile_async<D, kKeys, kThreads>(sV + b * TILE, v + head, key_begin + ns * kKeys, key_end);
       }
-      skip = (kf1 < lo - width) || (kf0 > hi + width);
+      cp_async_commit();
     }
-    if (!skip) {
-      const uint32_t kt = smem_u32(sK + (st & 1) * TILE), vt = smem_u32(sV + (st & 1) * TILE);
-      float s[kKeys / 8][4];
-      qk_frags<D, kKeys>(s, qa, kt, 0);
-      float mx[2] = {-INFINITY, -INFINITY};
+    if (st == 0) load_a_frags<D>(qa, smem_u32(sQ), row0);
+    const int key0 = key_begin + st * kKeys;
+    if (key0 >= whi || key0 + kKeys <= wlo) continue;  // no row of this warp sees the stage
+    const int b = st % kStages;
+    float s[kKeys / 8][4];
+    qk_frags<D, kKeys>(s, qa, smem_u32(sK + b * TILE), 0);
+    float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+    for (int n = 0; n < kKeys / 8; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int key = key0 + 8 * n + 2 * t4 + (e & 1);
+        const int h = e >> 1;
+        s[n][e] = (key >= lo[h] && key < hi[h]) ? s[n][e] * scale_log2 : -INFINITY;
+        mx[h] = fmaxf(mx[h], s[n][e]);
+      }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
+      mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
+      const float mn = fmaxf(m[h], mx[h]);
+      const float base = mn == -INFINITY ? 0.f : mn;
+      const float alpha = fast_exp2(m[h] - base);  // exp2(-inf) = 0 on the first stage
+      m[h] = mn;
+      l[h] *= alpha;
+#pragma unroll
+      for (int n = 0; n < D / 8; ++n) {
+        o[n][2 * h] *= alpha;
+        o[n][2 * h + 1] *= alpha;
+      }
 #pragma unroll
       for (int n = 0; n < kKeys / 8; ++n) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int key = key0 + 8 * n + 2 * t4 + (e & 1);
-          const int fr = (e < 2) ? fr0 : fr1;
-          bool ok = key < key_end;
-          if (variant == 1) ok = ok && abs(key / P - fr) <= width;
-          s[n][e] = ok ? s[n][e] * scale_log2 : -INFINITY;
-          mx[e >> 1] = fmaxf(mx[e >> 1], s[n][e]);
-        }
+        s[n][2 * h] = round_bf16(fast_exp2(s[n][2 * h] - base));
+        s[n][2 * h + 1] = round_bf16(fast_exp2(s[n][2 * h + 1] - base));
+        l[h] += s[n][2 * h] + s[n][2 * h + 1];
       }
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
-        mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
-        const float mn = fmaxf(m[h], mx[h]);
-        const float base = mn == -INFINITY ? 0.f : mn;
-        const float alpha = fast_exp2(m[h] - base);  // exp2(-inf) = 0 on the first stage
-        m[h] = mn;
-        l[h] *= alpha;
-#pragma unroll
-        for (int n = 0; n < D / 8; ++n) {
-          o[n][2 * h] *= alpha;
-          o[n][2 * h + 1] *= alpha;
-        }
-#pragma unroll
-        for (int n = 0; n < kKeys / 8; ++n) {
-          s[n][2 * h] = round_bf16(fast_exp2(s[n][2 * h] - base));
-          s[n][2 * h + 1] = round_bf16(fast_exp2(s[n][2 * h + 1] - base));
-          l[h] += s[n][2 * h] + s[n][2 * h + 1];
-        }
-      }
-      pv_frags<D, kKeys>(o, s, vt, 0);
     }
-    __syncthreads();  // stage (st & 1) is refilled next iteration
+    pv_frags<D, kKeys>(o, s, smem_u32(sV + b * TILE), 0);
   }
 
   // per-row partial state -> workspace [bh][variant][chunk][row][m, l, o[D]]
@@ -186,7 +203,7 @@ __global__ void __launch_bounds__(kThreads) profile_partial_bf16(
                          state_floats<D>();
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    const int r = warp * 16 + g + 8 * h;
+    const int r = row0 + g + 8 * h;
     float* row = base + r * state_floats<D>();
     if (t4 == 0) {
       row[0] = m[h];
@@ -202,7 +219,8 @@ __global__ void __launch_bounds__(kThreads) profile_partial_bf16(
 
 // --------------------------------------------------------------- fp32 partial
 
-// SIMT fp32: warp per sampled row, lanes split the head dimension.
+// SIMT fp32: warp per sampled row, lanes split the head dimension; grid z
+// selects the mask (0 dense, 1 spatial).
 template <int D>
 __global__ void __launch_bounds__(256) profile_partial_fp32(
     const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v,
@@ -230,7 +248,8 @@ __global__ void __launch_bounds__(256) profile_partial_fp32(
         if (variant == 1 && abs(j / P - fr) > width) continue;
         float dot = 0.f;
 #pragma unroll
-        for (int e = 0; e < E; ++e) dot = fmaf(qv[e], k[head + static_cast<long long>(j) * D + lane + 32 * e], dot);
+        for (int e = 0; e < E; ++e)
+          dot = fmaf(qv[e], k[head + static_cast<long long>(j) * D + lane + 32 * e], dot);
 #pragma unroll
         for (int o2 = 16; o2 > 0; o2 >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o2);
         const float t = dot * scale_log2;
@@ -272,12 +291,32 @@ __global__ void __launch_bounds__(256) profile_combine(
     const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
     const int32_t* __restrict__ idx, int S, int N, int F, int P, float scale_log2, int chunks,
     const float* __restrict__ ws, float* __restrict__ mse_out, int32_t* __restrict__ mode_out) {
-  __shared__ float o_t[kRows][D];  // temporal outputs
+  __shared__ float o_t[kRows][D];              // temporal outputs
+  __shared__ float wts[2][kRows][kMaxChunks];  // merge weight of each chunk state
   __shared__ float red[2][8];
   const int bh = blockIdx.x;
   const long long head = static_cast<long long>(bh) * N * D;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int E = D / 32;
+  const float* wsh = ws + static_cast<long long>(bh) * 2 * chunks * kRows * state_floats<D>();
+
+  // chunk weights per (mask, row): w_c = exp2(m_c - M) / sum_c exp2(m_c - M) l_c
+  for (int t = threadIdx.x; t < 2 * S; t += blockDim.x) {
+    const int var = t / S, r = t - var * S;
+    const float* st = wsh + (static_cast<long long>(var) * chunks * kRows + r) * state_floats<D>();
+    const int stride = kRows * state_floats<D>();
+    float M = -INFINITY;
+    for (int c = 0; c < chunks; ++c) M = fmaxf(M, st[c * stride]);
+    float L = 0.f;
+    for (int c = 0; c < chunks; ++c) {
+      const float mc = st[c * stride];
+      const float w = mc == -INFINITY ? 0.f : exp2f(mc - M);
+      wts[var][r][c] = w;
+      L += w * st[c * stride + 1];
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    for (int c = 0; c < chunks; ++c) wts[var][r][c] *= inv;
+  }
 
   // temporal mask: the F keys of the row's position, exact online softmax
   for (int r = warp; r < S; r += 8) {
@@ -310,36 +349,17 @@ __global__ void __launch_bounds__(256) profile_combine(
   }
   __syncthreads();
 
-  // merge the chunk states of the dense and spatial variants; accumulate errors
-  const float* wd = ws + (static_cast<long long>(bh) * 2 + 0) * chunks * kRows * state_floats<D>();
-  const float* wsp = ws + (static_cast<long long>(bh) * 2 + 1) * chunks * kRows * state_floats<D>();
+  // merged dense and spatial outputs; squared errors against dense
   float err_s = 0.f, err_t = 0.f;
   for (int t = threadIdx.x; t < S * D; t += blockDim.x) {
     const int r = t / D, c = t % D;
-    float od, os;
-    {
-      float M = -INFINITY;
-      for (int ch = 0; ch < chunks; ++ch) M = fmaxf(M, wd[(ch * kRows + r) * state_floats<D>()]);
-      float L = 0.f, O = 0.f;
-      for (int ch = 0; ch < chunks; ++ch) {
-        const float* st = wd + (ch * kRows + r) * state_floats<D>();
-        const float wgt = exp2f(st[0] - M);
-        L += st[1] * wgt;
-        O += st[2 + c] * wgt;
-      }
-      od = O / L;
-    }
-    {
-      float M = -INFINITY;
-      for (int ch = 0; ch < chunks; ++ch) M = fmaxf(M, wsp[(ch * kRows + r) * state_floats<D>()]);
-      float L = 0.f, O = 0.f;
-      for (int ch = 0; ch < chunks; ++ch) {
-        const float* st = wsp + (ch * kRows + r) * state_floats<D>();
-        const float wgt = st[0] == -INFINITY ? 0.f : exp2f(st[0] - M);
-        L += st[1] * wgt;
-        O += st[2 + c] * wgt;
-      }
-      os = O / L;
+    float od = 0.f, os = 0.f;
+    const float* sd = wsh + static_cast<long long>(r) * state_floats<D>() + 2 + c;
+    const float* ss = sd + static_cast<long long>(chunks) * kRows * state_floats<D>();
+    for (int ch = 0; ch < chunks; ++ch) {
+      const long long off = static_cast<long long>(ch) * kRows * state_floats<D>();
+      od = fmaf(wts[0][r][ch], sd[off], od);
+      os = fmaf(wts[1][r][ch], ss[off], os);
     }
     const float ds = os - od, dt = o_t[r][c] - od;
     err_s = fmaf(ds, ds, err_s);
@@ -372,37 +392,38 @@ __global__ void __launch_bounds__(256) profile_combine(
   }
 }
 
+// Launches partial + combine with the given key chunking and state buffer.
 template <int D>
-svg_status launch_profile(const void* q, const void* k, const void* v, int dtype, int B, int H,
-                          int N, int F, int P, int width, const int32_t* idx, int S,
-                          float* mse_out, int32_t* mode_out, float* ws, cudaStream_t s) {
-  ProfileShape ps = profile_shape(B, H, N);
+svg_status launch_profile_shaped(const void* q, const void* k, const void* v, int dtype, int B,
+                                 int H, int N, int F, int P, int width, const int32_t* idx, int S,
+                                 float* mse_out, int32_t* mode_out, float* ws, ProfileShape ps,
+                                 cudaStream_t s, const char* who) {
   const float scale_log2 = kLog2e / sqrtf(static_cast<float>(D));
-  dim3 grid(ps.chunks, B * H, 2);
   if (dtype == SVG_BF16) {
-    const size_t smem = static_cast<size_t>(kRows) * D * 2 + 4 * static_cast<size_t>(kKeys) * D * 2;
+    const size_t smem =
+        static_cast<size_t>(kRows) * D * 2 + 2 * kStages * static_cast<size_t>(kKeys) * D * 2;
     if (cudaFuncSetAttribute(profile_partial_bf16<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
-      return fail(SVG_ERR_CUDA, "profile: cannot reserve shared memory");
-    profile_partial_bf16<D><<<grid, kThreads, smem, s>>>(
+      return fail(SVG_ERR_CUDA, "%s: cannot reserve shared memory", who);
+    profile_partial_bf16<D><<<dim3(ps.chunks, B * H), kThreads, smem, s>>>(
         static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
         static_cast<const __nv_bfloat16*>(v), idx, S, N, P, width, scale_log2, ps.chunks,
         ps.chunk_len, ws);
-    if (svg_status st = check_launch("profile partial")) return st;
+    if (svg_status st = check_launch(who)) return st;
     profile_combine<D, __nv_bfloat16><<<B * H, 256, 0, s>>>(
         static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
         static_cast<const __nv_bfloat16*>(v), idx, S, N, F, P, scale_log2, ps.chunks, ws, mse_out,
         mode_out);
   } else {
-    profile_partial_fp32<D><<<grid, 256, 0, s>>>(
+    profile_partial_fp32<D><<<dim3(ps.chunks, B * H, 2), 256, 0, s>>>(
         static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
         idx, S, N, P, width, scale_log2, ps.chunks, ps.chunk_len, ws);
-    if (svg_status st = check_launch("profile partial")) return st;
+    if (svg_status st = check_launch(who)) return st;
     profile_combine<D, float><<<B * H, 256, 0, s>>>(
         static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
         idx, S, N, F, P, scale_log2, ps.chunks, ws, mse_out, mode_out);
   }
-  return check_launch("profile combine");
+  return check_launch(who);
 }
 
 }  // namespace
@@ -440,11 +461,14 @@ extern "C" svg_status svg_profile_heads(const void* q, const void* k, const void
     return fail(SVG_ERR_INVALID_ARG, "profile: workspace too small or not 256-byte aligned");
   auto* ws = static_cast<float*>(workspace);
   cudaStream_t s = as_stream(stream);
+  const ProfileShape ps = profile_shape(B, H, N);
   if (d == 64)
-    return launch_profile<64>(q, k, v, dtype, B, H, N, frames, tokens_per_frame, spatial_width,
-                              sample_idx, S, mse_out, mode_out, ws, s);
-  return launch_profile<128>(q, k, v, dtype, B, H, N, frames, tokens_per_frame, spatial_width,
-                             sample_idx, S, mse_out, mode_out, ws, s);
+    return launch_profile_shaped<64>(q, k, v, dtype, B, H, N, frames, tokens_per_frame,
+                                     spatial_width, sample_idx, S, mse_out, mode_out, ws, ps, s,
+                                     "profile");
+  return launch_profile_shaped<128>(q, k, v, dtype, B, H, N, frames, tokens_per_frame,
+                                    spatial_width, sample_idx, S, mse_out, mode_out, ws, ps, s,
+                                    "profile");
 }
 
 // ---------------------------------------------------------------------------
@@ -508,46 +532,8 @@ ProfileShape fixed_shape(int B, int H, int N, int d) {
   ProfileShape ps = profile_shape(B, H, N);
   const long long max_chunks =
       static_cast<long long>(kFixedScratchBytes / fixed_bytes_per_chunk(B, H, d));
-  if (ps.chunks > max_chunks) {
-    long long len = (N + max_chunks - 1) / max_chunks;
-    len = (len + kKeys - 1) / kKeys * kKeys;
-    ps.chunk_len = static_cast<int>(len);
-    ps.chunks = static_cast<int>((N + len - 1) / len);
-  }
+  if (ps.chunks > max_chunks) ps = shape_for(N, max_chunks);
   return ps;
-}
-
-template <int D>
-svg_status launch_profile_fixed(const void* q, const void* k, const void* v, int dtype, int B,
-                                int H, int N, int F, int P, int width, const int32_t* idx, int S,
-                                float* mse_out, int32_t* mode_out, float* ws, cudaStream_t s) {
-  const ProfileShape ps = fixed_shape(B, H, N, D);
-  const float scale_log2 = kLog2e / sqrtf(static_cast<float>(D));
-  dim3 grid(ps.chunks, B * H, 2);
-  if (dtype == SVG_BF16) {
-    const size_t smem = static_cast<size_t>(kRows) * D * 2 + 4 * static_cast<size_t>(kKeys) * D * 2;
-    if (cudaFuncSetAttribute(profile_partial_bf16<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-      return fail(SVG_ERR_CUDA, "profile_noalloc: cannot reserve shared memory");
-    profile_partial_bf16<D><<<grid, kThreads, smem, s>>>(
-        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-        static_cast<const __nv_bfloat16*>(v), idx, S, N, P, width, scale_log2, ps.chunks,
-        ps.chunk_len, ws);
-    if (svg_status st = check_launch("profile_noalloc partial")) return st;
-    profile_combine<D, __nv_bfloat16><<<B * H, 256, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-        static_cast<const __nv_bfloat16*>(v), idx, S, N, F, P, scale_log2, ps.chunks, ws, mse_out,
-        mode_out);
-  } else {
-    profile_partial_fp32<D><<<grid, 256, 0, s>>>(
-        static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
-        idx, S, N, P, width, scale_log2, ps.chunks, ps.chunk_len, ws);
-    if (svg_status st = check_launch("profile_noalloc partial")) return st;
-    profile_combine<D, float><<<B * H, 256, 0, s>>>(
-        static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
-        idx, S, N, F, P, scale_log2, ps.chunks, ws, mse_out, mode_out);
-  }
-  return check_launch("profile_noalloc combine");
 }
 
 }  // namespace
@@ -583,9 +569,12 @@ extern "C" svg_status svg_profile_heads_noalloc(const void* q, const void* k, co
   float* ws = nullptr;
   if (svg_status st = fixed_scratch(&ws)) return st;
   cudaStream_t s = as_stream(stream);
+  const ProfileShape ps = fixed_shape(B, H, N, d);
   if (d == 64)
-    return launch_profile_fixed<64>(q, k, v, dtype, B, H, N, frames, tokens_per_frame,
-                                    spatial_width, sample_idx, S, mse_out, mode_out, ws, s);
-  return launch_profile_fixed<128>(q, k, v, dtype, B, H, N, frames, tokens_per_frame,
-                                   spatial_width, sample_idx, S, mse_out, mode_out, ws, s);
+    return launch_profile_shaped<64>(q, k, v, dtype, B, H, N, frames, tokens_per_frame,
+                                     spatial_width, sample_idx, S, mse_out, mode_out, ws, ps, s,
+                                     "profile_noalloc");
+  return launch_profile_shaped<128>(q, k, v, dtype, B, H, N, frames, tokens_per_frame,
+                                    spatial_width, sample_idx, S, mse_out, mode_out, ws, ps, s,
+                                    "profile_noalloc");
 }
