@@ -131,8 +131,10 @@ svg_status svg_profile_heads(const void* q, const void* k, const void* v, int dt
  *  (every GPU that loads the library holds it until the process exits).
  *  The keys of each head are cut into fewer, longer ranges when needed so
  *  that the states fit; results agree with svg_profile_heads to rounding.
- *  Limit: B*H*2*64*(d+2)*4 bytes <= 16 MiB, i.e. B*H <= 496 at d = 64 and
- *  B*H <= 252 at d = 128; larger shapes return SVG_ERR_INVALID_ARG.
+ *  Limit: the states of one key range plus the per-row error sums,
+ *  B*H*(2*64*(d+2)*4 + 512) bytes, must fit in 16 MiB - 256, i.e.
+ *  B*H <= 489 at d = 64 and B*H <= 250 at d = 128; larger shapes return
+ *  SVG_ERR_INVALID_ARG.
  *  No device memory is allocated or freed by this call.
  *  The first call on a device looks up the array's device address
  *  (cudaGetSymbolAddress); make that first call on each device before any

@@ -16,10 +16,11 @@
 //            key range, tested with two compares; stages outside a warp's
 //            bands are skipped).  bf16: mma.sync tensor-core products;
 //            fp32: SIMT (one launch per mask, grid z).
-//   combine  grid (B*H): per row, the chunk weights exp2(m_c - M) / L are
-//            computed once; the merged dense and spatial outputs, the
+//   merge    grid (B*H, 16), one warp per sampled row: the chunk weights
+//            exp2(m_c - M) / L, the merged dense and spatial outputs, the
 //            temporal output (a row sees only the F keys of its position,
-//            computed directly), the two errors and the mode follow.
+//            computed directly) and the row's squared errors;
+//   finalize grid (B*H): mean errors and the mode.
 // The pass reads K and V once per head and costs a few percent of the
 // attention it configures.
 #include <float.h>
@@ -35,7 +36,7 @@ constexpr int kKeys = 64;          // keys per shared-memory stage
 constexpr int kStages = 3;         // cp.async ring depth
 constexpr int kThreads = 256;      // 8 warps: 4 dense + 4 spatial, 16 rows each
 constexpr int kTargetCtas = 592;   // partial-grid size the chunking aims for (4 x 148)
-constexpr int kMaxChunks = 24;     // combine keeps per-row chunk weights in smem
+constexpr int kMaxChunks = 32;     // merge holds one chunk weight per lane
 constexpr float kLog2e = 1.4426950408889634f;
 
 // Sampled indices outside [0, N) are clamped into range (never read out of bounds).
@@ -68,9 +69,19 @@ constexpr int state_floats() {
   return D + 2;
 }
 
+size_t states_bytes(int B, int H, int chunks, int d) {
+  const size_t b = static_cast<size_t>(B) * H * 2 * chunks * kRows * (d + 2) * sizeof(float);
+  return (b + 255) / 256 * 256;
+}
+
+// per (head, sampled row): squared errors of the spatial and temporal outputs
+size_t errors_bytes(int B, int H) {
+  return (static_cast<size_t>(B) * H * kRows * 2 * sizeof(float) + 255) / 256 * 256;
+}
+
 size_t partial_bytes(int B, int H, int N, int d) {
   ProfileShape ps = profile_shape(B, H, N);
-  return static_cast<size_t>(B) * H * 2 * ps.chunks * kRows * (d + 2) * sizeof(float);
+  return states_bytes(B, H, ps.chunks, d) + errors_bytes(B, H);
 }
 
 // --------------------------------------------------------------- bf16 partial
@@ -286,104 +297,119 @@ __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) {
   return __bfloat162float(x);
 }
 
+constexpr int kMergeRows = 4;  // sampled rows per merge CTA (one warp each)
+
+// Merges the chunk states of one sampled row (one warp per row), computes the
+// row's temporal output directly and writes the row's squared errors.
 template <int D, typename T>
-__global__ void __launch_bounds__(256) profile_combine(
+__global__ void __launch_bounds__(32 * kMergeRows) profile_merge(
     const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
     const int32_t* __restrict__ idx, int S, int N, int F, int P, float scale_log2, int chunks,
-    const float* __restrict__ ws, float* __restrict__ mse_out, int32_t* __restrict__ mode_out) {
-  __shared__ float o_t[kRows][D];              // temporal outputs
-  __shared__ float wts[2][kRows][kMaxChunks];  // merge weight of each chunk state
-  __shared__ float red[2][8];
-  const int bh = blockIdx.x;
-  const long long head = static_cast<long long>(bh) * N * D;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const float* __restrict__ ws, float* __restrict__ errs) {
   constexpr int E = D / 32;
-  const float* wsh = ws + static_cast<long long>(bh) * 2 * chunks * kRows * state_floats<D>();
-
-  // chunk weights per (mask, row): w_c = exp2(m_c - M) / sum_c exp2(m_c - M) l_c
-  for (int t = threadIdx.x; t < 2 * S; t += blockDim.x) {
-    const int var = t / S, r = t - var * S;
-    const float* st = wsh + (static_cast<long long>(var) * chunks * kRows + r) * state_floats<D>();
-    const int stride = kRows * state_floats<D>();
-    float M = -INFINITY;
-    for (int c = 0; c < chunks; ++c) M = fmaxf(M, st[c * stride]);
-    float L = 0.f;
+  const int bh = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.y * kMergeRows + warp;
+  if (r >= kRows) return;
+  float* err = errs + (static_cast<long long>(bh) * kRows + r) * 2;
+  if (r >= S) {
+    if (lane == 0) err[0] = err[1] = 0.f;
+    return;
+  }
+  const long long head = static_cast<long long>(bh) * N * D;
+  const int stride = kRows * state_floats<D>();  // between chunks
+  float om[2][E];
+#pragma unroll
+  for (int var = 0; var < 2; ++var) {
+    const float* st = ws + (static_cast<long long>(bh) * 2 + var) * chunks * stride +
+                      static_cast<long long>(r) * state_floats<D>();
+    // lane c holds chunk c's weight exp2(m_c - M) / sum_c exp2(m_c - M) l_c
+    const float mc = lane < chunks ? st[static_cast<long long>(lane) * stride] : -INFINITY;
+    float M = mc;
+#pragma unroll
+    for (int o2 = 16; o2 > 0; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o2));
+    float w = mc == -INFINITY ? 0.f : exp2f(mc - M);
+    float L = lane < chunks ? w * st[static_cast<long long>(lane) * stride + 1] : 0.f;
+#pragma unroll
+    for (int o2 = 16; o2 > 0; o2 >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o2);
+    w = L > 0.f ? w / L : 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) om[var][e] = 0.f;
     for (int c = 0; c < chunks; ++c) {
-      const float mc = st[c * stride];
-      const float w = mc == -INFINITY ? 0.f : exp2f(mc - M);
-      wts[var][r][c] = w;
-      L += w * st[c * stride + 1];
+      const float wc = __shfl_sync(0xffffffffu, w, c);
+      const float* oc = st + static_cast<long long>(c) * stride + 2;
+#pragma unroll
+      for (int e = 0; e < E; ++e) om[var][e] = fmaf(wc, oc[lane + 32 * e], om[var][e]);
     }
-    const float inv = L > 0.f ? 1.f / L : 0.f;
-    for (int c = 0; c < chunks; ++c) wts[var][r][c] *= inv;
   }
-
   // temporal mask: the F keys of the row's position, exact online softmax
-  for (int r = warp; r < S; r += 8) {
-    const int n = clamp_index(idx[r], N);
-    const int s = n % P;
-    float qv[E], acc[E], m = -INFINITY, l = 0.f;
+  const int n = clamp_index(idx[r], N);
+  const int sp = n % P;
+  float qv[E], acc[E], m = -INFINITY, l = 0.f;
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-      qv[e] = to_f(q[head + static_cast<long long>(n) * D + lane + 32 * e]);
-      acc[e] = 0.f;
-    }
-    for (int f = 0; f < F; ++f) {
-      const long long j = static_cast<long long>(f) * P + s;
-      float dot = 0.f;
-#pragma unroll
-      for (int e = 0; e < E; ++e) dot = fmaf(qv[e], to_f(k[head + j * D + lane + 32 * e]), dot);
-#pragma unroll
-      for (int o2 = 16; o2 > 0; o2 >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o2);
-      const float t = dot * scale_log2;
-      const float mn = fmaxf(m, t);
-      const float alpha = exp2f(m - mn);
-      const float p = exp2f(t - mn);
-      l = l * alpha + p;
-#pragma unroll
-      for (int e = 0; e < E; ++e) acc[e] = fmaf(p, to_f(v[head + j * D + lane + 32 * e]), acc[e] * alpha);
-      m = mn;
-    }
-#pragma unroll
-    for (int e = 0; e < E; ++e) o_t[r][lane + 32 * e] = acc[e] / l;
+  for (int e = 0; e < E; ++e) {
+    qv[e] = to_f(q[head + static_cast<long long>(n) * D + lane + 32 * e]);
+    acc[e] = 0.f;
   }
-  __syncthreads();
-
-  // merged dense and spatial outputs; squared errors against dense
-  float err_s = 0.f, err_t = 0.f;
-  for (int t = threadIdx.x; t < S * D; t += blockDim.x) {
-    const int r = t / D, c = t % D;
-    float od = 0.f, os = 0.f;
-    const float* sd = wsh + static_cast<long long>(r) * state_floats<D>() + 2 + c;
-    const float* ss = sd + static_cast<long long>(chunks) * kRows * state_floats<D>();
-    for (int ch = 0; ch < chunks; ++ch) {
-      const long long off = static_cast<long long>(ch) * kRows * state_floats<D>();
-      od = fmaf(wts[0][r][ch], sd[off], od);
-      os = fmaf(wts[1][r][ch], ss[off], os);
-    }
-    const float ds = os - od, dt = o_t[r][c] - od;
-    err_s = fmaf(ds, ds, err_s);
-    err_t = fmaf(dt, dt, err_t);
+  for (int f = 0; f < F; ++f) {
+    const long long j = static_cast<long long>(f) * P + sp;
+    float dot = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) dot = fmaf(qv[e], to_f(k[head + j * D + lane + 32 * e]), dot);
+#pragma unroll
+    for (int o2 = 16; o2 > 0; o2 >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o2);
+    const float t = dot * scale_log2;
+    const float mn = fmaxf(m, t);
+    const float alpha = exp2f(m - mn);
+    const float p = exp2f(t - mn);
+    l = l * alpha + p;
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] = fmaf(p, to_f(v[head + j * D + lane + 32 * e]), acc[e] * alpha);
+    m = mn;
+  }
+  float es = 0.f, et = 0.f;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const float ds = om[1][e] - om[0][e], dt = acc[e] / l - om[0][e];
+    es = fmaf(ds, ds, es);
+    et = fmaf(dt, dt, et);
   }
 #pragma unroll
   for (int o2 = 16; o2 > 0; o2 >>= 1) {
-    err_s += __shfl_xor_sync(0xffffffffu, err_s, o2);
-    err_t += __shfl_xor_sync(0xffffffffu, err_t, o2);
+    es += __shfl_xor_sync(0xffffffffu, es, o2);
+    et += __shfl_xor_sync(0xffffffffu, et, o2);
   }
   if (lane == 0) {
-    red[0][warp] = err_s;
-    red[1][warp] = err_t;
+    err[0] = es;
+    err[1] = et;
+  }
+}
+
+// Per head: mean squared errors over the S x d sampled outputs and the mode.
+__global__ void __launch_bounds__(kRows) profile_finalize(const float* __restrict__ errs, int S,
+                                                          int D, float* __restrict__ mse_out,
+                                                          int32_t* __restrict__ mode_out) {
+  __shared__ float red[2][2];
+  const int bh = blockIdx.x, r = threadIdx.x, lane = r & 31, warp = r >> 5;
+  float es = 0.f, et = 0.f;
+  if (r < S) {
+    es = errs[(static_cast<long long>(bh) * kRows + r) * 2];
+    et = errs[(static_cast<long long>(bh) * kRows + r) * 2 + 1];
+  }
+#pragma unroll
+  for (int o2 = 16; o2 > 0; o2 >>= 1) {
+    es += __shfl_xor_sync(0xffffffffu, es, o2);
+    et += __shfl_xor_sync(0xffffffffu, et, o2);
+  }
+  if (lane == 0) {
+    red[0][warp] = es;
+    red[1][warp] = et;
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    float es = 0.f, et = 0.f;
-    for (int w = 0; w < 8; ++w) {
-      es += red[0][w];
-      et += red[1][w];
-    }
+  if (r == 0) {
     const float denom = static_cast<float>(S) * D;
-    es /= denom;
-    et /= denom;
+    es = (red[0][0] + red[0][1]) / denom;
+    et = (red[1][0] + red[1][1]) / denom;
     if (mse_out != nullptr) {
       mse_out[2 * bh] = es;
       mse_out[2 * bh + 1] = et;
@@ -399,6 +425,7 @@ svg_status launch_profile_shaped(const void* q, const void* k, const void* v, in
                                  float* mse_out, int32_t* mode_out, float* ws, ProfileShape ps,
                                  cudaStream_t s, const char* who) {
   const float scale_log2 = kLog2e / sqrtf(static_cast<float>(D));
+  float* errs = ws + states_bytes(B, H, ps.chunks, D) / sizeof(float);
   if (dtype == SVG_BF16) {
     const size_t smem =
         static_cast<size_t>(kRows) * D * 2 + 2 * kStages * static_cast<size_t>(kKeys) * D * 2;
@@ -410,19 +437,20 @@ svg_status launch_profile_shaped(const void* q, const void* k, const void* v, in
         static_cast<const __nv_bfloat16*>(v), idx, S, N, P, width, scale_log2, ps.chunks,
         ps.chunk_len, ws);
     if (svg_status st = check_launch(who)) return st;
-    profile_combine<D, __nv_bfloat16><<<B * H, 256, 0, s>>>(
+    profile_merge<D, __nv_bfloat16><<<dim3(B * H, kRows / kMergeRows), 32 * kMergeRows, 0, s>>>(
         static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-        static_cast<const __nv_bfloat16*>(v), idx, S, N, F, P, scale_log2, ps.chunks, ws, mse_out,
-        mode_out);
+        static_cast<const __nv_bfloat16*>(v), idx, S, N, F, P, scale_log2, ps.chunks, ws, errs);
   } else {
     profile_partial_fp32<D><<<dim3(ps.chunks, B * H, 2), 256, 0, s>>>(
         static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
         idx, S, N, P, width, scale_log2, ps.chunks, ps.chunk_len, ws);
     if (svg_status st = check_launch(who)) return st;
-    profile_combine<D, float><<<B * H, 256, 0, s>>>(
+    profile_merge<D, float><<<dim3(B * H, kRows / kMergeRows), 32 * kMergeRows, 0, s>>>(
         static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
-        idx, S, N, F, P, scale_log2, ps.chunks, ws, mse_out, mode_out);
+        idx, S, N, F, P, scale_log2, ps.chunks, ws, errs);
   }
+  if (svg_status st = check_launch(who)) return st;
+  profile_finalize<<<B * H, kRows, 0, s>>>(errs, S, D, mse_out, mode_out);
   return check_launch(who);
 }
 
@@ -526,12 +554,18 @@ size_t fixed_bytes_per_chunk(int B, int H, int d) {
   return static_cast<size_t>(B) * H * 2 * kRows * (d + 2) * sizeof(float);
 }
 
+// Scratch left for the chunk states after the per-row error sums.
+size_t fixed_state_budget(int B, int H) {
+  const size_t e = errors_bytes(B, H) + 256;  // + rounding of the state region
+  return e < kFixedScratchBytes ? kFixedScratchBytes - e : 0;
+}
+
 // The chunking of profile_shape, reduced until the states fit the fixed
 // scratch (fewer, longer key ranges per head).
 ProfileShape fixed_shape(int B, int H, int N, int d) {
   ProfileShape ps = profile_shape(B, H, N);
   const long long max_chunks =
-      static_cast<long long>(kFixedScratchBytes / fixed_bytes_per_chunk(B, H, d));
+      static_cast<long long>(fixed_state_budget(B, H) / fixed_bytes_per_chunk(B, H, d));
   if (ps.chunks > max_chunks) ps = shape_for(N, max_chunks);
   return ps;
 }
@@ -560,12 +594,12 @@ extern "C" svg_status svg_profile_heads_noalloc(const void* q, const void* k, co
     return fail(SVG_ERR_INVALID_ARG, "profile_noalloc: S=%d not in [1,%d]", S, kRows);
   if (!aligned16(q) || !aligned16(k) || !aligned16(v))
     return fail(SVG_ERR_INVALID_ARG, "profile_noalloc: tensors must be 16-byte aligned");
-  if (fixed_bytes_per_chunk(B, H, d) > kFixedScratchBytes)
+  if (fixed_bytes_per_chunk(B, H, d) > fixed_state_budget(B, H))
     return fail(SVG_ERR_INVALID_ARG,
                 "profile_noalloc: B*H=%d heads at d=%d need %zu bytes of scratch per key range; the "
                 "fixed scratch holds %zu bytes (at most %zu heads)",
-                B * H, d, fixed_bytes_per_chunk(B, H, d), kFixedScratchBytes,
-                kFixedScratchBytes / fixed_bytes_per_chunk(1, 1, d));
+                B * H, d, fixed_bytes_per_chunk(B, H, d) + errors_bytes(B, H), kFixedScratchBytes,
+                kFixedScratchBytes / (fixed_bytes_per_chunk(1, 1, d) + kRows * 2 * sizeof(float)));
   float* ws = nullptr;
   if (svg_status st = fixed_scratch(&ws)) return st;
   cudaStream_t s = as_stream(stream);
