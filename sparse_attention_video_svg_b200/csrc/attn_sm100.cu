@@ -49,6 +49,7 @@ constexpr int kBox = 16384;           // one 128-row x 128-byte TMA box
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;  // lazy-rescale threshold (factor 256)
 constexpr uint32_t kSpinLimit = 1u << 22;
+constexpr int kPolyPairs = 7;         // of every 16 exp2 pairs, this many run on the FMA pipe
 constexpr int kBarMax = 1;            // named barriers of the 256 softmax threads
 constexpr int kBarSum = 2;
 
@@ -59,12 +60,17 @@ struct Cfg {
   static constexpr int kSlots = D == 64 ? 10 : 4;  // K/V ring entries
   static constexpr int kOffQ = 0;                  // 2 Q buffers
   static constexpr int kOffKV = 2 * kTile;
-  static constexpr int kOffRed = kOffKV + kSlots * kTile;  // float [2][2][128] + [2][128]
+  // d = 64: the row sums come out of the tensor core as an extra O column:
+  // V is extended by a 64-column atom whose first column is 1.0 (fp16)
+  static constexpr bool kSumOnTC = D == 64;
+  static constexpr int kNO = kSumOnTC ? D + 16 : D;  // O columns (N of P.V)
+  static constexpr int kOffOnes = kOffKV + kSlots * kTile;
+  static constexpr int kOffRed = kOffOnes + (kSumOnTC ? kBox : 0);  // float [2][2][128] + [2][128]
   static constexpr int kOffBar = kOffRed + 6 * 128 * 4;
   static constexpr int kBars = 2 + 2 + 3 * kSlots + 2 + 2 + 2 + 1;
   static constexpr int kSmem = kOffBar + kBars * 8 + 16 + 1024;  // + alignment slack
   static constexpr uint32_t kIdescQK = idesc_bf16(128, 128, false);
-  static constexpr uint32_t kIdescPV = idesc_f16(128, D, true);
+  static constexpr uint32_t kIdescPV = idesc_f16(128, kNO, true);
 };
 
 struct Maps {
@@ -118,6 +124,30 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
   return false;
 }
 
+// 2^t for a pair of arguments on the FMA pipe: t = n + f with n the nearest
+// integer (t + 1.5 * 2^23 rounds in the mantissa), 2^f from a degree-4
+// minimax polynomial on [-1/2, 1/2] (coefficients fitted for this kernel by
+// a Remez iteration; relative error < 3e-6 in fp32), and 2^n added into the
+// exponent field.  Arguments are clamped at -40: the fp16 weight of 2^-40 is
+// 0 either way.
+__device__ __forceinline__ void exp2_poly2(float t0, float t1, float& p0, float& p1) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  constexpr float c0 = 0.9999992847442627f, c1 = 0.6931217908859253f, c2 = 0.240247443318367f,
+                  c3 = 0.05591785907745361f, c4 = 0.009570102207362652f;
+  t0 = fmaxf(t0, -40.f);
+  t1 = fmaxf(t1, -40.f);
+  float j0, j1, n0, n1, f0, f1, q0, q1;
+  add2(j0, j1, t0, t1, kRound, kRound);
+  add2(n0, n1, j0, j1, -kRound, -kRound);
+  add2(f0, f1, t0, t1, -n0, -n1);
+  fma2(q0, q1, c4, c4, f0, f1, c3, c3);
+  fma2(q0, q1, q0, q1, f0, f1, c2, c2);
+  fma2(q0, q1, q0, q1, f0, f1, c1, c1);
+  fma2(q0, q1, q0, q1, f0, f1, c0, c0);
+  p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(j0) << 23));
+  p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(j1) << 23));
+}
+
 // Softmax of one column half (64 keys) of every S tile, and the matching half
 // of the output columns.
 template <int D>
@@ -131,6 +161,7 @@ __device__ __forceinline__ void softmax_half(const AttnArgs& a, const Bars& B,
   const int row = quarter * 32 + lane;
   const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
   const uint32_t t_o = tmem + lane_off + 256 + half * (D / 2);
+  const uint32_t t_sum = tmem + lane_off + 256 + D;  // row-sum column (d = 64)
   const float sl2 = a.scale * kLog2e;
   const int N = a.N;
   uint32_t g = 0;  // tiles so far
@@ -168,13 +199,14 @@ __device__ __forceinline__ void softmax_half(const AttnArgs& a, const Bars& B,
         for (int i = 0; i < 64; ++i)
           if (i >= valid_cols) s[i] = -INFINITY;
       }
-      float mx8[8];
+      float mx4[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-      for (int t = 0; t < 8; ++t) mx8[t] = s[t];
+      for (int i = 4; i < 60; i += 8) {  // s[4 .. 59]
 #pragma unroll
-      for (int i = 8; i < 64; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], s[i]);
-      float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        for (int c = 0; c < 4; ++c) mx4[c] = max3(mx4[c], s[i + c], s[i + 4 + c]);
+      }
+      float mx = max3(max3(mx4[0], mx4[1], s[60]), max3(mx4[2], mx4[3], s[61]),
+                      fmaxf(s[62], s[63]));
       // both halves have read all of S once they pass this barrier, so the P
       // writes below cannot overwrite scores the other half still needs
       float* rm = red_max + (sb * 2) * 128;
@@ -204,28 +236,51 @@ __device__ __forceinline__ void softmax_half(const AttnArgs& a, const Bars& B,
             tmem_st32(t_o + ch * 32, r);
             tmem_wait_st();  // r is reused by the next chunk
           }
-          l *= alpha;
+          if constexpr (Cfg<D>::kSumOnTC) {
+            if (half == 1) {  // the row-sum columns [D, D + 16)
+              uint32_t r16[16];
+              tmem_ld16(t_sum, r16);
+              tmem_wait_ld();
+              reg_fence16(r16);
+#pragma unroll
+              for (int i = 0; i < 16; ++i) r16[i] = __float_as_uint(__uint_as_float(r16[i]) * alpha);
+              tmem_st16(t_sum, r16);
+              tmem_wait_st();
+            }
+          } else {
+            l *= alpha;
+          }
           m_used = m_new;
         }
       }
       const float neg = -m_used;
+      float lx = 0.f, ly = 0.f;
 #pragma unroll
       for (int q2 = 0; q2 < 2; ++q2) {
         uint32_t ph[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float p0 = fast_exp2(fmaf(s[32 * q2 + 2 * i], sl2, neg));
-          const float p1 = fast_exp2(fmaf(s[32 * q2 + 2 * i + 1], sl2, neg));
+          float t0, t1, p0, p1;
+          fma2(t0, t1, s[32 * q2 + 2 * i], s[32 * q2 + 2 * i + 1], sl2, sl2, neg, neg);
+          if ((i & 1) == 0 && i < 2 * kPolyPairs) {
+            exp2_poly2(t0, t1, p0, p1);  // FMA pipe
+          } else {
+            p0 = fast_exp2(t0);  // MUFU
+            p1 = fast_exp2(t1);
+          }
           const __half2 h = __floats2half2_rn(p0, p1);
           ph[i] = *reinterpret_cast<const uint32_t*>(&h);
-          // the row sum uses the fp16-rounded weights the MMA sees
-          const float2 r = __half22float2(h);
-          l += r.x + r.y;
+          if constexpr (!Cfg<D>::kSumOnTC) {
+            // the row sum uses the fp16-rounded weights the MMA sees
+            const float2 r = __half22float2(h);
+            add2(lx, ly, lx, ly, r.x, r.y);
+          }
         }
         // P column c (fp16 pair) holds keys 2c, 2c+1
         tmem_st16(t_s + 32 * half + 16 * q2, ph);
         tmem_wait_st();  // ph is rewritten by the next quarter
       }
+      if constexpr (!Cfg<D>::kSumOnTC) l += lx + ly;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&B.p_ready[sb]);
@@ -240,9 +295,16 @@ __device__ __forceinline__ void softmax_half(const AttnArgs& a, const Bars& B,
       if (!(ok = wait_bar(&B.o_done[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_flag, a.status)))
         break;
       tc_fence_after();
-      red_sum[half * 128 + row] = l;
-      named_bar_sync(kBarSum, 256);
-      ltot = l + red_sum[(half ^ 1) * 128 + row];
+      if constexpr (Cfg<D>::kSumOnTC) {
+        uint32_t r1 = tmem_ld1(t_sum);
+        tmem_wait_ld();
+        reg_fence1(r1);
+        ltot = __uint_as_float(r1);
+      } else {
+        red_sum[half * 128 + row] = l;
+        named_bar_sync(kBarSum, 256);
+        ltot = l + red_sum[(half ^ 1) * 128 + row];
+      }
     }
     const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
     const int n = qt * 128 + row;
@@ -336,6 +398,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
+  if (C::kSumOnTC && (warp == 2 || warp == 3)) {
+    // 128 rows x 64 fp16 columns, swizzled like a V box: column 0 = 1.0
+    uint4* ones = reinterpret_cast<uint4*>(smem + C::kOffOnes);
+    for (int r = threadIdx.x - 64; r < 128; r += 64)
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc)
+        ones[r * 8 + cc] = make_uint4(cc == (r & 7) ? 0x3C00u : 0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -398,10 +469,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!wait_bar(&B.v_ready[slot], (lv / C::kSlots) & 1, abort_flag, a.status)) return false;
         tc_fence_after();
         const uint32_t vbase = smem_u32(smem + C::kOffKV + slot * C::kTile);
+        // second 64-column atom of B: V columns 64.. (d = 128) or the ones
+        // column that accumulates the row sums (d = 64)
+        const uint32_t lbo = C::kSumOnTC ? smem_u32(smem + C::kOffOnes) - vbase : kBox;
         // O (+)= P V, P (fp16) in S columns [0, 64), V converted to fp16
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem_o, tmem_s0 + sb * 128 + kk * 8, sdesc_sw128(vbase + kk * 2048, kBox, 1024),
+          mma_ts(tmem_o, tmem_s0 + sb * 128 + kk * 8, sdesc_sw128(vbase + kk * 2048, lbo, 1024),
                  C::kIdescPV, (first_of_item && kk == 0) ? 0u : 1u);
         tc_commit(&B.kv_empty[slot]);
         tc_commit(&B.o_done[sb]);
