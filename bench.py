@@ -46,6 +46,60 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+# DRAM bytes (read + write) of one attention launch on the CogVideoX-shaped
+# layer, from an ncu capture of the kernel built from the sources whose
+# sha256 is recorded here.  Reported only while the sources still match.
+ATTN_SOURCES = ("attn_sm100.cu", "sm100.cuh", "attn.cuh", "common.cuh")
+ATTN_TRAFFIC = {"cogvideox": {"sha256": "cc1096141835a399df2fc154f3eae3d5e6fc8a804b56af6430a52dd193db03db",
+                              "bytes": 324635392 + 87066880}}
+
+
+def attn_sources_sha256():
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "sparse_attention_video_svg_b200", "csrc")
+    for name in ATTN_SOURCES:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def attn_traffic(workload):
+    rec = ATTN_TRAFFIC.get(workload)
+    if rec is None or attn_sources_sha256() != rec["sha256"]:
+        return None
+    return rec["bytes"]
+
+
+def rank_seed(wl, rank):
+    """Each rank runs its own independent layer (weak scaling)."""
+    return wl.seed + rank
+
+
+def max_over_ranks(values, world, device):
+    """Element-wise max of per-rank timings (every rank gets the result)."""
+    if world == 1:
+        return [float(x) for x in values]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x) for x in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def aggregate(flops_per_rank, total_ms, steps, world, tokens_per_rank):
+    """Whole-job throughput: the work of all ranks over the slowest rank's
+    time per step.  Returns (TFLOPS, tokens/s, ms per step)."""
+    ms = total_ms / steps
+    return (flops_per_rank * world / (ms * 1e-3) / 1e12,
+            tokens_per_rank * world / (ms * 1e-3), ms)
+
+
+def workload_config(wl):
+    return {"workload": wl.name, "B": wl.B, "H": wl.H, "frames": wl.F, "tokens_per_frame": wl.P,
+            "N": wl.N, "d": wl.d, "sampled_queries": wl.S, "spatial_width": wl.width}
+
+
 def kept_pairs(indptr, indices, N, T=128):
     """Query-key pairs inside the kept tiles of one list (ragged tiles count
     their valid rows and columns)."""
@@ -122,7 +176,7 @@ def run_ours(args, rank, world, local_rank):
     wl = si.WORKLOADS[args.config]
     if wl.kind != "profiled":
         raise SystemExit(f"bench runs profiled layers; {wl.name} is {wl.kind}")
-    seed = wl.seed + rank
+    seed = rank_seed(wl, rank)
     q, k, v, types = si.generate(wl, seed=seed)
     idx = si.sample_queries(wl, seed=wl.seed)
     host = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in (q, k, v)]
@@ -161,15 +215,14 @@ def run_ours(args, rank, world, local_rank):
     clocks = ClockSampler(local_rank)
     clocks.start()
     time.sleep(0.3)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(K)]
+    ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(5)) for _ in range(K)]
     for i in range(K):
         flush.fill_(i & 0xff)
-        s0, a0, a1, s1 = ev[i]
+        s0, p0, a0, a1, s1 = ev[i]
         s0.record(stream)
         svg.svg_profile_heads(qd, kd, vd, F, P, w, idx_d, mse_out=bufs.mse, mode_out=bufs.mode,
                               workspace=bufs.ws)
+        p0.record(stream)
         for x, y in ((qd, bufs.qp), (kd, bufs.kp), (vd, bufs.vp)):
             svg.svg_permute_token_major(x, F, P, bufs.mode, out=y)
         a0.record(stream)
@@ -182,10 +235,14 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
     torch.cuda.synchronize()
     clk = clocks.stop()
-    step_ms = [e[0].elapsed_time(e[3]) for e in ev]
-    attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    step_ms = [e[0].elapsed_time(e[4]) for e in ev]
+    attn_ms = [e[2].elapsed_time(e[3]) for e in ev]
+    prof_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    perm_ms = [e[1].elapsed_time(e[2]) + e[3].elapsed_time(e[4]) for e in ev]
     total_ms = float(sum(step_ms))
     attn_avg = float(sum(attn_ms) / K)
+    prof_avg = float(sum(prof_ms) / K)
+    perm_avg = float(sum(perm_ms) / K)
 
     # end to end through the public API with host buffers
     out_host = torch.empty(qd.shape, dtype=torch.bfloat16).pin_memory()
@@ -211,22 +268,24 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
 
-    if world > 1:
-        t = torch.tensor([total_ms, e2e_ms, attn_avg], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, e2e_ms, attn_avg = (float(x) for x in t.tolist())
+    total_ms, e2e_ms, attn_avg, prof_avg, perm_avg = max_over_ranks(
+        [total_ms, e2e_ms, attn_avg, prof_avg, perm_avg], world, dev)
     if rank != 0:
         return None
 
     peaks, src = load_peaks()
     peak_tf = float(peaks["bf16_tflops"])
-    all_flops = flops * world
-    value = all_flops / (total_ms / K * 1e-3) / 1e12
-    tokens_s = wl.B * N * world / (total_ms / K * 1e-3)
+    value, tokens_s, step_ms_avg = aggregate(flops, total_ms, K, world, wl.B * N)
+    e2e_value, _, e2e_step_ms = aggregate(flops, e2e_ms, K, world, wl.B * N)
     attn_tf = flops / (attn_avg * 1e-3) / 1e12
+    hbm_gbs = float(peaks["hbm_gbs"])
+    elems = wl.B * wl.H * N * d
+    perm_bytes = 4 * 2 * elems * 2
+    prof_bytes = 2 * elems * 2      # K and V streamed once
     h2d = sum(h.numel() * 2 for h in host)
     d2h = out_host.numel() * 2 + mode_host.numel() * 4
-    launches_per_step = 2 + 3 + 1 + 1   # profile partial+combine, 3 permutes, attention, permute back
+    # profile partial, merge, finalize; 3 permutes; attention; permute back
+    launches_per_step = 3 + 3 + 1 + 1
     line = {
         "metric": METRIC,
         "value": round(value, 3),
@@ -234,14 +293,13 @@ def run_ours(args, rank, world, local_rank):
         "n_gpus": world,
         "steps": K,
         "warmup": W,
-        "ms_per_step": round(total_ms / K, 5),
+        "ms_per_step": round(step_ms_avg, 5),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded biased-Gaussian q/k/v, no model weights)",
-        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "frames": F, "tokens_per_frame": P,
-                   "N": N, "d": d, "sampled_queries": wl.S, "spatial_width": w,
+        "config": {**workload_config(wl),
                    "modes": {"spatial": int((modes == 0).sum()), "temporal": int((modes == 1).sum())},
                    "kept_fraction": {"spatial": round(kept_frac[0], 5),
                                      "temporal": round(kept_frac[1], 5)},
@@ -250,12 +308,20 @@ def run_ours(args, rank, world, local_rank):
         "tokens_per_s": round(tokens_s, 1),
         "pct_of_bf16_peak": round(100 * value / world / peak_tf, 2),
         "attention_only": {"ms": round(attn_avg, 5), "effective_tflops": round(attn_tf, 3)},
+        # 4 permutes per step (q, k, v forward; o back), every head written:
+        # 2 * B*H*N*d * 2 bytes each; L2 flushed only before the step
+        "permute": {"ms": round(perm_avg, 5),
+                    "gbs": round(perm_bytes / (perm_avg * 1e-3) / 1e9, 1),
+                    "frac_of_hbm": round(perm_bytes / (perm_avg * 1e-3) / 1e9 / hbm_gbs, 4),
+                    "hbm_peak_gbs": hbm_gbs},
+        "profile": {"ms": round(prof_avg, 5),
+                    "kv_gbs": round(prof_bytes / (prof_avg * 1e-3) / 1e9, 1)},
         "roofline": {"kernel": "svg_sparse_attn", "bound": "tensor", "achieved": round(attn_tf, 3),
                      "peak": peak_tf, "unit": "TFLOP/s", "frac": round(attn_tf / peak_tf, 4),
-                     "peak_source": f"{src} bf16 burst", "traffic": None},
-        "e2e": {"value": round(all_flops / (e2e_ms / K * 1e-3) / 1e12, 3), "unit": "TFLOPS",
+                     "peak_source": f"{src} bf16 burst", "traffic": attn_traffic(wl.name)},
+        "e2e": {"value": round(e2e_value, 3), "unit": "TFLOPS",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": round(e2e_ms / K, 5)},
+                "ms_per_step": round(e2e_step_ms, 5)},
         "gpu_launches": launches_per_step * K,
         "clocks": clk,
     }
@@ -316,20 +382,24 @@ def cpu_baseline(wl, budget_s=15.0, seed=None):
                       f"block-sparse attention (float64 NumPy), {dt:.1f} s"}
 
 
-def run_reference(args):
+def run_reference(args, world=1):
     wl = si.WORKLOADS[args.config]
     K, W = args.steps, args.warmup
     budget = max(1.0, args.cpu_budget / max(1, K + W))
     for _ in range(W):
         cpu_baseline(wl, budget_s=budget)
-    vals = [cpu_baseline(wl, budget_s=budget) for _ in range(K)]
+    vals, wall = [], []
+    for _ in range(K):
+        t0 = time.perf_counter()
+        vals.append(cpu_baseline(wl, budget_s=budget))
+        wall.append(time.perf_counter() - t0)
     value = statistics.mean(v["value"] for v in vals)
     return {
         "impl": "reference",
-        "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": 1, "steps": K, "warmup": W,
-        "ms_per_step": None, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": round(1e3 * statistics.mean(wall), 3), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic (seeded biased-Gaussian q/k/v, no model weights)",
-        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "N": wl.N, "d": wl.d},
+        "config": {**workload_config(wl), "oracle": "rank 0 host cores only"},
         "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": vals[-1]["cores"],
                          "kind": "oracle", "sample": vals[-1]["sample"]},
         "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0,
@@ -354,7 +424,7 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         if rank == 0:
-            print(json.dumps(run_reference(args)), flush=True)
+            print(json.dumps(run_reference(args, world)), flush=True)
         return
     if world > 1:
         import datetime

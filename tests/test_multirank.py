@@ -1,0 +1,111 @@
+"""Multi-rank host logic of bench.py on CPU (gloo, world size 2).
+
+The layer shards by (batch, head) with no exchange step, so N GPUs run N
+independent layers (weak scaling); the only cross-rank operations are the
+barrier and the max-over-ranks of the step timings.  These tests run that
+logic as real gloo ranks and launch the reference arm through torchrun."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+import svg_inputs as si  # noqa: E402
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, results):
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        # per-rank timings that differ in every slot
+        mine = [10.0 + rank, 5.0 - rank, 1.0 + 0.5 * rank]
+        got = bench.max_over_ranks(mine, world, torch.device("cpu"))
+        wl = si.WORKLOADS["cogvideox"]
+        value, tok, ms = bench.aggregate(2.0e12, got[0], 4, world, wl.B * wl.N)
+        dist.barrier()
+        results[rank] = {"max": got, "value": value, "tokens": tok, "ms": ms,
+                         "seed": bench.rank_seed(wl, rank)}
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_aggregate_gloo():
+    world = 2
+    mgr = mp.get_context("spawn").Manager()
+    results = mgr.dict()
+    mp.start_processes(_rank_main, args=(world, _free_port(), results), nprocs=world,
+                       join=True, start_method="spawn")
+    r0, r1 = results[0], results[1]
+    assert r0["max"] == r1["max"] == [11.0, 5.0, 1.5]
+    # whole-job value: both ranks' work over the slowest rank's step time
+    assert r0["ms"] == pytest.approx(11.0 / 4)
+    assert r0["value"] == pytest.approx(2 * 2.0e12 / (11.0 / 4 * 1e-3) / 1e12)
+    assert r0["tokens"] == pytest.approx(2 * 17550 / (11.0 / 4 * 1e-3))
+    assert r0["value"] == r1["value"]
+    # independent inputs per rank
+    assert r0["seed"] != r1["seed"]
+
+
+def test_single_rank_passthrough():
+    assert bench.max_over_ranks([3, 2.5], 1, None) == [3.0, 2.5]
+    v, t, ms = bench.aggregate(1.0e12, 20.0, 10, 1, 100)
+    assert ms == 2.0 and v == pytest.approx(500.0) and t == pytest.approx(5.0e4)
+
+
+def test_rank_inputs_differ():
+    wl = si.small("cogvideox")
+    a = si.generate(wl, seed=bench.rank_seed(wl, 0))[0]
+    b = si.generate(wl, seed=bench.rank_seed(wl, 1))[0]
+    assert a.shape == b.shape and (a != b).any()
+
+
+def test_reference_arm_under_torchrun_prints_once():
+    """torchrun with 2 ranks: rank 0 alone runs the oracle and prints one JSON
+    line carrying the contract's keys; the other rank exits 0 without work."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()),
+           os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+           "--steps", "1", "--warmup", "3", "--cpu-budget", "1"]
+    env = dict(os.environ, OMP_NUM_THREADS="2")
+    out = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, out.stdout
+    line = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e", "impl"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["n_gpus"] == 2
+    assert line["config"]["workload"] == "cogvideox"
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    assert line["value"] > 0
+
+
+def test_traffic_tracks_kernel_sources(monkeypatch):
+    """DRAM traffic is reported only for the kernel sources it was measured on."""
+    rec = bench.ATTN_TRAFFIC["cogvideox"]
+    monkeypatch.setattr(bench, "attn_sources_sha256", lambda: rec["sha256"])
+    assert bench.attn_traffic("cogvideox") == rec["bytes"]
+    monkeypatch.setattr(bench, "attn_sources_sha256", lambda: "0" * 64)
+    assert bench.attn_traffic("cogvideox") is None
+    assert bench.attn_traffic("wan480") is None
