@@ -6,32 +6,42 @@
 // keep/skip decisions on 128 x 128 tiles, walked through a per-query-block
 // list of kept key blocks.
 //
-// Persistent kernel, one CTA per SM, work item = (head, 128-row query tile).
+// Persistent kernel, one CTA per SM.  A work item is a pair of adjacent
+// 128-row query tiles of one head (members 0 and 1).  The producer walks the
+// two members' key lists as one merged sequence of steps, so a key block that
+// both keep is loaded once and feeds both; each member then runs its own
+// pipeline on the tensor core.
 // Warp roles (384 threads, three warpgroups):
-//   warp 0      TMA producer: the Q tile of each item (double-buffered across
-//               items), then K and V of every kept key block into a ring;
-//   warp 1      MMA issuer (one thread): S = Q K^T into TMEM (two S buffers,
-//               bf16 operands) and O += P V (fp16 operands), P read from
-//               TMEM, V from smem;
-//   warps 2-3   convert each V tile in shared memory from bf16 to fp16;
-//   warps 4-7   softmax of S columns [0, 64), warps 8-11 of [64, 128): one
-//               thread per (query row, column half).  The two halves swap
-//               their row maxima through shared memory, then each computes
-//               fp32 online-softmax weights for its 64 keys with lazy
-//               rescaling (O is rescaled only when the running max grows by
-//               more than 2^8) and writes them into the S buffer as fp16
-//               (11 significant bits; the row sum uses the same rounded
-//               values).  In the
-//               epilogue each half writes its half of the columns of O / l as
-//               bf16 straight from registers to global memory.
-// MMA order per item: QK_0, QK_1, PV_0, QK_2, PV_1, ... so the tensor core
-// computes S_{j+1} while the softmax works on S_j.
+//   warp 0      TMA producer: each member's Q tile, then K and V of every
+//               step into a ring, with a step record (which members keep the
+//               block, item boundaries) in shared memory;
+//   warps 1, 2  MMA issuers of members 0 and 1 (one thread each):
+//               S_t = Q_t K^T into TMEM (bf16 operands) and O_t += P_t V
+//               (fp16 operands, P_t read from TMEM, V from smem).  A K/V ring
+//               entry is released when both issuers have passed it;
+//   warp 3      converts each V tile in shared memory from bf16 to fp16;
+//   warps 4-7   softmax of member 0, warps 8-11 of member 1: one thread per
+//               query row holds the tile's 128 scores, fp32 online softmax
+//               with lazy rescaling (O is rescaled only when the running max
+//               grows by more than 2^8); the weights go to TMEM as fp16
+//               (11 significant bits) and the row sums add the same rounded
+//               values (mixed-precision adds).  The epilogue writes O / l as
+//               bf16 from registers.
+// Every exponential runs on the MUFU (ex2.approx): FMA-pipe work in the
+// softmax warps measurably slows the issue of the tensor-core instructions,
+// so the softmax keeps its FMA-pipe share small.  Each tile's MMAs are
+// issued from one asm block (about two instructions per MMA).
+// d = 64: P_t has TMEM columns of its own, so the next S_t = Q_t K^T is
+// issued as soon as the softmax has read S_t and runs during the softmax.
+// d = 128 (TMEM is full with two S and two O): P_t overwrites S_t, and the
+// next Q_t K^T is issued after O_t += P_t V; tcgen05 operations of one thread
+// complete in issue order, so "S_t full" also means that P.V finished.
 //
-// TMEM columns: S buffer b at [128 b, 128 b + 128), O at [256, 256 + d).
 // Every mbarrier wait is bounded; a wait that gives up sets
 // SVG_DEVICE_TIMEOUT, raises a CTA-wide abort flag and every role drains out.
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
+#include <limits.h>
 
 #include <mutex>
 
@@ -49,28 +59,42 @@ constexpr int kBox = 16384;           // one 128-row x 128-byte TMA box
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;  // lazy-rescale threshold (factor 256)
 constexpr uint32_t kSpinLimit = 1u << 22;
-constexpr int kPolyPairs = 7;         // of every 16 exp2 pairs, this many run on the FMA pipe
-constexpr int kBarMax = 1;            // named barriers of the 256 softmax threads
-constexpr int kBarSum = 2;
+constexpr uint32_t kDrainLimit = 1u << 20;
+constexpr int kLaunchRegs = 168;      // 65536 / 384, rounded down to a multiple of 8
 
 template <int D>
 struct Cfg {
   static constexpr int kTile = 128 * D * 2;        // bytes of a Q / K / V tile
   static constexpr int kBoxes = D / 64;            // 64-column boxes per tile
-  static constexpr int kSlots = D == 64 ? 10 : 4;  // K/V ring entries
-  static constexpr int kOffQ = 0;                  // 2 Q buffers
-  static constexpr int kOffKV = 2 * kTile;
-  // d = 64: the row sums come out of the tensor core as an extra O column:
-  // V is extended by a 64-column atom whose first column is 1.0 (fp16)
-  static constexpr bool kSumOnTC = D == 64;
-  static constexpr int kNO = kSumOnTC ? D + 16 : D;  // O columns (N of P.V)
-  static constexpr int kOffOnes = kOffKV + kSlots * kTile;
-  static constexpr int kOffRed = kOffOnes + (kSumOnTC ? kBox : 0);  // float [2][2][128] + [2][128]
-  static constexpr int kOffBar = kOffRed + 6 * 128 * 4;
-  static constexpr int kBars = 2 + 2 + 3 * kSlots + 2 + 2 + 2 + 1;
+  static constexpr int kQDepth = D == 64 ? 2 : 1;  // Q buffers per member
+  // K/V ring entries; even, so K tiles always sit in even and V tiles in odd
+  // entries
+  static constexpr int kSlots = D == 64 ? 8 : 4;
+  static constexpr int kSteps = kSlots / 2;        // merged-walk steps in flight
+  static constexpr bool kSepP = D == 64;           // P_t in TMEM columns of its own
+  static constexpr int kOffQ = 0;                  // [member][depth]
+  static constexpr int kOffKV = 2 * kQDepth * kTile;
+  static constexpr int kOffInfo = kOffKV + kSlots * kTile;  // uint32 [kSteps]
+  static constexpr int kOffBar = kOffInfo + 64;
+  static constexpr int kBars = 4 * kQDepth + 3 * kSlots + 5 * 2;
   static constexpr int kSmem = kOffBar + kBars * 8 + 16 + 1024;  // + alignment slack
+  // TMEM columns
+  static constexpr uint32_t kColS = 0;                   // S_t at 128 t
+  static constexpr uint32_t kColP = kSepP ? 256 : 0;     // P_t at kColP + kPStride t
+  static constexpr uint32_t kPStride = kSepP ? 64 : 128;
+  static constexpr uint32_t kColO = kSepP ? 384 : 256;   // O_t at kColO + kOStride t
+  static constexpr uint32_t kOStride = kSepP ? 64 : 128;
+  // Register split of the 384 x 168 launch registers: warpgroup 0
+  // (producer, MMA issuers, converter) drops to kRegsLow, the two softmax
+  // warpgroups rise to kRegsHigh (the split with the fewest spills ptxas reports).
+  static constexpr int kRegsLow = 80;
+  static constexpr int kRegsHigh = 208;
+  static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kLaunchRegs, "register split");
   static constexpr uint32_t kIdescQK = idesc_bf16(128, 128, false);
-  static constexpr uint32_t kIdescPV = idesc_f16(128, kNO, true);
+  static constexpr uint32_t kIdescPV = idesc_f16(128, D, true);
+  static_assert(kSlots % 2 == 0, "K and V must alternate between even and odd ring entries");
+  static_assert(kSmem <= 227 * 1024, "shared memory budget");
+  static_assert(kColO + 2 * kOStride <= 512, "TMEM budget");
 };
 
 struct Maps {
@@ -78,21 +102,31 @@ struct Maps {
 };
 
 struct Bars {
-  uint64_t* q_full;    // [2]
-  uint64_t* q_empty;   // [2]
+  uint64_t* q_full;    // [2][depth]
+  uint64_t* q_empty;   // [2][depth]
   uint64_t* kv_full;   // [slots]
-  uint64_t* kv_empty;  // [slots]
+  uint64_t* kv_empty;  // [slots] one commit from each member's issuer
   uint64_t* v_ready;   // [slots] V tile converted to fp16
-  uint64_t* s_full;    // [2]
-  uint64_t* p_ready;   // [2]
-  uint64_t* o_done;    // [2]
-  uint64_t* o_free;    // [1]
+  uint64_t* s_full;    // [2] S_t written
+  uint64_t* s_free;    // [2] S_t read by the softmax (4 warps; separate-P layout)
+  uint64_t* p_ready;   // [2] P_t written (4 warps)
+  uint64_t* o_done;    // [2] O_t += P_t V finished
+  uint64_t* drain;     // [2] every MMA of an issuer finished
 };
 
-// The list of (bh, qt): [beg, end) into indices, or empty.
-__device__ __forceinline__ void item_list(const AttnArgs& a, int bh, int qt, int& beg, int& end,
-                                          bool report = false) {
+__device__ __forceinline__ bool valid_tile(int j, int nb) { return j >= 0 && j < nb; }
+
+// Step record the producer publishes with each K/V pair: bits 0-1 the members
+// that keep the block, bits 2-3 the members for which it is the first block
+// of the item, bits 4-5 the last; bit 6 marks the end (no tile loaded).
+constexpr uint32_t kStepEnd = 1u << 6;
+
+// Entries [beg, end) of `indices` for query tile qt of head bh; empty for a
+// tile past the end or a bad list.
+__device__ __forceinline__ void member_list(const AttnArgs& a, int bh, int qt, int nb, int& beg,
+                                            int& end, bool report) {
   beg = end = 0;
+  if (qt >= nb) return;
   const int lid = a.list_id[bh];
   if (lid < 0 || lid >= a.n_lists) {
     if (report) set_status(a.status, SVG_DEVICE_BAD_LIST_ID);
@@ -108,7 +142,35 @@ __device__ __forceinline__ void item_list(const AttnArgs& a, int bh, int qt, int
   end = e;
 }
 
-__device__ __forceinline__ bool valid_tile(int j, int nb) { return j >= 0 && j < nb; }
+__device__ __forceinline__ void skip_invalid(const AttnArgs& a, int nb, int& p, int e,
+                                             bool report) {
+  while (p < e && !valid_tile(a.indices[p], nb)) {
+    if (report) set_status(a.status, SVG_DEVICE_BAD_INDEX);
+    ++p;
+  }
+}
+
+// Next key block of the merged walk over both members' lists, whose heads
+// are valid (or exhausted).  mask bit t: member t keeps block j.  Every entry
+// of either list is visited exactly once, in whatever order the lists come;
+// equal heads are shared.  Afterwards both heads are again valid or
+// exhausted.
+__device__ __forceinline__ bool merge_next(const AttnArgs& a, int nb, int (&p)[2],
+                                           const int (&e)[2], int& j, int& mask) {
+  int jj[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) jj[t] = p[t] < e[t] ? a.indices[p[t]] : INT_MAX;
+  j = min(jj[0], jj[1]);
+  if (j == INT_MAX) return false;
+  mask = (jj[0] == j ? 1 : 0) | (jj[1] == j ? 2 : 0);
+#pragma unroll
+  for (int t = 0; t < 2; ++t)
+    if (mask >> t & 1) {
+      ++p[t];
+      skip_invalid(a, nb, p[t], e[t], true);
+    }
+  return true;
+}
 
 // Bounded wait on an mbarrier phase; false if it timed out or another role
 // aborted.
@@ -124,224 +186,183 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
   return false;
 }
 
-// 2^t for a pair of arguments on the FMA pipe: t = n + f with n the nearest
-// integer (t + 1.5 * 2^23 rounds in the mantissa), 2^f from a degree-4
-// minimax polynomial on [-1/2, 1/2] (coefficients fitted for this kernel by
-// a Remez iteration; relative error < 3e-6 in fp32), and 2^n added into the
-// exponent field.  Arguments are clamped at -40: the fp16 weight of 2^-40 is
-// 0 either way.
-__device__ __forceinline__ void exp2_poly2(float t0, float t1, float& p0, float& p1) {
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  constexpr float c0 = 0.9999992847442627f, c1 = 0.6931217908859253f, c2 = 0.240247443318367f,
-                  c3 = 0.05591785907745361f, c4 = 0.009570102207362652f;
-  t0 = fmaxf(t0, -40.f);
-  t1 = fmaxf(t1, -40.f);
-  float j0, j1, n0, n1, f0, f1, q0, q1;
-  add2(j0, j1, t0, t1, kRound, kRound);
-  add2(n0, n1, j0, j1, -kRound, -kRound);
-  add2(f0, f1, t0, t1, -n0, -n1);
-  fma2(q0, q1, c4, c4, f0, f1, c3, c3);
-  fma2(q0, q1, q0, q1, f0, f1, c2, c2);
-  fma2(q0, q1, q0, q1, f0, f1, c1, c1);
-  fma2(q0, q1, q0, q1, f0, f1, c0, c0);
-  p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(j0) << 23));
-  p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(j1) << 23));
+// Bounded wait that ignores the abort flag (used to drain copies and MMAs in
+// flight before the CTA exits).
+__device__ __forceinline__ void drain_bar(uint64_t* bar, uint32_t parity) {
+  const uint32_t addr = smem_u32(bar);
+  for (uint32_t i = 0; i < kDrainLimit; ++i)
+    if (mbar_try_wait(addr, parity)) return;
 }
 
-// Softmax of one column half (64 keys) of every S tile, and the matching half
-// of the output columns.
+// Softmax and epilogue of member t (warps 4 + 4t .. 7 + 4t).
 template <int D>
-__device__ __forceinline__ void softmax_half(const AttnArgs& a, const Bars& B,
-                                             volatile int* abort_flag, uint32_t tmem,
-                                             float* red_max, float* red_sum, int n_items,
-                                             int nb) {
+__device__ __forceinline__ void softmax_member(const AttnArgs& a, const Bars& B,
+                                               volatile int* abort_flag, uint32_t tmem,
+                                               int n_items, int n_pairs, int nb) {
+  using C = Cfg<D>;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int half = (warp >> 2) - 1;  // 0: S columns [0, 64), 1: [64, 128)
-  const int quarter = warp & 3;      // TMEM lane quarter this warp may access
+  const int t = (warp - 4) >> 2;  // member
+  const int quarter = warp & 3;   // TMEM lane quarter this warp may access
   const int row = quarter * 32 + lane;
   const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-  const uint32_t t_o = tmem + lane_off + 256 + half * (D / 2);
-  const uint32_t t_sum = tmem + lane_off + 256 + D;  // row-sum column (d = 64)
+  const uint32_t t_s = tmem + lane_off + C::kColS + 128 * t;
+  const uint32_t t_p = tmem + lane_off + C::kColP + C::kPStride * t;
+  const uint32_t t_o = tmem + lane_off + C::kColO + C::kOStride * t;
   const float sl2 = a.scale * kLog2e;
   const int N = a.N;
-  uint32_t g = 0;  // tiles so far
+  uint32_t g = 0;  // tiles of this member so far
   bool ok = true;
   for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
-    const int bh = item / nb, qt = item - bh * nb;
+    const int bh = item / n_pairs;
+    const int qt = 2 * (item - bh * n_pairs) + t;
+    if (qt >= nb) continue;
     int beg, end;
-    item_list(a, bh, qt, beg, end);
+    member_list(a, bh, qt, nb, beg, end, false);
     float m_used = -INFINITY, l = 0.f;
     bool first = true;
-    for (int e = beg; e < end && ok; ++e) {
+    for (int e = beg; e < end; ++e) {
       const int j = a.indices[e];
       if (!valid_tile(j, nb)) continue;
-      const int sb = g & 1;
-      if (!(ok = wait_bar(&B.s_full[sb], (g >> 1) & 1, abort_flag, a.status))) break;
+      if (!(ok = wait_bar(&B.s_full[t], g & 1, abort_flag, a.status))) break;
       tc_fence_after();
-      const uint32_t t_s = tmem + lane_off + sb * 128;
-      float s[64];
+      float s[128];
       {
-        uint32_t r0[32], r1[32];
-        tmem_ld32(t_s + 64 * half, r0);
-        tmem_ld32(t_s + 64 * half + 32, r1);
-        tmem_wait_ld();
-        reg_fence32(r0);
-        reg_fence32(r1);
+        uint32_t r[4][32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          s[i] = __uint_as_float(r0[i]);
-          s[32 + i] = __uint_as_float(r1[i]);
+        for (int c = 0; c < 4; ++c) tmem_ld32(t_s + 32 * c, r[c]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          reg_fence32(r[c]);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(r[c][i]);
         }
       }
-      const int valid_cols = min(128, N - j * 128) - 64 * half;
-      if (valid_cols < 64) {
+      if constexpr (C::kSepP) {
+        // S_t is in registers: the next Q_t K^T may overwrite it
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&B.s_free[t]);
+      }
+      const int valid_cols = min(128, N - j * 128);
+      if (valid_cols < 128) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i)
+        for (int i = 0; i < 128; ++i)
           if (i >= valid_cols) s[i] = -INFINITY;
       }
       float mx4[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-      for (int i = 4; i < 60; i += 8) {  // s[4 .. 59]
+      for (int i = 4; i < 124; i += 8) {  // s[4 .. 123]
 #pragma unroll
         for (int c = 0; c < 4; ++c) mx4[c] = max3(mx4[c], s[i + c], s[i + 4 + c]);
       }
-      float mx = max3(max3(mx4[0], mx4[1], s[60]), max3(mx4[2], mx4[3], s[61]),
-                      fmaxf(s[62], s[63]));
-      // both halves have read all of S once they pass this barrier, so the P
-      // writes below cannot overwrite scores the other half still needs
-      float* rm = red_max + (sb * 2) * 128;
-      rm[half * 128 + row] = mx;
-      named_bar_sync(kBarMax, 256);
-      mx = fmaxf(mx, rm[(half ^ 1) * 128 + row]);
+      const float mx = max3(max3(mx4[0], s[124], s[125]), max3(mx4[1], s[126], s[127]),
+                            fmaxf(mx4[2], mx4[3]));
       const float tm = mx * sl2;
+      float alpha = 1.f;
+      bool rescale = false;
       if (first) {
         m_used = tm;
       } else {
         const bool need = tm > m_used + kRescaleLog2;
         if (__any_sync(0xffffffffu, need)) {
-          // O must hold PV of the previous tile before it is rescaled
-          if (!(ok = wait_bar(&B.o_done[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_flag, a.status)))
-            break;
-          tc_fence_after();
+          rescale = true;
           const float m_new = need ? tm : m_used;
-          const float alpha = exp2f(m_used - m_new);
-          uint32_t r[32];
-#pragma unroll
-          for (int ch = 0; ch < D / 64; ++ch) {
-            tmem_ld32(t_o + ch * 32, r);
-            tmem_wait_ld();
-            reg_fence32(r);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            tmem_st32(t_o + ch * 32, r);
-            tmem_wait_st();  // r is reused by the next chunk
-          }
-          if constexpr (Cfg<D>::kSumOnTC) {
-            if (half == 1) {  // the row-sum columns [D, D + 16)
-              uint32_t r16[16];
-              tmem_ld16(t_sum, r16);
-              tmem_wait_ld();
-              reg_fence16(r16);
-#pragma unroll
-              for (int i = 0; i < 16; ++i) r16[i] = __float_as_uint(__uint_as_float(r16[i]) * alpha);
-              tmem_st16(t_sum, r16);
-              tmem_wait_st();
-            }
-          } else {
-            l *= alpha;
-          }
+          alpha = exp2f(m_used - m_new);
           m_used = m_new;
         }
       }
       const float neg = -m_used;
       float lx = 0.f, ly = 0.f;
+      uint32_t ph[4][16];
 #pragma unroll
-      for (int q2 = 0; q2 < 2; ++q2) {
-        uint32_t ph[16];
+      for (int c = 0; c < 4; ++c) {
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           float t0, t1, p0, p1;
-          fma2(t0, t1, s[32 * q2 + 2 * i], s[32 * q2 + 2 * i + 1], sl2, sl2, neg, neg);
-          if ((i & 1) == 0 && i < 2 * kPolyPairs) {
-            exp2_poly2(t0, t1, p0, p1);  // FMA pipe
-          } else {
-            p0 = fast_exp2(t0);  // MUFU
-            p1 = fast_exp2(t1);
-          }
+          fma2(t0, t1, s[32 * c + 2 * i], s[32 * c + 2 * i + 1], sl2, sl2, neg, neg);
+          p0 = fast_exp2(t0);
+          p1 = fast_exp2(t1);
           const __half2 h = __floats2half2_rn(p0, p1);
-          ph[i] = *reinterpret_cast<const uint32_t*>(&h);
-          if constexpr (!Cfg<D>::kSumOnTC) {
-            // the row sum uses the fp16-rounded weights the MMA sees
-            const float2 r = __half22float2(h);
-            add2(lx, ly, lx, ly, r.x, r.y);
-          }
+          ph[c][i] = *reinterpret_cast<const uint32_t*>(&h);
+          // the row sum uses the fp16-rounded weights the MMA sees
+          add_f16x2_to_f32(lx, ly, ph[c][i]);
         }
-        // P column c (fp16 pair) holds keys 2c, 2c+1
-        tmem_st16(t_s + 32 * half + 16 * q2, ph);
-        tmem_wait_st();  // ph is rewritten by the next quarter
       }
-      if constexpr (!Cfg<D>::kSumOnTC) l += lx + ly;
+      if constexpr (C::kSepP) {
+        // P_t and O_t are free once the previous P.V of this member is done
+        // (waited for only now, so that P.V overlaps the exponentials)
+        if (g > 0) {
+          if (!(ok = wait_bar(&B.o_done[t], (g - 1) & 1, abort_flag, a.status))) break;
+          tc_fence_after();
+        }
+      }
+      // (separate-P layout off: S_t full implies every earlier P.V of this
+      // member has completed)
+      // P column 16 c + i (fp16 pair) holds keys 32 c + 2 i, 32 c + 2 i + 1
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_st16(t_p + 16 * c, ph[c]);
+      if (rescale) {
+        uint32_t r[32];
+#pragma unroll
+        for (int ch = 0; ch < D / 32; ++ch) {
+          tmem_ld32(t_o + ch * 32, r);
+          tmem_wait_ld();
+          reg_fence32(r);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+          tmem_st32(t_o + ch * 32, r);
+        }
+      }
+      l = l * alpha + (lx + ly);
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&B.p_ready[sb]);
+      if (lane == 0) mbar_arrive(&B.p_ready[t]);
       first = false;
       ++g;
     }
     if (!ok) break;
     // -------------------------------------------------------------- epilogue
     const bool empty = first;
-    float ltot = 0.f;
+    float inv = 0.f;
     if (!empty) {
-      if (!(ok = wait_bar(&B.o_done[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_flag, a.status)))
-        break;
+      if (!(ok = wait_bar(&B.o_done[t], (g - 1) & 1, abort_flag, a.status))) break;
       tc_fence_after();
-      if constexpr (Cfg<D>::kSumOnTC) {
-        uint32_t r1 = tmem_ld1(t_sum);
-        tmem_wait_ld();
-        reg_fence1(r1);
-        ltot = __uint_as_float(r1);
-      } else {
-        red_sum[half * 128 + row] = l;
-        named_bar_sync(kBarSum, 256);
-        ltot = l + red_sum[(half ^ 1) * 128 + row];
-      }
+      inv = l > 0.f ? 1.f / l : 0.f;
     }
-    const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
     const int n = qt * 128 + row;
-    __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.o) +
-                          (static_cast<long long>(bh) * N + n) * D + half * (D / 2);
+    __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.o) + (static_cast<long long>(bh) * N + n) * D;
 #pragma unroll
-    for (int ch = 0; ch < D / 64; ++ch) {
-      uint32_t r[32];
+    for (int ch = 0; ch < D / 32; ch += 2) {
+      uint32_t r[2][32];
       if (!empty) {
-        tmem_ld32(t_o + ch * 32, r);
+        tmem_ld32(t_o + ch * 32, r[0]);
+        tmem_ld32(t_o + ch * 32 + 32, r[1]);
         tmem_wait_ld();
-        reg_fence32(r);
+        reg_fence32(r[0]);
+        reg_fence32(r[1]);
       } else {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) r[i] = 0u;
+        for (int i = 0; i < 32; ++i) r[0][i] = r[1][i] = 0u;
       }
       if (n < N) {
 #pragma unroll
-        for (int c16 = 0; c16 < 4; ++c16) {
-          uint4 v;
-          v.x = pack_bf16x2(__uint_as_float(r[8 * c16 + 0]) * inv,
-                            __uint_as_float(r[8 * c16 + 1]) * inv);
-          v.y = pack_bf16x2(__uint_as_float(r[8 * c16 + 2]) * inv,
-                            __uint_as_float(r[8 * c16 + 3]) * inv);
-          v.z = pack_bf16x2(__uint_as_float(r[8 * c16 + 4]) * inv,
-                            __uint_as_float(r[8 * c16 + 5]) * inv);
-          v.w = pack_bf16x2(__uint_as_float(r[8 * c16 + 6]) * inv,
-                            __uint_as_float(r[8 * c16 + 7]) * inv);
-          *reinterpret_cast<uint4*>(orow + ch * 32 + c16 * 8) = v;
-        }
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int c16 = 0; c16 < 4; ++c16) {
+            const uint32_t* x = &r[h][8 * c16];
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(x[0]) * inv, __uint_as_float(x[1]) * inv);
+            v.y = pack_bf16x2(__uint_as_float(x[2]) * inv, __uint_as_float(x[3]) * inv);
+            v.z = pack_bf16x2(__uint_as_float(x[4]) * inv, __uint_as_float(x[5]) * inv);
+            v.w = pack_bf16x2(__uint_as_float(x[6]) * inv, __uint_as_float(x[7]) * inv);
+            *reinterpret_cast<uint4*>(orow + (ch + h) * 32 + c16 * 8) = v;
+          }
       }
     }
-    if (!empty) {
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(B.o_free);
-    }
+    // the next item's first P.V (accumulate off) is issued after this
+    // member's next p_ready, which follows these TMEM reads in program order
   }
 }
 
@@ -349,43 +370,48 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_sm100_kernel(const __grid_constant__ Maps maps, const AttnArgs a) {
   using C = Cfg<D>;
+  constexpr int QD = C::kQDepth, S = C::kSlots;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* bar_base = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   Bars B;
   B.q_full = bar_base;
-  B.q_empty = bar_base + 2;
-  B.kv_full = bar_base + 4;
-  B.kv_empty = B.kv_full + C::kSlots;
-  B.v_ready = B.kv_empty + C::kSlots;
-  B.s_full = B.v_ready + C::kSlots;
-  B.p_ready = B.s_full + 2;
+  B.q_empty = B.q_full + 2 * QD;
+  B.kv_full = B.q_empty + 2 * QD;
+  B.kv_empty = B.kv_full + S;
+  B.v_ready = B.kv_empty + S;
+  B.s_full = B.v_ready + S;
+  B.s_free = B.s_full + 2;
+  B.p_ready = B.s_free + 2;
   B.o_done = B.p_ready + 2;
-  B.o_free = B.o_done + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(B.o_free + 1);
+  B.drain = B.o_done + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(B.drain + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* red_max = reinterpret_cast<float*>(smem + C::kOffRed);  // [S buffer][half][row]
-  float* red_sum = red_max + 4 * 128;                             // [half][row]
+  volatile uint32_t* step_info = reinterpret_cast<volatile uint32_t*>(smem + C::kOffInfo);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int N = a.N, nb = n_tiles(N);
-  const int n_items = a.B * a.H * nb;
+  const int n_pairs = (nb + 1) / 2;
+  const int n_items = a.B * a.H * n_pairs;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 2 * QD; ++i) {
       mbar_init(&B.q_full[i], 1);
       mbar_init(&B.q_empty[i], 1);
-      mbar_init(&B.s_full[i], 1);
-      mbar_init(&B.p_ready[i], 8);
-      mbar_init(&B.o_done[i], 1);
     }
-    for (int i = 0; i < C::kSlots; ++i) {
+    for (int i = 0; i < S; ++i) {
       mbar_init(&B.kv_full[i], 1);
-      mbar_init(&B.kv_empty[i], 1);
-      mbar_init(&B.v_ready[i], 2);
+      mbar_init(&B.kv_empty[i], 2);
+      mbar_init(&B.v_ready[i], 1);
     }
-    mbar_init(B.o_free, 8);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&B.s_full[t], 1);
+      mbar_init(&B.s_free[t], 4);
+      mbar_init(&B.p_ready[t], 4);
+      mbar_init(&B.o_done[t], 1);
+      mbar_init(&B.drain[t], 1);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -398,173 +424,193 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
-  if (C::kSumOnTC && (warp == 2 || warp == 3)) {
-    // 128 rows x 64 fp16 columns, swizzled like a V box: column 0 = 1.0
-    uint4* ones = reinterpret_cast<uint4*>(smem + C::kOffOnes);
-    for (int r = threadIdx.x - 64; r < 128; r += 64)
-#pragma unroll
-      for (int cc = 0; cc < 8; ++cc)
-        ones[r * 8 + cc] = make_uint4(cc == (r & 7) ? 0x3C00u : 0u, 0u, 0u, 0u);
-    fence_proxy_async_smem();
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tmem_s0 = tmem, tmem_o = tmem + 256;
 
   if (warp == 0) {
+    reg_dealloc<C::kRegsLow>();
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      uint32_t L = 0, c = 0;
+      uint32_t L = 0, cq[2] = {0, 0};
       bool ok = true;
+      // waits until the K and V entries of the step at ring index L are free
+      auto claim = [&]() -> bool {
+        return wait_bar(&B.kv_empty[L % S], ((L / S) & 1) ^ 1, abort_flag, a.status) &&
+               wait_bar(&B.kv_empty[(L + 1) % S], (((L + 1) / S) & 1) ^ 1, abort_flag, a.status);
+      };
       for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
-        const int bh = item / nb, qt = item - bh * nb;
-        int beg, end;
-        item_list(a, bh, qt, beg, end, true);
-        int first = beg;
-        while (first < end && !valid_tile(a.indices[first], nb)) {
-          set_status(a.status, SVG_DEVICE_BAD_INDEX);
-          ++first;
+        const int bh = item / n_pairs, qt0 = 2 * (item - bh * n_pairs);
+        int p[2], e[2];
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          member_list(a, bh, qt0 + t, nb, p[t], e[t], true);
+          skip_invalid(a, nb, p[t], e[t], true);
         }
-        if (first == end) continue;
-        const int qb = c & 1;
-        if (!(ok = wait_bar(&B.q_empty[qb], ((c >> 1) & 1) ^ 1, abort_flag, a.status))) break;
-        mbar_arrive_expect_tx(&B.q_full[qb], C::kTile);
-        for (int bx = 0; bx < C::kBoxes; ++bx)
-          tma_load_3d(smem + C::kOffQ + qb * C::kTile + bx * kBox, &maps.q, &B.q_full[qb], 64 * bx,
-                      qt * 128, bh);
-        for (int e = first; e < end && ok; ++e) {
-          const int j = a.indices[e];
-          if (!valid_tile(j, nb)) {
-            set_status(a.status, SVG_DEVICE_BAD_INDEX);
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          if (p[t] >= e[t] || !ok) continue;
+          const uint32_t qs = cq[t] % QD;
+          if (!(ok = wait_bar(&B.q_empty[t * QD + qs], ((cq[t] / QD) & 1) ^ 1, abort_flag,
+                              a.status)))
             continue;
-          }
-          for (int t = 0; t < 2; ++t, ++L) {
-            const int slot = L % C::kSlots;
-            if (!(ok = wait_bar(&B.kv_empty[slot], ((L / C::kSlots) & 1) ^ 1, abort_flag,
-                                a.status)))
-              break;
+          mbar_arrive_expect_tx(&B.q_full[t * QD + qs], C::kTile);
+          for (int bx = 0; bx < C::kBoxes; ++bx)
+            tma_load_3d(smem + C::kOffQ + (t * QD + qs) * C::kTile + bx * kBox, &maps.q,
+                        &B.q_full[t * QD + qs], 64 * bx, (qt0 + t) * 128, bh);
+          ++cq[t];
+        }
+        uint32_t seen = 0;  // members that already had a block in this item
+        int j, mask;
+        while (ok && merge_next(a, nb, p, e, j, mask)) {
+          const uint32_t m = static_cast<uint32_t>(mask);
+          const uint32_t last = (m & 1u) * (p[0] >= e[0] ? 1u : 0u) |
+                                (m & 2u) * (p[1] >= e[1] ? 1u : 0u);
+          const uint32_t info = m | ((m & ~seen) << 2) | (last << 4);
+          seen |= m;
+          if (!(ok = claim())) break;
+          step_info[(L / 2) % C::kSteps] = info;  // released by the arrives below
+          for (int kv = 0; kv < 2; ++kv, ++L) {
+            const uint32_t slot = L % S;
             mbar_arrive_expect_tx(&B.kv_full[slot], C::kTile);
-            const CUtensorMap* m = t == 0 ? &maps.k : &maps.v;
+            const CUtensorMap* map = kv == 0 ? &maps.k : &maps.v;
             for (int bx = 0; bx < C::kBoxes; ++bx)
-              tma_load_3d(smem + C::kOffKV + slot * C::kTile + bx * kBox, m, &B.kv_full[slot],
+              tma_load_3d(smem + C::kOffKV + slot * C::kTile + bx * kBox, map, &B.kv_full[slot],
                           64 * bx, j * 128, bh);
           }
         }
-        ++c;
+      }
+      // end record in the next step's entries; plain arrives complete their
+      // phases
+      if (ok && (ok = claim())) {
+        step_info[(L / 2) % C::kSteps] = kStepEnd;
+        mbar_arrive(&B.kv_full[L % S]);
+        mbar_arrive(&B.kv_full[(L + 1) % S]);
+      }
+      if (!ok) {
+        // let the copies already issued land before the CTA can exit
+        for (uint32_t l = L > S ? L - S : 0; l < L; ++l) drain_bar(&B.kv_full[l % S], (l / S) & 1);
+        for (int t = 0; t < 2; ++t)
+          for (uint32_t c = cq[t] > QD ? cq[t] - QD : 0; c < cq[t]; ++c)
+            drain_bar(&B.q_full[t * QD + c % QD], (c / QD) & 1);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == 2) {
+    reg_dealloc<C::kRegsLow>();
+    // ------------------------------------------------------------ MMA issuers
     if (lane == 0) {
-      uint32_t L = 0, g = 0, c = 0;
-      bool ok = true;
-      auto issue_pv = [&](uint32_t gp, uint32_t lv, bool first_of_item) -> bool {
-        const int sb = gp & 1;
-        if (!wait_bar(&B.p_ready[sb], (gp >> 1) & 1, abort_flag, a.status)) return false;
-        if (first_of_item && c > 0 && !wait_bar(B.o_free, (c - 1) & 1, abort_flag, a.status))
-          return false;
-        const int slot = lv % C::kSlots;
-        if (!wait_bar(&B.v_ready[slot], (lv / C::kSlots) & 1, abort_flag, a.status)) return false;
+      const int t = warp - 1;  // member
+      const uint32_t t_s = tmem + C::kColS + 128 * t;
+      const uint32_t t_p = tmem + C::kColP + C::kPStride * t;
+      const uint32_t t_o = tmem + C::kColO + C::kOStride * t;
+      // descriptors of the first Q buffer and of ring entry 0; a buffer at
+      // byte offset x adds x >> 4 (the start-address field)
+      const uint64_t dq = sdesc_sw128(smem_u32(smem + C::kOffQ + t * QD * C::kTile), 16, 1024);
+      const uint64_t dk = sdesc_sw128(smem_u32(smem + C::kOffKV), 16, 1024);
+      const uint64_t dv = sdesc_sw128(smem_u32(smem + C::kOffKV), kBox, 1024);
+      uint32_t L = 0, cq = 0, nq = 0, np = 0;
+      bool ok = true, pend = false, pend_first = false;
+      uint32_t pend_lv = 0;
+      auto issue_pv = [&]() -> bool {
+        if (!wait_bar(&B.p_ready[t], np & 1, abort_flag, a.status)) return false;
+        const uint32_t slot = pend_lv % S;
+        if (!wait_bar(&B.v_ready[slot], (pend_lv / S) & 1, abort_flag, a.status)) return false;
         tc_fence_after();
-        const uint32_t vbase = smem_u32(smem + C::kOffKV + slot * C::kTile);
-        // second 64-column atom of B: V columns 64.. (d = 128) or the ones
-        // column that accumulates the row sums (d = 64)
-        const uint32_t lbo = C::kSumOnTC ? smem_u32(smem + C::kOffOnes) - vbase : kBox;
-        // O (+)= P V, P (fp16) in S columns [0, 64), V converted to fp16
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem_o, tmem_s0 + sb * 128 + kk * 8, sdesc_sw128(vbase + kk * 2048, lbo, 1024),
-                 C::kIdescPV, (first_of_item && kk == 0) ? 0u : 1u);
+        const uint64_t d0 = dv + ((slot * C::kTile) >> 4);
+        mma_ts_k128(t_o, t_p, d0, C::kIdescPV, pend_first ? 0u : 1u);
+        tc_commit(&B.o_done[t]);
         tc_commit(&B.kv_empty[slot]);
-        tc_commit(&B.o_done[sb]);
+        ++np;
+        pend = false;
         return true;
       };
-      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
-        const int bh = item / nb, qt = item - bh * nb;
-        int beg, end;
-        item_list(a, bh, qt, beg, end);
-        bool any = false;
-        for (int e = beg; e < end && !any; ++e) any = valid_tile(a.indices[e], nb);
-        if (!any) continue;
-        const int qb = c & 1;
-        if (!(ok = wait_bar(&B.q_full[qb], (c >> 1) & 1, abort_flag, a.status))) break;
-        const uint32_t qbase = smem_u32(smem + C::kOffQ + qb * C::kTile);
-        bool have_pending = false, pending_first = false;
-        uint32_t pend_g = 0, pend_lv = 0;
-        bool first = true;
-        for (int e = beg; e < end && ok; ++e) {
-          if (!valid_tile(a.indices[e], nb)) continue;
-          const int slot = L % C::kSlots;
-          if (!(ok = wait_bar(&B.kv_full[slot], (L / C::kSlots) & 1, abort_flag, a.status))) break;
-          tc_fence_after();
-          const int sb = g & 1;
-          const uint32_t kbase = smem_u32(smem + C::kOffKV + slot * C::kTile);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
-            mma_ss(tmem_s0 + sb * 128, sdesc_sw128(qbase + off, 16, 1024),
-                   sdesc_sw128(kbase + off, 16, 1024), C::kIdescQK, kk > 0 ? 1u : 0u);
-          }
-          tc_commit(&B.s_full[sb]);
-          tc_commit(&B.kv_empty[slot]);
-          if (have_pending && !(ok = issue_pv(pend_g, pend_lv, pending_first))) break;
-          have_pending = true;
-          pending_first = first;
-          pend_g = g;
-          pend_lv = L + 1;
+      while (ok) {
+        const uint32_t kslot = L % S;
+        if (!(ok = wait_bar(&B.kv_full[kslot], (L / S) & 1, abort_flag, a.status))) break;
+        const uint32_t info = step_info[(L / 2) % C::kSteps];
+        if (info & kStepEnd) break;
+        if (!(info >> t & 1u)) {
+          // this member skips the block: its pending P.V goes now (otherwise
+          // that V entry could stay held past the point where the producer
+          // needs it again), then its share of both entries is released
+          if (pend && !(ok = issue_pv())) break;
+          tc_commit(&B.kv_empty[kslot]);
+          tc_commit(&B.kv_empty[kslot + 1]);
           L += 2;
-          ++g;
-          first = false;
+          continue;
         }
-        if (!ok) break;
-        tc_commit(&B.q_empty[qb]);  // Q buffer free once its last QK^T completes
-        if (!(ok = issue_pv(pend_g, pend_lv, pending_first))) break;
-        ++c;
-      }
-    }
-  } else if (warp == 2 || warp == 3) {
-    // ------------------------------------------------------------ V to fp16
-    // Converts every V tile in place, in the order the MMA issuer consumes
-    // them.  bf16 -> fp16 is exact for |v| <= 65504 (fp16 subnormals keep
-    // the absolute error below 2^-25); larger values become inf and are
-    // reported as SVG_DEVICE_RANGE.
-    const int t = threadIdx.x - 64;  // 0..63
-    uint32_t L = 0;
-    bool ok = true, range = false;
-    for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
-      const int bh = item / nb, qt = item - bh * nb;
-      int beg, end;
-      item_list(a, bh, qt, beg, end);
-      for (int e = beg; e < end && ok; ++e) {
-        if (!valid_tile(a.indices[e], nb)) continue;
-        const uint32_t lv = L + 1;
-        const int slot = lv % C::kSlots;
-        if (!(ok = wait_bar(&B.kv_full[slot], (lv / C::kSlots) & 1, abort_flag, a.status))) break;
-        uint4* tile = reinterpret_cast<uint4*>(smem + C::kOffKV + slot * C::kTile);
-#pragma unroll 4
-        for (int c = t; c < C::kTile / 16; c += 64) {
-          uint4 v = tile[c];
-          uint32_t* w = reinterpret_cast<uint32_t*>(&v);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xffff0000u);
-            range |= fabsf(lo) > 65504.f || fabsf(hi) > 65504.f;
-            const __half2 h = __floats2half2_rn(lo, hi);
-            w[i] = *reinterpret_cast<const uint32_t*>(&h);
-          }
-          tile[c] = v;
+        if constexpr (!C::kSepP) {
+          // P_t lives in S_t: the previous P.V goes first (tensor-core order)
+          if (pend && !(ok = issue_pv())) break;
+        } else if (nq > 0) {
+          if (!(ok = wait_bar(&B.s_free[t], (nq - 1) & 1, abort_flag, a.status))) break;
         }
-        fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&B.v_ready[slot]);
+        const uint32_t qs = cq % QD;
+        if (info >> (2 + t) & 1u) {  // first block of the item: a new Q tile
+          if (!(ok = wait_bar(&B.q_full[t * QD + qs], (cq / QD) & 1, abort_flag, a.status))) break;
+        }
+        tc_fence_after();
+        const uint64_t q0 = dq + ((qs * C::kTile) >> 4), k0 = dk + ((kslot * C::kTile) >> 4);
+        if constexpr (D == 64)
+          mma_ss_k64(t_s, q0, k0, C::kIdescQK);
+        else
+          mma_ss_k128(t_s, q0, k0, C::kIdescQK, kBox >> 4);
+        tc_commit(&B.s_full[t]);
+        tc_commit(&B.kv_empty[kslot]);
+        if (info >> (4 + t) & 1u) {  // last block of the item: its Q buffer is free
+          tc_commit(&B.q_empty[t * QD + qs]);
+          ++cq;
+        }
+        ++nq;
+        if constexpr (C::kSepP) {
+          if (pend && !(ok = issue_pv())) break;
+        }
+        pend = true;
+        pend_first = (info >> (2 + t)) & 1u;
+        pend_lv = L + 1;
         L += 2;
       }
+      if (ok && pend) ok = issue_pv();
+      // every MMA issued by this thread completes before TMEM is released
+      tc_commit(&B.drain[t]);
+      drain_bar(&B.drain[t], 0);
+    }
+  } else if (warp == 3) {
+    reg_dealloc<C::kRegsLow>();
+    // ------------------------------------------------------------ V to fp16
+    // Converts every V tile in place, in ring order.  bf16 -> fp16 is exact
+    // for |v| <= 65504 (fp16 subnormals keep the absolute error below
+    // 2^-25); larger values become inf and are reported as SVG_DEVICE_RANGE.
+    uint32_t L = 0;
+    bool ok = true, range = false;
+    while (ok) {
+      const uint32_t slot = (L + 1) % S;
+      if (!(ok = wait_bar(&B.kv_full[slot], ((L + 1) / S) & 1, abort_flag, a.status))) break;
+      if (step_info[(L / 2) % C::kSteps] & kStepEnd) break;
+      uint4* tile = reinterpret_cast<uint4*>(smem + C::kOffKV + slot * C::kTile);
+#pragma unroll 4
+      for (int c = lane; c < C::kTile / 16; c += 32) {
+        uint4 v = tile[c];
+        uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xffff0000u);
+          range |= fabsf(lo) > 65504.f || fabsf(hi) > 65504.f;
+          const __half2 h = __floats2half2_rn(lo, hi);
+          w[i] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+        tile[c] = v;
+      }
+      fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&B.v_ready[slot]);
+      L += 2;
     }
     if (__any_sync(0xffffffffu, range) && lane == 0) set_status(a.status, SVG_DEVICE_RANGE);
-  } else if (warp >= 4) {
-    softmax_half<D>(a, B, abort_flag, tmem, red_max, red_sum, n_items, nb);
+  } else {
+    reg_alloc<C::kRegsHigh>();
+    softmax_member<D>(a, B, abort_flag, tmem, n_items, n_pairs, nb);
   }
   tc_fence_before();
   __syncthreads();
@@ -617,7 +663,7 @@ svg_status launch_attn_sm100(const AttnArgs& a, cudaStream_t s) {
   if (cudaFuncSetAttribute(attn_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            C::kSmem) != cudaSuccess)
     return fail(SVG_ERR_CUDA, "sparse_attn: cannot reserve %d bytes of shared memory", C::kSmem);
-  const long long items = static_cast<long long>(BH) * n_tiles(a.N);
+  const long long items = static_cast<long long>(BH) * ((n_tiles(a.N) + 1) / 2);
   const int grid = static_cast<int>(items < sm_count() ? items : sm_count());
   attn_sm100_kernel<D><<<grid, kThreads, C::kSmem, s>>>(maps, a);
   return check_launch("sparse_attn sm100");

@@ -124,6 +124,78 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       : "memory");
 }
 
+// The K-steps of one tile in a single asm block, so the issuing thread
+// spends about two instructions per MMA (a 32-bit add on the descriptor's
+// start-address field and the MMA itself).  Start addresses are in 16-byte
+// units inside the low word; every buffer lies below 256 KB, so the field
+// never carries into the high word.
+//
+// S (+)= A B^T, K = 64 (four K-steps of 32 bytes inside one 128-byte
+// swizzle atom); A and B from shared memory, K-major.
+__device__ __forceinline__ void mma_ss_k64(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                           uint32_t idesc) {
+  asm volatile(
+      "{\n .reg .pred p0, p1;\n .reg .b32 al, ah, bl, bh, x, y;\n .reg .b64 da, db;\n"
+      " setp.ne.b32 p0, %4, %4;\n setp.eq.b32 p1, %4, %4;\n"
+      " mov.b64 {al, ah}, %1;\n mov.b64 {bl, bh}, %2;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p0;\n"
+      " add.u32 x, al, 2;\n add.u32 y, bl, 2;\n mov.b64 da, {x, ah};\n mov.b64 db, {y, bh};\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, p1;\n"
+      " add.u32 x, al, 4;\n add.u32 y, bl, 4;\n mov.b64 da, {x, ah};\n mov.b64 db, {y, bh};\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, p1;\n"
+      " add.u32 x, al, 6;\n add.u32 y, bl, 6;\n mov.b64 da, {x, ah};\n mov.b64 db, {y, bh};\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, p1;\n}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(0u)
+      : "memory");
+}
+// K = 128 as two 64-column atoms `atom_units` (16-byte units) apart.
+__device__ __forceinline__ void mma_ss_k128(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t atom_units) {
+  mma_ss_k64(d_tmem, adesc, bdesc, idesc);
+  asm volatile(
+      "{\n .reg .pred p1;\n .reg .b32 al, ah, bl, bh, x, y;\n .reg .b64 da, db;\n"
+      " setp.eq.b32 p1, %4, %4;\n"
+      " mov.b64 {al, ah}, %1;\n mov.b64 {bl, bh}, %2;\n"
+      " add.u32 al, al, %4;\n add.u32 bl, bl, %4;\n"
+      " mov.b64 da, {al, ah};\n mov.b64 db, {bl, bh};\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, p1;\n"
+      " add.u32 x, al, 2;\n add.u32 y, bl, 2;\n mov.b64 da, {x, ah};\n mov.b64 db, {y, bh};\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, p1;\n"
+      " add.u32 x, al, 4;\n add.u32 y, bl, 4;\n mov.b64 da, {x, ah};\n mov.b64 db, {y, bh};\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, p1;\n"
+      " add.u32 x, al, 6;\n add.u32 y, bl, 6;\n mov.b64 da, {x, ah};\n mov.b64 db, {y, bh};\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, p1;\n}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(atom_units)
+      : "memory");
+}
+// O (+)= P V over 128 keys: eight K-steps of 16 keys, P from TMEM (8
+// columns per step), V from shared memory (16 rows of 128 bytes per step,
+// MN-major).  accumulate == 0 overwrites O in the first step.
+__device__ __forceinline__ void mma_ts_k128(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p0, p1;\n .reg .b32 bl, bh, x, ta;\n .reg .b64 db;\n"
+      " setp.ne.b32 p0, %4, 0;\n setp.eq.b32 p1, %4, %4;\n"
+      " mov.b64 {bl, bh}, %2;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p0;\n"
+      " add.u32 ta, %1, 8;\n add.u32 x, bl, 128;\n mov.b64 db, {x, bh};\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, p1;\n"
+      " add.u32 ta, %1, 16;\n add.u32 x, bl, 256;\n mov.b64 db, {x, bh};\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, p1;\n"
+      " add.u32 ta, %1, 24;\n add.u32 x, bl, 384;\n mov.b64 db, {x, bh};\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, p1;\n"
+      " add.u32 ta, %1, 32;\n add.u32 x, bl, 512;\n mov.b64 db, {x, bh};\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, p1;\n"
+      " add.u32 ta, %1, 40;\n add.u32 x, bl, 640;\n mov.b64 db, {x, bh};\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, p1;\n"
+      " add.u32 ta, %1, 48;\n add.u32 x, bl, 768;\n mov.b64 db, {x, bh};\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, p1;\n"
+      " add.u32 ta, %1, 56;\n add.u32 x, bl, 896;\n mov.b64 db, {x, bh};\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, p1;\n}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Instruction descriptor, kind::f16: bf16 A and B, fp32 D, K-major A,
 // B K-major (QK^T) or MN-major (PV), shape M x N.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major) {
@@ -221,6 +293,14 @@ __device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1, f
       " add.rn.f32x2 rd, ra, rb;\n mov.b64 {%0, %1}, rd;\n}\n"
       : "=f"(d0), "=f"(d1)
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+// (acc0, acc1) += (lo, hi) of an fp16 pair, each converted exactly to fp32
+// inside the add (mixed-precision add, sm_100).
+__device__ __forceinline__ void add_f16x2_to_f32(float& acc0, float& acc1, uint32_t h2) {
+  asm("{\n .reg .f16 lo, hi;\n mov.b32 {lo, hi}, %2;\n add.rn.f32.f16 %0, lo, %0;\n"
+      " add.rn.f32.f16 %1, hi, %1;\n}\n"
+      : "+f"(acc0), "+f"(acc1)
+      : "r"(h2));
 }
 // max of three floats in one instruction.
 __device__ __forceinline__ float max3(float a, float b, float c) {
