@@ -32,12 +32,15 @@ __device__ __forceinline__ void qk_frags(float (&s)[NK / 8][4], const uint32_t (
   const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int n = 0; n < NK / 8; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
+  // K-steps outer, key groups inner: consecutive MMAs accumulate into
+  // different s[n], so they pipeline (each s[n] still sums its K-steps in
+  // order)
 #pragma unroll
-  for (int np = 0; np < NK / 16; ++np) {
-    const int r = key0 + np * 16 + (lane & 7) + ((lane >> 4) << 3);
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const int c = 2 * kk + ((lane >> 3) & 1);
 #pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const int c = 2 * kk + ((lane >> 3) & 1);
+    for (int np = 0; np < NK / 16; ++np) {
+      const int r = key0 + np * 16 + (lane & 7) + ((lane >> 4) << 3);
       uint32_t b0, b1, b2, b3;
       ldmatrix_x4(b0, b1, b2, b3, ktile + swz(r, c, 2 * D));
       const uint32_t bA[2] = {b0, b1};

@@ -9,12 +9,14 @@
 //
 // Work split (one layer, all heads, one launch each):
 //   partial  grid (chunks, B*H): the keys of a head are cut into `chunks`
-//            contiguous ranges.  A CTA streams one range through a 3-stage
-//            cp.async ring; warps 0-3 keep the dense online-softmax state
-//            (max, sum, o) of the 64 sampled rows, warps 4-7 the state under
+//            contiguous ranges.  A CTA of 4 warps streams one range through
+//            a cp.async ring (4 stages of 64 keys at d = 64, 3 at d = 128);
+//            each warp owns 16 of the 64 sampled rows and keeps two
+//            online-softmax states (max, sum, o) for them: dense and under
 //            the spatial mask (each row's band of frames is one contiguous
-//            key range, tested with two compares; stages outside a warp's
-//            bands are skipped).  bf16: mma.sync tensor-core products;
+//            key range, tested with two compares; the spatial update is
+//            skipped for stages outside the warp's bands).  Both updates
+//            share one Q K^T per stage.  bf16: mma.sync tensor-core products;
 //            fp32: SIMT (one launch per mask, grid z).
 //   merge    grid (B*H, 16), one warp per sampled row: the chunk weights
 //            exp2(m_c - M) / L, the merged dense and spatial outputs, the
@@ -33,9 +35,8 @@ namespace {
 
 constexpr int kRows = 64;          // sampled rows per head (S padded to 64)
 constexpr int kKeys = 64;          // keys per shared-memory stage
-constexpr int kStages = 3;         // cp.async ring depth
-constexpr int kThreads = 256;      // 8 warps: 4 dense + 4 spatial, 16 rows each
-constexpr int kTargetCtas = 592;   // partial-grid size the chunking aims for (4 x 148)
+constexpr int kThreads = 128;      // bf16 partial: 4 warps, 16 rows each
+constexpr int kTargetCtas = 888;   // partial-grid size the chunking aims for (6 x 148)
 constexpr int kMaxChunks = 32;     // merge holds one chunk weight per lane
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -87,22 +88,99 @@ size_t partial_bytes(int B, int H, int N, int d) {
 // --------------------------------------------------------------- bf16 partial
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) profile_partial_bf16(
+constexpr int stages_for() {
+  return D == 64 ? 4 : 3;  // cp.async ring depth (shared memory: 3 or 2 CTAs per SM)
+}
+template <int D>
+constexpr size_t partial_smem() {
+  return static_cast<size_t>(kRows) * D * 2 + 2 * static_cast<size_t>(stages_for<D>()) * kKeys * D * 2;
+}
+
+// One stage's online-softmax update of a warp's 16 rows: s holds the scores
+// (scale * log2 e applied below), keys outside [lo[h], hi[h]) are masked for
+// the thread's row h; P is rounded to bf16 and the row sum adds the rounded
+// values.
+template <int D>
+__device__ __forceinline__ void stage_update(float (&m)[2], float (&l)[2], float (&o)[D / 8][4],
+                                             float (&s)[kKeys / 8][4], const int (&lo)[2],
+                                             const int (&hi)[2], int key0, float scale_log2,
+                                             uint32_t vtile) {
+  const int t4 = threadIdx.x & 3;
+  float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+  for (int n = 0; n < kKeys / 8; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int key = key0 + 8 * n + 2 * t4 + (e & 1);
+      const int h = e >> 1;
+      s[n][e] = (key >= lo[h] && key < hi[h]) ? s[n][e] * scale_log2 : -INFINITY;
+      mx[h] = fmaxf(mx[h], s[n][e]);
+    }
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
+    mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
+    const float mn = fmaxf(m[h], mx[h]);
+    const float base = mn == -INFINITY ? 0.f : mn;
+    const float alpha = fast_exp2(m[h] - base);  // exp2(-inf) = 0 on the first update
+    m[h] = mn;
+    l[h] *= alpha;
+#pragma unroll
+    for (int n = 0; n < D / 8; ++n) {
+      o[n][2 * h] *= alpha;
+      o[n][2 * h + 1] *= alpha;
+    }
+#pragma unroll
+    for (int n = 0; n < kKeys / 8; ++n) {
+      s[n][2 * h] = round_bf16(fast_exp2(s[n][2 * h] - base));
+      s[n][2 * h + 1] = round_bf16(fast_exp2(s[n][2 * h + 1] - base));
+      l[h] += s[n][2 * h] + s[n][2 * h + 1];
+    }
+  }
+  pv_frags<D, kKeys>(o, s, vtile, 0);
+}
+
+template <int D>
+__device__ __forceinline__ void store_state(float* base, int row0, const float (&m)[2],
+                                            float (&l)[2], const float (&o)[D / 8][4]) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t4 = lane & 3;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    l[h] += __shfl_xor_sync(0xffffffffu, l[h], 1);
+    l[h] += __shfl_xor_sync(0xffffffffu, l[h], 2);
+  }
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    float* row = base + (row0 + g + 8 * h) * state_floats<D>();
+    if (t4 == 0) {
+      row[0] = m[h];
+      row[1] = l[h];
+    }
+#pragma unroll
+    for (int n = 0; n < D / 8; ++n) {
+      row[2 + 8 * n + 2 * t4] = o[n][2 * h];
+      row[2 + 8 * n + 2 * t4 + 1] = o[n][2 * h + 1];
+    }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, D == 64 ? 3 : 2) profile_partial_bf16(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
     const __nv_bfloat16* __restrict__ v, const int32_t* __restrict__ idx, int S, int N, int P,
     int width, float scale_log2, int chunks, int chunk_len, float* __restrict__ ws) {
-  extern __shared__ __align__(128) unsigned char smem[];
+  constexpr int ST = stages_for<D>();
   constexpr int TILE = kKeys * D * 2;  // bytes of one K or V stage
+  extern __shared__ __align__(128) unsigned char smem[];
   unsigned char* sQ = smem;
   unsigned char* sK = smem + kRows * D * 2;
-  unsigned char* sV = sK + kStages * TILE;
+  unsigned char* sV = sK + ST * TILE;
 
   const int chunk = blockIdx.x, bh = blockIdx.y;
   const long long head = static_cast<long long>(bh) * N * D;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int variant = warp >> 2;  // 0 dense, 1 spatial
-  const int row0 = (warp & 3) * 16;
-  const int g = lane >> 2, t4 = lane & 3;
+  const int row0 = warp * 16;
+  const int g = lane >> 2;
   const int key_begin = chunk * chunk_len;
   const int key_end = min(N, key_begin + chunk_len);
   const int n_stages = (key_end - key_begin + kKeys - 1) / kKeys;
@@ -114,23 +192,24 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) profile_partial_bf1
     const int n = ok ? clamp_index(idx[r], N) : 0;
     cp_async16(sQ + swz(r, c, 2 * D), q + head + static_cast<long long>(n) * D + c * 8, ok);
   }
-  // the keys each of this thread's two rows may see, clipped to the chunk
-  int lo[2], hi[2];
+  // the keys each of this thread's two rows may see, clipped to the chunk:
+  // every key of the chunk (dense) and the row's band of frames (spatial)
+  int dlo[2], dhi[2], slo[2], shi[2];
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const int r = row0 + g + 8 * h;
-    lo[h] = key_begin;
-    hi[h] = key_end;
+    dlo[h] = slo[h] = key_begin;
+    dhi[h] = shi[h] = key_end;
     if (r >= S) {
-      hi[h] = lo[h];  // padding row: no keys
-    } else if (variant == 1) {
+      dhi[h] = shi[h] = key_begin;  // padding row: no keys
+    } else {
       const int f = clamp_index(idx[r], N) / P;
-      lo[h] = max(key_begin, max(0, f - width) * P);
-      hi[h] = min(key_end, static_cast<int>(min(static_cast<long long>(N),
-                                                static_cast<long long>(f + width + 1) * P)));
+      slo[h] = max(key_begin, max(0, f - width) * P);
+      shi[h] = min(key_end, static_cast<int>(min(static_cast<long long>(N),
+                                                 static_cast<long long>(f + width + 1) * P)));
     }
   }
-  int wlo = min(lo[0], lo[1]), whi = max(hi[0], hi[1]);
+  int wlo = min(slo[0], slo[1]), whi = max(shi[0], shi[1]);
 #pragma unroll
   for (int o2 = 4; o2 < 32; o2 <<= 1) {
     wlo = min(wlo, __shfl_xor_sync(0xffffffffu, wlo, o2));
@@ -138,7 +217,7 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) profile_partial_bf1
   }
 
 #pragma unroll
-  for (int st = 0; st < kStages - 1; ++st) {
+  for (int st = 0; st < ST - 1; ++st) {
     if (st < n_stages) {
       load_tile_async<D, kKeys, kThreads>(sK + st * TILE, k + head, key_begin + st * kKeys, key_end);
       load_tile_async<D, kKeys, kThreads>(sV + st * TILE, v + head, key_begin + st * kKeys, key_end);
@@ -146,19 +225,22 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) profile_partial_bf1
     cp_async_commit();
   }
 
-  float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
-  float o[D / 8][4];
+  float md[2] = {-INFINITY, -INFINITY}, ld[2] = {0.f, 0.f};
+  float ms[2] = {-INFINITY, -INFINITY}, ls[2] = {0.f, 0.f};
+  float od[D / 8][4], os[D / 8][4];
 #pragma unroll
-  for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+  for (int n = 0; n < D / 8; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) od[n][e] = os[n][e] = 0.f;
   uint32_t qa[D / 16][4];
 
   for (int st = 0; st < n_stages; ++st) {
-    cp_async_wait<kStages - 2>();
+    cp_async_wait<ST - 2>();
     __syncthreads();  // stage st landed; the buffer refilled below is free
     {
-      const int ns = st + kStages - 1;
+      const int ns = st + ST - 1;
       if (ns < n_stages) {
-        const int b = ns % kStages;
+        const int b = ns % ST;
         load_tile_async<D, kKeys, kThreads>(sK + b * TILE, k + head, key_begin + ns * kKeys, key_end);
         load_tile_async<D, kKeys, kThreads>(sV + b * TILE, v + head, key_begin + ns * kKeys, key_end);
       }
@@ -166,66 +248,25 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) profile_partial_bf1
     }
     if (st == 0) load_a_frags<D>(qa, smem_u32(sQ), row0);
     const int key0 = key_begin + st * kKeys;
-    if (key0 >= whi || key0 + kKeys <= wlo) continue;  // no row of this warp sees the stage
-    const int b = st % kStages;
+    const int b = st % ST;
     float s[kKeys / 8][4];
     qk_frags<D, kKeys>(s, qa, smem_u32(sK + b * TILE), 0);
-    float mx[2] = {-INFINITY, -INFINITY};
+    if (key0 < whi && key0 + kKeys > wlo) {  // some row of this warp has band keys here
+      float sp[kKeys / 8][4];
 #pragma unroll
-    for (int n = 0; n < kKeys / 8; ++n)
+      for (int n = 0; n < kKeys / 8; ++n)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int key = key0 + 8 * n + 2 * t4 + (e & 1);
-        const int h = e >> 1;
-        s[n][e] = (key >= lo[h] && key < hi[h]) ? s[n][e] * scale_log2 : -INFINITY;
-        mx[h] = fmaxf(mx[h], s[n][e]);
-      }
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
-      mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
-      const float mn = fmaxf(m[h], mx[h]);
-      const float base = mn == -INFINITY ? 0.f : mn;
-      const float alpha = fast_exp2(m[h] - base);  // exp2(-inf) = 0 on the first stage
-      m[h] = mn;
-      l[h] *= alpha;
-#pragma unroll
-      for (int n = 0; n < D / 8; ++n) {
-        o[n][2 * h] *= alpha;
-        o[n][2 * h + 1] *= alpha;
-      }
-#pragma unroll
-      for (int n = 0; n < kKeys / 8; ++n) {
-        s[n][2 * h] = round_bf16(fast_exp2(s[n][2 * h] - base));
-        s[n][2 * h + 1] = round_bf16(fast_exp2(s[n][2 * h + 1] - base));
-        l[h] += s[n][2 * h] + s[n][2 * h + 1];
-      }
+        for (int e = 0; e < 4; ++e) sp[n][e] = s[n][e];
+      stage_update<D>(ms, ls, os, sp, slo, shi, key0, scale_log2, smem_u32(sV + b * TILE));
     }
-    pv_frags<D, kKeys>(o, s, smem_u32(sV + b * TILE), 0);
+    stage_update<D>(md, ld, od, s, dlo, dhi, key0, scale_log2, smem_u32(sV + b * TILE));
   }
 
-  // per-row partial state -> workspace [bh][variant][chunk][row][m, l, o[D]]
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    l[h] += __shfl_xor_sync(0xffffffffu, l[h], 1);
-    l[h] += __shfl_xor_sync(0xffffffffu, l[h], 2);
-  }
-  float* base = ws + ((static_cast<long long>(bh) * 2 + variant) * chunks + chunk) * kRows *
-                         state_floats<D>();
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int r = row0 + g + 8 * h;
-    float* row = base + r * state_floats<D>();
-    if (t4 == 0) {
-      row[0] = m[h];
-      row[1] = l[h];
-    }
-#pragma unroll
-    for (int n = 0; n < D / 8; ++n) {
-      row[2 + 8 * n + 2 * t4] = o[n][2 * h];
-      row[2 + 8 * n + 2 * t4 + 1] = o[n][2 * h + 1];
-    }
-  }
+  // per-row partial states -> workspace [bh][variant][chunk][row][m, l, o[D]]
+  const long long stride = static_cast<long long>(chunks) * kRows * state_floats<D>();
+  float* base = ws + (static_cast<long long>(bh) * 2 * chunks + chunk) * kRows * state_floats<D>();
+  store_state<D>(base, row0, md, ld, od);
+  store_state<D>(base + stride, row0, ms, ls, os);
 }
 
 // --------------------------------------------------------------- fp32 partial
@@ -297,7 +338,8 @@ __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) {
   return __bfloat162float(x);
 }
 
-constexpr int kMergeRows = 4;  // sampled rows per merge CTA (one warp each)
+constexpr int kMergeRows = 4;      // sampled rows per merge CTA (one warp each)
+constexpr int kTemporalBatch = 8;  // temporal keys whose loads are in flight together
 
 // Merges the chunk states of one sampled row (one warp per row), computes the
 // row's temporal output directly and writes the row's squared errors.
@@ -351,21 +393,37 @@ __global__ void __launch_bounds__(32 * kMergeRows) profile_merge(
     qv[e] = to_f(q[head + static_cast<long long>(n) * D + lane + 32 * e]);
     acc[e] = 0.f;
   }
-  for (int f = 0; f < F; ++f) {
-    const long long j = static_cast<long long>(f) * P + sp;
-    float dot = 0.f;
+  // keys in groups of kTemporalBatch: all their K and V loads are issued
+  // before any of them is used, so the group costs one memory latency
+  for (int f0 = 0; f0 < F; f0 += kTemporalBatch) {
+    float kx[kTemporalBatch][E], vx[kTemporalBatch][E];
 #pragma unroll
-    for (int e = 0; e < E; ++e) dot = fmaf(qv[e], to_f(k[head + j * D + lane + 32 * e]), dot);
+    for (int b = 0; b < kTemporalBatch; ++b) {
+      const int f = min(f0 + b, F - 1);
+      const long long j = static_cast<long long>(f) * P + sp;
 #pragma unroll
-    for (int o2 = 16; o2 > 0; o2 >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o2);
-    const float t = dot * scale_log2;
-    const float mn = fmaxf(m, t);
-    const float alpha = exp2f(m - mn);
-    const float p = exp2f(t - mn);
-    l = l * alpha + p;
+      for (int e = 0; e < E; ++e) {
+        kx[b][e] = to_f(k[head + j * D + lane + 32 * e]);
+        vx[b][e] = to_f(v[head + j * D + lane + 32 * e]);
+      }
+    }
 #pragma unroll
-    for (int e = 0; e < E; ++e) acc[e] = fmaf(p, to_f(v[head + j * D + lane + 32 * e]), acc[e] * alpha);
-    m = mn;
+    for (int b = 0; b < kTemporalBatch; ++b) {
+      if (f0 + b >= F) break;
+      float dot = 0.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) dot = fmaf(qv[e], kx[b][e], dot);
+#pragma unroll
+      for (int o2 = 16; o2 > 0; o2 >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o2);
+      const float t = dot * scale_log2;
+      const float mn = fmaxf(m, t);
+      const float alpha = exp2f(m - mn);
+      const float p = exp2f(t - mn);
+      l = l * alpha + p;
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[e] = fmaf(p, vx[b][e], acc[e] * alpha);
+      m = mn;
+    }
   }
   float es = 0.f, et = 0.f;
 #pragma unroll
@@ -427,8 +485,7 @@ svg_status launch_profile_shaped(const void* q, const void* k, const void* v, in
   const float scale_log2 = kLog2e / sqrtf(static_cast<float>(D));
   float* errs = ws + states_bytes(B, H, ps.chunks, D) / sizeof(float);
   if (dtype == SVG_BF16) {
-    const size_t smem =
-        static_cast<size_t>(kRows) * D * 2 + 2 * kStages * static_cast<size_t>(kKeys) * D * 2;
+    const size_t smem = partial_smem<D>();
     if (cudaFuncSetAttribute(profile_partial_bf16<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
       return fail(SVG_ERR_CUDA, "%s: cannot reserve shared memory", who);
