@@ -1,8 +1,11 @@
 """Benchmark of one sparse spatial/temporal attention layer on B200.
 
 A step is one pass of the whole hot path over one layer's inputs:
-    profile heads -> permute q, k, v (temporal heads) -> block-sparse attention
-    -> permute the output back.
+    profile heads -> permute q, k, v of temporal heads to token-major ->
+    block-sparse attention that writes its output back frame-major
+    (svg_sparse_attn_fused with the output side of the reordering fused).
+The permutation kernel is also timed on its own beside the step, and the
+unfused layer (permute -> attention -> permute back) for comparison.
 Workload (default): the CogVideoX-shaped layer, B=1 H=48 N=17550 (13 frames x
 30x45 tokens) d=64 bf16, synthetic biased-Gaussian q/k/v, 64 sampled queries.
 
@@ -215,10 +218,10 @@ def run_ours(args, rank, world, local_rank):
     clocks = ClockSampler(local_rank)
     clocks.start()
     time.sleep(0.3)
-    ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(5)) for _ in range(K)]
+    ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(4)) for _ in range(K)]
     for i in range(K):
         flush.fill_(i & 0xff)
-        s0, p0, a0, a1, s1 = ev[i]
+        s0, p0, a0, s1 = ev[i]
         s0.record(stream)
         svg.svg_profile_heads(qd, kd, vd, F, P, w, idx_d, mse_out=bufs.mse, mode_out=bufs.mode,
                               workspace=bufs.ws)
@@ -226,23 +229,49 @@ def run_ours(args, rank, world, local_rank):
         for x, y in ((qd, bufs.qp), (kd, bufs.kp), (vd, bufs.vp)):
             svg.svg_permute_token_major(x, F, P, bufs.mode, out=y)
         a0.record(stream)
-        svg.svg_sparse_attn(bufs.qp, bufs.kp, bufs.vp, bufs.mode, lists, out=bufs.op)
-        a1.record(stream)
-        svg.svg_permute_frame_major(bufs.op, F, P, bufs.mode, out=bufs.o)
+        svg.svg_sparse_attn_fused(bufs.qp, bufs.kp, bufs.vp, F, P, bufs.mode, lists,
+                                  layout=svg._lib.SVG_FUSE_OUTPUT, out=bufs.o)
         s1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     clk = clocks.stop()
-    step_ms = [e[0].elapsed_time(e[4]) for e in ev]
+    step_ms = [e[0].elapsed_time(e[3]) for e in ev]
     attn_ms = [e[2].elapsed_time(e[3]) for e in ev]
     prof_ms = [e[0].elapsed_time(e[1]) for e in ev]
-    perm_ms = [e[1].elapsed_time(e[2]) + e[3].elapsed_time(e[4]) for e in ev]
+    fwd_perm_ms = [e[1].elapsed_time(e[2]) for e in ev]
     total_ms = float(sum(step_ms))
     attn_avg = float(sum(attn_ms) / K)
     prof_avg = float(sum(prof_ms) / K)
-    perm_avg = float(sum(perm_ms) / K)
+    fwd_perm_avg = float(sum(fwd_perm_ms) / K)
+
+    # the permutation kernels on their own (one token-major pass of q over
+    # every head, L2 flushed before each) and the unfused layer
+    tmp = [torch.empty_like(qd) for _ in range(4)]
+    perm_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(K)]
+    unf_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(K)]
+    for i in range(K):
+        flush.fill_(i & 0xff)
+        perm_ev[i][0].record(stream)
+        svg.svg_permute_token_major(qd, F, P, None, out=tmp[0])
+        perm_ev[i][1].record(stream)
+    for i in range(K):
+        flush.fill_(i & 0xff)
+        unf_ev[i][0].record(stream)
+        svg.svg_profile_heads(qd, kd, vd, F, P, w, idx_d, mse_out=bufs.mse, mode_out=bufs.mode,
+                              workspace=bufs.ws)
+        for x, y in zip((qd, kd, vd), tmp):
+            svg.svg_permute_token_major(x, F, P, bufs.mode, out=y)
+        svg.svg_sparse_attn(tmp[0], tmp[1], tmp[2], bufs.mode, lists, out=tmp[3])
+        svg.svg_permute_frame_major(tmp[3], F, P, bufs.mode, out=bufs.o)
+        unf_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    perm_avg = float(sum(e[0].elapsed_time(e[1]) for e in perm_ev) / K)
+    unf_avg = float(sum(e[0].elapsed_time(e[1]) for e in unf_ev) / K)
+    del tmp
 
     # end to end through the public API with host buffers
     out_host = torch.empty(qd.shape, dtype=torch.bfloat16).pin_memory()
@@ -268,8 +297,8 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
 
-    total_ms, e2e_ms, attn_avg, prof_avg, perm_avg = max_over_ranks(
-        [total_ms, e2e_ms, attn_avg, prof_avg, perm_avg], world, dev)
+    total_ms, e2e_ms, attn_avg, prof_avg, perm_avg, unf_avg, fwd_perm_avg = max_over_ranks(
+        [total_ms, e2e_ms, attn_avg, prof_avg, perm_avg, unf_avg, fwd_perm_avg], world, dev)
     if rank != 0:
         return None
 
@@ -280,12 +309,12 @@ def run_ours(args, rank, world, local_rank):
     attn_tf = flops / (attn_avg * 1e-3) / 1e12
     hbm_gbs = float(peaks["hbm_gbs"])
     elems = wl.B * wl.H * N * d
-    perm_bytes = 4 * 2 * elems * 2
+    perm_bytes = 2 * elems * 2      # one tensor read and written once
     prof_bytes = 2 * elems * 2      # K and V streamed once
     h2d = sum(h.numel() * 2 for h in host)
     d2h = out_host.numel() * 2 + mode_host.numel() * 4
-    # profile partial, merge, finalize; 3 permutes; attention; permute back
-    launches_per_step = 3 + 3 + 1 + 1
+    # profile partial, merge, finalize; 3 permutes; attention (output reordering fused)
+    launches_per_step = 3 + 3 + 1
     line = {
         "metric": METRIC,
         "value": round(value, 3),
@@ -307,16 +336,20 @@ def run_ours(args, rank, world, local_rank):
                    "parallelism": f"independent layer per GPU x{world}"},
         "tokens_per_s": round(tokens_s, 1),
         "pct_of_bf16_peak": round(100 * value / world / peak_tf, 2),
-        "attention_only": {"ms": round(attn_avg, 5), "effective_tflops": round(attn_tf, 3)},
-        # 4 permutes per step (q, k, v forward; o back), every head written:
-        # 2 * B*H*N*d * 2 bytes each; L2 flushed only before the step
+        "attention_only": {"ms": round(attn_avg, 5), "effective_tflops": round(attn_tf, 3),
+                           "kernel": "svg_sparse_attn_fused (output fused)"},
+        "step_permutes_ms": round(fwd_perm_avg, 5),
+        "unfused_layer_ms": round(unf_avg, 5),
+        # the permutation kernel alone: one [B,H,N,d] tensor, every head
+        # reordered, 2 * B*H*N*d * 2 bytes, L2 flushed before each launch
         "permute": {"ms": round(perm_avg, 5),
                     "gbs": round(perm_bytes / (perm_avg * 1e-3) / 1e9, 1),
                     "frac_of_hbm": round(perm_bytes / (perm_avg * 1e-3) / 1e9 / hbm_gbs, 4),
                     "hbm_peak_gbs": hbm_gbs},
         "profile": {"ms": round(prof_avg, 5),
                     "kv_gbs": round(prof_bytes / (prof_avg * 1e-3) / 1e9, 1)},
-        "roofline": {"kernel": "svg_sparse_attn", "bound": "tensor", "achieved": round(attn_tf, 3),
+        "roofline": {"kernel": "svg_sparse_attn_fused", "bound": "tensor",
+                     "achieved": round(attn_tf, 3),
                      "peak": peak_tf, "unit": "TFLOP/s", "frac": round(attn_tf / peak_tf, 4),
                      "peak_source": f"{src} bf16 burst", "traffic": attn_traffic(wl.name)},
         "e2e": {"value": round(e2e_value, 3), "unit": "TFLOPS",

@@ -81,6 +81,10 @@ typedef enum {
 
 #define SVG_TILE 128
 
+/* Layout bits of svg_sparse_attn_fused (section 4b). */
+#define SVG_FUSE_INPUT 0x1   /* q, k, v frame-major; temporal heads gathered  */
+#define SVG_FUSE_OUTPUT 0x2  /* o written frame-major for temporal heads      */
+
 /* Library identification, e.g. "svg_b200 0.1 sm_100a". */
 const char* svg_version(void);
 
@@ -276,6 +280,40 @@ svg_status svg_sparse_attn(const void* q, const void* k, const void* v, void* o,
                            const int32_t* list_id, int n_lists, int n_qblocks,
                            const int32_t* indptr, const int32_t* indices,
                            float scale, int32_t* device_status, void* stream);
+
+/* --------------------------------------------------------------------------
+ * 4b. Block-sparse attention with the layout transformation fused in
+ *    [SVG] sections "Temporal Head" and "Layout Transformation + Kernel 加速":
+ *    temporal heads attend in token-major order (a token's keys across frames
+ *    are contiguous there).  With layout = SVG_FUSE_INPUT | SVG_FUSE_OUTPUT,
+ *    svg_sparse_attn_fused computes exactly
+ *        x' = svg_permute_token_major(x, mode) for x in q, k, v
+ *        o' = svg_sparse_attn(q', k', v', list_id = mode)
+ *        o  = svg_permute_frame_major(o', mode)
+ *    without the intermediate tensors.  Each side can be fused on its own:
+ *      SVG_FUSE_INPUT   q, k, v are FRAME-MAJOR for every head; heads with
+ *                       mode == SVG_MODE_TEMPORAL gather their rows in
+ *                       token-major order (otherwise such heads' q, k, v are
+ *                       already token-major, e.g. from svg_permute_token_major);
+ *      SVG_FUSE_OUTPUT  o is written FRAME-MAJOR for every head (otherwise
+ *                       temporal heads' o is token-major).
+ *    layout 0 is svg_sparse_attn with list_id = mode.
+ *
+ *  q, k, v, o   device [B, H, N, d] in the layouts above.
+ *  frames, tokens_per_frame   F and P with F * P == N (unused for layout 0).
+ *  mode         device int32 [B*H]: the list id of each head (as list_id in
+ *               svg_sparse_attn, e.g. the profiling output with the three
+ *               geometric lists concatenated) and its token order.
+ *  layout       0 or an OR of SVG_FUSE_INPUT and SVG_FUSE_OUTPUT.
+ *  Other arguments, errors and arithmetic as in svg_sparse_attn; a mode
+ *  outside [0, n_lists) sets SVG_DEVICE_BAD_LIST_ID and gives o = 0 for the
+ *  head.
+ * ------------------------------------------------------------------------ */
+svg_status svg_sparse_attn_fused(const void* q, const void* k, const void* v, void* o, int dtype,
+                                 int B, int H, int N, int d, int frames, int tokens_per_frame,
+                                 const int32_t* mode, int layout, int n_lists, int n_qblocks,
+                                 const int32_t* indptr, const int32_t* indices,
+                                 float scale, int32_t* device_status, void* stream);
 
 #ifdef __cplusplus
 }

@@ -209,18 +209,36 @@ def svg_sparse_attn(q, k, v, list_id: torch.Tensor, lists: BlockLists, *, scale:
     return out
 
 
+def svg_sparse_attn_fused(q, k, v, frames: int, tokens_per_frame: int, mode: torch.Tensor,
+                          lists: BlockLists, *, layout: int = 3, scale: float = 0.0, out=None,
+                          status=None, stream=None):
+    """Block-sparse attention with the token-major reordering of temporal
+    heads fused in: layout bit 1 (SVG_FUSE_INPUT) gathers q, k, v from
+    frame-major memory, bit 2 (SVG_FUSE_OUTPUT) writes o frame-major."""
+    B, H, N, d = _check_qkv(q, k, v)
+    if out is None:
+        out = torch.empty_like(q)
+    _lib.call("svg_sparse_attn_fused", q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+              _dt(q), B, H, N, d, frames, tokens_per_frame, mode.data_ptr(), int(layout),
+              lists.n_lists, lists.n_qblocks, lists.indptr.data_ptr(), lists.indices.data_ptr(),
+              float(scale), _ptr(status), _stream(stream))
+    return out
+
+
 # --------------------------------------------------------------------- layer
 
 class LayerBuffers:
     """Preallocated buffers for svg_layer at one shape (reused across steps)."""
 
-    def __init__(self, q: torch.Tensor, S: int):
+    def __init__(self, q: torch.Tensor, S: int, layout: int = _lib.SVG_FUSE_OUTPUT):
         B, H, N, d = q.shape
         dev = q.device
-        self.qp = torch.empty_like(q)
-        self.kp = torch.empty_like(q)
-        self.vp = torch.empty_like(q)
-        self.op = torch.empty_like(q)
+        if not layout & _lib.SVG_FUSE_INPUT:  # token-major copies of q, k, v
+            self.qp = torch.empty_like(q)
+            self.kp = torch.empty_like(q)
+            self.vp = torch.empty_like(q)
+        if not layout & _lib.SVG_FUSE_OUTPUT:  # token-major output
+            self.op = torch.empty_like(q)
         self.o = torch.empty_like(q)
         self.mse = torch.empty(B * H, 2, dtype=torch.float32, device=dev)
         self.mode = torch.empty(B * H, dtype=torch.int32, device=dev)
@@ -229,17 +247,30 @@ class LayerBuffers:
 
 def svg_layer(q, k, v, frames: int, tokens_per_frame: int, spatial_width: int,
               sample_idx: torch.Tensor, lists: BlockLists, bufs: Optional[LayerBuffers] = None,
-              stream=None):
-    """One attention layer: profile -> permute temporal heads -> block-sparse
-    attention on the list the mode selects -> permute back.
+              stream=None, layout: int = _lib.SVG_FUSE_OUTPUT):
+    """One attention layer: profile -> block-sparse attention on the list the
+    mode selects, temporal heads in token-major order.  `layout` picks which
+    side of the reordering runs inside the attention kernel
+    (svg_sparse_attn_fused); the other side runs as permutation kernels.
+    The default fuses only the output side: on B200 the permutation kernel
+    moves q, k, v faster than row gathers inside the attention kernel.
     Returns (o, mode, mse)."""
     if bufs is None:
         bufs = LayerBuffers(q, sample_idx.numel())
     F, P = frames, tokens_per_frame
     svg_profile_heads(q, k, v, F, P, spatial_width, sample_idx, mse_out=bufs.mse,
                       mode_out=bufs.mode, workspace=bufs.ws, stream=stream)
-    for x, y in ((q, bufs.qp), (k, bufs.kp), (v, bufs.vp)):
-        svg_permute_token_major(x, F, P, bufs.mode, out=y, stream=stream)
-    svg_sparse_attn(bufs.qp, bufs.kp, bufs.vp, bufs.mode, lists, out=bufs.op, stream=stream)
-    svg_permute_frame_major(bufs.op, F, P, bufs.mode, out=bufs.o, stream=stream)
+    if layout & _lib.SVG_FUSE_INPUT:
+        ins = (q, k, v)
+    else:
+        for x, y in ((q, bufs.qp), (k, bufs.kp), (v, bufs.vp)):
+            svg_permute_token_major(x, F, P, bufs.mode, out=y, stream=stream)
+        ins = (bufs.qp, bufs.kp, bufs.vp)
+    if layout & _lib.SVG_FUSE_OUTPUT:
+        svg_sparse_attn_fused(*ins, F, P, bufs.mode, lists, layout=layout, out=bufs.o,
+                              stream=stream)
+    else:
+        svg_sparse_attn_fused(*ins, F, P, bufs.mode, lists, layout=layout, out=bufs.op,
+                              stream=stream)
+        svg_permute_frame_major(bufs.op, F, P, bufs.mode, out=bufs.o, stream=stream)
     return bufs.o, bufs.mode, bufs.mse

@@ -15,6 +15,8 @@ SVG_BF16, SVG_FP32 = 0, 1
 SVG_MODE_SPATIAL, SVG_MODE_TEMPORAL, SVG_MODE_DENSE = 0, 1, 2
 SVG_DEVICE_BAD_LIST_ID, SVG_DEVICE_BAD_INDEX, SVG_DEVICE_TIMEOUT, SVG_DEVICE_CAPACITY = 1, 2, 4, 8
 SVG_DEVICE_RANGE = 16
+SVG_FUSE_INPUT = 1
+SVG_FUSE_OUTPUT = 2
 SVG_TILE = 128
 
 _p = C.c_void_p
@@ -42,6 +44,8 @@ SIGNATURES = {
     "svg_build_block_mask_calibrated": (_i, [_p, _i, _i, _i, _i, _d, _d, _p, _p, _i64, _p, _p, _p,
                                              _sz, _p]),
     "svg_sparse_attn": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _i, _p, _i, _i, _p, _p, _f, _p, _p]),
+    "svg_sparse_attn_fused": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p, _i, _i, _i, _p,
+                                   _p, _f, _p, _p]),
 }
 
 

@@ -18,7 +18,29 @@ struct AttnArgs {
   const int32_t* indices;
   float scale;
   int32_t* status;         // optional device status word
+  // Optional fused layout transformation for heads whose order[b*H + h] is
+  // SVG_MODE_TEMPORAL (they run in token-major order, m = s * F + f):
+  // SVG_FUSE_INPUT  q, k, v of such heads are frame-major in memory
+  //                 (n = f * P + s) and gathered row by row;
+  // SVG_FUSE_OUTPUT o of such heads is written frame-major.
+  // order == nullptr or layout == 0: every tensor is in the heads' order.
+  const int32_t* order;
+  int frames, tokens_per_frame;
+  int layout;
 };
+
+__device__ __forceinline__ bool temporal_head(const AttnArgs& a, int bh) {
+  return a.order != nullptr && a.order[bh] == SVG_MODE_TEMPORAL;
+}
+__device__ __forceinline__ bool gathers_input(const AttnArgs& a, int bh) {
+  return (a.layout & SVG_FUSE_INPUT) != 0 && temporal_head(a, bh);
+}
+__device__ __forceinline__ bool scatters_output(const AttnArgs& a, int bh) {
+  return (a.layout & SVG_FUSE_OUTPUT) != 0 && temporal_head(a, bh);
+}
+
+// Frame-major memory row of token-major row m.
+__device__ __forceinline__ int token_major_row(int m, int F, int P) { return (m % F) * P + m / F; }
 
 template <int D>
 svg_status launch_attn_fp32(const AttnArgs& a, cudaStream_t s);

@@ -48,11 +48,17 @@ __global__ void __launch_bounds__(256) attn_fp32(AttnArgs a) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const RowList lst = row_list(a, bh, qt);
   const float scale_log2 = a.scale * kLog2e;
+  const bool gin = gathers_input(a, bh), sout = scatters_output(a, bh);
+  const int F = a.frames, P = a.tokens_per_frame;
+  // memory row of sequence position x in the inputs
+  auto row = [&](int x) -> long long { return gin ? token_major_row(x, F, P) : x; };
   for (int r = qt * SVG_TILE + warp; r < min(N, (qt + 1) * SVG_TILE); r += 8) {
     float qv[E], acc[E], m = -INFINITY, l = 0.f;
+    const long long rq = row(r);
+    const long long ro = sout ? token_major_row(r, F, P) : r;
 #pragma unroll
     for (int e = 0; e < E; ++e) {
-      qv[e] = q[static_cast<long long>(r) * D + lane + 32 * e];
+      qv[e] = q[rq * D + lane + 32 * e];
       acc[e] = 0.f;
     }
     for (int t = 0; t < lst.len; ++t) {
@@ -62,9 +68,10 @@ __global__ void __launch_bounds__(256) attn_fp32(AttnArgs a) {
         continue;
       }
       for (int c = j * SVG_TILE; c < min(N, (j + 1) * SVG_TILE); ++c) {
+        const long long rc = row(c);
         float dot = 0.f;
 #pragma unroll
-        for (int e = 0; e < E; ++e) dot = fmaf(qv[e], k[static_cast<long long>(c) * D + lane + 32 * e], dot);
+        for (int e = 0; e < E; ++e) dot = fmaf(qv[e], k[rc * D + lane + 32 * e], dot);
 #pragma unroll
         for (int o2 = 16; o2 > 0; o2 >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o2);
         const float tt = dot * scale_log2;
@@ -73,13 +80,13 @@ __global__ void __launch_bounds__(256) attn_fp32(AttnArgs a) {
         const float p = exp2f(tt - mn);
         l = l * alpha + p;
 #pragma unroll
-        for (int e = 0; e < E; ++e) acc[e] = fmaf(p, v[static_cast<long long>(c) * D + lane + 32 * e], acc[e] * alpha);
+        for (int e = 0; e < E; ++e) acc[e] = fmaf(p, v[rc * D + lane + 32 * e], acc[e] * alpha);
         m = mn;
       }
     }
     const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
-    for (int e = 0; e < E; ++e) o[static_cast<long long>(r) * D + lane + 32 * e] = acc[e] * inv;
+    for (int e = 0; e < E; ++e) o[ro * D + lane + 32 * e] = acc[e] * inv;
   }
 }
 

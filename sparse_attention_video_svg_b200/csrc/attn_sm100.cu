@@ -120,6 +120,7 @@ __device__ __forceinline__ bool valid_tile(int j, int nb) { return j >= 0 && j <
 // that keep the block, bits 2-3 the members for which it is the first block
 // of the item, bits 4-5 the last; bit 6 marks the end (no tile loaded).
 constexpr uint32_t kStepEnd = 1u << 6;
+constexpr uint32_t kStepGathered = 1u << 7;  // Q / K / V of this step came through cp.async
 
 // Entries [beg, end) of `indices` for query tile qt of head bh; empty for a
 // tile past the end or a bad list.
@@ -156,7 +157,7 @@ __device__ __forceinline__ void skip_invalid(const AttnArgs& a, int nb, int& p, 
 // equal heads are shared.  Afterwards both heads are again valid or
 // exhausted.
 __device__ __forceinline__ bool merge_next(const AttnArgs& a, int nb, int (&p)[2],
-                                           const int (&e)[2], int& j, int& mask) {
+                                           const int (&e)[2], int& j, int& mask, bool report) {
   int jj[2];
 #pragma unroll
   for (int t = 0; t < 2; ++t) jj[t] = p[t] < e[t] ? a.indices[p[t]] : INT_MAX;
@@ -167,7 +168,7 @@ __device__ __forceinline__ bool merge_next(const AttnArgs& a, int nb, int (&p)[2
   for (int t = 0; t < 2; ++t)
     if (mask >> t & 1) {
       ++p[t];
-      skip_invalid(a, nb, p[t], e[t], true);
+      skip_invalid(a, nb, p[t], e[t], report);
     }
   return true;
 }
@@ -332,7 +333,9 @@ __device__ __forceinline__ void softmax_member(const AttnArgs& a, const Bars& B,
       inv = l > 0.f ? 1.f / l : 0.f;
     }
     const int n = qt * 128 + row;
-    __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.o) + (static_cast<long long>(bh) * N + n) * D;
+    // token-major heads over frame-major memory write row n back to its frame-major place
+    const int nm = (scatters_output(a, bh) && n < N) ? token_major_row(n, a.frames, a.tokens_per_frame) : n;
+    __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.o) + (static_cast<long long>(bh) * N + nm) * D;
 #pragma unroll
     for (int ch = 0; ch < D / 32; ch += 2) {
       uint32_t r[2][32];
@@ -363,6 +366,150 @@ __device__ __forceinline__ void softmax_member(const AttnArgs& a, const Bars& B,
     }
     // the next item's first P.V (accumulate off) is issued after this
     // member's next p_ready, which follows these TMEM reads in program order
+  }
+}
+
+// 128 token-major rows m0 .. m0 + 127 of one head's frame-major [N][D]
+// matrix (row m is memory row (m mod F) P + m div F), copied by the 32 lanes
+// of a warp into a tile laid out exactly like the 128-byte-swizzled TMA
+// boxes (box bx holds columns 64 bx .. 64 bx + 63; the 16-byte chunk c of
+// row r sits at chunk position c ^ (r mod 8)).  Rows at or past N are
+// zero-filled.
+template <int D>
+__device__ __forceinline__ void gather_rows(unsigned char* dst, const __nv_bfloat16* src, int m0,
+                                            int N, int F, int P) {
+  constexpr int CH = D / 8;       // 16-byte chunks per row
+  constexpr int RSTEP = 32 / CH;  // rows between one lane's copies
+  const int lane = threadIdx.x & 31;
+  const int c = lane % CH;
+  int r = lane / CH;
+  int m = m0 + r;
+  int f = m % F, sp = m / F;  // m = sp * F + f
+#pragma unroll 4
+  for (; r < 128; r += RSTEP) {
+    const bool ok = m < N;
+    const long long n = ok ? static_cast<long long>(f) * P + sp : 0;
+    cp_async16(dst + (c >> 3) * kBox + r * 128 + (((c & 7) ^ (r & 7)) << 4), src + n * D + c * 8,
+               ok);
+    m += RSTEP;
+    f += RSTEP;
+    while (f >= F) {
+      f -= F;
+      ++sp;
+    }
+  }
+}
+
+// TMA producer (warp 0, all lanes): Q tiles and the merged walk's K / V
+// tiles.  Heads in memory order load with TMA; heads that run token-major
+// over frame-major memory gather their rows with cp.async: every lane hands
+// its copies to the tile's mbarrier (cp.async.mbarrier.arrive) and the leader
+// adds the phase's regular arrival, so the barrier completes when the rows
+// have landed.  The consumers fence the async proxy after their wait, as the
+// tensor core reads what the generic proxy wrote.
+template <int D>
+__device__ __forceinline__ void producer(const AttnArgs& a, const Maps& maps, const Bars& B,
+                                         unsigned char* smem, volatile uint32_t* step_info,
+                                         volatile int* abort_flag, int n_items, int n_pairs,
+                                         int nb) {
+  using C = Cfg<D>;
+  constexpr int QD = C::kQDepth, S = C::kSlots;
+  const int lane = threadIdx.x & 31;
+  const bool leader = lane == 0;
+  const int N = a.N, F = a.frames, P = a.tokens_per_frame;
+  uint32_t L = 0, cq[2] = {0, 0};
+  bool ok = true;
+  auto leader_wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+    int r = 1;
+    if (leader) r = wait_bar(bar, parity, abort_flag, a.status) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, r, 0) != 0;
+  };
+  // gathered tile: lanes' copies, then the barrier takes them over
+  auto gather_into = [&](unsigned char* dst, const void* src, int m0, uint64_t* bar) {
+    gather_rows<D>(dst, static_cast<const __nv_bfloat16*>(src), m0, N, F, P);
+    cp_async_mbar_arrive(bar);
+    __syncwarp();
+    if (leader) mbar_arrive(bar);
+  };
+  auto claim = [&]() -> bool {  // the K and V entries of the step at ring index L are free
+    return leader_wait(&B.kv_empty[L % S], ((L / S) & 1) ^ 1) &&
+           leader_wait(&B.kv_empty[(L + 1) % S], (((L + 1) / S) & 1) ^ 1);
+  };
+  for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+    const int bh = item / n_pairs, qt0 = 2 * (item - bh * n_pairs);
+    const bool tm = gathers_input(a, bh);
+    const long long head = static_cast<long long>(bh) * N * D;
+    int p[2], e[2];
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      member_list(a, bh, qt0 + t, nb, p[t], e[t], leader);
+      skip_invalid(a, nb, p[t], e[t], leader);
+    }
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      if (p[t] >= e[t] || !ok) continue;
+      const uint32_t qs = cq[t] % QD, qb = t * QD + qs;
+      if (!(ok = leader_wait(&B.q_empty[qb], ((cq[t] / QD) & 1) ^ 1))) continue;
+      unsigned char* dst = smem + C::kOffQ + qb * C::kTile;
+      if (!tm) {
+        if (leader) {
+          mbar_arrive_expect_tx(&B.q_full[qb], C::kTile);
+          for (int bx = 0; bx < C::kBoxes; ++bx)
+            tma_load_3d(dst + bx * kBox, &maps.q, &B.q_full[qb], 64 * bx, (qt0 + t) * 128, bh);
+        }
+      } else {
+        gather_into(dst, static_cast<const __nv_bfloat16*>(a.q) + head, (qt0 + t) * 128,
+                    &B.q_full[qb]);
+      }
+      ++cq[t];
+    }
+    uint32_t seen = 0;  // members that already had a block in this item
+    int j, mask;
+    while (ok && merge_next(a, nb, p, e, j, mask, leader)) {
+      const uint32_t m = static_cast<uint32_t>(mask);
+      const uint32_t last = (m & 1u) * (p[0] >= e[0] ? 1u : 0u) |
+                            (m & 2u) * (p[1] >= e[1] ? 1u : 0u);
+      const uint32_t info = m | ((m & ~seen) << 2) | (last << 4) | (tm ? kStepGathered : 0u);
+      seen |= m;
+      if (!(ok = claim())) break;
+      if (leader) step_info[(L / 2) % C::kSteps] = info;  // released by the step's arrives
+      for (int kv = 0; kv < 2; ++kv) {
+        const uint32_t slot = (L + kv) % S;
+        unsigned char* dst = smem + C::kOffKV + slot * C::kTile;
+        const void* src = kv == 0 ? a.k : a.v;
+        if (!tm) {
+          if (leader) {
+            mbar_arrive_expect_tx(&B.kv_full[slot], C::kTile);
+            const CUtensorMap* map = kv == 0 ? &maps.k : &maps.v;
+            for (int bx = 0; bx < C::kBoxes; ++bx)
+              tma_load_3d(dst + bx * kBox, map, &B.kv_full[slot], 64 * bx, j * 128, bh);
+          }
+        } else {
+          gather_into(dst, static_cast<const __nv_bfloat16*>(src) + head, j * 128,
+                      &B.kv_full[slot]);
+        }
+      }
+      L += 2;
+    }
+  }
+  // end record in the next step's entries; plain arrives complete their
+  // phases
+  if (ok && (ok = claim())) {
+    if (leader) {
+      step_info[(L / 2) % C::kSteps] = kStepEnd;
+      mbar_arrive(&B.kv_full[L % S]);
+      mbar_arrive(&B.kv_full[(L + 1) % S]);
+    }
+  }
+  if (!ok) {
+    // let the copies already issued land before the CTA can exit
+    cp_async_wait<0>();
+    if (leader) {
+      for (uint32_t l = L > S ? L - S : 0; l < L; ++l) drain_bar(&B.kv_full[l % S], (l / S) & 1);
+      for (int t = 0; t < 2; ++t)
+        for (uint32_t c = cq[t] > QD ? cq[t] - QD : 0; c < cq[t]; ++c)
+          drain_bar(&B.q_full[t * QD + c % QD], (c / QD) & 1);
+    }
   }
 }
 
@@ -432,70 +579,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     reg_dealloc<C::kRegsLow>();
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      uint32_t L = 0, cq[2] = {0, 0};
-      bool ok = true;
-      // waits until the K and V entries of the step at ring index L are free
-      auto claim = [&]() -> bool {
-        return wait_bar(&B.kv_empty[L % S], ((L / S) & 1) ^ 1, abort_flag, a.status) &&
-               wait_bar(&B.kv_empty[(L + 1) % S], (((L + 1) / S) & 1) ^ 1, abort_flag, a.status);
-      };
-      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
-        const int bh = item / n_pairs, qt0 = 2 * (item - bh * n_pairs);
-        int p[2], e[2];
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          member_list(a, bh, qt0 + t, nb, p[t], e[t], true);
-          skip_invalid(a, nb, p[t], e[t], true);
-        }
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          if (p[t] >= e[t] || !ok) continue;
-          const uint32_t qs = cq[t] % QD;
-          if (!(ok = wait_bar(&B.q_empty[t * QD + qs], ((cq[t] / QD) & 1) ^ 1, abort_flag,
-                              a.status)))
-            continue;
-          mbar_arrive_expect_tx(&B.q_full[t * QD + qs], C::kTile);
-          for (int bx = 0; bx < C::kBoxes; ++bx)
-            tma_load_3d(smem + C::kOffQ + (t * QD + qs) * C::kTile + bx * kBox, &maps.q,
-                        &B.q_full[t * QD + qs], 64 * bx, (qt0 + t) * 128, bh);
-          ++cq[t];
-        }
-        uint32_t seen = 0;  // members that already had a block in this item
-        int j, mask;
-        while (ok && merge_next(a, nb, p, e, j, mask)) {
-          const uint32_t m = static_cast<uint32_t>(mask);
-          const uint32_t last = (m & 1u) * (p[0] >= e[0] ? 1u : 0u) |
-                                (m & 2u) * (p[1] >= e[1] ? 1u : 0u);
-          const uint32_t info = m | ((m & ~seen) << 2) | (last << 4);
-          seen |= m;
-          if (!(ok = claim())) break;
-          step_info[(L / 2) % C::kSteps] = info;  // released by the arrives below
-          for (int kv = 0; kv < 2; ++kv, ++L) {
-            const uint32_t slot = L % S;
-            mbar_arrive_expect_tx(&B.kv_full[slot], C::kTile);
-            const CUtensorMap* map = kv == 0 ? &maps.k : &maps.v;
-            for (int bx = 0; bx < C::kBoxes; ++bx)
-              tma_load_3d(smem + C::kOffKV + slot * C::kTile + bx * kBox, map, &B.kv_full[slot],
-                          64 * bx, j * 128, bh);
-          }
-        }
-      }
-      // end record in the next step's entries; plain arrives complete their
-      // phases
-      if (ok && (ok = claim())) {
-        step_info[(L / 2) % C::kSteps] = kStepEnd;
-        mbar_arrive(&B.kv_full[L % S]);
-        mbar_arrive(&B.kv_full[(L + 1) % S]);
-      }
-      if (!ok) {
-        // let the copies already issued land before the CTA can exit
-        for (uint32_t l = L > S ? L - S : 0; l < L; ++l) drain_bar(&B.kv_full[l % S], (l / S) & 1);
-        for (int t = 0; t < 2; ++t)
-          for (uint32_t c = cq[t] > QD ? cq[t] - QD : 0; c < cq[t]; ++c)
-            drain_bar(&B.q_full[t * QD + c % QD], (c / QD) & 1);
-      }
-    }
+    producer<D>(a, maps, B, smem, step_info, abort_flag, n_items, n_pairs, nb);
   } else if (warp == 1 || warp == 2) {
     reg_dealloc<C::kRegsLow>();
     // ------------------------------------------------------------ MMA issuers
@@ -529,6 +613,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t kslot = L % S;
         if (!(ok = wait_bar(&B.kv_full[kslot], (L / S) & 1, abort_flag, a.status))) break;
         const uint32_t info = step_info[(L / 2) % C::kSteps];
+        // gathered tiles were written through the generic proxy
+        if (info & kStepGathered) fence_proxy_async_smem();
         if (info & kStepEnd) break;
         if (!(info >> t & 1u)) {
           // this member skips the block: its pending P.V goes now (otherwise
@@ -549,6 +635,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t qs = cq % QD;
         if (info >> (2 + t) & 1u) {  // first block of the item: a new Q tile
           if (!(ok = wait_bar(&B.q_full[t * QD + qs], (cq / QD) & 1, abort_flag, a.status))) break;
+          if (info & kStepGathered) fence_proxy_async_smem();
         }
         tc_fence_after();
         const uint64_t q0 = dq + ((qs * C::kTile) >> 4), k0 = dk + ((kslot * C::kTile) >> 4);

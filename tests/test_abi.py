@@ -77,6 +77,17 @@ class TestHostValidation:
         expect(INVALID, "svg_sparse_attn", *(base[:14] + [-1.0] + base[15:]), match="scale")
         expect(INVALID, "svg_sparse_attn", *([None] + base[1:]), match="null")
 
+    def test_sparse_attn_fused(self):
+        # q k v o dtype B H N d F P mode layout n_lists n_qblocks indptr indices scale status
+        # stream
+        base = [FAKE, FAKE2, FAKE3, FAKE4 * 4, 0, 1, 2, 256, 64, 4, 64, FAKE, 3, 3, 2, FAKE, FAKE,
+                0.0, None, None]
+        expect(INVALID, "svg_sparse_attn_fused", *(base[:9] + [5] + base[10:]), match="frames")
+        expect(INVALID, "svg_sparse_attn_fused", *(base[:8] + [96] + base[9:]), match="d=96")
+        expect(INVALID, "svg_sparse_attn_fused", *(base[:11] + [None] + base[12:]), match="null")
+        expect(INVALID, "svg_sparse_attn_fused", *(base[:3] + [FAKE] + base[4:]), match="overlaps")
+        expect(INVALID, "svg_sparse_attn_fused", *(base[:12] + [4] + base[13:]), match="layout")
+
     def test_permute(self):
         args = [FAKE, FAKE4 * 4, 0, 1, 2, 12, 64, 3, 4, None, None]
         expect(INVALID, "svg_permute_token_major", *(args[:7] + [5] + args[8:]), match="!= N")

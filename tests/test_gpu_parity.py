@@ -263,6 +263,90 @@ def test_sparse_attn_ragged_dense(N, d):
         assert_close(o[b, 0], ref, f"N={N} d={d} b={b}")
 
 
+# ------------------------------------------------- fused layout transformation
+
+def _unfused(qd, kd, vd, F, P, mode, lists):
+    perm = [svg.svg_permute_token_major(x, F, P, mode) for x in (qd, kd, vd)]
+    op = svg.svg_sparse_attn(*perm, mode, lists)
+    return svg.svg_permute_frame_major(op, F, P, mode)
+
+
+FUSE_IN, FUSE_OUT = 1, 2
+
+
+@pytest.mark.parametrize("wl", SMALL, ids=lambda w: w.name)
+def test_sparse_attn_fused_small(wl):
+    """Every fused layout == permute -> attention -> permute back, bit for
+    bit, and element-wise against the oracle, with mixed modes (incl. dense)."""
+    (q, k, v), (qd, kd, vd), _ = workload_tensors(wl)
+    lists = svg.geometric_lists(wl.F, wl.P, wl.width, wl.N)
+    modes = np.array([(O.MODE_TEMPORAL, O.MODE_SPATIAL, O.MODE_DENSE, O.MODE_TEMPORAL)[h % 4]
+                      for h in range(wl.B * wl.H)], dtype=np.int32)
+    mode = torch.from_numpy(modes).to(DEV)
+    ref_bits = bits(_unfused(qd, kd, vd, wl.F, wl.P, mode, lists))
+    perm = [svg.svg_permute_token_major(x, wl.F, wl.P, mode) for x in (qd, kd, vd)]
+    for layout in (FUSE_IN, FUSE_OUT, FUSE_IN | FUSE_OUT):
+        ins = (qd, kd, vd) if layout & FUSE_IN else perm
+        status = torch.zeros(1, dtype=torch.int32, device=DEV)
+        o = svg.svg_sparse_attn_fused(*ins, wl.F, wl.P, mode, lists, layout=layout, status=status)
+        assert status.item() == 0
+        if not layout & FUSE_OUT:
+            o = svg.svg_permute_frame_major(o, wl.F, wl.P, mode)
+        np.testing.assert_array_equal(bits(o), ref_bits, err_msg=f"layout {layout}")
+    got = to_float64(o)
+    for h in range(wl.H):
+        md = int(modes[h])
+        ip, ix = O.geometric_block_lists(md, wl.F, wl.P, wl.width, wl.N)
+        qh, kh, vh = head64(q, 0, h), head64(k, 0, h), head64(v, 0, h)
+        if md == O.MODE_TEMPORAL:
+            qh, kh, vh = (O.permute_token_major(t, wl.F, wl.P) for t in (qh, kh, vh))
+        ref = O.block_sparse_attention(qh, kh, vh, ip, ix)
+        if md == O.MODE_TEMPORAL:
+            ref = O.permute_frame_major(ref, wl.F, wl.P)
+        assert_close(got[0, h], ref, f"{wl.name} mode {md} head {h}", bf16=wl.dtype == "bf16")
+
+
+@pytest.mark.parametrize("name", ["wan480", "hunyuan720"])
+def test_sparse_attn_fused_full_size_sampled(name, full_inputs):
+    """Token-major gathers at the full sizes (F = 21 and 33 frames)."""
+    wl = si.WORKLOADS[name]
+    (q, k, v), (qd, kd, vd), types = full_inputs(name)
+    lists = svg.geometric_lists(wl.F, wl.P, wl.width, wl.N)
+    mode = torch.from_numpy(types).to(DEV)
+    o = svg.svg_sparse_attn_fused(qd, kd, vd, wl.F, wl.P, mode, lists)
+    src = O.token_major_source(wl.F, wl.P)
+    rng = np.random.default_rng(13)
+    nb = svg.n_tiles(wl.N)
+    temporal = np.flatnonzero(types == O.MODE_TEMPORAL)
+    for h in list(rng.choice(temporal, size=3, replace=False)) + [int(np.flatnonzero(types == 0)[0])]:
+        md = int(types[h])
+        ip, ix = O.geometric_block_lists(md, wl.F, wl.P, wl.width, wl.N)
+        qh, kh, vh = head64(q, 0, h), head64(k, 0, h), head64(v, 0, h)
+        if md == O.MODE_TEMPORAL:
+            qh, kh, vh = (O.permute_token_major(t, wl.F, wl.P) for t in (qh, kh, vh))
+        for t in np.r_[rng.choice(nb - 1, size=2, replace=False), nb - 1]:
+            rows = O.tile_rows(int(t), wl.N)
+            ref = O.block_sparse_rows(qh, kh, vh, rows, ip, ix)
+            out_rows = src[rows] if md == O.MODE_TEMPORAL else rows
+            got = to_float64(o[0, h][torch.from_numpy(out_rows).to(DEV)])
+            assert_close(got, ref, f"{name} fused head {h} tile {t}")
+
+
+def test_sparse_attn_fused_bad_mode():
+    wl = si.small("cogvideox")
+    (q, k, v), (qd, kd, vd), _ = workload_tensors(wl)
+    lists = svg.geometric_lists(wl.F, wl.P, wl.width, wl.N)
+    mode = torch.tensor([1, 7, 0, 1], dtype=torch.int32, device=DEV)  # head 1: not a list
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o = svg.svg_sparse_attn_fused(qd, kd, vd, wl.F, wl.P, mode, lists, status=status)
+    assert status.item() & svg._lib.SVG_DEVICE_BAD_LIST_ID
+    assert (to_float64(o[0, 1]) == 0).all()
+    good = torch.tensor([1, 0, 0, 1], dtype=torch.int32, device=DEV)
+    ref = svg.svg_sparse_attn_fused(qd, kd, vd, wl.F, wl.P, good, lists)
+    for h in (0, 2, 3):
+        np.testing.assert_array_equal(bits(o[0, h]), bits(ref[0, h]))
+
+
 # ---------------------------------------------------------------- the layer
 
 @pytest.mark.parametrize("wl", SMALL, ids=lambda w: w.name)
@@ -279,6 +363,23 @@ def test_layer_small(wl):
     got = to_float64(o)
     for h in range(wl.H):
         assert_close(got[0, h], o_ref[0, h], f"{wl.name} head {h}", bf16=wl.dtype == "bf16")
+
+
+@pytest.mark.parametrize("wl", SMALL[:3], ids=lambda w: w.name)
+def test_layer_small_layouts_agree(wl):
+    """The layer gives the same bits whichever side of the reordering is
+    fused into the attention kernel."""
+    (q, k, v), (qd, kd, vd), _ = workload_tensors(wl)
+    idx = torch.from_numpy(si.sample_queries(wl)).to(DEV)
+    lists = svg.geometric_lists(wl.F, wl.P, wl.width, wl.N)
+    outs = []
+    for layout in (0, FUSE_IN, FUSE_OUT, FUSE_IN | FUSE_OUT):
+        bufs = svg.LayerBuffers(qd, idx.numel(), layout=layout)
+        o, m, _ = svg.svg_layer(qd, kd, vd, wl.F, wl.P, wl.width, idx, lists, bufs, layout=layout)
+        outs.append((bits(o), m.cpu().numpy()))
+    for o, m in outs[1:]:
+        np.testing.assert_array_equal(m, outs[0][1])
+        np.testing.assert_array_equal(o, outs[0][0])
 
 
 def test_layer_full_size_cogvideox_sampled(full_inputs):
