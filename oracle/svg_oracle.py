@@ -31,7 +31,11 @@ notes):
   to 1); the kept set is the shortest prefix, in descending energy with ties
   to the smaller block index, whose sum reaches eps; a block survives the
   cross-input vote when its keep frequency is >= rho; an empty voted row keeps
-  the block of largest summed energy.
+  the block of largest summed energy;
+* the energy threshold decays exponentially in the denoising-step index from
+  0.99 (first step) to 0.84 (last step); the skip list holds each row's
+  maximal runs of consecutive kept blocks; the bitmap holds one bit per
+  (query block, key block) in 32-bit words.
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
 (library cross-checks, closed forms, invariants, brute force, and worked
@@ -343,6 +347,89 @@ def calibrate_lists(E_list: Sequence[np.ndarray], eps: float, rho: float):
                 tot = tot + np.asarray(E[r], np.float64)
             kept = [int(np.argmax(tot))]
         indices.extend(kept)
+        indptr.append(len(indices))
+    return np.asarray(indptr, np.int32), np.asarray(indices, np.int32)
+
+
+# ---------------------------------------------------------------------------
+# O10: timestep schedule of the energy threshold and mask encodings
+#      ([CAL] 3.1: eps(t) decays exponentially, about 0.99 early and 0.84
+#      late; 3.3: the mask as a skip list of contiguous block intervals and
+#      as a bitmap, 32x smaller)
+# ---------------------------------------------------------------------------
+
+def epsilon_schedule(n_steps: int, eps_first: float = 0.99, eps_last: float = 0.84) -> np.ndarray:
+    """eps at denoising steps 0 .. n_steps-1, decaying exponentially in the
+    step index from eps_first to eps_last: eps_i = eps_first *
+    (eps_last / eps_first) ** (i / (n_steps - 1)); a single step uses
+    eps_first.  (The pages give the two end values and the decay shape, not
+    the formula; this is the plainest exponential between them.)"""
+    if n_steps <= 0:
+        return np.zeros(0)
+    if n_steps == 1:
+        return np.array([float(eps_first)])
+    i = np.arange(n_steps, dtype=np.float64)
+    return float(eps_first) * (float(eps_last) / float(eps_first)) ** (i / (n_steps - 1))
+
+
+def lists_to_intervals(indptr, indices):
+    """Skip list: each row's set of kept key blocks as maximal runs of
+    consecutive blocks [start, end), ascending.  Returns (iptr [rows + 1],
+    starts, ends)."""
+    iptr = [0]
+    starts: List[int] = []
+    ends: List[int] = []
+    for r in range(len(indptr) - 1):
+        kept = sorted(set(int(c) for c in indices[indptr[r]:indptr[r + 1]]))
+        run_start = None
+        prev = None
+        for c in kept:
+            if run_start is None:
+                run_start = c
+            elif c != prev + 1:
+                starts.append(run_start)
+                ends.append(prev + 1)
+                run_start = c
+            prev = c
+        if run_start is not None:
+            starts.append(run_start)
+            ends.append(prev + 1)
+        iptr.append(len(starts))
+    return (np.asarray(iptr, np.int32), np.asarray(starts, np.int32), np.asarray(ends, np.int32))
+
+
+def intervals_to_lists(iptr, starts, ends):
+    """Inverse of lists_to_intervals: CSR with ascending indices."""
+    indptr = [0]
+    indices: List[int] = []
+    for r in range(len(iptr) - 1):
+        for t in range(iptr[r], iptr[r + 1]):
+            indices.extend(range(int(starts[t]), int(ends[t])))
+        indptr.append(len(indices))
+    return np.asarray(indptr, np.int32), np.asarray(indices, np.int32)
+
+
+def lists_to_bitmap(indptr, indices, n_cols: int) -> np.ndarray:
+    """Bitmap of the kept blocks: uint32 words [rows][ceil(n_cols / 32)],
+    block c of row r is bit (c mod 32) of word (c div 32)."""
+    rows = len(indptr) - 1
+    words = (n_cols + 31) // 32
+    bm = np.zeros((rows, words), dtype=np.uint32)
+    for r in range(rows):
+        for c in indices[indptr[r]:indptr[r + 1]]:
+            c = int(c)
+            bm[r, c // 32] |= np.uint32(1) << np.uint32(c % 32)
+    return bm
+
+
+def bitmap_to_lists(bm: np.ndarray, n_cols: int):
+    """Inverse of lists_to_bitmap: CSR with ascending indices."""
+    indptr = [0]
+    indices: List[int] = []
+    for r in range(bm.shape[0]):
+        for c in range(n_cols):
+            if (int(bm[r, c // 32]) >> (c % 32)) & 1:
+                indices.append(c)
         indptr.append(len(indices))
     return np.asarray(indptr, np.int32), np.asarray(indices, np.int32)
 

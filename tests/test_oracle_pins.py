@@ -438,3 +438,69 @@ def test_layer_composes_steps_on_tiny():
     half = (n % P) // 32
     M = half[:, None] == half[None, :]
     np.testing.assert_allclose(o[0, 1], sdpa64(q64[0, 1], k64[0, 1], v64[0, 1], M), atol=1e-12)
+
+
+# ------------------------------------------- eps(t) schedule and mask encodings
+
+def random_lists(rows, n_cols, seed):
+    rng = np.random.default_rng(seed)
+    ip, ix = [0], []
+    for _ in range(rows):
+        k = int(rng.integers(0, n_cols + 1))
+        ix.extend(sorted(rng.choice(n_cols, size=k, replace=False).tolist()))
+        ip.append(len(ix))
+    return np.asarray(ip, np.int32), np.asarray(ix, np.int32)
+
+
+class TestScheduleAndEncodings:
+    def test_schedule_end_values_and_exponential_shape(self):
+        e = O.epsilon_schedule(50)
+        assert e[0] == pytest.approx(0.99, abs=1e-15) and e[-1] == pytest.approx(0.84, abs=1e-15)
+        assert (np.diff(e) < 0).all()
+        # exponential decay: constant ratio between consecutive steps, and the
+        # log is linear in the step index
+        r = e[1:] / e[:-1]
+        np.testing.assert_allclose(r, (0.84 / 0.99) ** (1 / 49), rtol=1e-13)
+        np.testing.assert_allclose(np.diff(np.log(e), 2), 0.0, atol=1e-13)
+        assert O.epsilon_schedule(1).tolist() == [0.99]
+        assert O.epsilon_schedule(0).size == 0
+        np.testing.assert_allclose(O.epsilon_schedule(3, 0.9, 0.9), 0.9, rtol=1e-15)
+
+    def test_golden_intervals_and_bitmap(self):
+        g = golden("mask_encodings.json")
+        ip, ix = np.asarray(g["indptr"]), np.asarray(g["indices"])
+        iptr, st, en = O.lists_to_intervals(ip, ix)
+        assert iptr.tolist() == g["intervals"]["iptr"]
+        assert st.tolist() == g["intervals"]["starts"]
+        assert en.tolist() == g["intervals"]["ends"]
+        bm = O.lists_to_bitmap(ip, ix, g["n_cols"])
+        assert [[f"0x{int(w):08x}" for w in row] for row in bm] == g["bitmap_hex"]
+
+    def test_round_trips_on_random_sets(self):
+        for seed in range(20):
+            n_cols = [1, 31, 32, 33, 64, 138, 591][seed % 7]
+            ip, ix = random_lists(9, n_cols, seed)
+            iptr, st, en = O.lists_to_intervals(ip, ix)
+            ip2, ix2 = O.intervals_to_lists(iptr, st, en)
+            assert ip2.tolist() == ip.tolist() and ix2.tolist() == ix.tolist()
+            # maximal runs: no two intervals of a row touch
+            for r in range(len(iptr) - 1):
+                for t in range(iptr[r] + 1, iptr[r + 1]):
+                    assert st[t] > en[t - 1]
+            bm = O.lists_to_bitmap(ip, ix, n_cols)
+            ip3, ix3 = O.bitmap_to_lists(bm, n_cols)
+            assert ip3.tolist() == ip.tolist() and ix3.tolist() == ix.tolist()
+            # popcount of the bitmap = number of kept blocks
+            assert sum(bin(int(w)).count("1") for w in bm.ravel()) == len(ix)
+
+    def test_bitmap_is_32x_smaller_than_an_int32_mask(self):
+        # [CAL] 3.3: bitmap storage of the mask takes 32x less memory than one
+        # 32-bit value per (query block, key block)
+        for n_cols in (32, 64, 640):
+            ip, ix = random_lists(5, n_cols, n_cols)
+            bm = O.lists_to_bitmap(ip, ix, n_cols)
+            assert bm.nbytes * 32 == 5 * n_cols * 4
+
+    def test_duplicates_and_unsorted_rows_become_sets(self):
+        iptr, st, en = O.lists_to_intervals(np.array([0, 5]), np.array([4, 2, 3, 3, 9]))
+        assert st.tolist() == [2, 9] and en.tolist() == [5, 10]
