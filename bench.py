@@ -273,6 +273,33 @@ def run_ours(args, rank, world, local_rank):
     unf_avg = float(sum(e[0].elapsed_time(e[1]) for e in unf_ev) / K)
     del tmp
 
+    # mask encodings of the layer's three lists ([CAL] 3.3): skip list and bitmap
+    rows = 3 * nb
+    ix_host = lists.indices.cpu().numpy()
+    segs = [ix_host[ip[kk][r]:ip[kk][r + 1]] for kk in range(3) for r in range(nb)]
+    ip_all = torch.from_numpy(np.cumsum([0] + [len(x) for x in segs]).astype(np.int32)).to(dev)
+    ix_all = torch.from_numpy(np.concatenate(segs).astype(np.int32)).to(dev)
+    enc = {}
+    for kind, fn in (("intervals", lambda: svg.svg_lists_to_intervals(ip_all, ix_all, nb)),
+                     ("bitmap", lambda: svg.svg_lists_to_bitmap(ip_all, ix_all, nb))):
+        fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(10):
+            res = fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        enc[kind] = (e0.elapsed_time(e1) / 10 * 1e3, res)
+    iptr_e, starts_e, _ = enc["intervals"][1]
+    encodings = {"rows": rows, "csr_bytes": int(4 * (rows + 1 + ix_all.numel())),
+                 "intervals_bytes": int(4 * (rows + 1 + 2 * starts_e.numel())),
+                 "bitmap_bytes": int(enc["bitmap"][1].numel() * 4),
+                 "int32_mask_bytes": int(rows * nb * 4),
+                 "intervals_us": round(enc["intervals"][0], 2),
+                 "bitmap_us": round(enc["bitmap"][0], 2),
+                 "note": "host-synchronising size query included in intervals_us"}
+
     # end to end through the public API with host buffers
     out_host = torch.empty(qd.shape, dtype=torch.bfloat16).pin_memory()
     mode_host = torch.empty(modes.shape, dtype=torch.int32).pin_memory()
@@ -339,6 +366,7 @@ def run_ours(args, rank, world, local_rank):
         "attention_only": {"ms": round(attn_avg, 5), "effective_tflops": round(attn_tf, 3),
                            "kernel": "svg_sparse_attn_fused (output fused)"},
         "step_permutes_ms": round(fwd_perm_avg, 5),
+        "mask_encodings": encodings,
         "unfused_layer_ms": round(unf_avg, 5),
         # the permutation kernel alone: one [B,H,N,d] tensor, every head
         # reordered, 2 * B*H*N*d * 2 bytes, L2 flushed before each launch

@@ -249,6 +249,50 @@ svg_status svg_build_block_mask_calibrated(const float* energy, int R, int L,
                                            void* stream);
 
 /* --------------------------------------------------------------------------
+ * 3c. Threshold schedule and mask encodings
+ *    [CAL] section 3.1: the energy threshold eps(t) of the calibration decays
+ *    exponentially over the denoising steps, about 0.99 at the first and
+ *    0.84 at the last; section 3.3: the sparse mask is precomputed as a skip
+ *    list of contiguous block intervals and stored as a bitmap (32x less
+ *    memory than one 32-bit value per block pair).
+ *
+ *  svg_epsilon_schedule (host only, no device work):
+ *    eps_out[i] = eps_first * (eps_last / eps_first)^(i / (n_steps - 1)),
+ *    i in [0, n_steps); one step gives eps_first.  eps_out is a HOST array of
+ *    n_steps doubles; thresholds must lie in (0, 1].  Feed eps_out[t] to
+ *    svg_build_block_mask_calibrated for the lists of step t.
+ *
+ *  svg_lists_to_intervals:
+ *    indptr / indices  device CSR of n_rows rows over n_cols key blocks,
+ *                      indices ascending within a row (duplicates allowed);
+ *    iptr     device int32 [n_rows + 1]: row r's runs are
+ *             [iptr[r], iptr[r + 1]) of starts / ends;
+ *    starts, ends  device int32 [capacity]: maximal runs of consecutive kept
+ *             blocks, half-open [start, end), ascending;
+ *    n_out    device int64: total runs (written in every case);
+ *    capacity 0 is a size query (only iptr and n_out are written).
+ *    Indices outside [0, n_cols) or a descending row set
+ *    SVG_DEVICE_BAD_INDEX (the row's runs are then unspecified); runs past
+ *    capacity are dropped and set SVG_DEVICE_CAPACITY.
+ *
+ *  svg_lists_to_bitmap:
+ *    bitmap   device uint32 [n_rows][ceil(n_cols / 32)]: block c of row r is
+ *             bit (c mod 32) of word (c div 32); every word is written.
+ *    Indices outside [0, n_cols) are skipped and set SVG_DEVICE_BAD_INDEX.
+ * Integer work: bit-exact.
+ * ------------------------------------------------------------------------ */
+svg_status svg_epsilon_schedule(int n_steps, double eps_first, double eps_last, double* eps_out);
+
+svg_status svg_lists_to_intervals(int n_rows, int n_cols, const int32_t* indptr,
+                                  const int32_t* indices, int32_t* iptr, int32_t* starts,
+                                  int32_t* ends, int64_t capacity, int64_t* n_out,
+                                  int32_t* device_status, void* stream);
+
+svg_status svg_lists_to_bitmap(int n_rows, int n_cols, const int32_t* indptr,
+                               const int32_t* indices, uint32_t* bitmap, int32_t* device_status,
+                               void* stream);
+
+/* --------------------------------------------------------------------------
  * 4. Block-sparse attention
  *    [SURV] section 2.1 (softmax(Q K^T / sqrt(d)) V), [CAL] sections 2.2 and
  *    3.3 (128x128 tiles, per-query-block list of kept key blocks).  For every

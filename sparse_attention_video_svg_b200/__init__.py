@@ -22,6 +22,8 @@ from __future__ import annotations
 
 from typing import NamedTuple, Optional, Sequence
 
+import ctypes as C
+
 import torch
 
 from . import _lib
@@ -32,7 +34,9 @@ __all__ = [
     "SVG_MODE_SPATIAL", "SVG_MODE_TEMPORAL", "SVG_MODE_DENSE", "SVG_TILE", "SvgError",
     "BlockLists", "svg_version", "svg_profile_heads", "svg_permute_token_major",
     "svg_permute_frame_major", "svg_build_block_mask", "svg_block_energy",
-    "svg_build_block_mask_calibrated", "svg_sparse_attn", "geometric_lists", "svg_layer",
+    "svg_build_block_mask_calibrated", "svg_sparse_attn", "svg_sparse_attn_fused",
+    "svg_epsilon_schedule", "svg_lists_to_intervals", "svg_lists_to_bitmap", "geometric_lists",
+    "svg_layer",
     "n_tiles",
 ]
 
@@ -222,6 +226,47 @@ def svg_sparse_attn_fused(q, k, v, frames: int, tokens_per_frame: int, mode: tor
               _dt(q), B, H, N, d, frames, tokens_per_frame, mode.data_ptr(), int(layout),
               lists.n_lists, lists.n_qblocks, lists.indptr.data_ptr(), lists.indices.data_ptr(),
               float(scale), _ptr(status), _stream(stream))
+    return out
+
+
+# ------------------------------------------- threshold schedule, mask encodings
+
+def svg_epsilon_schedule(n_steps: int, eps_first: float = 0.99, eps_last: float = 0.84):
+    """Energy threshold for each denoising step (host computation)."""
+    out = (C.c_double * max(n_steps, 1))()
+    _lib.call("svg_epsilon_schedule", int(n_steps), float(eps_first), float(eps_last),
+              C.cast(out, C.c_void_p))
+    return [out[i] for i in range(n_steps)]
+
+
+def svg_lists_to_intervals(indptr: torch.Tensor, indices: torch.Tensor, n_cols: int, *,
+                           status=None, stream=None):
+    """CSR rows -> skip list of maximal block runs: (iptr, starts, ends)."""
+    n_rows = indptr.numel() - 1
+    dev = indptr.device
+    iptr = torch.empty(n_rows + 1, dtype=torch.int32, device=dev)
+    n = torch.zeros(1, dtype=torch.int64, device=dev)
+    _lib.call("svg_lists_to_intervals", n_rows, int(n_cols), indptr.data_ptr(),
+              indices.data_ptr(), iptr.data_ptr(), None, None, 0, n.data_ptr(), _ptr(status),
+              _stream(stream))
+    cap = max(int(n.item()), 1)
+    starts = torch.empty(cap, dtype=torch.int32, device=dev)
+    ends = torch.empty(cap, dtype=torch.int32, device=dev)
+    _lib.call("svg_lists_to_intervals", n_rows, int(n_cols), indptr.data_ptr(),
+              indices.data_ptr(), iptr.data_ptr(), starts.data_ptr(), ends.data_ptr(), cap,
+              n.data_ptr(), _ptr(status), _stream(stream))
+    total = int(n.item())
+    return iptr, starts[:total], ends[:total]
+
+
+def svg_lists_to_bitmap(indptr: torch.Tensor, indices: torch.Tensor, n_cols: int, *,
+                        out=None, status=None, stream=None):
+    """CSR rows -> bitmap, uint32 words [rows][ceil(n_cols / 32)] (as int32)."""
+    n_rows = indptr.numel() - 1
+    if out is None:
+        out = torch.empty(n_rows, (n_cols + 31) // 32, dtype=torch.int32, device=indptr.device)
+    _lib.call("svg_lists_to_bitmap", n_rows, int(n_cols), indptr.data_ptr(), indices.data_ptr(),
+              out.data_ptr(), _ptr(status), _stream(stream))
     return out
 
 

@@ -1,6 +1,6 @@
 """ctypes loader of libsvg_b200.so with the C ABI signatures of include/svg.h.
 
-The library is built in-tree (``python -m sparse_attention_video_svg_b200.build``).
+The library is built in-tree (``python sparse_attention_video_svg_b200/build.py``).
 There is no fallback: if the shared library is missing, importing this module
 raises."""
 from __future__ import annotations
@@ -44,6 +44,9 @@ SIGNATURES = {
     "svg_build_block_mask_calibrated": (_i, [_p, _i, _i, _i, _i, _d, _d, _p, _p, _i64, _p, _p, _p,
                                              _sz, _p]),
     "svg_sparse_attn": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _i, _p, _i, _i, _p, _p, _f, _p, _p]),
+    "svg_epsilon_schedule": (_i, [_i, C.c_double, C.c_double, _p]),
+    "svg_lists_to_intervals": (_i, [_i, _i, _p, _p, _p, _p, _p, C.c_int64, _p, _p, _p]),
+    "svg_lists_to_bitmap": (_i, [_i, _i, _p, _p, _p, _p, _p]),
     "svg_sparse_attn_fused": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p, _i, _i, _i, _p,
                                    _p, _f, _p, _p]),
 }
@@ -58,7 +61,7 @@ class SvgError(RuntimeError):
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is missing; build it with `python -m sparse_attention_video_svg_b200.build`"
+            f"{LIB_PATH} is missing; build it with `python sparse_attention_video_svg_b200/build.py`"
             " (there is no CPU fallback)")
     lib = C.CDLL(LIB_PATH)
     for name, (res, args) in SIGNATURES.items():

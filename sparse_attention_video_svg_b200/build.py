@@ -1,6 +1,7 @@
 """Builds libsvg_b200.so in-tree with nvcc for sm_100a.
 
-Usage: python -m sparse_attention_video_svg_b200.build [--force] [--ptxas-v]
+Usage: python sparse_attention_video_svg_b200/build.py [--force] [--ptxas-v]
+(run as a file: importing the package loads the library this builds)
 """
 from __future__ import annotations
 

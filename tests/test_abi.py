@@ -6,6 +6,7 @@ import ctypes as C
 import os
 import re
 
+import numpy as np
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -122,3 +123,27 @@ class TestHostValidation:
     def test_block_energy(self):
         expect(INVALID, "svg_block_energy", FAKE, FAKE2, 0, 1, 2, 256, 64, FAKE3, FAKE4 * 2, 10,
                None, match="workspace")
+
+
+def test_epsilon_schedule_host_matches_oracle():
+    """svg_epsilon_schedule runs on the host: same values as the oracle's
+    schedule (libm pow against NumPy's, a few ulp at most)."""
+    import ctypes as C
+
+    from oracle import svg_oracle as O
+    for n, a, b in ((50, 0.99, 0.84), (1, 0.99, 0.84), (7, 0.95, 0.5), (2, 1.0, 0.9)):
+        out = (C.c_double * n)()
+        assert L.svg_epsilon_schedule(n, a, b, C.cast(out, C.c_void_p)) == _lib.SVG_OK
+        np.testing.assert_allclose(list(out), O.epsilon_schedule(n, a, b), rtol=4e-16)
+    out = (C.c_double * 1)()
+    assert L.svg_epsilon_schedule(3, 1.5, 0.8, C.cast(out, C.c_void_p)) == INVALID
+    assert L.svg_epsilon_schedule(-1, 0.9, 0.8, C.cast(out, C.c_void_p)) == INVALID
+
+
+def test_encoding_validation():
+    expect(INVALID, "svg_lists_to_intervals", 0, 10, FAKE, FAKE2, FAKE3, FAKE4, FAKE4 * 2, 8,
+           FAKE4 * 3, None, None, match="bad sizes")
+    expect(INVALID, "svg_lists_to_intervals", 3, 10, FAKE, FAKE2, FAKE3, None, None, 8,
+           FAKE4 * 3, None, None, match="null starts")
+    expect(INVALID, "svg_lists_to_bitmap", 3, 0, FAKE, FAKE2, FAKE3, None, None, match="bad sizes")
+    expect(INVALID, "svg_lists_to_bitmap", 3, 10, FAKE, None, FAKE3, None, None, match="null")

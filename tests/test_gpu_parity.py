@@ -482,3 +482,77 @@ def test_calibration_end_to_end_small():
         hx = ix[ip[h][0]:ip[h][-1]]
         ref = O.block_sparse_attention(head64(q, 0, h), head64(k, 0, h), head64(v, 0, h), hp, hx)
         assert_close(o[0, h], ref, f"calibrated head {h}")
+
+
+# ------------------------------------------------ mask encodings (skip list, bitmap)
+
+def _rand_csr(rows, n_cols, seed, dup=False):
+    rng = np.random.default_rng(seed)
+    ip, ix = [0], []
+    for _ in range(rows):
+        k = int(rng.integers(0, min(n_cols, 80) + 1))
+        r = sorted(rng.choice(n_cols, size=k, replace=False).tolist())
+        if dup and r:
+            r = sorted(r + rng.choice(r, size=min(3, len(r))).tolist())
+        ix.extend(r)
+        ip.append(len(ix))
+    return np.asarray(ip, np.int32), np.asarray(ix, np.int32)
+
+
+def _check_encodings(ip, ix, n_cols, what):
+    ipd = torch.from_numpy(ip).to(DEV)
+    ixd = torch.from_numpy(ix if ix.size else np.zeros(1, np.int32)).to(DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    iptr, st, en = svg.svg_lists_to_intervals(ipd, ixd, n_cols, status=status)
+    bm = svg.svg_lists_to_bitmap(ipd, ixd, n_cols, status=status)
+    assert status.item() == 0, what
+    r_iptr, r_st, r_en = O.lists_to_intervals(ip, ix)
+    np.testing.assert_array_equal(iptr.cpu().numpy(), r_iptr, err_msg=what)
+    np.testing.assert_array_equal(st.cpu().numpy(), r_st, err_msg=what)
+    np.testing.assert_array_equal(en.cpu().numpy(), r_en, err_msg=what)
+    np.testing.assert_array_equal(bm.cpu().numpy().view(np.uint32),
+                                  O.lists_to_bitmap(ip, ix, n_cols), err_msg=what)
+
+
+@pytest.mark.parametrize("n_cols", [1, 31, 32, 33, 138, 929, 2000])
+def test_encodings_random(n_cols):
+    ip, ix = _rand_csr(300, n_cols, n_cols)
+    _check_encodings(ip, ix, n_cols, f"random n_cols={n_cols}")
+    ip, ix = _rand_csr(57, n_cols, n_cols + 1, dup=True)  # duplicates merge into runs
+    _check_encodings(ip, ix, n_cols, f"duplicates n_cols={n_cols}")
+
+
+@pytest.mark.parametrize("name", si.ORDER)
+def test_encodings_geometric_lists(name):
+    wl = si.WORKLOADS[name]
+    nb = svg.n_tiles(wl.N)
+    for kind in (O.MODE_SPATIAL, O.MODE_TEMPORAL, O.MODE_DENSE):
+        ip, ix = O.geometric_block_lists(kind, wl.F, wl.P, wl.width, wl.N)
+        _check_encodings(ip, ix, nb, f"{name} kind {kind}")
+
+
+def test_encodings_capacity_and_bad_index():
+    ip, ix = _rand_csr(40, 100, 3)
+    ipd, ixd = torch.from_numpy(ip).to(DEV), torch.from_numpy(ix).to(DEV)
+    n_runs = len(O.lists_to_intervals(ip, ix)[1])
+    iptr = torch.empty(41, dtype=torch.int32, device=DEV)
+    starts = torch.full((n_runs - 1,), -7, dtype=torch.int32, device=DEV)
+    ends = torch.full((n_runs - 1,), -7, dtype=torch.int32, device=DEV)
+    n = torch.zeros(1, dtype=torch.int64, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    svg._lib.call("svg_lists_to_intervals", 40, 100, ipd.data_ptr(), ixd.data_ptr(),
+                  iptr.data_ptr(), starts.data_ptr(), ends.data_ptr(), n_runs - 1, n.data_ptr(),
+                  status.data_ptr(), None)
+    assert status.item() & svg._lib.SVG_DEVICE_CAPACITY and n.item() == n_runs
+    _, r_st, r_en = O.lists_to_intervals(ip, ix)
+    np.testing.assert_array_equal(starts.cpu().numpy(), r_st[:n_runs - 1])
+    np.testing.assert_array_equal(ends.cpu().numpy(), r_en[:n_runs - 1])
+    bad = ix.copy()
+    bad[5] = 100  # outside [0, n_cols)
+    status.zero_()
+    bm = svg.svg_lists_to_bitmap(ipd, torch.from_numpy(bad).to(DEV), 100, status=status)
+    assert status.item() & svg._lib.SVG_DEVICE_BAD_INDEX
+    good = np.delete(bad, 5)
+    ip2 = ip.copy()
+    ip2[np.searchsorted(ip, 5, side="right"):] -= 1
+    np.testing.assert_array_equal(bm.cpu().numpy().view(np.uint32), O.lists_to_bitmap(ip2, good, 100))
