@@ -342,8 +342,14 @@ svg_status svg_sparse_attn(const void* q, const void* k, const void* v, void* o,
  *      SVG_FUSE_OUTPUT  o is written FRAME-MAJOR for every head (otherwise
  *                       temporal heads' o is token-major).
  *    layout 0 is svg_sparse_attn with list_id = mode.
+ *    Token-major copies: q_tm, k_tm, v_tm (all three or none; not with
+ *    SVG_FUSE_INPUT) hold every head in token-major order, e.g. from
+ *    svg_permute_token_major with mode NULL; temporal heads read them and the
+ *    other heads read q, k, v (frame-major).  The copies then do not depend
+ *    on the modes, so they can be made while the heads are being profiled.
  *
  *  q, k, v, o   device [B, H, N, d] in the layouts above.
+ *  q_tm, k_tm, v_tm   device [B, H, N, d] or NULL.
  *  frames, tokens_per_frame   F and P with F * P == N (unused for layout 0).
  *  mode         device int32 [B*H]: the list id of each head (as list_id in
  *               svg_sparse_attn, e.g. the profiling output with the three
@@ -353,11 +359,13 @@ svg_status svg_sparse_attn(const void* q, const void* k, const void* v, void* o,
  *  outside [0, n_lists) sets SVG_DEVICE_BAD_LIST_ID and gives o = 0 for the
  *  head.
  * ------------------------------------------------------------------------ */
-svg_status svg_sparse_attn_fused(const void* q, const void* k, const void* v, void* o, int dtype,
-                                 int B, int H, int N, int d, int frames, int tokens_per_frame,
-                                 const int32_t* mode, int layout, int n_lists, int n_qblocks,
-                                 const int32_t* indptr, const int32_t* indices,
-                                 float scale, int32_t* device_status, void* stream);
+svg_status svg_sparse_attn_fused(const void* q, const void* k, const void* v,
+                                 const void* q_tm, const void* k_tm, const void* v_tm, void* o,
+                                 int dtype, int B, int H, int N, int d, int frames,
+                                 int tokens_per_frame, const int32_t* mode, int layout,
+                                 int n_lists, int n_qblocks, const int32_t* indptr,
+                                 const int32_t* indices, float scale, int32_t* device_status,
+                                 void* stream);
 
 #ifdef __cplusplus
 }

@@ -214,18 +214,21 @@ def svg_sparse_attn(q, k, v, list_id: torch.Tensor, lists: BlockLists, *, scale:
 
 
 def svg_sparse_attn_fused(q, k, v, frames: int, tokens_per_frame: int, mode: torch.Tensor,
-                          lists: BlockLists, *, layout: int = 3, scale: float = 0.0, out=None,
-                          status=None, stream=None):
+                          lists: BlockLists, *, layout: int = 3, copies=None, scale: float = 0.0,
+                          out=None, status=None, stream=None):
     """Block-sparse attention with the token-major reordering of temporal
     heads fused in: layout bit 1 (SVG_FUSE_INPUT) gathers q, k, v from
-    frame-major memory, bit 2 (SVG_FUSE_OUTPUT) writes o frame-major."""
+    frame-major memory, bit 2 (SVG_FUSE_OUTPUT) writes o frame-major.
+    copies = (q_tm, k_tm, v_tm): token-major copies of every head, read by
+    the temporal heads instead (q, k, v then frame-major)."""
     B, H, N, d = _check_qkv(q, k, v)
     if out is None:
         out = torch.empty_like(q)
-    _lib.call("svg_sparse_attn_fused", q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-              _dt(q), B, H, N, d, frames, tokens_per_frame, mode.data_ptr(), int(layout),
-              lists.n_lists, lists.n_qblocks, lists.indptr.data_ptr(), lists.indices.data_ptr(),
-              float(scale), _ptr(status), _stream(stream))
+    qt, kt, vt = (None, None, None) if copies is None else (c.data_ptr() for c in copies)
+    _lib.call("svg_sparse_attn_fused", q.data_ptr(), k.data_ptr(), v.data_ptr(), qt, kt, vt,
+              out.data_ptr(), _dt(q), B, H, N, d, frames, tokens_per_frame, mode.data_ptr(),
+              int(layout), lists.n_lists, lists.n_qblocks, lists.indptr.data_ptr(),
+              lists.indices.data_ptr(), float(scale), _ptr(status), _stream(stream))
     return out
 
 
@@ -282,6 +285,9 @@ class LayerBuffers:
             self.qp = torch.empty_like(q)
             self.kp = torch.empty_like(q)
             self.vp = torch.empty_like(q)
+            # the copies of every head are made on this stream while the
+            # heads are profiled
+            self.side = torch.cuda.Stream(device=dev) if dev.type == "cuda" else None
         if not layout & _lib.SVG_FUSE_OUTPUT:  # token-major output
             self.op = torch.empty_like(q)
         self.o = torch.empty_like(q)
@@ -292,17 +298,46 @@ class LayerBuffers:
 
 def svg_layer(q, k, v, frames: int, tokens_per_frame: int, spatial_width: int,
               sample_idx: torch.Tensor, lists: BlockLists, bufs: Optional[LayerBuffers] = None,
-              stream=None, layout: int = _lib.SVG_FUSE_OUTPUT):
+              stream=None, layout: int = _lib.SVG_FUSE_OUTPUT, overlap: bool = True):
     """One attention layer: profile -> block-sparse attention on the list the
     mode selects, temporal heads in token-major order.  `layout` picks which
     side of the reordering runs inside the attention kernel
     (svg_sparse_attn_fused); the other side runs as permutation kernels.
     The default fuses only the output side: on B200 the permutation kernel
-    moves q, k, v faster than row gathers inside the attention kernel.
+    moves q, k, v faster than row gathers inside the attention kernel.  With
+    overlap (input side not fused), the token-major copies of every head are
+    made on a side stream while the heads are profiled.
     Returns (o, mode, mse)."""
     if bufs is None:
-        bufs = LayerBuffers(q, sample_idx.numel())
+        bufs = LayerBuffers(q, sample_idx.numel(), layout)
     F, P = frames, tokens_per_frame
+    if overlap and not layout & _lib.SVG_FUSE_INPUT:
+        # token-major copies of every head on a side stream, concurrent with
+        # the (latency-bound) profiling; temporal heads read the copies
+        if stream is None:
+            main = torch.cuda.current_stream()
+        elif hasattr(stream, "wait_event"):
+            main = stream
+        else:  # a raw cudaStream_t handle
+            main = torch.cuda.ExternalStream(int(stream), device=q.device)
+        ready = torch.cuda.Event()
+        ready.record(main)
+        bufs.side.wait_event(ready)
+        for x, y in ((q, bufs.qp), (k, bufs.kp), (v, bufs.vp)):
+            svg_permute_token_major(x, F, P, None, out=y, stream=bufs.side)
+        copied = torch.cuda.Event()
+        copied.record(bufs.side)
+        svg_profile_heads(q, k, v, F, P, spatial_width, sample_idx, mse_out=bufs.mse,
+                          mode_out=bufs.mode, workspace=bufs.ws, stream=main)
+        main.wait_event(copied)
+        for t in (bufs.qp, bufs.kp, bufs.vp):
+            t.record_stream(main)
+        out = bufs.o if layout & _lib.SVG_FUSE_OUTPUT else bufs.op
+        svg_sparse_attn_fused(q, k, v, F, P, bufs.mode, lists, layout=layout,
+                              copies=(bufs.qp, bufs.kp, bufs.vp), out=out, stream=main)
+        if not layout & _lib.SVG_FUSE_OUTPUT:
+            svg_permute_frame_major(bufs.op, F, P, bufs.mode, out=bufs.o, stream=main)
+        return bufs.o, bufs.mode, bufs.mse
     svg_profile_heads(q, k, v, F, P, spatial_width, sample_idx, mse_out=bufs.mse,
                       mode_out=bufs.mode, workspace=bufs.ws, stream=stream)
     if layout & _lib.SVG_FUSE_INPUT:

@@ -47,8 +47,8 @@ SIGNATURES = {
     "svg_epsilon_schedule": (_i, [_i, C.c_double, C.c_double, _p]),
     "svg_lists_to_intervals": (_i, [_i, _i, _p, _p, _p, _p, _p, C.c_int64, _p, _p, _p]),
     "svg_lists_to_bitmap": (_i, [_i, _i, _p, _p, _p, _p, _p]),
-    "svg_sparse_attn_fused": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p, _i, _i, _i, _p,
-                                   _p, _f, _p, _p]),
+    "svg_sparse_attn_fused": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p,
+                                   _i, _i, _i, _p, _p, _f, _p, _p]),
 }
 
 

@@ -27,7 +27,16 @@ struct AttnArgs {
   const int32_t* order;
   int frames, tokens_per_frame;
   int layout;
+  // Optional token-major copies of q, k, v (every head reordered, e.g. by
+  // svg_permute_token_major with no mode): heads whose order is
+  // SVG_MODE_TEMPORAL read these, the others read q, k, v.  Set together or
+  // not at all; exclusive with SVG_FUSE_INPUT.
+  const void* q_tm;
+  const void* k_tm;
+  const void* v_tm;
 };
+
+__device__ __forceinline__ bool reads_copies(const AttnArgs& a, int bh);
 
 __device__ __forceinline__ bool temporal_head(const AttnArgs& a, int bh) {
   return a.order != nullptr && a.order[bh] == SVG_MODE_TEMPORAL;
@@ -37,6 +46,9 @@ __device__ __forceinline__ bool gathers_input(const AttnArgs& a, int bh) {
 }
 __device__ __forceinline__ bool scatters_output(const AttnArgs& a, int bh) {
   return (a.layout & SVG_FUSE_OUTPUT) != 0 && temporal_head(a, bh);
+}
+__device__ __forceinline__ bool reads_copies(const AttnArgs& a, int bh) {
+  return a.q_tm != nullptr && temporal_head(a, bh);
 }
 
 // Frame-major memory row of token-major row m.

@@ -12,7 +12,7 @@ svg_status sparse_attn_impl(const char* who, const void* q, const void* k, const
                             int n_lists, int n_qblocks, const int32_t* indptr,
                             const int32_t* indices, float scale, int32_t* device_status,
                             const int32_t* order, int frames, int tokens_per_frame, int layout,
-                            void* stream) {
+                            const void* q_tm, const void* k_tm, const void* v_tm, void* stream) {
   clear_error();
   if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || list_id == nullptr ||
       indptr == nullptr || indices == nullptr)
@@ -32,11 +32,18 @@ svg_status sparse_attn_impl(const char* who, const void* q, const void* k, const
       (frames <= 0 || tokens_per_frame <= 0 ||
        static_cast<long long>(frames) * tokens_per_frame != N))
     return fail(SVG_ERR_INVALID_ARG, "%s: frames * tokens_per_frame must equal N", who);
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+  const bool copies = q_tm != nullptr || k_tm != nullptr || v_tm != nullptr;
+  if (copies && (q_tm == nullptr || k_tm == nullptr || v_tm == nullptr))
+    return fail(SVG_ERR_INVALID_ARG, "%s: give all three token-major copies or none", who);
+  if (copies && (layout & SVG_FUSE_INPUT) != 0)
+    return fail(SVG_ERR_INVALID_ARG, "%s: token-major copies exclude SVG_FUSE_INPUT", who);
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (copies && (!aligned16(q_tm) || !aligned16(k_tm) || !aligned16(v_tm))))
     return fail(SVG_ERR_INVALID_ARG, "%s: tensors must be 16-byte aligned", who);
   const long long bytes = static_cast<long long>(B) * H * N * d * elt_bytes(dtype);
   const char* ob = static_cast<const char*>(o);
-  for (const void* t : {q, k, v}) {
+  for (const void* t : {q, k, v, q_tm, k_tm, v_tm}) {
+    if (t == nullptr) continue;
     const char* tb = static_cast<const char*>(t);
     if (ob < tb + bytes && tb < ob + bytes)
       return fail(SVG_ERR_INVALID_ARG, "%s: o overlaps an input", who);
@@ -44,7 +51,7 @@ svg_status sparse_attn_impl(const char* who, const void* q, const void* k, const
   if (!(scale >= 0.f) || isinf(scale)) return fail(SVG_ERR_INVALID_ARG, "%s: bad scale", who);
   AttnArgs a{q, k, v, o, dtype, B, H, N, d, list_id, n_lists, n_qblocks, indptr, indices,
              scale == 0.f ? 1.f / sqrtf(static_cast<float>(d)) : scale, device_status,
-             order, frames, tokens_per_frame, layout};
+             order, frames, tokens_per_frame, layout, q_tm, k_tm, v_tm};
   cudaStream_t s = as_stream(stream);
   if (dtype == SVG_FP32) return d == 64 ? launch_attn_fp32<64>(a, s) : launch_attn_fp32<128>(a, s);
   return d == 64 ? launch_attn_sm100<64>(a, s) : launch_attn_sm100<128>(a, s);
@@ -58,16 +65,19 @@ extern "C" svg_status svg_sparse_attn(const void* q, const void* k, const void* 
                                       const int32_t* indptr, const int32_t* indices, float scale,
                                       int32_t* device_status, void* stream) {
   return sparse_attn_impl("sparse_attn", q, k, v, o, dtype, B, H, N, d, list_id, n_lists,
-                          n_qblocks, indptr, indices, scale, device_status, nullptr, 0, 0, 0, stream);
+                          n_qblocks, indptr, indices, scale, device_status, nullptr, 0, 0, 0,
+                          nullptr, nullptr, nullptr, stream);
 }
 
-extern "C" svg_status svg_sparse_attn_fused(const void* q, const void* k, const void* v, void* o,
-                                            int dtype, int B, int H, int N, int d, int frames,
-                                            int tokens_per_frame, const int32_t* mode,
-                                            int layout, int n_lists, int n_qblocks,
-                                            const int32_t* indptr, const int32_t* indices,
-                                            float scale, int32_t* device_status, void* stream) {
+extern "C" svg_status svg_sparse_attn_fused(const void* q, const void* k, const void* v,
+                                            const void* q_tm, const void* k_tm,
+                                            const void* v_tm, void* o, int dtype, int B, int H,
+                                            int N, int d, int frames, int tokens_per_frame,
+                                            const int32_t* mode, int layout, int n_lists,
+                                            int n_qblocks, const int32_t* indptr,
+                                            const int32_t* indices, float scale,
+                                            int32_t* device_status, void* stream) {
   return sparse_attn_impl("sparse_attn_fused", q, k, v, o, dtype, B, H, N, d, mode, n_lists,
                           n_qblocks, indptr, indices, scale, device_status, mode, frames,
-                          tokens_per_frame, layout, stream);
+                          tokens_per_frame, layout, q_tm, k_tm, v_tm, stream);
 }

@@ -41,9 +41,10 @@ __global__ void __launch_bounds__(256) attn_fp32(AttnArgs a) {
   const int qt = blockIdx.x, bh = blockIdx.y;
   const int N = a.N, nb = n_tiles(N);
   const long long head = static_cast<long long>(bh) * N * D;
-  auto* q = static_cast<const float*>(a.q) + head;
-  auto* k = static_cast<const float*>(a.k) + head;
-  auto* v = static_cast<const float*>(a.v) + head;
+  const bool copies = reads_copies(a, bh);
+  auto* q = static_cast<const float*>(copies ? a.q_tm : a.q) + head;
+  auto* k = static_cast<const float*>(copies ? a.k_tm : a.k) + head;
+  auto* v = static_cast<const float*>(copies ? a.v_tm : a.v) + head;
   auto* o = static_cast<float*>(a.o) + head;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const RowList lst = row_list(a, bh, qt);

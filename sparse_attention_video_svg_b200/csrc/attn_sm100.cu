@@ -99,6 +99,7 @@ struct Cfg {
 
 struct Maps {
   CUtensorMap q, k, v;
+  CUtensorMap qt, kt, vt;  // token-major copies (encoded only when given)
 };
 
 struct Bars {
@@ -438,6 +439,10 @@ __device__ __forceinline__ void producer(const AttnArgs& a, const Maps& maps, co
   for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
     const int bh = item / n_pairs, qt0 = 2 * (item - bh * n_pairs);
     const bool tm = gathers_input(a, bh);
+    const bool cp = reads_copies(a, bh);
+    const CUtensorMap* mq = cp ? &maps.qt : &maps.q;
+    const CUtensorMap* mk = cp ? &maps.kt : &maps.k;
+    const CUtensorMap* mv = cp ? &maps.vt : &maps.v;
     const long long head = static_cast<long long>(bh) * N * D;
     int p[2], e[2];
 #pragma unroll
@@ -455,7 +460,7 @@ __device__ __forceinline__ void producer(const AttnArgs& a, const Maps& maps, co
         if (leader) {
           mbar_arrive_expect_tx(&B.q_full[qb], C::kTile);
           for (int bx = 0; bx < C::kBoxes; ++bx)
-            tma_load_3d(dst + bx * kBox, &maps.q, &B.q_full[qb], 64 * bx, (qt0 + t) * 128, bh);
+            tma_load_3d(dst + bx * kBox, mq, &B.q_full[qb], 64 * bx, (qt0 + t) * 128, bh);
         }
       } else {
         gather_into(dst, static_cast<const __nv_bfloat16*>(a.q) + head, (qt0 + t) * 128,
@@ -480,7 +485,7 @@ __device__ __forceinline__ void producer(const AttnArgs& a, const Maps& maps, co
         if (!tm) {
           if (leader) {
             mbar_arrive_expect_tx(&B.kv_full[slot], C::kTile);
-            const CUtensorMap* map = kv == 0 ? &maps.k : &maps.v;
+            const CUtensorMap* map = kv == 0 ? mk : mv;
             for (int bx = 0; bx < C::kBoxes; ++bx)
               tma_load_3d(dst + bx * kBox, map, &B.kv_full[slot], 64 * bx, j * 128, bh);
           }
@@ -566,6 +571,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&maps.q);
     prefetch_tmap(&maps.k);
     prefetch_tmap(&maps.v);
+    if (a.q_tm != nullptr) {
+      prefetch_tmap(&maps.qt);
+      prefetch_tmap(&maps.kt);
+      prefetch_tmap(&maps.vt);
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
@@ -742,10 +752,13 @@ bool make_map(CUtensorMap* m, const void* base, int BH, int N, int d) {
 template <int D>
 svg_status launch_attn_sm100(const AttnArgs& a, cudaStream_t s) {
   using C = Cfg<D>;
-  Maps maps;
+  Maps maps = {};
   const int BH = a.B * a.H;
   if (!make_map(&maps.q, a.q, BH, a.N, D) || !make_map(&maps.k, a.k, BH, a.N, D) ||
-      !make_map(&maps.v, a.v, BH, a.N, D))
+      !make_map(&maps.v, a.v, BH, a.N, D) ||
+      (a.q_tm != nullptr &&
+       (!make_map(&maps.qt, a.q_tm, BH, a.N, D) || !make_map(&maps.kt, a.k_tm, BH, a.N, D) ||
+        !make_map(&maps.vt, a.v_tm, BH, a.N, D))))
     return fail(SVG_ERR_CUDA, "sparse_attn: cannot encode TMA descriptors");
   if (cudaFuncSetAttribute(attn_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            C::kSmem) != cudaSuccess)

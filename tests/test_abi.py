@@ -79,15 +79,20 @@ class TestHostValidation:
         expect(INVALID, "svg_sparse_attn", *([None] + base[1:]), match="null")
 
     def test_sparse_attn_fused(self):
-        # q k v o dtype B H N d F P mode layout n_lists n_qblocks indptr indices scale status
-        # stream
-        base = [FAKE, FAKE2, FAKE3, FAKE4 * 4, 0, 1, 2, 256, 64, 4, 64, FAKE, 3, 3, 2, FAKE, FAKE,
-                0.0, None, None]
-        expect(INVALID, "svg_sparse_attn_fused", *(base[:9] + [5] + base[10:]), match="frames")
-        expect(INVALID, "svg_sparse_attn_fused", *(base[:8] + [96] + base[9:]), match="d=96")
-        expect(INVALID, "svg_sparse_attn_fused", *(base[:11] + [None] + base[12:]), match="null")
-        expect(INVALID, "svg_sparse_attn_fused", *(base[:3] + [FAKE] + base[4:]), match="overlaps")
-        expect(INVALID, "svg_sparse_attn_fused", *(base[:12] + [4] + base[13:]), match="layout")
+        # q k v q_tm k_tm v_tm o dtype B H N d F P mode layout n_lists n_qblocks indptr
+        # indices scale status stream
+        base = [FAKE, FAKE2, FAKE3, None, None, None, FAKE4 * 4, 0, 1, 2, 256, 64, 4, 64, FAKE,
+                3, 3, 2, FAKE, FAKE, 0.0, None, None]
+        expect(INVALID, "svg_sparse_attn_fused", *(base[:12] + [5] + base[13:]), match="frames")
+        expect(INVALID, "svg_sparse_attn_fused", *(base[:11] + [96] + base[12:]), match="d=96")
+        expect(INVALID, "svg_sparse_attn_fused", *(base[:14] + [None] + base[15:]), match="null")
+        expect(INVALID, "svg_sparse_attn_fused", *(base[:6] + [FAKE] + base[7:]), match="overlaps")
+        expect(INVALID, "svg_sparse_attn_fused", *(base[:15] + [4] + base[16:]), match="layout")
+        expect(INVALID, "svg_sparse_attn_fused", *(base[:3] + [FAKE4 * 5] + base[4:]),
+               match="all three")
+        expect(INVALID, "svg_sparse_attn_fused",
+               *(base[:3] + [FAKE4 * 5, FAKE4 * 6, FAKE4 * 7] + base[6:15] + [1] + base[16:]),
+               match="exclude")
 
     def test_permute(self):
         args = [FAKE, FAKE4 * 4, 0, 1, 2, 12, 64, 3, 4, None, None]

@@ -306,6 +306,24 @@ def test_sparse_attn_fused_small(wl):
         assert_close(got[0, h], ref, f"{wl.name} mode {md} head {h}", bf16=wl.dtype == "bf16")
 
 
+@pytest.mark.parametrize("wl", SMALL, ids=lambda w: w.name)
+def test_sparse_attn_fused_with_copies(wl):
+    """Temporal heads read token-major copies of every head, the others the
+    frame-major inputs: same bits as the unfused composition."""
+    (q, k, v), (qd, kd, vd), _ = workload_tensors(wl)
+    lists = svg.geometric_lists(wl.F, wl.P, wl.width, wl.N)
+    modes = np.array([(O.MODE_SPATIAL, O.MODE_TEMPORAL)[h % 2] for h in range(wl.H)], np.int32)
+    mode = torch.from_numpy(modes).to(DEV)
+    copies = tuple(svg.svg_permute_token_major(x, wl.F, wl.P, None) for x in (qd, kd, vd))
+    ref = bits(_unfused(qd, kd, vd, wl.F, wl.P, mode, lists))
+    for layout in (0, FUSE_OUT):
+        o = svg.svg_sparse_attn_fused(qd, kd, vd, wl.F, wl.P, mode, lists, layout=layout,
+                                      copies=copies)
+        if not layout & FUSE_OUT:
+            o = svg.svg_permute_frame_major(o, wl.F, wl.P, mode)
+        np.testing.assert_array_equal(bits(o), ref, err_msg=f"layout {layout}")
+
+
 @pytest.mark.parametrize("name", ["wan480", "hunyuan720"])
 def test_sparse_attn_fused_full_size_sampled(name, full_inputs):
     """Token-major gathers at the full sizes (F = 21 and 33 frames)."""
@@ -373,9 +391,12 @@ def test_layer_small_layouts_agree(wl):
     idx = torch.from_numpy(si.sample_queries(wl)).to(DEV)
     lists = svg.geometric_lists(wl.F, wl.P, wl.width, wl.N)
     outs = []
-    for layout in (0, FUSE_IN, FUSE_OUT, FUSE_IN | FUSE_OUT):
+    for layout, overlap in ((0, False), (0, True), (FUSE_IN, False), (FUSE_OUT, False),
+                            (FUSE_OUT, True), (FUSE_IN | FUSE_OUT, False)):
         bufs = svg.LayerBuffers(qd, idx.numel(), layout=layout)
-        o, m, _ = svg.svg_layer(qd, kd, vd, wl.F, wl.P, wl.width, idx, lists, bufs, layout=layout)
+        o, m, _ = svg.svg_layer(qd, kd, vd, wl.F, wl.P, wl.width, idx, lists, bufs, layout=layout,
+                                overlap=overlap)
+        torch.cuda.synchronize()
         outs.append((bits(o), m.cpu().numpy()))
     for o, m in outs[1:]:
         np.testing.assert_array_equal(m, outs[0][1])
