@@ -32,6 +32,10 @@ notes):
   to the smaller block index, whose sum reaches eps; a block survives the
   cross-input vote when its keep frequency is >= rho; an empty voted row keeps
   the block of largest summed energy;
+* QK-Norm is an RMS normalisation over the head dimension with a per-channel
+  weight and an epsilon inside the square root; RoPE rotates interleaved
+  channel pairs (2i, 2i+1) by caller-supplied per-token angles (cos / sin
+  tables); QK-Norm runs first;
 * the energy threshold decays exponentially in the denoising-step index from
   0.99 (first step) to 0.84 (last step); the skip list holds each row's
   maximal runs of consecutive kept blocks; the bitmap holds one bit per
@@ -435,15 +439,64 @@ def bitmap_to_lists(bm: np.ndarray, n_cols: int):
 
 
 # ---------------------------------------------------------------------------
+# QK-Norm and rotary position embedding before attention
+#   ([SVG] "Layout Transformation + Kernel 加速": the method ships its own
+#   QK-Norm and RoPE kernels next to the attention kernels)
+# ---------------------------------------------------------------------------
+
+def qk_rms_norm(x, gamma=None, eps: float = 1e-6) -> np.ndarray:
+    """RMS normalisation of every row over the head dimension:
+    x_hat = x / sqrt(mean_c x_c^2 + eps) * gamma (gamma = 1 when None)."""
+    x = np.asarray(x, np.float64)
+    ms = np.mean(x * x, axis=-1, keepdims=True)
+    y = x / np.sqrt(ms + eps)
+    if gamma is not None:
+        y = y * np.asarray(gamma, np.float64)
+    return y
+
+
+def rope_rotate(x, cos, sin) -> np.ndarray:
+    """Rotary embedding on interleaved channel pairs: pair i of row n,
+    (a, b) = (x[n, 2i], x[n, 2i+1]), becomes (a cos - b sin, a sin + b cos)
+    with cos = cos[n, i], sin = sin[n, i].  x [..., N, d], tables [N, d/2]."""
+    x = np.asarray(x, np.float64)
+    c = np.asarray(cos, np.float64)
+    s = np.asarray(sin, np.float64)
+    a = x[..., 0::2]
+    b = x[..., 1::2]
+    y = np.empty_like(x)
+    y[..., 0::2] = a * c - b * s
+    y[..., 1::2] = a * s + b * c
+    return y
+
+
+def qk_norm_rope(x, gamma=None, eps: float = 1e-6, cos=None, sin=None,
+                 norm: bool = True, rope: bool = True) -> np.ndarray:
+    """The pre-attention transform of q or k: QK-Norm first, then RoPE
+    (either may be switched off)."""
+    y = np.asarray(x, np.float64)
+    if norm:
+        y = qk_rms_norm(y, gamma, eps)
+    if rope:
+        y = rope_rotate(y, cos, sin)
+    return y
+
+
+# ---------------------------------------------------------------------------
 # The whole layer: profile -> permute temporal heads -> block-sparse -> back
 # ---------------------------------------------------------------------------
 
-def svg_layer(q, k, v, idx, F: int, P: int, width: int, T: int = 128):
+def svg_layer(q, k, v, idx, F: int, P: int, width: int, T: int = 128, qk=None):
     """One attention layer of the method for [B, H, N, d] inputs: profile each
     head, run spatial heads on their frame-major lists, temporal heads in
     token-major order on their lists, and map temporal outputs back.
-    Returns (o [B, H, N, d], mode [B*H], mse [B*H, 2])."""
+    qk = (gamma_q, gamma_k, eps, cos, sin) first applies QK-Norm + RoPE to q
+    and k.  Returns (o [B, H, N, d], mode [B*H], mse [B*H, 2])."""
     B, H, N, d = q.shape
+    if qk is not None:
+        gq, gk, eps, cos, sin = qk
+        q = qk_norm_rope(q, gq, eps, cos, sin)
+        k = qk_norm_rope(k, gk, eps, cos, sin)
     mse, mode = profile_heads(q, k, v, idx, F, P, width)
     lists = {MODE_SPATIAL: geometric_block_lists(MODE_SPATIAL, F, P, width, N, T),
              MODE_TEMPORAL: geometric_block_lists(MODE_TEMPORAL, F, P, width, N, T)}

@@ -21,6 +21,8 @@ q/k/v are synthetic:
 The same bias vector is added to q, k and v, so q.k is large between tokens of
 one frame (spatial-type heads) or of one spatial position (temporal-type
 heads).  Tokens are frame-major: n = f * P + s with P = ph * pw tokens per frame.
+QK-Norm weights and 3D rotary tables for the fused QK-Norm + RoPE step are
+synthetic inputs too (``qk_norm_weights``, ``rope_tables``).
 All draws use numpy's PCG64 ``default_rng(seed)`` in float32; bf16 workloads
 are rounded to bf16 with round-to-nearest-even and both sides consume the
 rounded values.
@@ -195,6 +197,39 @@ def as_float64(x: np.ndarray) -> np.ndarray:
     if x.dtype == np.uint16:
         return bf16_bits_to_f32(x).astype(np.float64)
     return np.asarray(x, dtype=np.float64)
+
+
+def qk_norm_weights(wl: Workload, seed: Optional[int] = None):
+    """Per-channel QK-Norm weights gamma_q, gamma_k (float32 [d]): 1 + 0.25 z
+    with z ~ N(0, 1) from default_rng(2000 + seed), q's then k's.  Synthetic
+    stand-ins for a model's learned weights."""
+    seed = wl.seed if seed is None else seed
+    rng = np.random.default_rng(2000 + seed)
+    g = np.float32(1.0) + np.float32(0.25) * rng.standard_normal((2, wl.d), dtype=np.float32)
+    return np.ascontiguousarray(g[0]), np.ascontiguousarray(g[1])
+
+
+def rope_tables(wl: Workload, theta: float = 10000.0):
+    """3D rotary-position tables cos, sin (float32 [N, d / 2]) for frame-major
+    tokens n = f * P + y * pw + x.  The d / 2 channel pairs are split over the
+    three axes as (d / 8, 3 d / 16, 3 d / 16) pairs for (f, y, x); pair i of
+    an axis with n_a pairs turns at frequency theta^(-i / n_a), so the angle
+    is the token's coordinate on that axis times that frequency.  These are
+    inputs (a model computes them from its own positional scheme); both sides
+    read the same float32 tables."""
+    d, F, ph, pw = wl.d, wl.F, wl.ph, wl.pw
+    n_t = d // 8
+    n_y = (d // 2 - n_t) // 2
+    n_x = d // 2 - n_t - n_y
+    n = np.arange(wl.N)
+    coords = (n // (ph * pw), (n // pw) % ph, n % pw)
+    parts = []
+    for c, n_a in zip(coords, (n_t, n_y, n_x)):
+        freq = theta ** (-np.arange(n_a, dtype=np.float64) / n_a)
+        parts.append(c[:, None].astype(np.float64) * freq[None, :])
+    ang = np.concatenate(parts, axis=1)
+    return (np.ascontiguousarray(np.cos(ang).astype(np.float32)),
+            np.ascontiguousarray(np.sin(ang).astype(np.float32)))
 
 
 def sample_queries(wl: Workload, seed: Optional[int] = None) -> np.ndarray:

@@ -504,3 +504,108 @@ class TestScheduleAndEncodings:
     def test_duplicates_and_unsorted_rows_become_sets(self):
         iptr, st, en = O.lists_to_intervals(np.array([0, 5]), np.array([4, 2, 3, 3, 9]))
         assert st.tolist() == [2, 9] and en.tolist() == [5, 10]
+
+
+# ------------------------------------------------------- QK-Norm and RoPE
+
+class TestQkNormRope:
+    def test_rms_norm_matches_torch(self):
+        x = rand((7, 64), 1, 3.0)
+        g = 1.0 + 0.3 * rand(64, 2)
+        for eps in (0.0, 1e-6, 0.5):
+            want = torch.nn.functional.rms_norm(torch.from_numpy(x), (64,),
+                                                weight=torch.from_numpy(g), eps=eps).numpy()
+            np.testing.assert_allclose(O.qk_rms_norm(x, g, eps), want, rtol=1e-13, atol=1e-14)
+
+    def test_rms_norm_closed_forms(self):
+        x = rand((5, 128), 3, 7.0)
+        y = O.qk_rms_norm(x, None, 0.0)
+        np.testing.assert_allclose(np.mean(y * y, axis=1), 1.0, rtol=1e-13)
+        # scale invariance without epsilon, and a constant row a -> a / sqrt(a^2 + eps)
+        np.testing.assert_allclose(O.qk_rms_norm(4.5 * x, None, 0.0), y, rtol=1e-12)
+        c = O.qk_rms_norm(np.full((1, 8), 3.0), None, 0.25)
+        np.testing.assert_allclose(c, 3.0 / math.sqrt(9.25), rtol=1e-15)
+        # the weight scales channel c alone
+        g = np.arange(1, 129, dtype=np.float64)
+        np.testing.assert_allclose(O.qk_rms_norm(x, g, 0.0), y * g, rtol=1e-13)
+
+    def test_rope_matches_complex_multiplication(self):
+        x = rand((9, 64), 4)
+        ang = rand((9, 32), 5, 2.0)
+        z = (x[:, 0::2] + 1j * x[:, 1::2]) * np.exp(1j * ang)
+        want = np.empty_like(x)
+        want[:, 0::2], want[:, 1::2] = z.real, z.imag
+        np.testing.assert_allclose(O.rope_rotate(x, np.cos(ang), np.sin(ang)), want,
+                                   rtol=1e-12, atol=1e-13)
+
+    def test_rope_closed_forms(self):
+        x = rand((4, 16), 6)
+        zero = np.zeros((4, 8))
+        np.testing.assert_array_equal(O.rope_rotate(x, np.cos(zero), np.sin(zero)), x)
+        a, b = rand((4, 8), 7), rand((4, 8), 8)
+        y = O.rope_rotate(O.rope_rotate(x, np.cos(a), np.sin(a)), np.cos(b), np.sin(b))
+        np.testing.assert_allclose(y, O.rope_rotate(x, np.cos(a + b), np.sin(a + b)),
+                                   rtol=1e-12, atol=1e-13)
+        # every pair keeps its length
+        r = O.rope_rotate(x, np.cos(a), np.sin(a))
+        np.testing.assert_allclose(r[:, 0::2] ** 2 + r[:, 1::2] ** 2,
+                                   x[:, 0::2] ** 2 + x[:, 1::2] ** 2, rtol=1e-12)
+
+    def test_rope_relative_position(self):
+        # angles pos * freq: the score of a rotated query and key depends on
+        # the position difference only
+        d = 32
+        freq = 10000.0 ** (-np.arange(d // 2) / (d // 2))
+        tab = lambda pos: (np.cos(pos * freq)[None], np.sin(pos * freq)[None])
+        q, k = rand((1, d), 9), rand((1, d), 10)
+        s = lambda m, n: float((O.rope_rotate(q, *tab(m)) @ O.rope_rotate(k, *tab(n)).T)[0, 0])
+        for m, n, t in ((3, 1, 5), (0, 7, 11), (20, 20, 3)):
+            assert s(m, n) == pytest.approx(s(m + t, n + t), rel=1e-11)
+        assert s(0, 0) == pytest.approx(float((q @ k.T)[0, 0]), rel=1e-12)
+
+    def test_worked_example(self):
+        # x = (1, 2, 3, 4): rms = sqrt(30 / 4); pair 0 turned by pi/2 maps
+        # (a, b) -> (-b, a); pair 1 turned by pi maps (a, b) -> (-a, -b)
+        x = np.array([[1.0, 2.0, 3.0, 4.0]])
+        ang = np.array([[math.pi / 2, math.pi]])
+        y = O.qk_norm_rope(x, None, 0.0, np.cos(ang), np.sin(ang))
+        np.testing.assert_allclose(y, np.array([[-2.0, 1.0, -3.0, -4.0]]) / math.sqrt(7.5),
+                                   rtol=1e-14, atol=1e-15)
+
+    def test_norm_commutes_with_rope_at_unit_weight(self):
+        # the rotation keeps every row's sum of squares, so with gamma = 1 the
+        # two orders agree (up to cos^2 + sin^2 = 1 in the float32 tables);
+        # with a non-uniform weight they do not
+        wl = si.small("cogvideox")
+        cos, sin = si.rope_tables(wl)
+        x = rand((wl.N, wl.d), 11, 2.0)
+        a = O.qk_norm_rope(x, None, 1e-6, cos, sin)
+        b = O.qk_rms_norm(O.rope_rotate(x, cos, sin), None, 1e-6)
+        np.testing.assert_allclose(a, b, rtol=1e-6, atol=1e-6)
+        g = si.qk_norm_weights(wl)[0]
+        a = O.qk_norm_rope(x, g, 1e-6, cos, sin)
+        b = O.qk_rms_norm(O.rope_rotate(x, cos, sin), g, 1e-6)
+        assert np.abs(a - b).max() > 1e-3
+
+    def test_layer_with_unit_transform_is_the_plain_layer(self):
+        wl = si.WORKLOADS["tiny"]
+        q, k, v, _ = si.generate(wl)
+        q, k, v = (si.as_float64(t) for t in (q, k, v))
+        idx = si.sample_queries(wl)
+        ones = np.ones((wl.N, wl.d // 2))
+        zeros = np.zeros((wl.N, wl.d // 2))
+        o1, m1, e1 = O.svg_layer(q, k, v, idx, wl.F, wl.P, wl.width,
+                                 qk=(None, None, 0.0, ones, zeros))
+        nrm = lambda t: torch.nn.functional.rms_norm(torch.from_numpy(t), (wl.d,)).numpy()
+        o2, m2, e2 = O.svg_layer(nrm(q), nrm(k), v, idx, wl.F, wl.P, wl.width)
+        np.testing.assert_array_equal(m1, m2)
+        np.testing.assert_allclose(o1, o2, rtol=1e-12, atol=1e-12)
+
+    def test_rope_tables_input(self):
+        wl = si.small("wan480")
+        cos, sin = si.rope_tables(wl)
+        assert cos.shape == (wl.N, wl.d // 2) and cos.dtype == np.float32
+        np.testing.assert_allclose(cos.astype(np.float64) ** 2 + sin.astype(np.float64) ** 2,
+                                   1.0, atol=1e-6)
+        np.testing.assert_array_equal(cos[0], 1.0)  # token 0 sits at the origin
+        np.testing.assert_array_equal(sin[0], 0.0)
