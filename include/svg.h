@@ -77,7 +77,7 @@ typedef enum {
 #define SVG_DEVICE_BAD_INDEX 0x2     /* a key-block index outside [0, nB)   */
 #define SVG_DEVICE_TIMEOUT 0x4       /* a bounded pipeline wait gave up      */
 #define SVG_DEVICE_CAPACITY 0x8      /* a list did not fit the given buffer */
-#define SVG_DEVICE_RANGE 0x10        /* a bf16 V value exceeded the fp16 range */
+#define SVG_DEVICE_RANGE 0x10        /* a bf16 V value is outside the fp16 range, inf or NaN */
 
 #define SVG_TILE 128
 
@@ -315,7 +315,8 @@ svg_status svg_lists_to_bitmap(int n_rows, int n_cols, const int32_t* indptr,
  * Arithmetic (bf16): Q.K^T on bf16 tensor cores with fp32 accumulation, fp32
  * online softmax; P.V on fp16 tensor cores (P in [0, 256] with an 11-bit
  * significand; V converted from bf16 to fp16 on chip, exact for
- * |v| <= 65504 -- larger values become inf and set SVG_DEVICE_RANGE) with
+ * |v| <= 65504 -- a larger, infinite or NaN value in a visited key block
+ * sets SVG_DEVICE_RANGE; larger values become inf) with
  * fp32 accumulation; output rounded to nearest bf16.  fp32 inputs use fp32
  * arithmetic throughout.
  * ------------------------------------------------------------------------ */

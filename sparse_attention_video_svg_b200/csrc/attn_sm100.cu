@@ -679,8 +679,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Converts every V tile in place, in ring order.  bf16 -> fp16 is exact
     // for |v| <= 65504 (fp16 subnormals keep the absolute error below
     // 2^-25); larger values become inf and are reported as SVG_DEVICE_RANGE.
-    uint32_t L = 0;
-    bool ok = true, range = false;
+    // The check is on the bf16 bits: a magnitude field of 0x4780 (65536) or
+    // more, inf and NaN included, carries into bit 15 of its half once
+    // 0x3880 is added, and the 15-bit fields cannot carry into each other.
+    uint32_t L = 0, over = 0;
+    bool ok = true;
     while (ok) {
       const uint32_t slot = (L + 1) % S;
       if (!(ok = wait_bar(&B.kv_full[slot], ((L + 1) / S) & 1, abort_flag, a.status))) break;
@@ -693,7 +696,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xffff0000u);
-          range |= fabsf(lo) > 65504.f || fabsf(hi) > 65504.f;
+          over |= (w[i] & 0x7fff7fffu) + 0x38803880u;
           const __half2 h = __floats2half2_rn(lo, hi);
           w[i] = *reinterpret_cast<const uint32_t*>(&h);
         }
@@ -704,7 +707,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(&B.v_ready[slot]);
       L += 2;
     }
-    if (__any_sync(0xffffffffu, range) && lane == 0) set_status(a.status, SVG_DEVICE_RANGE);
+    if (__any_sync(0xffffffffu, (over & 0x80008000u) != 0u) && lane == 0)
+      set_status(a.status, SVG_DEVICE_RANGE);
   } else {
     reg_alloc<C::kRegsHigh>();
     softmax_member<D>(a, B, abort_flag, tmem, n_items, n_pairs, nb);

@@ -11,8 +11,8 @@ import torch
 
 import svg_inputs as si
 from oracle import svg_oracle as O
-from tests.helpers import (MODE_MARGIN, assert_close, bits, to_device, to_float64,
-                           workload_tensors)
+from tests.helpers import (MAX_ABS, MODE_MARGIN, assert_close, bits, half_ulp_bf16, to_device,
+                           to_float64, workload_tensors)
 
 pytestmark = pytest.mark.gpu
 
@@ -363,6 +363,38 @@ def test_sparse_attn_fused_bad_mode():
     ref = svg.svg_sparse_attn_fused(qd, kd, vd, wl.F, wl.P, good, lists)
     for h in (0, 2, 3):
         np.testing.assert_array_equal(bits(o[0, h]), bits(ref[0, h]))
+
+
+@pytest.mark.parametrize("value,flagged", [(65280.0, False), (-65280.0, False), (65536.0, True),
+                                           (-1.0e6, True), (float("inf"), True),
+                                           (float("nan"), True)])
+def test_sparse_attn_v_range_flag(value, flagged):
+    """bf16 -> fp16 conversion of V on chip: the largest bf16 below the fp16
+    limit 65504 passes; larger magnitudes, inf and NaN set SVG_DEVICE_RANGE."""
+    wl = si.small("cogvideox")
+    (q, k, v), (qd, kd, vd), _ = workload_tensors(wl)
+    lists = svg.geometric_lists(wl.F, wl.P, wl.width, wl.N)
+    dense = torch.full((wl.B * wl.H,), O.MODE_DENSE, dtype=torch.int32, device=DEV)
+    vd = vd.clone()
+    vd[0, 1, wl.N - 1, 5] = value  # last (ragged) key tile of head 1
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o = svg.svg_sparse_attn(qd, kd, vd, dense, lists, status=status)
+    torch.cuda.synchronize()
+    assert bool(status.item() & svg._lib.SVG_DEVICE_RANGE) == flagged
+    if not flagged:
+        # the value is exact in fp16, so head 1 matches the oracle; with |v|
+        # this large the fp16 rounding of P (2^-12 relative per term, and as
+        # much again through the row sum) is no longer below the bf16 output
+        # rounding, so the bound adds 2^-11 |o| to half a bf16 ulp
+        vh = head64(v, 0, 1)
+        vh[wl.N - 1, 5] = value
+        ip, ix = O.geometric_block_lists(O.MODE_DENSE, wl.F, wl.P, wl.width, wl.N)
+        rows = np.arange(wl.N)
+        want = O.block_sparse_rows(head64(q, 0, 1), head64(k, 0, 1), vh, rows, ip, ix)
+        got = to_float64(o[0, 1])
+        bound = np.maximum(MAX_ABS, half_ulp_bf16(want) + 1e-3 + 2.0 ** -11 * np.abs(want))
+        err = np.abs(got - want)
+        assert (err <= bound).all(), f"v = {value}: worst excess {(err - bound).max():.4g}"
 
 
 # ---------------------------------------------------------------- the layer
