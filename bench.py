@@ -53,8 +53,8 @@ def load_peaks():
 # layer, from an ncu capture of the kernel built from the sources whose
 # sha256 is recorded here.  Reported only while the sources still match.
 ATTN_SOURCES = ("attn_sm100.cu", "sm100.cuh", "attn.cuh", "common.cuh")
-ATTN_TRAFFIC = {"cogvideox": {"sha256": "6819d80f9416009b3f31b8b87e78683b95a4af22a36552ed53d8caadf75d4511",
-                              "bytes": 327064064 + 84521472}}
+ATTN_TRAFFIC = {"cogvideox": {"sha256": "69b305cdbe530f99bc8a8765c1846ab9b147187ad62f564c4cb15e738271a2c4",
+                              "bytes": 328518912 + 84531456}}
 
 
 def attn_sources_sha256():
@@ -308,6 +308,40 @@ def run_ours(args, rank, world, local_rank):
                  "bitmap_us": round(enc["bitmap"][0], 2),
                  "note": "host-synchronising size query included in intervals_us"}
 
+    # QK-Norm + RoPE of q and k, writing the token-major copies in the same
+    # pass, on its own; then the layer with it in front (the pass makes the
+    # copies of q and k, only v is permuted on the side stream) against the
+    # pass followed by the plain layer (which reorders q and k again)
+    gq, gk = si.qk_norm_weights(wl)
+    cos, sin = si.rope_tables(wl)
+    to_dev = lambda a: torch.from_numpy(a).to(dev)
+    qk = svg.QKTransform(to_dev(gq), to_dev(gk), 1e-6, to_dev(cos), to_dev(sin))
+    qk_bufs = svg.LayerBuffers(qd, wl.S, qk=True)
+    qn, kn = torch.empty_like(qd), torch.empty_like(kd)
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        evs = []
+        for i in range(K):
+            flush.fill_(i & 0xff)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            evs.append((e0, e1))
+        torch.cuda.synchronize()
+        return float(sum(a.elapsed_time(b) for a, b in evs) / K)
+
+    qk_ms = timed(lambda: svg.svg_qk_norm_rope(qd, kd, qk, out=(qn, kn),
+                                               tm_out=(qk_bufs.qp, qk_bufs.kp), frames=F,
+                                               tokens_per_frame=P))
+    qk_layer_ms = timed(lambda: svg.svg_layer(qd, kd, vd, F, P, w, idx_d, lists, qk_bufs, qk=qk))
+    qk_modes = qk_bufs.mode.cpu().numpy()  # QK-Norm changes what profiling picks
+    qk_then_layer_ms = timed(lambda: (svg.svg_qk_norm_rope(qd, kd, qk, out=(qn, kn)),
+                                      svg.svg_layer(qn, kn, vd, F, P, w, idx_d, lists, bufs)))
+    del qk_bufs, qn, kn
+
     # end to end through the public API with host buffers
     out_host = torch.empty(qd.shape, dtype=torch.bfloat16).pin_memory()
     mode_host = torch.empty(modes.shape, dtype=torch.int32).pin_memory()
@@ -332,8 +366,10 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
 
-    total_ms, e2e_ms, attn_avg, prof_avg, perm_avg, unf_avg, fwd_perm_avg = max_over_ranks(
-        [total_ms, e2e_ms, attn_avg, prof_avg, perm_avg, unf_avg, fwd_perm_avg], world, dev)
+    (total_ms, e2e_ms, attn_avg, prof_avg, perm_avg, unf_avg, fwd_perm_avg, qk_ms, qk_layer_ms,
+     qk_then_layer_ms) = max_over_ranks(
+        [total_ms, e2e_ms, attn_avg, prof_avg, perm_avg, unf_avg, fwd_perm_avg, qk_ms,
+         qk_layer_ms, qk_then_layer_ms], world, dev)
     if rank != 0:
         return None
 
@@ -346,6 +382,8 @@ def run_ours(args, rank, world, local_rank):
     elems = wl.B * wl.H * N * d
     perm_bytes = 2 * elems * 2      # one tensor read and written once
     prof_bytes = 2 * elems * 2      # K and V streamed once
+    # q, k read once; q, k written frame-major and token-major; cos, sin once
+    qk_bytes = 6 * elems * 2 + 2 * N * (d // 2) * 4
     h2d = sum(h.numel() * 2 for h in host)
     d2h = out_host.numel() * 2 + mode_host.numel() * 4
     # profile partial, merge, finalize; 3 permutes; attention (output reordering fused)
@@ -382,6 +420,15 @@ def run_ours(args, rank, world, local_rank):
                     "gbs": round(perm_bytes / (perm_avg * 1e-3) / 1e9, 1),
                     "frac_of_hbm": round(perm_bytes / (perm_avg * 1e-3) / 1e9 / hbm_gbs, 4),
                     "hbm_peak_gbs": hbm_gbs},
+        "qk_norm_rope": {"ms": round(qk_ms, 5),
+                         "gbs": round(qk_bytes / (qk_ms * 1e-3) / 1e9, 1),
+                         "frac_of_hbm": round(qk_bytes / (qk_ms * 1e-3) / 1e9 / hbm_gbs, 4),
+                         "bytes": qk_bytes,
+                         "note": "q, k -> QK-Norm + RoPE, frame-major and token-major copies"},
+        "layer_with_qk_norm_rope_ms": round(qk_layer_ms, 5),
+        "layer_with_qk_norm_rope_modes": {"spatial": int((qk_modes == 0).sum()),
+                                          "temporal": int((qk_modes == 1).sum())},
+        "qk_norm_rope_then_layer_ms": round(qk_then_layer_ms, 5),
         "profile": {"ms": round(prof_avg, 5),
                     "kv_gbs": round(prof_bytes / (prof_avg * 1e-3) / 1e9, 1)},
         "roofline": {"kernel": "svg_sparse_attn_fused", "bound": "tensor",

@@ -85,6 +85,10 @@ typedef enum {
 #define SVG_FUSE_INPUT 0x1   /* q, k, v frame-major; temporal heads gathered  */
 #define SVG_FUSE_OUTPUT 0x2  /* o written frame-major for temporal heads      */
 
+/* Operation bits of svg_qk_norm_rope (section 2b). */
+#define SVG_QK_NORM 0x1  /* RMS-normalise each row over d, times gamma       */
+#define SVG_QK_ROPE 0x2  /* rotate channel pairs (2i, 2i+1) by cos / sin    */
+
 /* Library identification, e.g. "svg_b200 0.1 sm_100a". */
 const char* svg_version(void);
 
@@ -175,6 +179,44 @@ svg_status svg_permute_frame_major(const void* x, void* y, int dtype,
                                    int B, int H, int N, int d,
                                    int frames, int tokens_per_frame,
                                    const int32_t* mode, void* stream);
+
+/* --------------------------------------------------------------------------
+ * 2b. QK-Norm + RoPE of q and k, with optional token-major copies
+ *    [SVG] section "Layout Transformation + Kernel 加速": next to the
+ *    attention kernels the method ships its own QK-Norm and RoPE kernels.
+ *    The pages give no formulas; this call reads them as
+ *      QK-Norm: x_hat = x / sqrt(mean_c x_c^2 + eps) * gamma over the d
+ *               channels of each (b, h, n) row;
+ *      RoPE:    channel pair (2i, 2i+1) = (a, b) of row n becomes
+ *               (a cos[n][i] - b sin[n][i], a sin[n][i] + b cos[n][i]);
+ *    with the norm first.  One pass reads q and k once and writes the
+ *    results frame-major and, when asked, token-major (every head), which
+ *    is the reordering the temporal heads need.
+ *
+ *  q, k          device [B, H, N, d] inputs, frame-major.
+ *  q_out, k_out  device [B, H, N, d] results, frame-major.  q_out may be q
+ *                itself and k_out k itself (in place); no other overlap.
+ *  q_tm_out, k_tm_out  device [B, H, N, d] token-major copies of the
+ *                results (row m = s * F + f holds token n = f * P + s), or
+ *                both NULL.  When given, frames * tokens_per_frame == N;
+ *                otherwise frames and tokens_per_frame are ignored.
+ *  ops           SVG_QK_NORM | SVG_QK_ROPE (either, both, or 0 for a copy).
+ *  gamma_q, gamma_k  device float [d] per-channel weights, or NULL for 1.
+ *  eps           added to the mean square inside the square root; finite,
+ *                >= 0 (eps = 0 turns an all-zero row into NaN).
+ *  rope_cos, rope_sin  device float [N][d/2] (pair i of token n), required
+ *                with SVG_QK_ROPE.
+ * Every pointer is 16-byte aligned.  Arithmetic in fp32 (row sums of squares
+ * in fp32, reciprocal square root), results rounded to the tensor dtype
+ * (bf16: to nearest even).  Bytes: reads 2 B H N d elt, writes 2 or 4 times
+ * that, plus the tables once per group of heads.
+ * ------------------------------------------------------------------------ */
+svg_status svg_qk_norm_rope(const void* q, const void* k, void* q_out, void* k_out,
+                            void* q_tm_out, void* k_tm_out, int dtype,
+                            int B, int H, int N, int d,
+                            int frames, int tokens_per_frame, int ops,
+                            const float* gamma_q, const float* gamma_k, float eps,
+                            const float* rope_cos, const float* rope_sin, void* stream);
 
 /* --------------------------------------------------------------------------
  * 3a. Geometric key-block lists

@@ -470,6 +470,15 @@ def rope_rotate(x, cos, sin) -> np.ndarray:
     return y
 
 
+def round_bf16(x) -> np.ndarray:
+    """x rounded to the nearest bf16 value (8 significant bits, ties to
+    even), kept in float64: with x = m 2^e, 0.5 <= |m| < 1, the result is
+    round_half_even(m 2^8) 2^(e-8).  Models a bf16 tensor holding a
+    result; no overflow or subnormal handling (not reached here)."""
+    m, e = np.frexp(np.asarray(x, np.float64))
+    return np.ldexp(np.round(m * 256.0), e - 8)
+
+
 def qk_norm_rope(x, gamma=None, eps: float = 1e-6, cos=None, sin=None,
                  norm: bool = True, rope: bool = True) -> np.ndarray:
     """The pre-attention transform of q or k: QK-Norm first, then RoPE
@@ -486,17 +495,22 @@ def qk_norm_rope(x, gamma=None, eps: float = 1e-6, cos=None, sin=None,
 # The whole layer: profile -> permute temporal heads -> block-sparse -> back
 # ---------------------------------------------------------------------------
 
-def svg_layer(q, k, v, idx, F: int, P: int, width: int, T: int = 128, qk=None):
+def svg_layer(q, k, v, idx, F: int, P: int, width: int, T: int = 128, qk=None,
+              qk_bf16: bool = False):
     """One attention layer of the method for [B, H, N, d] inputs: profile each
     head, run spatial heads on their frame-major lists, temporal heads in
     token-major order on their lists, and map temporal outputs back.
     qk = (gamma_q, gamma_k, eps, cos, sin) first applies QK-Norm + RoPE to q
-    and k.  Returns (o [B, H, N, d], mode [B*H], mse [B*H, 2])."""
+    and k; qk_bf16 stores that result as bf16 (the tensor type of a bf16
+    layer) before attention reads it.
+    Returns (o [B, H, N, d], mode [B*H], mse [B*H, 2])."""
     B, H, N, d = q.shape
     if qk is not None:
         gq, gk, eps, cos, sin = qk
         q = qk_norm_rope(q, gq, eps, cos, sin)
         k = qk_norm_rope(k, gk, eps, cos, sin)
+        if qk_bf16:
+            q, k = round_bf16(q), round_bf16(k)
     mse, mode = profile_heads(q, k, v, idx, F, P, width)
     lists = {MODE_SPATIAL: geometric_block_lists(MODE_SPATIAL, F, P, width, N, T),
              MODE_TEMPORAL: geometric_block_lists(MODE_TEMPORAL, F, P, width, N, T)}

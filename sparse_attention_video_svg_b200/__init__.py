@@ -16,7 +16,8 @@ m.jxzklqfsx.com/article/815093.html; CalibAtt article, lpnh.cn/news/568491):
     o'        = svg_sparse_attn(q', k', v', mode, *lists)
     o         = svg_permute_frame_major(o', F, P, mode)
 
-``svg_layer`` runs exactly that sequence.
+``svg_layer`` runs exactly that sequence (optionally after
+``svg_qk_norm_rope``, QK-Norm + RoPE of q and k).
 """
 from __future__ import annotations
 
@@ -36,7 +37,7 @@ __all__ = [
     "svg_permute_frame_major", "svg_build_block_mask", "svg_block_energy",
     "svg_build_block_mask_calibrated", "svg_sparse_attn", "svg_sparse_attn_fused",
     "svg_epsilon_schedule", "svg_lists_to_intervals", "svg_lists_to_bitmap", "geometric_lists",
-    "svg_layer",
+    "QKTransform", "svg_qk_norm_rope", "svg_layer",
     "n_tiles",
 ]
 
@@ -232,6 +233,42 @@ def svg_sparse_attn_fused(q, k, v, frames: int, tokens_per_frame: int, mode: tor
     return out
 
 
+class QKTransform(NamedTuple):
+    """Parameters of the QK-Norm + RoPE step before attention: per-channel
+    weights (float32 [d] CUDA tensors, or None for 1), epsilon, and the rotary
+    tables cos, sin (float32 [N, d/2] CUDA tensors, or None for no RoPE)."""
+    gamma_q: Optional[torch.Tensor]
+    gamma_k: Optional[torch.Tensor]
+    eps: float
+    cos: Optional[torch.Tensor]
+    sin: Optional[torch.Tensor]
+    norm: bool = True
+
+
+def svg_qk_norm_rope(q, k, qk: QKTransform, *, out=None, tm_out=None, frames: int = 0,
+                     tokens_per_frame: int = 0, stream=None):
+    """QK-Norm then RoPE of q and k in one pass.  out = (q_out, k_out)
+    (allocated when None; may be (q, k) for in place); tm_out = (q_tm, k_tm)
+    also writes the token-major copies of every head (needs frames and
+    tokens_per_frame).  Returns (q_out, k_out)."""
+    B, H, N, d = _check_qkv(q, k)
+    if out is None:
+        out = (torch.empty_like(q), torch.empty_like(k))
+    _check_qkv(q, *out)
+    qt, kt = (None, None) if tm_out is None else (tm_out[0].data_ptr(), tm_out[1].data_ptr())
+    if tm_out is not None:
+        _check_qkv(q, *tm_out)
+    ops = (_lib.SVG_QK_NORM if qk.norm else 0) | (_lib.SVG_QK_ROPE if qk.cos is not None else 0)
+    for t in (qk.gamma_q, qk.gamma_k, qk.cos, qk.sin):
+        if t is not None and (t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("QK-Norm weights and RoPE tables must be contiguous float32 CUDA")
+    _lib.call("svg_qk_norm_rope", q.data_ptr(), k.data_ptr(), out[0].data_ptr(),
+              out[1].data_ptr(), qt, kt, _dt(q), B, H, N, d, int(frames), int(tokens_per_frame),
+              ops, _ptr(qk.gamma_q), _ptr(qk.gamma_k), float(qk.eps), _ptr(qk.cos), _ptr(qk.sin),
+              _stream(stream))
+    return out
+
+
 # ------------------------------------------- threshold schedule, mask encodings
 
 def svg_epsilon_schedule(n_steps: int, eps_first: float = 0.99, eps_last: float = 0.84):
@@ -278,9 +315,13 @@ def svg_lists_to_bitmap(indptr: torch.Tensor, indices: torch.Tensor, n_cols: int
 class LayerBuffers:
     """Preallocated buffers for svg_layer at one shape (reused across steps)."""
 
-    def __init__(self, q: torch.Tensor, S: int, layout: int = _lib.SVG_FUSE_OUTPUT):
+    def __init__(self, q: torch.Tensor, S: int, layout: int = _lib.SVG_FUSE_OUTPUT,
+                 qk: bool = False):
         B, H, N, d = q.shape
         dev = q.device
+        if qk:  # q and k after QK-Norm + RoPE
+            self.qn = torch.empty_like(q)
+            self.kn = torch.empty_like(q)
         if not layout & _lib.SVG_FUSE_INPUT:  # token-major copies of q, k, v
             self.qp = torch.empty_like(q)
             self.kp = torch.empty_like(q)
@@ -298,7 +339,8 @@ class LayerBuffers:
 
 def svg_layer(q, k, v, frames: int, tokens_per_frame: int, spatial_width: int,
               sample_idx: torch.Tensor, lists: BlockLists, bufs: Optional[LayerBuffers] = None,
-              stream=None, layout: int = _lib.SVG_FUSE_OUTPUT, overlap: bool = True):
+              stream=None, layout: int = _lib.SVG_FUSE_OUTPUT, overlap: bool = True,
+              qk: Optional[QKTransform] = None):
     """One attention layer: profile -> block-sparse attention on the list the
     mode selects, temporal heads in token-major order.  `layout` picks which
     side of the reordering runs inside the attention kernel
@@ -307,9 +349,12 @@ def svg_layer(q, k, v, frames: int, tokens_per_frame: int, spatial_width: int,
     moves q, k, v faster than row gathers inside the attention kernel.  With
     overlap (input side not fused), the token-major copies of every head are
     made on a side stream while the heads are profiled.
+    qk applies QK-Norm + RoPE to q and k first (svg_qk_norm_rope); with
+    overlap that pass also writes the token-major copies of q and k, and only
+    v is permuted on the side stream.
     Returns (o, mode, mse)."""
     if bufs is None:
-        bufs = LayerBuffers(q, sample_idx.numel(), layout)
+        bufs = LayerBuffers(q, sample_idx.numel(), layout, qk=qk is not None)
     F, P = frames, tokens_per_frame
     if overlap and not layout & _lib.SVG_FUSE_INPUT:
         # token-major copies of every head on a side stream, concurrent with
@@ -323,10 +368,16 @@ def svg_layer(q, k, v, frames: int, tokens_per_frame: int, spatial_width: int,
         ready = torch.cuda.Event()
         ready.record(main)
         bufs.side.wait_event(ready)
-        for x, y in ((q, bufs.qp), (k, bufs.kp), (v, bufs.vp)):
+        side_work = ((v, bufs.vp),) if qk is not None else \
+            ((q, bufs.qp), (k, bufs.kp), (v, bufs.vp))
+        for x, y in side_work:
             svg_permute_token_major(x, F, P, None, out=y, stream=bufs.side)
         copied = torch.cuda.Event()
         copied.record(bufs.side)
+        if qk is not None:
+            svg_qk_norm_rope(q, k, qk, out=(bufs.qn, bufs.kn), tm_out=(bufs.qp, bufs.kp),
+                             frames=F, tokens_per_frame=P, stream=main)
+            q, k = bufs.qn, bufs.kn
         svg_profile_heads(q, k, v, F, P, spatial_width, sample_idx, mse_out=bufs.mse,
                           mode_out=bufs.mode, workspace=bufs.ws, stream=main)
         main.wait_event(copied)
@@ -338,6 +389,9 @@ def svg_layer(q, k, v, frames: int, tokens_per_frame: int, spatial_width: int,
         if not layout & _lib.SVG_FUSE_OUTPUT:
             svg_permute_frame_major(bufs.op, F, P, bufs.mode, out=bufs.o, stream=main)
         return bufs.o, bufs.mode, bufs.mse
+    if qk is not None:
+        svg_qk_norm_rope(q, k, qk, out=(bufs.qn, bufs.kn), stream=stream)
+        q, k = bufs.qn, bufs.kn
     svg_profile_heads(q, k, v, F, P, spatial_width, sample_idx, mse_out=bufs.mse,
                       mode_out=bufs.mode, workspace=bufs.ws, stream=stream)
     if layout & _lib.SVG_FUSE_INPUT:

@@ -17,6 +17,8 @@ SVG_DEVICE_BAD_LIST_ID, SVG_DEVICE_BAD_INDEX, SVG_DEVICE_TIMEOUT, SVG_DEVICE_CAP
 SVG_DEVICE_RANGE = 16
 SVG_FUSE_INPUT = 1
 SVG_FUSE_OUTPUT = 2
+SVG_QK_NORM = 1
+SVG_QK_ROPE = 2
 SVG_TILE = 128
 
 _p = C.c_void_p
@@ -49,6 +51,8 @@ SIGNATURES = {
     "svg_lists_to_bitmap": (_i, [_i, _i, _p, _p, _p, _p, _p]),
     "svg_sparse_attn_fused": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p,
                                    _i, _i, _i, _p, _p, _f, _p, _p]),
+    "svg_qk_norm_rope": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _p, _p, _f,
+                              _p, _p, _p]),
 }
 
 

@@ -94,6 +94,24 @@ class TestHostValidation:
                *(base[:3] + [FAKE4 * 5, FAKE4 * 6, FAKE4 * 7] + base[6:15] + [1] + base[16:]),
                match="exclude")
 
+    def test_qk_norm_rope(self):
+        # q k q_out k_out q_tm k_tm dtype B H N d F P ops gamma_q gamma_k eps cos sin stream
+        both = _lib.SVG_QK_NORM | _lib.SVG_QK_ROPE
+        base = [FAKE, FAKE2, FAKE3, FAKE4, FAKE4 * 2, FAKE4 * 3, 0, 1, 2, 256, 64, 4, 64, both,
+                FAKE4 * 4, None, 1e-6, FAKE4 * 5, FAKE4 * 6, None]
+        f = "svg_qk_norm_rope"
+        expect(INVALID, f, *(base[:13] + [4] + base[14:]), match="bad ops")
+        expect(INVALID, f, *(base[:16] + [-1.0] + base[17:]), match="eps")
+        expect(INVALID, f, *(base[:17] + [None] + base[18:]), match="cos and sin")
+        expect(INVALID, f, *(base[:5] + [None] + base[6:]), match="both token-major")
+        expect(INVALID, f, *(base[:11] + [5] + base[12:]), match="frames")
+        expect(INVALID, f, *(base[:2] + [FAKE2] + base[3:]), match="overlap")
+        expect(INVALID, f, *(base[:4] + [FAKE3 + 4096] + base[5:]), match="token-major outputs")
+        expect(INVALID, f, *(base[:14] + [FAKE4 * 4 + 4] + base[15:]), match="aligned")
+        expect(INVALID, f, *(base[:10] + [96] + base[11:]), match="d=96")
+        expect(INVALID, f, *(base[:6] + [3] + base[7:]), match="dtype")
+        expect(INVALID, f, *([None] + base[1:]), match="null")
+
     def test_permute(self):
         args = [FAKE, FAKE4 * 4, 0, 1, 2, 12, 64, 3, 4, None, None]
         expect(INVALID, "svg_permute_token_major", *(args[:7] + [5] + args[8:]), match="!= N")

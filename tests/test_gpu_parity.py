@@ -609,3 +609,130 @@ def test_encodings_capacity_and_bad_index():
     ip2 = ip.copy()
     ip2[np.searchsorted(ip, 5, side="right"):] -= 1
     np.testing.assert_array_equal(bm.cpu().numpy().view(np.uint32), O.lists_to_bitmap(ip2, good, 100))
+
+
+# ------------------------------------------------------- QK-Norm + RoPE (f2)
+
+def qk_inputs(wl):
+    (q, k, _), (qd, kd, _), _ = workload_tensors(wl)
+    gq, gk = si.qk_norm_weights(wl)
+    cos, sin = si.rope_tables(wl)
+    dev = lambda a: torch.from_numpy(a).to(DEV)
+    qk = svg.QKTransform(dev(gq), dev(gk), 1e-6, dev(cos), dev(sin))
+    return (q, k), (qd, kd), (gq, gk, cos, sin), qk
+
+
+def check_qk(got, x64, gamma, eps, cos, sin, bf16, what, norm=True, rope=True):
+    """got vs the float64 oracle.  Bound per element: fp32 arithmetic (a few
+    2^-24 of the rotated magnitudes |a c| + |b s|, with margin 2^-17) plus,
+    for bf16 results, half a bf16 ulp of the rounding."""
+    ref = O.qk_norm_rope(x64, gamma, eps, cos, sin, norm=norm, rope=rope)
+    pre = np.abs(O.qk_rms_norm(x64, gamma, eps) if norm else x64)
+    if rope:
+        c, s = np.abs(cos), np.abs(sin)
+        mag = np.empty_like(pre)
+        mag[..., 0::2] = pre[..., 0::2] * c + pre[..., 1::2] * s
+        mag[..., 1::2] = pre[..., 0::2] * s + pre[..., 1::2] * c
+    else:
+        mag = pre
+    slack = 2.0 ** -17 * mag + 1e-30
+    bound = slack + (half_ulp_bf16(np.abs(ref) + slack) if bf16 else 0.0)
+    err = np.abs(got - ref)
+    assert (err <= bound).all(), f"{what}: worst excess {(err - bound).max():.3g}"
+
+
+@pytest.mark.parametrize("wl", SMALL, ids=lambda w: w.name)
+def test_qk_norm_rope_small(wl):
+    (q, k), (qd, kd), (gq, gk, cos, sin), qk = qk_inputs(wl)
+    q_tm, k_tm = torch.empty_like(qd), torch.empty_like(kd)
+    qo, ko = svg.svg_qk_norm_rope(qd, kd, qk, tm_out=(q_tm, k_tm), frames=wl.F,
+                                  tokens_per_frame=wl.P)
+    bf16 = wl.dtype == "bf16"
+    for x, g, got in ((q, gq, qo), (k, gk, ko)):
+        check_qk(to_float64(got), si.as_float64(x), g, 1e-6, cos, sin, bf16, wl.name)
+    # the token-major copies hold the same bits, reordered m = s F + f <- n = f P + s
+    src = O.token_major_source(wl.F, wl.P)
+    for fm, tm in ((qo, q_tm), (ko, k_tm)):
+        np.testing.assert_array_equal(bits(tm), bits(fm)[:, :, src])
+
+
+@pytest.mark.parametrize("which", ["norm", "rope", "copy", "unit_weight"])
+def test_qk_norm_rope_ops(which):
+    wl = si.small("wan480")
+    (q, k), (qd, kd), (gq, gk, cos, sin), qk = qk_inputs(wl)
+    norm, rope = which in ("norm", "unit_weight"), which == "rope"
+    if which == "unit_weight":
+        qk = qk._replace(gamma_q=None, gamma_k=None)
+        gq = gk = None
+    qk = qk._replace(norm=norm, cos=qk.cos if rope else None, sin=qk.sin if rope else None)
+    qo, ko = svg.svg_qk_norm_rope(qd, kd, qk)
+    if which == "copy":
+        np.testing.assert_array_equal(bits(qo), bits(qd))
+        np.testing.assert_array_equal(bits(ko), bits(kd))
+        return
+    for x, g, got in ((q, gq, qo), (k, gk, ko)):
+        check_qk(to_float64(got), si.as_float64(x), g, 1e-6, cos, sin, True, which,
+                 norm=norm, rope=rope)
+
+
+def test_qk_norm_rope_in_place():
+    wl = si.small("cogvideox")
+    _, (qd, kd), _, qk = qk_inputs(wl)
+    want = svg.svg_qk_norm_rope(qd, kd, qk)
+    qi, ki = qd.clone(), kd.clone()
+    svg.svg_qk_norm_rope(qi, ki, qk, out=(qi, ki))
+    np.testing.assert_array_equal(bits(qi), bits(want[0]))
+    np.testing.assert_array_equal(bits(ki), bits(want[1]))
+
+
+@pytest.mark.parametrize("name", ["cogvideox", "hunyuan720"])
+def test_qk_norm_rope_full_sampled(name, full_inputs):
+    wl = si.WORKLOADS[name]
+    (q, k, _), (qd, kd, _), _ = full_inputs(name)
+    gq, gk = si.qk_norm_weights(wl)
+    cos, sin = si.rope_tables(wl)
+    dev = lambda a: torch.from_numpy(a).to(DEV)
+    qk = svg.QKTransform(dev(gq), dev(gk), 1e-6, dev(cos), dev(sin))
+    q_tm, k_tm = torch.empty_like(qd), torch.empty_like(kd)
+    qo, ko = svg.svg_qk_norm_rope(qd, kd, qk, tm_out=(q_tm, k_tm), frames=wl.F,
+                                  tokens_per_frame=wl.P)
+    rng = np.random.default_rng(17)
+    heads = rng.choice(wl.H, size=4, replace=False)
+    rows = np.r_[rng.choice(wl.N - 1, size=509, replace=False), wl.N - 1]
+    src = O.token_major_source(wl.F, wl.P)
+    inv = np.empty_like(src)
+    inv[src] = np.arange(wl.N)  # token-major row of token n
+    rows_d = torch.from_numpy(rows).to(DEV)
+    inv_d = torch.from_numpy(inv[rows]).to(DEV)
+    for h in heads:
+        for x, g, got, tm in ((q, gq, qo, q_tm), (k, gk, ko, k_tm)):
+            sel = got[0, h][rows_d]
+            check_qk(to_float64(sel), si.as_float64(x[0, h][rows]), g, 1e-6, cos[rows],
+                     sin[rows], True, f"{name} head {h}")
+            np.testing.assert_array_equal(bits(tm[0, h][inv_d]), bits(sel))
+
+
+@pytest.mark.parametrize("overlap", [True, False])
+@pytest.mark.parametrize("name", ["cogvideox", "wan480"])
+def test_layer_small_with_qk_norm_rope(name, overlap):
+    wl = si.small(name)
+    (q, k, v), (qd, kd, vd), _ = workload_tensors(wl)
+    gq, gk = si.qk_norm_weights(wl)
+    cos, sin = si.rope_tables(wl)
+    dev = lambda a: torch.from_numpy(a).to(DEV)
+    qk = svg.QKTransform(dev(gq), dev(gk), 1e-6, dev(cos), dev(sin))
+    idx = si.sample_queries(wl)
+    lists = svg.geometric_lists(wl.F, wl.P, wl.width, wl.N)
+    o, mode, mse = svg.svg_layer(qd, kd, vd, wl.F, wl.P, wl.width,
+                                 torch.from_numpy(idx).to(DEV), lists, overlap=overlap, qk=qk)
+    o_ref, mode_ref, mse_ref = O.svg_layer(si.as_float64(q), si.as_float64(k), si.as_float64(v),
+                                           idx, wl.F, wl.P, wl.width,
+                                           qk=(gq, gk, 1e-6, cos, sin),
+                                           qk_bf16=wl.dtype == "bf16")
+    check_profile(mse.cpu().numpy(), mode.cpu().numpy(), mse_ref, mode_ref, wl.name)
+    m = mode.cpu().numpy()
+    for bh in range(wl.B * wl.H):
+        if m[bh] != mode_ref[bh]:
+            continue  # a near-tie decided the other way (checked above)
+        b, h = divmod(bh, wl.H)
+        assert_close(to_float64(o[b, h]), o_ref[b, h], f"{wl.name} head {h}")

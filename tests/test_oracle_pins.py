@@ -601,6 +601,21 @@ class TestQkNormRope:
         np.testing.assert_array_equal(m1, m2)
         np.testing.assert_allclose(o1, o2, rtol=1e-12, atol=1e-12)
 
+    def test_round_bf16(self):
+        # library cross-check: torch's float32 -> bf16 cast (round to nearest
+        # even) on float32 values, where no double rounding can occur
+        x = (rand(4000, 12, 3.0) * np.exp(rand(4000, 13, 4.0))).astype(np.float32)
+        want = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+        np.testing.assert_array_equal(O.round_bf16(x.astype(np.float64)), want)
+        # ties go to even; just above a tie goes up; sign symmetry; exact values stay
+        u = 2.0 ** -8
+        assert O.round_bf16(1 + u) == 1.0 and O.round_bf16(1 + 3 * u) == 1 + 4 * u
+        assert O.round_bf16(1 + u * (1 + 2.0 ** -30)) == 1 + 2 * u
+        assert O.round_bf16(-(1 + 3 * u)) == -(1 + 4 * u)
+        assert O.round_bf16(0.0) == 0.0 and O.round_bf16(-40.0) == -40.0
+        np.testing.assert_array_equal(O.round_bf16(O.round_bf16(x.astype(np.float64))),
+                                      O.round_bf16(x.astype(np.float64)))
+
     def test_rope_tables_input(self):
         wl = si.small("wan480")
         cos, sin = si.rope_tables(wl)
