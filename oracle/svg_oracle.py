@@ -36,6 +36,12 @@ notes):
   weight and an epsilon inside the square root; RoPE rotates interleaved
   channel pairs (2i, 2i+1) by caller-supplied per-token angles (cos / sin
   tables); QK-Norm runs first;
+* spatial repetition ([CAL] 3.2): a row's attention pattern is the block of
+  dense probabilities of its pw query tokens over all keys; the head score
+  is the mean pairwise cosine over the rows of each evaluated frame; anchors
+  are the middle rows of k equal bands and each row copies the anchor of its
+  band; anchor rows attend exactly as in the full layer (query tiles with no
+  anchor row are skipped);
 * the energy threshold decays exponentially in the denoising-step index from
   0.99 (first step) to 0.84 (last step); the skip list holds each row's
   maximal runs of consecutive kept blocks; the bitmap holds one bit per
@@ -489,6 +495,106 @@ def qk_norm_rope(x, gamma=None, eps: float = 1e-6, cos=None, sin=None,
     if rope:
         y = rope_rotate(y, cos, sin)
     return y
+
+
+# ---------------------------------------------------------------------------
+# Spatial-repetition heads   ([CAL] 3.2)
+#   Some heads attend almost identically from every image row of a frame:
+#   they are found by the mean cosine similarity of the rows' attention
+#   patterns (> gamma = 0.87), and for them only k = 5 equally spaced anchor
+#   rows per frame are computed; every other row takes its anchor's output.
+# ---------------------------------------------------------------------------
+
+def row_similarity(q, k, F: int, ph: int, pw: int, frames=None, scale=None) -> float:
+    """Mean cosine similarity between the attention patterns of the image
+    rows of a frame.  The pattern of row y of frame f is the pw x N block of
+    dense attention probabilities of its query tokens n = f P + y pw + x
+    (x < pw) over all N keys; the cosine of rows y, y' is the Frobenius inner
+    product of their blocks over the product of their Frobenius norms.  The
+    mean runs over all pairs y < y' of a frame, then over the evaluated
+    frames (all when None).  Needs ph >= 2."""
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    P = ph * pw
+    N = k.shape[0]
+    scale = softmax_scale(q.shape[-1]) if scale is None else scale
+    frames = range(F) if frames is None else frames
+    iu = np.triu_indices(ph, 1)
+    per_frame = []
+    for f in frames:
+        p = attention_probs(q[f * P:(f + 1) * P], k, scale)   # rows in order y pw + x
+        A = p.reshape(ph, pw * N)                             # row y -> its flattened block
+        G = A @ A.T
+        nrm = np.sqrt(np.diag(G))
+        per_frame.append(np.mean((G / np.outer(nrm, nrm))[iu]))
+    return float(np.mean(per_frame))
+
+
+def is_repetitive(similarity, gamma: float = 0.87):
+    """A head repeats spatially when its mean row similarity exceeds gamma."""
+    return np.asarray(similarity) > gamma
+
+
+def anchor_rows(ph: int, k: int = 5) -> np.ndarray:
+    """k equally spaced anchor rows: the ph rows fall into k equal bands
+    (band j = the rows y with floor(y k / ph) = j, i.e. y in
+    [ceil(j ph / k), ceil((j+1) ph / k))) and each band's anchor is its
+    middle row (the upper one of two); every row when k >= ph."""
+    if k >= ph:
+        return np.arange(ph)
+    out = []
+    for j in range(k):
+        lo = -(-j * ph // k)
+        hi = -(-(j + 1) * ph // k)
+        out.append(lo + (hi - lo) // 2)
+    return np.array(out)
+
+
+def row_anchor(ph: int, k: int = 5) -> np.ndarray:
+    """The anchor row each row y takes its output from: the anchor of band
+    floor(y k / ph)."""
+    if k >= ph:
+        return np.arange(ph)
+    a = anchor_rows(ph, k)
+    return np.array([a[(y * k) // ph] for y in range(ph)])
+
+
+def anchor_token_mask(F: int, ph: int, pw: int, k: int = 5) -> np.ndarray:
+    """Boolean [N]: frame-major tokens that lie on an anchor row."""
+    rows = np.zeros(ph, dtype=bool)
+    rows[anchor_rows(ph, k)] = True
+    return np.tile(np.repeat(rows, pw), F)
+
+
+def anchor_tile_lists(indptr, indices, F: int, ph: int, pw: int, k: int = 5, T: int = 128):
+    """The lists of the query tiles that hold an anchor-row token; the other
+    tiles get empty lists (their rows are all filled by the broadcast)."""
+    N = F * ph * pw
+    on = anchor_token_mask(F, ph, pw, k)
+    keep = [bool(on[tile_rows(i, N, T)].any()) for i in range(len(indptr) - 1)]
+    ip, ix = [0], []
+    for i, kp in enumerate(keep):
+        if kp:
+            ix.extend(indices[indptr[i]:indptr[i + 1]])
+        ip.append(len(ix))
+    return np.array(ip, dtype=np.int64), np.array(ix, dtype=np.int64)
+
+
+def broadcast_rows(o, F: int, ph: int, pw: int, k: int = 5) -> np.ndarray:
+    """o'[f, y, x] = o[f, anchor(y), x] for [N, d] frame-major rows."""
+    o = np.asarray(o)
+    src = row_anchor(ph, k)
+    y = o.reshape(F, ph, pw, -1)[:, src]
+    return y.reshape(o.shape).copy()
+
+
+def repeat_head_attention(q, k, v, indptr, indices, F: int, ph: int, pw: int, kk: int = 5,
+                          T: int = 128, scale=None) -> np.ndarray:
+    """Attention of a spatially repeating head: block-sparse attention over
+    the anchor-tile lists, then every row takes its anchor's output."""
+    ip, ix = anchor_tile_lists(indptr, indices, F, ph, pw, kk, T)
+    o = block_sparse_attention(q, k, v, ip, ix, T, scale)
+    return broadcast_rows(o, F, ph, pw, kk)
 
 
 # ---------------------------------------------------------------------------

@@ -624,3 +624,120 @@ class TestQkNormRope:
                                    1.0, atol=1e-6)
         np.testing.assert_array_equal(cos[0], 1.0)  # token 0 sits at the origin
         np.testing.assert_array_equal(sin[0], 0.0)
+
+
+# ------------------------------------------------- spatial repetition ([CAL] 3.2)
+
+class TestSpatialRepetition:
+    def brute_similarity(self, q, k, F, ph, pw, frames):
+        # explicit loops over row pairs, columns and keys; probabilities from
+        # torch's softmax in float64
+        P, N = ph * pw, k.shape[0]
+        s = torch.from_numpy(q @ k.T / math.sqrt(q.shape[1]))
+        p = torch.softmax(s, dim=1).numpy()
+        vals = []
+        for f in frames:
+            pairs = []
+            for y in range(ph):
+                for y2 in range(y + 1, ph):
+                    num = na = nb = 0.0
+                    for x in range(pw):
+                        a = p[f * P + y * pw + x]
+                        b = p[f * P + y2 * pw + x]
+                        for j in range(N):
+                            num += a[j] * b[j]
+                            na += a[j] * a[j]
+                            nb += b[j] * b[j]
+                    pairs.append(num / math.sqrt(na * nb))
+            vals.append(sum(pairs) / len(pairs))
+        return sum(vals) / len(vals)
+
+    def test_similarity_brute_force(self):
+        F, ph, pw, d = 2, 3, 4, 8
+        N = F * ph * pw
+        q, k = rand((N, d), 20, 1.5), rand((N, d), 21, 1.5)
+        for frames in ([0, 1], [1]):
+            want = self.brute_similarity(q, k, F, ph, pw, frames)
+            assert O.row_similarity(q, k, F, ph, pw, frames) == pytest.approx(want, rel=1e-12)
+
+    def test_identical_rows_give_one(self):
+        # queries that depend on (frame, column) only: every row of a frame
+        # has the same pattern
+        F, ph, pw, d = 3, 5, 4, 16
+        base = rand((F, 1, pw, d), 22)
+        q = np.broadcast_to(base, (F, ph, pw, d)).reshape(-1, d)
+        k = rand((F * ph * pw, d), 23)
+        assert O.row_similarity(q, k, F, ph, pw) == pytest.approx(1.0, abs=1e-12)
+        assert O.is_repetitive(O.row_similarity(q, k, F, ph, pw))
+
+    def test_key_order_and_frame_mean(self):
+        F, ph, pw, d = 3, 4, 5, 8
+        N = F * ph * pw
+        q, k = rand((N, d), 24, 2.0), rand((N, d), 25, 2.0)
+        perm = np.random.default_rng(26).permutation(N)
+        a = O.row_similarity(q, k, F, ph, pw)
+        assert O.row_similarity(q, k[perm], F, ph, pw) == pytest.approx(a, rel=1e-12)
+        per = [O.row_similarity(q, k, F, ph, pw, [f]) for f in range(F)]
+        assert a == pytest.approx(np.mean(per), rel=1e-12)
+        assert 0.0 < a < 1.0
+
+    def test_threshold_is_strict(self):
+        assert not O.is_repetitive(0.87)
+        assert O.is_repetitive(0.87 + 1e-9)
+        assert not O.is_repetitive(0.5)
+
+    def test_anchor_rows(self):
+        assert O.anchor_rows(30, 5).tolist() == [3, 9, 15, 21, 27]
+        assert O.anchor_rows(45, 5).tolist() == [4, 13, 22, 31, 40]
+        assert O.anchor_rows(4, 5).tolist() == [0, 1, 2, 3]
+        assert O.anchor_rows(6, 5).tolist() == [1, 2, 3, 4, 5]  # bands [0,2) [2] [3] [4] [5]
+        assert O.anchor_rows(7, 2).tolist() == [2, 5]           # bands [0,4) [4,7)
+        for ph in range(1, 50):
+            for k in (1, 2, 5, 7):
+                a, src = O.anchor_rows(ph, k), O.row_anchor(ph, k)
+                assert len(a) == min(k, ph) and (np.diff(a) > 0).all()
+                assert (src[a] == a).all()          # an anchor takes itself
+                assert set(src.tolist()) == set(a.tolist())
+                assert (np.diff(src) >= 0).all()    # bands are contiguous
+                # every row takes the anchor of its own band floor(y k / ph)
+                for y in range(ph):
+                    if k < ph:
+                        assert (src[y] * k) // ph == (y * k) // ph
+                    assert abs(y - src[y]) <= (ph + k - 1) // k
+
+    def test_broadcast_rows(self):
+        F, ph, pw, d = 2, 7, 3, 2
+        o = np.arange(F * ph * pw * d, dtype=np.float64).reshape(-1, d)
+        b = O.broadcast_rows(o, F, ph, pw, 3)
+        src = O.row_anchor(ph, 3)
+        for f in range(F):
+            for y in range(ph):
+                for x in range(pw):
+                    n, m = f * ph * pw + y * pw + x, f * ph * pw + src[y] * pw + x
+                    assert (b[n] == o[m]).all()
+        np.testing.assert_array_equal(O.broadcast_rows(o, F, ph, pw, ph), o)
+
+    def test_anchor_tile_lists_brute_force(self):
+        F, ph, pw, T = 3, 20, 13, 16
+        N = F * ph * pw
+        ip, ix = O.geometric_block_lists(O.MODE_SPATIAL, F, ph * pw, 1, N, T)
+        aip, aix = O.anchor_tile_lists(ip, ix, F, ph, pw, 5, T)
+        anchors = set(O.anchor_rows(ph, 5).tolist())
+        for i in range(len(ip) - 1):
+            has = any(((n % (ph * pw)) // pw) in anchors for n in range(i * T, min(N, i * T + T)))
+            got = aix[aip[i]:aip[i + 1]].tolist()
+            assert got == (ix[ip[i]:ip[i + 1]].tolist() if has else [])
+        assert aip[-1] < ip[-1]  # some tiles hold no anchor row
+
+    def test_repeat_head_is_broadcast_of_full_attention(self):
+        F, ph, pw, d, T = 3, 6, 10, 8, 16
+        N = F * ph * pw
+        q, k, v = rand((N, d), 27), rand((N, d), 28), rand((N, d), 29)
+        ip, ix = O.geometric_block_lists(O.MODE_SPATIAL, F, ph * pw, 1, N, T)
+        full = O.block_sparse_attention(q, k, v, ip, ix, T)
+        got = O.repeat_head_attention(q, k, v, ip, ix, F, ph, pw, 2, T)
+        np.testing.assert_allclose(got, O.broadcast_rows(full, F, ph, pw, 2), rtol=1e-13,
+                                   atol=1e-14)
+        # anchor rows are exactly the full layer's rows
+        on = O.anchor_token_mask(F, ph, pw, 2)
+        np.testing.assert_allclose(got[on], full[on], rtol=1e-13, atol=1e-14)
