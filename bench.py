@@ -53,8 +53,8 @@ def load_peaks():
 # layer, from an ncu capture of the kernel built from the sources whose
 # sha256 is recorded here.  Reported only while the sources still match.
 ATTN_SOURCES = ("attn_sm100.cu", "sm100.cuh", "attn.cuh", "common.cuh")
-ATTN_TRAFFIC = {"cogvideox": {"sha256": "69b305cdbe530f99bc8a8765c1846ab9b147187ad62f564c4cb15e738271a2c4",
-                              "bytes": 328518912 + 84531456}}
+ATTN_TRAFFIC = {"cogvideox": {"sha256": "5793729729a2ea2d4d1d452ea9e0c9819a1ec3f6f3b12116b7b62140d84f2c2b",
+                              "bytes": 330266368 + 84697856}}
 
 
 def attn_sources_sha256():
@@ -342,6 +342,33 @@ def run_ours(args, rank, world, local_rank):
                                       svg.svg_layer(qn, kn, vd, F, P, w, idx_d, lists, bufs)))
     del qk_bufs, qn, kn
 
+    # spatial-repetition heads ([CAL] 3.2): the row-similarity test on one
+    # frame of every head, and the layer with every spatial head taken as
+    # repeating (anchor tiles only, then the broadcast)
+    ph, pw = wl.ph, wl.pw
+    mid = torch.tensor([F // 2], dtype=torch.int32, device=dev)
+    rs_ws = torch.empty(max(256, svg._lib.lib.svg_row_similarity_workspace_size(
+        svg._lib.SVG_BF16, wl.B, wl.H, ph, pw, 1)), dtype=torch.uint8, device=dev)
+    sims = svg.svg_row_similarity(qd, kd, F, ph, pw, mid, workspace=rs_ws)
+    rs_ms = timed(lambda: svg.svg_row_similarity(qd, kd, F, ph, pw, mid, out=sims,
+                                                 workspace=rs_ws))
+    sims_h = sims.cpu().numpy()
+    rep_all = torch.from_numpy((modes == 0).astype(np.int32)).to(dev)  # every spatial head
+    modes_d = torch.from_numpy(modes.astype(np.int32)).to(dev)  # this layer's profiled modes
+    alists, ids = svg.svg_anchor_lists(lists, N, F, ph, pw, modes_d, rep_all,
+                                       skip_list=svg._lib.SVG_MODE_TEMPORAL)
+    rep_attn_ms = timed(lambda: svg.svg_sparse_attn_fused(
+        qd, kd, vd, F, P, ids, alists, layout=svg._lib.SVG_FUSE_OUTPUT,
+        copies=(bufs.qp, bufs.kp, bufs.vp), out=bufs.o))
+    rep_layer_ms = timed(lambda: svg.svg_layer(qd, kd, vd, F, P, w, idx_d, lists, bufs,
+                                               repeat=rep_all, frame_shape=(ph, pw)))
+    aip = alists.indptr.cpu().numpy().reshape(6, nb + 1)
+    aix = alists.indices.cpu().numpy()
+    anchor_pairs = kept_pairs(aip[3] - aip[3][0], aix[aip[3][0]:aip[3][-1]], N)
+    rep_attn_pairs_ms = timed(lambda: svg.svg_sparse_attn_fused(
+        qd, kd, vd, F, P, ids, alists._replace(tile_order=None),
+        layout=svg._lib.SVG_FUSE_OUTPUT, copies=(bufs.qp, bufs.kp, bufs.vp), out=bufs.o))
+
     # end to end through the public API with host buffers
     out_host = torch.empty(qd.shape, dtype=torch.bfloat16).pin_memory()
     mode_host = torch.empty(modes.shape, dtype=torch.int32).pin_memory()
@@ -367,9 +394,10 @@ def run_ours(args, rank, world, local_rank):
     e2e_ms = e0.elapsed_time(e1)
 
     (total_ms, e2e_ms, attn_avg, prof_avg, perm_avg, unf_avg, fwd_perm_avg, qk_ms, qk_layer_ms,
-     qk_then_layer_ms) = max_over_ranks(
+     qk_then_layer_ms, rs_ms, rep_attn_ms, rep_layer_ms, rep_attn_pairs_ms) = max_over_ranks(
         [total_ms, e2e_ms, attn_avg, prof_avg, perm_avg, unf_avg, fwd_perm_avg, qk_ms,
-         qk_layer_ms, qk_then_layer_ms], world, dev)
+         qk_layer_ms, qk_then_layer_ms, rs_ms, rep_attn_ms, rep_layer_ms, rep_attn_pairs_ms],
+        world, dev)
     if rank != 0:
         return None
 
@@ -429,6 +457,16 @@ def run_ours(args, rank, world, local_rank):
         "layer_with_qk_norm_rope_modes": {"spatial": int((qk_modes == 0).sum()),
                                           "temporal": int((qk_modes == 1).sum())},
         "qk_norm_rope_then_layer_ms": round(qk_then_layer_ms, 5),
+        "repeat_heads": {
+            "similarity_one_frame_ms": round(rs_ms, 5),
+            "similarity": {"min": round(float(sims_h.min()), 4),
+                           "max": round(float(sims_h.max()), 4),
+                           "above_0.87": int((sims_h > 0.87).sum())},
+            "spatial_kept_fraction_anchor_tiles": round(anchor_pairs / float(N * N), 5),
+            "attention_ms_spatial_heads_repeating": round(rep_attn_ms, 5),
+            "attention_ms_spatial_heads_repeating_index_pairs": round(rep_attn_pairs_ms, 5),
+            "layer_ms_spatial_heads_repeating": round(rep_layer_ms, 5),
+            "note": "anchors k=5 per frame; every spatial head forced to repeat for timing"},
         "profile": {"ms": round(prof_avg, 5),
                     "kv_gbs": round(prof_bytes / (prof_avg * 1e-3) / 1e9, 1)},
         "roofline": {"kernel": "svg_sparse_attn_fused", "bound": "tensor",

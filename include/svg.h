@@ -15,7 +15,9 @@
  *      svg_build_block_mask_calibrated   lists from cumulative-energy calibration;
  *   4. svg_sparse_attn          block-sparse attention over 128x128 tiles that
  *                               walks only the kept key blocks;
- *   5. svg_permute_frame_major  the inverse reordering of the output.
+ *   5. svg_permute_frame_major  the inverse reordering of the output;
+ *   6. svg_row_similarity, svg_anchor_lists, svg_row_broadcast
+ *                               spatial-repetition heads (anchor rows only).
  *
  * Sources (cited by page title and section):
  *   [SVG]  Sparse VideoGen article, m.jxzklqfsx.com/article/815093.html
@@ -398,6 +400,14 @@ svg_status svg_sparse_attn(const void* q, const void* k, const void* v, void* o,
  *               svg_sparse_attn, e.g. the profiling output with the three
  *               geometric lists concatenated) and its token order.
  *  layout       0 or an OR of SVG_FUSE_INPUT and SVG_FUSE_OUTPUT.
+ *  tile_order   device int32 [n_lists][n_qblocks] or NULL: per list, the
+ *               query tiles in the order the kernel pairs them into work
+ *               items (each row a permutation of 0 .. n_qblocks-1, e.g. from
+ *               svg_anchor_lists, which puts the tiles with work first).
+ *               A scheduling choice only: results do not depend on it.  An
+ *               entry outside [0, n_qblocks) is skipped and sets
+ *               SVG_DEVICE_BAD_INDEX; a row that is not a permutation leaves
+ *               missing tiles unwritten.  fp32 inputs ignore it.
  *  Other arguments, errors and arithmetic as in svg_sparse_attn; a mode
  *  outside [0, n_lists) sets SVG_DEVICE_BAD_LIST_ID and gives o = 0 for the
  *  head.
@@ -407,8 +417,87 @@ svg_status svg_sparse_attn_fused(const void* q, const void* k, const void* v,
                                  int dtype, int B, int H, int N, int d, int frames,
                                  int tokens_per_frame, const int32_t* mode, int layout,
                                  int n_lists, int n_qblocks, const int32_t* indptr,
-                                 const int32_t* indices, float scale, int32_t* device_status,
-                                 void* stream);
+                                 const int32_t* indices, const int32_t* tile_order, float scale,
+                                 int32_t* device_status, void* stream);
+
+/* --------------------------------------------------------------------------
+ * 6. Spatial-repetition heads
+ *    [CAL] section 3.2: in some heads the image rows of a frame attend almost
+ *    alike.  They are found by the mean cosine similarity of the rows'
+ *    attention patterns (repeating when it exceeds gamma = 0.87, a caller
+ *    decision on the returned value); for them only k = 5 equally spaced
+ *    anchor rows per frame are computed and every other row takes its
+ *    anchor's output.  A frame is `rows` x `cols` tokens (P = rows * cols,
+ *    token n = f P + y cols + x).  Anchors: band j holds the rows y with
+ *    floor(y k / rows) = j; its anchor is the band's middle row (the upper
+ *    of two); every row is an anchor when k >= rows.
+ *
+ *  svg_row_similarity -- per head, for each evaluated frame the mean over
+ *    all row pairs y < y' of cos(A_y, A_y') = <A_y, A_y'> / (|A_y| |A_y'|),
+ *    A_y = the cols x N block of dense attention probabilities
+ *    softmax(q k^T / sqrt(d)) of row y's tokens over all N keys (Frobenius
+ *    products); then the mean over the evaluated frames.
+ *      q, k          device [B, H, N, d], frame-major; N = frames*rows*cols.
+ *      rows          2 .. 128.
+ *      eval_frames   device int32 [n_frames] frame indices, or NULL for
+ *                    frames 0 .. n_frames-1.  Out-of-range values are
+ *                    clamped and flagged (SVG_DEVICE_BAD_INDEX).
+ *      sim_out       device float [B*H].
+ *      workspace     device scratch of svg_row_similarity_workspace_size().
+ *    Arithmetic (bf16): scores on bf16 tensor cores with fp32 accumulation,
+ *    probabilities exp2(t - lse) rounded to fp16 and multiplied on fp16
+ *    tensor cores with fp32 accumulation; fp32 inputs: fp32 SIMT.  An
+ *    offline step (two dense passes over the evaluated frames' queries).
+ *
+ *  svg_anchor_lists -- lists for a layer with repeating heads.  Output lists
+ *    0 .. n_lists-1 are the input lists; lists n_lists .. 2 n_lists-1 are
+ *    copies in which every query tile that holds no anchor-row token has an
+ *    empty list (its rows are all filled by svg_row_broadcast).
+ *      indptr, indices  input CSR as for svg_sparse_attn (n_qblocks = nB).
+ *      list_id, repeat  device int32 [n_heads]: a head with repeat != 0 and
+ *                    a list id in [0, n_lists) other than skip_list gets
+ *                    list_id + n_lists in list_id_out; others keep theirs.
+ *                    repeat may be NULL (no head moves).  skip_list: a list
+ *                    id never moved (e.g. SVG_MODE_TEMPORAL, whose heads
+ *                    run token-major), or -1.  list_id NULL builds the lists
+ *                    (and order) only; svg_anchor_list_ids then maps the ids
+ *                    alone, e.g. every step for lists built once.
+ *      out_indptr    device int32 [2 n_lists][n_qblocks + 1], absolute.
+ *      out_indices   device int32 [capacity]; 2 x the input entries always
+ *                    fit.  Entries past capacity are not written
+ *                    (SVG_DEVICE_CAPACITY).
+ *      list_id_out   device int32 [n_heads].
+ *      tile_order_out  device int32 [2 n_lists][n_qblocks] or NULL: per
+ *                    output list the pairing order for svg_sparse_attn_fused
+ *                    (index order for the first n_lists; for the copies the
+ *                    tiles holding anchor rows first, then the others).
+ *
+ *  svg_row_broadcast -- in place on o [B, H, N, d] (frame-major): for each
+ *    head with list_id[b*H+h] >= n_lists (as set by svg_anchor_lists), row
+ *    (f, y, x) takes the value of row (f, anchor(y), x); anchor rows and
+ *    other heads are untouched.
+ * ------------------------------------------------------------------------ */
+size_t svg_row_similarity_workspace_size(int dtype, int B, int H, int rows, int cols,
+                                         int n_frames);
+
+svg_status svg_row_similarity(const void* q, const void* k, int dtype, int B, int H, int N, int d,
+                              int frames, int rows, int cols, const int32_t* eval_frames,
+                              int n_frames, float* sim_out, void* workspace,
+                              size_t workspace_bytes, int32_t* device_status, void* stream);
+
+svg_status svg_anchor_lists(int n_lists, int n_qblocks, const int32_t* indptr,
+                            const int32_t* indices, int N, int frames, int rows, int cols,
+                            int anchors, const int32_t* list_id, const int32_t* repeat,
+                            int n_heads, int skip_list, int32_t* out_indptr,
+                            int32_t* out_indices, int64_t capacity, int32_t* list_id_out,
+                            int32_t* tile_order_out, int32_t* device_status, void* stream);
+
+svg_status svg_anchor_list_ids(const int32_t* list_id, const int32_t* repeat, int n_heads,
+                               int n_lists, int skip_list, int32_t* list_id_out, void* stream);
+
+svg_status svg_row_broadcast(void* o, int dtype, int B, int H, int N, int d, int frames, int rows,
+                             int cols, int anchors, const int32_t* list_id, int n_lists,
+                             void* stream);
 
 #ifdef __cplusplus
 }

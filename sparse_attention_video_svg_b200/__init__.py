@@ -37,7 +37,8 @@ __all__ = [
     "svg_permute_frame_major", "svg_build_block_mask", "svg_block_energy",
     "svg_build_block_mask_calibrated", "svg_sparse_attn", "svg_sparse_attn_fused",
     "svg_epsilon_schedule", "svg_lists_to_intervals", "svg_lists_to_bitmap", "geometric_lists",
-    "QKTransform", "svg_qk_norm_rope", "svg_layer",
+    "QKTransform", "svg_qk_norm_rope", "svg_row_similarity", "svg_anchor_lists",
+    "svg_anchor_list_ids", "svg_row_broadcast", "svg_repeat_attention", "svg_layer",
     "n_tiles",
 ]
 
@@ -90,6 +91,9 @@ class BlockLists(NamedTuple):
     indices: torch.Tensor
     n_lists: int
     n_qblocks: int
+    # optional int32 [n_lists * n_qblocks]: per list, the order in which the
+    # attention kernel pairs query tiles (scheduling only)
+    tile_order: Optional[torch.Tensor] = None
 
 
 # --------------------------------------------------------------------- steps
@@ -229,7 +233,8 @@ def svg_sparse_attn_fused(q, k, v, frames: int, tokens_per_frame: int, mode: tor
     _lib.call("svg_sparse_attn_fused", q.data_ptr(), k.data_ptr(), v.data_ptr(), qt, kt, vt,
               out.data_ptr(), _dt(q), B, H, N, d, frames, tokens_per_frame, mode.data_ptr(),
               int(layout), lists.n_lists, lists.n_qblocks, lists.indptr.data_ptr(),
-              lists.indices.data_ptr(), float(scale), _ptr(status), _stream(stream))
+              lists.indices.data_ptr(), _ptr(lists.tile_order), float(scale), _ptr(status),
+              _stream(stream))
     return out
 
 
@@ -267,6 +272,93 @@ def svg_qk_norm_rope(q, k, qk: QKTransform, *, out=None, tm_out=None, frames: in
               ops, _ptr(qk.gamma_q), _ptr(qk.gamma_k), float(qk.eps), _ptr(qk.cos), _ptr(qk.sin),
               _stream(stream))
     return out
+
+
+# ------------------------------------------------ spatial-repetition heads
+
+def svg_row_similarity(q, k, frames: int, rows: int, cols: int, eval_frames=None, *,
+                       n_frames: Optional[int] = None, out=None, workspace=None, status=None,
+                       stream=None):
+    """Mean row-pattern cosine similarity per head ([CAL] 3.2) over the
+    frames in eval_frames (int32 CUDA tensor) or frames 0 .. n_frames-1
+    (all frames when both are None).  Returns float32 [B*H]."""
+    B, H, N, d = _check_qkv(q, k)
+    if eval_frames is None:
+        nf = frames if n_frames is None else int(n_frames)
+        fptr = None
+    else:
+        nf = eval_frames.numel()
+        fptr = eval_frames.data_ptr()
+    if out is None:
+        out = torch.empty(B * H, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = _scratch(_lib.lib.svg_row_similarity_workspace_size(
+            _dt(q), B, H, rows, cols, nf), q.device)
+    _lib.call("svg_row_similarity", q.data_ptr(), k.data_ptr(), _dt(q), B, H, N, d, frames, rows,
+              cols, fptr, nf, out.data_ptr(), workspace.data_ptr(), workspace.numel(),
+              _ptr(status), _stream(stream))
+    return out
+
+
+def svg_anchor_lists(lists: BlockLists, N: int, frames: int, rows: int, cols: int,
+                     list_id: Optional[torch.Tensor] = None,
+                     repeat: Optional[torch.Tensor] = None, *, anchors: int = 5,
+                     skip_list: int = -1, status=None, stream=None):
+    """Lists 0 .. L-1 unchanged, L .. 2L-1 with anchor-free query tiles
+    emptied (with a pairing order that puts the tiles with work first);
+    repeating heads move to the second half.  Returns (BlockLists with 2L
+    lists, list_id_out), list_id_out None when list_id is None."""
+    L, nqb = lists.n_lists, lists.n_qblocks
+    dev = lists.indptr.device
+    indptr = torch.empty(2 * L * (nqb + 1), dtype=torch.int32, device=dev)
+    cap = max(2 * lists.indices.numel(), 1)
+    indices = torch.empty(cap, dtype=torch.int32, device=dev)
+    ids = None if list_id is None else torch.empty_like(list_id)
+    order = torch.empty(2 * L * nqb, dtype=torch.int32, device=dev)
+    _lib.call("svg_anchor_lists", L, nqb, lists.indptr.data_ptr(), lists.indices.data_ptr(), N,
+              frames, rows, cols, int(anchors), _ptr(list_id), _ptr(repeat),
+              0 if list_id is None else list_id.numel(), int(skip_list), indptr.data_ptr(),
+              indices.data_ptr(), cap, _ptr(ids), order.data_ptr(), _ptr(status),
+              _stream(stream))
+    return BlockLists(indptr, indices, 2 * L, nqb, order), ids
+
+
+def svg_anchor_list_ids(list_id: torch.Tensor, repeat: Optional[torch.Tensor], n_lists: int, *,
+                        skip_list: int = -1, out=None, stream=None):
+    """list_id + n_lists for heads with repeat != 0 (and a list other than
+    skip_list), list_id otherwise."""
+    if out is None:
+        out = torch.empty_like(list_id)
+    _lib.call("svg_anchor_list_ids", list_id.data_ptr(), _ptr(repeat), list_id.numel(),
+              int(n_lists), int(skip_list), out.data_ptr(), _stream(stream))
+    return out
+
+
+def svg_row_broadcast(o, frames: int, rows: int, cols: int, list_id: torch.Tensor, n_lists: int,
+                      *, anchors: int = 5, stream=None):
+    """In place: non-anchor rows of heads with list_id >= n_lists take their
+    anchor row's output."""
+    B, H, N, d = _check_qkv(o)
+    _lib.call("svg_row_broadcast", o.data_ptr(), _dt(o), B, H, N, d, frames, rows, cols,
+              int(anchors), list_id.data_ptr(), int(n_lists), _stream(stream))
+    return o
+
+
+def svg_repeat_attention(q, k, v, frames: int, rows: int, cols: int, list_id: torch.Tensor,
+                         lists: BlockLists, repeat: torch.Tensor, *, anchors: int = 5,
+                         skip_list: int = -1, out=None, status=None, stream=None):
+    """Block-sparse attention in which heads flagged in `repeat` compute
+    only the query tiles holding anchor rows and broadcast the anchors'
+    outputs to the other rows."""
+    N = q.shape[2]
+    alists, ids = svg_anchor_lists(lists, N, frames, rows, cols, list_id, repeat,
+                                   anchors=anchors, skip_list=skip_list, status=status,
+                                   stream=stream)
+    # layout 0: svg_sparse_attn with list_id = ids, plus the pairing order
+    o = svg_sparse_attn_fused(q, k, v, frames, rows * cols, ids, alists, layout=0, out=out,
+                              status=status, stream=stream)
+    svg_row_broadcast(o, frames, rows, cols, ids, lists.n_lists, anchors=anchors, stream=stream)
+    return o
 
 
 # ------------------------------------------- threshold schedule, mask encodings
@@ -340,7 +432,8 @@ class LayerBuffers:
 def svg_layer(q, k, v, frames: int, tokens_per_frame: int, spatial_width: int,
               sample_idx: torch.Tensor, lists: BlockLists, bufs: Optional[LayerBuffers] = None,
               stream=None, layout: int = _lib.SVG_FUSE_OUTPUT, overlap: bool = True,
-              qk: Optional[QKTransform] = None):
+              qk: Optional[QKTransform] = None, repeat: Optional[torch.Tensor] = None,
+              frame_shape: Optional[Sequence[int]] = None, anchors: int = 5):
     """One attention layer: profile -> block-sparse attention on the list the
     mode selects, temporal heads in token-major order.  `layout` picks which
     side of the reordering runs inside the attention kernel
@@ -352,10 +445,37 @@ def svg_layer(q, k, v, frames: int, tokens_per_frame: int, spatial_width: int,
     qk applies QK-Norm + RoPE to q and k first (svg_qk_norm_rope); with
     overlap that pass also writes the token-major copies of q and k, and only
     v is permuted on the side stream.
+    repeat (int32 [B*H], nonzero = spatially repeating head, e.g. from
+    svg_row_similarity > 0.87) with frame_shape = (rows, cols): those heads,
+    unless profiled temporal, compute only the query tiles holding anchor
+    rows and take the anchors' outputs on the other rows.
     Returns (o, mode, mse)."""
     if bufs is None:
         bufs = LayerBuffers(q, sample_idx.numel(), layout, qk=qk is not None)
     F, P = frames, tokens_per_frame
+    if repeat is not None and (frame_shape is None or frame_shape[0] * frame_shape[1] != P):
+        raise ValueError("repeat needs frame_shape = (rows, cols) with rows * cols = P")
+
+    def select_lists(st):
+        """The lists and per-head ids the attention runs with (anchor lists
+        are built once per buffers, lists and frame shape)."""
+        if repeat is None:
+            return lists, bufs.mode
+        key = (lists.indptr.data_ptr(), lists.indices.data_ptr(), tuple(frame_shape), anchors)
+        cached = getattr(bufs, "anchor_lists", None)
+        if cached is None or cached[0] != key:
+            alists, _ = svg_anchor_lists(lists, q.shape[2], F, frame_shape[0], frame_shape[1],
+                                         anchors=anchors, stream=st)
+            bufs.anchor_lists = cached = (key, alists, torch.empty_like(bufs.mode))
+        _, alists, ids = cached
+        svg_anchor_list_ids(bufs.mode, repeat, lists.n_lists, skip_list=SVG_MODE_TEMPORAL,
+                            out=ids, stream=st)
+        return alists, ids
+
+    def broadcast(ids, st):
+        if repeat is not None:
+            svg_row_broadcast(bufs.o, F, frame_shape[0], frame_shape[1], ids, lists.n_lists,
+                              anchors=anchors, stream=st)
     if overlap and not layout & _lib.SVG_FUSE_INPUT:
         # token-major copies of every head on a side stream, concurrent with
         # the (latency-bound) profiling; temporal heads read the copies
@@ -384,10 +504,12 @@ def svg_layer(q, k, v, frames: int, tokens_per_frame: int, spatial_width: int,
         for t in (bufs.qp, bufs.kp, bufs.vp):
             t.record_stream(main)
         out = bufs.o if layout & _lib.SVG_FUSE_OUTPUT else bufs.op
-        svg_sparse_attn_fused(q, k, v, F, P, bufs.mode, lists, layout=layout,
+        use_lists, ids = select_lists(main)
+        svg_sparse_attn_fused(q, k, v, F, P, ids, use_lists, layout=layout,
                               copies=(bufs.qp, bufs.kp, bufs.vp), out=out, stream=main)
         if not layout & _lib.SVG_FUSE_OUTPUT:
             svg_permute_frame_major(bufs.op, F, P, bufs.mode, out=bufs.o, stream=main)
+        broadcast(ids, main)
         return bufs.o, bufs.mode, bufs.mse
     if qk is not None:
         svg_qk_norm_rope(q, k, qk, out=(bufs.qn, bufs.kn), stream=stream)
@@ -400,11 +522,13 @@ def svg_layer(q, k, v, frames: int, tokens_per_frame: int, spatial_width: int,
         for x, y in ((q, bufs.qp), (k, bufs.kp), (v, bufs.vp)):
             svg_permute_token_major(x, F, P, bufs.mode, out=y, stream=stream)
         ins = (bufs.qp, bufs.kp, bufs.vp)
+    use_lists, ids = select_lists(stream)
     if layout & _lib.SVG_FUSE_OUTPUT:
-        svg_sparse_attn_fused(*ins, F, P, bufs.mode, lists, layout=layout, out=bufs.o,
+        svg_sparse_attn_fused(*ins, F, P, ids, use_lists, layout=layout, out=bufs.o,
                               stream=stream)
     else:
-        svg_sparse_attn_fused(*ins, F, P, bufs.mode, lists, layout=layout, out=bufs.op,
+        svg_sparse_attn_fused(*ins, F, P, ids, use_lists, layout=layout, out=bufs.op,
                               stream=stream)
         svg_permute_frame_major(bufs.op, F, P, bufs.mode, out=bufs.o, stream=stream)
+    broadcast(ids, stream)
     return bufs.o, bufs.mode, bufs.mse

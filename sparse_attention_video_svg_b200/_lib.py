@@ -50,9 +50,16 @@ SIGNATURES = {
     "svg_lists_to_intervals": (_i, [_i, _i, _p, _p, _p, _p, _p, C.c_int64, _p, _p, _p]),
     "svg_lists_to_bitmap": (_i, [_i, _i, _p, _p, _p, _p, _p]),
     "svg_sparse_attn_fused": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p,
-                                   _i, _i, _i, _p, _p, _f, _p, _p]),
+                                   _i, _i, _i, _p, _p, _p, _f, _p, _p]),
     "svg_qk_norm_rope": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _p, _p, _f,
                               _p, _p, _p]),
+    "svg_row_similarity_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "svg_row_similarity": (_i, [_p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _p, _i, _p, _p, _sz, _p,
+                                _p]),
+    "svg_anchor_lists": (_i, [_i, _i, _p, _p, _i, _i, _i, _i, _i, _p, _p, _i, _i, _p, _p, _i64,
+                              _p, _p, _p, _p]),
+    "svg_anchor_list_ids": (_i, [_p, _p, _i, _i, _i, _p, _p]),
+    "svg_row_broadcast": (_i, [_p, _i, _i, _i, _i, _i, _i, _i, _i, _i, _p, _i, _p]),
 }
 
 

@@ -34,6 +34,11 @@ struct AttnArgs {
   const void* q_tm;
   const void* k_tm;
   const void* v_tm;
+  // Optional [n_lists][n_qblocks] pairing order: the tcgen05 kernel takes
+  // the query tiles of a head two at a time in this order (a permutation of
+  // 0 .. n_qblocks-1 per list); null = index order.  Results never depend
+  // on it.
+  const int32_t* tile_order;
 };
 
 __device__ __forceinline__ bool reads_copies(const AttnArgs& a, int bh);
@@ -49,6 +54,17 @@ __device__ __forceinline__ bool scatters_output(const AttnArgs& a, int bh) {
 }
 __device__ __forceinline__ bool reads_copies(const AttnArgs& a, int bh) {
   return a.q_tm != nullptr && temporal_head(a, bh);
+}
+
+// Query tile in pairing slot `slot` of head bh (the list's tile order, or
+// the slot itself); -1 past the end or for an out-of-range order entry.
+__device__ __forceinline__ int query_tile(const AttnArgs& a, int bh, int slot, int nb) {
+  if (slot >= nb) return -1;
+  if (a.tile_order == nullptr) return slot;
+  const int lid = a.list_id[bh];
+  if (lid < 0 || lid >= a.n_lists) return slot;  // the list walk reports the bad id
+  const int qt = a.tile_order[static_cast<long long>(lid) * a.n_qblocks + slot];
+  return (qt >= 0 && qt < nb) ? qt : -1;
 }
 
 // Frame-major memory row of token-major row m.

@@ -12,7 +12,8 @@ svg_status sparse_attn_impl(const char* who, const void* q, const void* k, const
                             int n_lists, int n_qblocks, const int32_t* indptr,
                             const int32_t* indices, float scale, int32_t* device_status,
                             const int32_t* order, int frames, int tokens_per_frame, int layout,
-                            const void* q_tm, const void* k_tm, const void* v_tm, void* stream) {
+                            const void* q_tm, const void* k_tm, const void* v_tm,
+                            const int32_t* tile_order, void* stream) {
   clear_error();
   if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || list_id == nullptr ||
       indptr == nullptr || indices == nullptr)
@@ -51,7 +52,7 @@ svg_status sparse_attn_impl(const char* who, const void* q, const void* k, const
   if (!(scale >= 0.f) || isinf(scale)) return fail(SVG_ERR_INVALID_ARG, "%s: bad scale", who);
   AttnArgs a{q, k, v, o, dtype, B, H, N, d, list_id, n_lists, n_qblocks, indptr, indices,
              scale == 0.f ? 1.f / sqrtf(static_cast<float>(d)) : scale, device_status,
-             order, frames, tokens_per_frame, layout, q_tm, k_tm, v_tm};
+             order, frames, tokens_per_frame, layout, q_tm, k_tm, v_tm, tile_order};
   cudaStream_t s = as_stream(stream);
   if (dtype == SVG_FP32) return d == 64 ? launch_attn_fp32<64>(a, s) : launch_attn_fp32<128>(a, s);
   return d == 64 ? launch_attn_sm100<64>(a, s) : launch_attn_sm100<128>(a, s);
@@ -66,7 +67,7 @@ extern "C" svg_status svg_sparse_attn(const void* q, const void* k, const void* 
                                       int32_t* device_status, void* stream) {
   return sparse_attn_impl("sparse_attn", q, k, v, o, dtype, B, H, N, d, list_id, n_lists,
                           n_qblocks, indptr, indices, scale, device_status, nullptr, 0, 0, 0,
-                          nullptr, nullptr, nullptr, stream);
+                          nullptr, nullptr, nullptr, nullptr, stream);
 }
 
 extern "C" svg_status svg_sparse_attn_fused(const void* q, const void* k, const void* v,
@@ -75,9 +76,9 @@ extern "C" svg_status svg_sparse_attn_fused(const void* q, const void* k, const 
                                             int N, int d, int frames, int tokens_per_frame,
                                             const int32_t* mode, int layout, int n_lists,
                                             int n_qblocks, const int32_t* indptr,
-                                            const int32_t* indices, float scale,
-                                            int32_t* device_status, void* stream) {
+                                            const int32_t* indices, const int32_t* tile_order,
+                                            float scale, int32_t* device_status, void* stream) {
   return sparse_attn_impl("sparse_attn_fused", q, k, v, o, dtype, B, H, N, d, mode, n_lists,
                           n_qblocks, indptr, indices, scale, device_status, mode, frames,
-                          tokens_per_frame, layout, q_tm, k_tm, v_tm, stream);
+                          tokens_per_frame, layout, q_tm, k_tm, v_tm, tile_order, stream);
 }

@@ -128,7 +128,7 @@ constexpr uint32_t kStepGathered = 1u << 7;  // Q / K / V of this step came thro
 __device__ __forceinline__ void member_list(const AttnArgs& a, int bh, int qt, int nb, int& beg,
                                             int& end, bool report) {
   beg = end = 0;
-  if (qt >= nb) return;
+  if (qt < 0 || qt >= nb) return;
   const int lid = a.list_id[bh];
   if (lid < 0 || lid >= a.n_lists) {
     if (report) set_status(a.status, SVG_DEVICE_BAD_LIST_ID);
@@ -216,8 +216,8 @@ __device__ __forceinline__ void softmax_member(const AttnArgs& a, const Bars& B,
   bool ok = true;
   for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
     const int bh = item / n_pairs;
-    const int qt = 2 * (item - bh * n_pairs) + t;
-    if (qt >= nb) continue;
+    const int qt = query_tile(a, bh, 2 * (item - bh * n_pairs) + t, nb);
+    if (qt < 0) continue;
     int beg, end;
     member_list(a, bh, qt, nb, beg, end, false);
     float m_used = -INFINITY, l = 0.f;
@@ -444,10 +444,12 @@ __device__ __forceinline__ void producer(const AttnArgs& a, const Maps& maps, co
     const CUtensorMap* mk = cp ? &maps.kt : &maps.k;
     const CUtensorMap* mv = cp ? &maps.vt : &maps.v;
     const long long head = static_cast<long long>(bh) * N * D;
-    int p[2], e[2];
+    int p[2], e[2], qtile[2];
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
-      member_list(a, bh, qt0 + t, nb, p[t], e[t], leader);
+      qtile[t] = query_tile(a, bh, qt0 + t, nb);
+      if (qtile[t] < 0 && qt0 + t < nb && leader) set_status(a.status, SVG_DEVICE_BAD_INDEX);
+      member_list(a, bh, qtile[t], nb, p[t], e[t], leader);
       skip_invalid(a, nb, p[t], e[t], leader);
     }
 #pragma unroll
@@ -460,10 +462,10 @@ __device__ __forceinline__ void producer(const AttnArgs& a, const Maps& maps, co
         if (leader) {
           mbar_arrive_expect_tx(&B.q_full[qb], C::kTile);
           for (int bx = 0; bx < C::kBoxes; ++bx)
-            tma_load_3d(dst + bx * kBox, mq, &B.q_full[qb], 64 * bx, (qt0 + t) * 128, bh);
+            tma_load_3d(dst + bx * kBox, mq, &B.q_full[qb], 64 * bx, qtile[t] * 128, bh);
         }
       } else {
-        gather_into(dst, static_cast<const __nv_bfloat16*>(a.q) + head, (qt0 + t) * 128,
+        gather_into(dst, static_cast<const __nv_bfloat16*>(a.q) + head, qtile[t] * 128,
                     &B.q_full[qb]);
       }
       ++cq[t];

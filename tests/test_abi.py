@@ -80,9 +80,9 @@ class TestHostValidation:
 
     def test_sparse_attn_fused(self):
         # q k v q_tm k_tm v_tm o dtype B H N d F P mode layout n_lists n_qblocks indptr
-        # indices scale status stream
+        # indices tile_order scale status stream
         base = [FAKE, FAKE2, FAKE3, None, None, None, FAKE4 * 4, 0, 1, 2, 256, 64, 4, 64, FAKE,
-                3, 3, 2, FAKE, FAKE, 0.0, None, None]
+                3, 3, 2, FAKE, FAKE, None, 0.0, None, None]
         expect(INVALID, "svg_sparse_attn_fused", *(base[:12] + [5] + base[13:]), match="frames")
         expect(INVALID, "svg_sparse_attn_fused", *(base[:11] + [96] + base[12:]), match="d=96")
         expect(INVALID, "svg_sparse_attn_fused", *(base[:14] + [None] + base[15:]), match="null")
@@ -111,6 +111,38 @@ class TestHostValidation:
         expect(INVALID, f, *(base[:10] + [96] + base[11:]), match="d=96")
         expect(INVALID, f, *(base[:6] + [3] + base[7:]), match="dtype")
         expect(INVALID, f, *([None] + base[1:]), match="null")
+
+    def test_repetition(self):
+        ws = L.svg_row_similarity_workspace_size(0, 1, 2, 4, 16, 2)
+        assert ws > 0
+        # q k dtype B H N d frames rows cols eval_frames n_frames sim ws ws_bytes status stream
+        base = [FAKE, FAKE2, 0, 1, 2, 256, 64, 4, 4, 16, None, 2, FAKE3, FAKE4 * 2, ws, None, None]
+        f = "svg_row_similarity"
+        expect(INVALID, f, *(base[:8] + [5] + base[9:]), match="!= N")
+        expect(INVALID, f, *(base[:7] + [256, 1, 1] + base[10:]), match="rows=1")
+        expect(INVALID, f, *(base[:11] + [5] + base[12:]), match="n_frames")
+        expect(INVALID, f, *(base[:14] + [ws - 256] + base[15:]), match="workspace")
+        expect(INVALID, f, *(base[:6] + [32] + base[7:]), match="d=32")
+        # n_lists nqb indptr indices N frames rows cols anchors list_id repeat n_heads skip
+        # out_indptr out_indices capacity list_id_out tile_order_out status stream
+        base = [3, 2, FAKE, FAKE2, 256, 4, 4, 16, 5, FAKE3, None, 2, 1, FAKE4, FAKE4 * 2, 100,
+                FAKE4 * 3, None, None, None]
+        f = "svg_anchor_lists"
+        expect(INVALID, f, *(base[:1] + [3] + base[2:]), match="n_qblocks")
+        expect(INVALID, f, *(base[:8] + [0] + base[9:]), match="anchors")
+        expect(INVALID, f, *(base[:15] + [0] + base[16:]), match="capacity")
+        expect(INVALID, f, *(base[:6] + [5] + base[7:]), match="!= N")
+        expect(INVALID, f, *(base[:2] + [None] + base[3:]), match="null")
+        # list_id given without list_id_out
+        expect(INVALID, f, *(base[:16] + [None] + base[17:]), match="null")
+        expect(INVALID, "svg_anchor_list_ids", FAKE, None, 0, 3, 1, FAKE2, None, match="sizes")
+        expect(INVALID, "svg_anchor_list_ids", FAKE, None, 4, 3, 1, None, None, match="null")
+        # o dtype B H N d frames rows cols anchors list_id n_lists stream
+        base = [FAKE, 0, 1, 2, 256, 64, 4, 4, 16, 5, FAKE2, 3, None]
+        f = "svg_row_broadcast"
+        expect(INVALID, f, *(base[:7] + [5] + base[8:]), match="!= N")
+        expect(INVALID, f, *(base[:11] + [0] + base[12:]), match="n_lists")
+        expect(INVALID, f, *([FAKE + 8] + base[1:]), match="aligned")
 
     def test_permute(self):
         args = [FAKE, FAKE4 * 4, 0, 1, 2, 12, 64, 3, 4, None, None]

@@ -736,3 +736,172 @@ def test_layer_small_with_qk_norm_rope(name, overlap):
             continue  # a near-tie decided the other way (checked above)
         b, h = divmod(bh, wl.H)
         assert_close(to_float64(o[b, h]), o_ref[b, h], f"{wl.name} head {h}")
+
+
+# ------------------------------------------- spatial-repetition heads (f4)
+
+def sim_tol(wl):
+    # probabilities are rounded to fp16 (2^-11 relative) before the Gram
+    # products: every G entry within 2^-10 relative, a cosine within 2e-3
+    return 2e-3 if wl.dtype == "bf16" else 1e-5
+
+
+@pytest.mark.parametrize("wl", SMALL, ids=lambda w: w.name)
+def test_row_similarity_small(wl):
+    (q, k, _), (qd, kd, _), _ = workload_tensors(wl)
+    sim = svg.svg_row_similarity(qd, kd, wl.F, wl.ph, wl.pw).cpu().numpy()
+    pick = [wl.F - 1, 1]
+    sub = torch.tensor(pick, dtype=torch.int32, device=DEV)
+    sim_sub = svg.svg_row_similarity(qd, kd, wl.F, wl.ph, wl.pw, sub).cpu().numpy()
+    for b in range(wl.B):
+        for h in range(wl.H):
+            q64, k64 = head64(q, b, h), head64(k, b, h)
+            want = O.row_similarity(q64, k64, wl.F, wl.ph, wl.pw)
+            want_sub = O.row_similarity(q64, k64, wl.F, wl.ph, wl.pw, pick)
+            i = b * wl.H + h
+            assert abs(sim[i] - want) <= sim_tol(wl), (wl.name, h, sim[i], want)
+            assert abs(sim_sub[i] - want_sub) <= sim_tol(wl), (wl.name, h, sim_sub[i], want_sub)
+
+
+def test_row_similarity_identical_rows():
+    # queries that depend on (frame, column) only: every row attends alike
+    wl = si.small("wan480")
+    (q, k, _), _, _ = workload_tensors(wl)
+    qr = q.reshape(wl.B, wl.H, wl.F, wl.ph, wl.pw, wl.d)
+    qr = np.ascontiguousarray(np.broadcast_to(qr[:, :, :, :1], qr.shape)).reshape(q.shape)
+    sim = svg.svg_row_similarity(to_device(qr), to_device(k), wl.F, wl.ph, wl.pw).cpu().numpy()
+    assert (np.abs(sim - 1.0) <= sim_tol(wl)).all(), sim
+    assert (sim > 0.87).all()
+    want = O.row_similarity(head64(qr, 0, 0), head64(k, 0, 0), wl.F, wl.ph, wl.pw)
+    assert want == pytest.approx(1.0, abs=1e-12)
+
+
+def test_row_similarity_full_sampled(full_inputs):
+    name = "cogvideox"
+    wl = si.WORKLOADS[name]
+    (q, k, _), (qd, kd, _), types = full_inputs(name)
+    frames = torch.tensor([6], dtype=torch.int32, device=DEV)
+    sim = svg.svg_row_similarity(qd, kd, wl.F, wl.ph, wl.pw, frames).cpu().numpy()
+    for h in (0, int(np.flatnonzero(types == 1)[0]), wl.H - 1):
+        want = O.row_similarity(head64(q, 0, h), head64(k, 0, h), wl.F, wl.ph, wl.pw, [6])
+        assert abs(sim[h] - want) <= sim_tol(wl), (h, sim[h], want)
+
+
+def test_anchor_lists_bit_exact():
+    wl = si.small("cogvideox")
+    lists = svg.geometric_lists(wl.F, wl.P, wl.width, wl.N)
+    nb = svg.n_tiles(wl.N)
+    rng = np.random.default_rng(5)
+    H = 12
+    lid = rng.integers(0, 3, size=H).astype(np.int32)
+    rep = rng.integers(0, 2, size=H).astype(np.int32)
+    alists, ids = svg.svg_anchor_lists(lists, wl.N, wl.F, wl.ph, wl.pw,
+                                       torch.from_numpy(lid).to(DEV),
+                                       torch.from_numpy(rep).to(DEV), skip_list=1)
+    ip = alists.indptr.cpu().numpy().reshape(6, nb + 1)
+    ix = alists.indices.cpu().numpy()
+    for c in range(6):
+        kind = c % 3
+        op, ox = O.geometric_block_lists(kind, wl.F, wl.P, wl.width, wl.N)
+        if c >= 3:
+            op, ox = O.anchor_tile_lists(op, ox, wl.F, wl.ph, wl.pw, 5)
+        np.testing.assert_array_equal(ip[c] - ip[c][0], op)
+        np.testing.assert_array_equal(ix[ip[c][0]:ip[c][-1]], ox)
+    want = np.where((rep != 0) & (lid != 1), lid + 3, lid)
+    np.testing.assert_array_equal(ids.cpu().numpy(), want)
+    # lists alone, then the ids alone, give the same
+    only, none = svg.svg_anchor_lists(lists, wl.N, wl.F, wl.ph, wl.pw)
+    assert none is None
+    np.testing.assert_array_equal(only.indptr.cpu().numpy(), alists.indptr.cpu().numpy())
+    n_used = int(ip[-1][-1])
+    np.testing.assert_array_equal(only.indices.cpu().numpy()[:n_used], ix[:n_used])
+    np.testing.assert_array_equal(only.tile_order.cpu().numpy(), alists.tile_order.cpu().numpy())
+    ids2 = svg.svg_anchor_list_ids(torch.from_numpy(lid).to(DEV), torch.from_numpy(rep).to(DEV),
+                                   3, skip_list=1)
+    np.testing.assert_array_equal(ids2.cpu().numpy(), want)
+    # pairing order: index order for the plain copies, tiles holding anchor
+    # rows first for the anchor copies
+    order = alists.tile_order.cpu().numpy().reshape(6, nb)
+    on = O.anchor_token_mask(wl.F, wl.ph, wl.pw, 5)
+    live = [i for i in range(nb) if on[O.tile_rows(i, wl.N)].any()]
+    idle = [i for i in range(nb) if i not in live]
+    for c in range(6):
+        assert order[c].tolist() == (list(range(nb)) if c < 3 else live + idle)
+
+
+def test_tile_order_changes_no_result():
+    # the pairing order is scheduling only: outputs are bit-identical with and
+    # without it, and an out-of-range entry is flagged, not faulted
+    wl = si.small("wan480")
+    (_, _, _), (qd, kd, vd), types = workload_tensors(wl)
+    lists = svg.geometric_lists(wl.F, wl.P, wl.width, wl.N)
+    mode = torch.from_numpy(types).to(DEV)
+    rep = torch.ones(wl.H, dtype=torch.int32, device=DEV)
+    alists, ids = svg.svg_anchor_lists(lists, wl.N, wl.F, wl.ph, wl.pw, mode, rep, skip_list=1)
+    a = svg.svg_sparse_attn_fused(qd, kd, vd, wl.F, wl.P, ids, alists)
+    b = svg.svg_sparse_attn_fused(qd, kd, vd, wl.F, wl.P, ids, alists._replace(tile_order=None))
+    np.testing.assert_array_equal(bits(a), bits(b))
+    rev = torch.flip(alists.tile_order.view(6, -1), dims=[1]).contiguous().view(-1)
+    c = svg.svg_sparse_attn_fused(qd, kd, vd, wl.F, wl.P, ids, alists._replace(tile_order=rev))
+    np.testing.assert_array_equal(bits(c), bits(b))
+    bad = alists.tile_order.clone()
+    bad[3 * svg.n_tiles(wl.N)] = 10 ** 6  # first slot of anchor list 3
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    svg.svg_sparse_attn_fused(qd, kd, vd, wl.F, wl.P, ids, alists._replace(tile_order=bad),
+                              status=status)
+    assert status.item() & svg._lib.SVG_DEVICE_BAD_INDEX
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_row_broadcast_bit_exact(dtype):
+    wl = si.small("hunyuan720")
+    g = torch.Generator().manual_seed(3)
+    o = torch.randn(wl.B, wl.H, wl.N, wl.d, generator=g).to(dtype).to(DEV)
+    ids = torch.tensor([0, 4, 2, 5], dtype=torch.int32, device=DEV)  # heads 1, 3 repeat
+    want = o.clone()
+    svg.svg_row_broadcast(o, wl.F, wl.ph, wl.pw, ids, 3)
+    got, ref = bits(o), bits(want)
+    for h in range(wl.H):
+        exp = ref[0, h]
+        if h in (1, 3):
+            exp = O.broadcast_rows(exp, wl.F, wl.ph, wl.pw, 5)
+        np.testing.assert_array_equal(got[0, h], exp)
+
+
+@pytest.mark.parametrize("wl", [si.small(n) for n in ("tiny", "cogvideox", "wan720")],
+                         ids=lambda w: w.name)
+def test_repeat_attention_small(wl):
+    (q, k, v), (qd, kd, vd), _ = workload_tensors(wl)
+    lists = svg.geometric_lists(wl.F, wl.P, wl.width, wl.N)
+    lid = np.resize(np.array([0, 2, 0, 0], dtype=np.int32), wl.H)   # spatial / dense lists
+    rep = np.resize(np.array([1, 1, 0, 1], dtype=np.int32), wl.H)
+    o = svg.svg_repeat_attention(qd, kd, vd, wl.F, wl.ph, wl.pw, torch.from_numpy(lid).to(DEV),
+                                 lists, torch.from_numpy(rep).to(DEV))
+    for h in range(wl.H):
+        ip, ix = O.geometric_block_lists(int(lid[h]), wl.F, wl.P, wl.width, wl.N)
+        q64, k64, v64 = head64(q, 0, h), head64(k, 0, h), head64(v, 0, h)
+        if rep[h]:
+            ref = O.repeat_head_attention(q64, k64, v64, ip, ix, wl.F, wl.ph, wl.pw, 5)
+        else:
+            ref = O.block_sparse_attention(q64, k64, v64, ip, ix)
+        assert_close(to_float64(o[0, h]), ref, f"{wl.name} head {h}", bf16=wl.dtype == "bf16")
+
+
+@pytest.mark.parametrize("overlap", [True, False])
+def test_layer_small_with_repeat(overlap):
+    wl = si.small("cogvideox")
+    (q, k, v), (qd, kd, vd), _ = workload_tensors(wl)
+    idx = si.sample_queries(wl)
+    lists = svg.geometric_lists(wl.F, wl.P, wl.width, wl.N)
+    rep = np.array([1, 1, 0, 1], dtype=np.int32)
+    o, mode, mse = svg.svg_layer(qd, kd, vd, wl.F, wl.P, wl.width, torch.from_numpy(idx).to(DEV),
+                                 lists, overlap=overlap, repeat=torch.from_numpy(rep).to(DEV),
+                                 frame_shape=(wl.ph, wl.pw))
+    o_ref, mode_ref, mse_ref = O.svg_layer(si.as_float64(q), si.as_float64(k), si.as_float64(v),
+                                           idx, wl.F, wl.P, wl.width)
+    np.testing.assert_array_equal(mode.cpu().numpy(), mode_ref)
+    for h in range(wl.H):
+        ref = o_ref[0, h]
+        if rep[h] and mode_ref[h] != O.MODE_TEMPORAL:
+            ref = O.broadcast_rows(ref, wl.F, wl.ph, wl.pw, 5)
+        assert_close(to_float64(o[0, h]), ref, f"layer head {h}")
