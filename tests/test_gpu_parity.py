@@ -905,3 +905,29 @@ def test_layer_small_with_repeat(overlap):
         if rep[h] and mode_ref[h] != O.MODE_TEMPORAL:
             ref = O.broadcast_rows(ref, wl.F, wl.ph, wl.pw, 5)
         assert_close(to_float64(o[0, h]), ref, f"layer head {h}")
+
+
+def test_layer_small_with_qk_norm_rope_and_repeat():
+    wl = si.small("wan480")
+    (q, k, v), (qd, kd, vd), _ = workload_tensors(wl)
+    gq, gk = si.qk_norm_weights(wl)
+    cos, sin = si.rope_tables(wl)
+    dev = lambda a: torch.from_numpy(a).to(DEV)
+    qk = svg.QKTransform(dev(gq), dev(gk), 1e-6, dev(cos), dev(sin))
+    idx = si.sample_queries(wl)
+    lists = svg.geometric_lists(wl.F, wl.P, wl.width, wl.N)
+    rep = np.array([1, 0, 1, 1], dtype=np.int32)
+    o, mode, mse = svg.svg_layer(qd, kd, vd, wl.F, wl.P, wl.width, torch.from_numpy(idx).to(DEV),
+                                 lists, qk=qk, repeat=dev(rep), frame_shape=(wl.ph, wl.pw))
+    o_ref, mode_ref, mse_ref = O.svg_layer(si.as_float64(q), si.as_float64(k), si.as_float64(v),
+                                           idx, wl.F, wl.P, wl.width, qk=(gq, gk, 1e-6, cos, sin),
+                                           qk_bf16=True)
+    check_profile(mse.cpu().numpy(), mode.cpu().numpy(), mse_ref, mode_ref, wl.name)
+    m = mode.cpu().numpy()
+    for h in range(wl.H):
+        if m[h] != mode_ref[h]:
+            continue  # a near tie decided the other way (checked above)
+        ref = o_ref[0, h]
+        if rep[h] and m[h] != O.MODE_TEMPORAL:
+            ref = O.broadcast_rows(ref, wl.F, wl.ph, wl.pw, 5)
+        assert_close(to_float64(o[0, h]), ref, f"head {h}")
