@@ -452,6 +452,8 @@ def svg_layer(q, k, v, frames: int, tokens_per_frame: int, spatial_width: int,
     Returns (o, mode, mse)."""
     if bufs is None:
         bufs = LayerBuffers(q, sample_idx.numel(), layout, qk=qk is not None)
+    if qk is not None and not hasattr(bufs, "qn"):
+        raise ValueError("QK-Norm + RoPE needs LayerBuffers(..., qk=True)")
     F, P = frames, tokens_per_frame
     if repeat is not None and (frame_shape is None or frame_shape[0] * frame_shape[1] != P):
         raise ValueError("repeat needs frame_shape = (rows, cols) with rows * cols = P")

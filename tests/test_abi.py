@@ -202,3 +202,23 @@ def test_encoding_validation():
            FAKE4 * 3, None, None, match="null starts")
     expect(INVALID, "svg_lists_to_bitmap", 3, 0, FAKE, FAKE2, FAKE3, None, None, match="bad sizes")
     expect(INVALID, "svg_lists_to_bitmap", 3, 10, FAKE, None, FAKE3, None, None, match="null")
+
+
+def test_layer_argument_checks_before_any_launch():
+    # these raise in the binding before anything reaches the library or a GPU
+    import torch
+    import sparse_attention_video_svg_b200 as svg
+    q = torch.zeros(1, 2, 256, 64, dtype=torch.bfloat16)
+    lists = svg.BlockLists(torch.zeros(3 * 3, dtype=torch.int32),
+                           torch.zeros(1, dtype=torch.int32), 3, 2)
+    idx = torch.zeros(16, dtype=torch.int32)
+    bufs = svg.LayerBuffers(q, 16)
+    qk = svg.QKTransform(None, None, 1e-6, None, None)
+    with pytest.raises(ValueError, match="qk=True"):
+        svg.svg_layer(q, q, q, 4, 64, 1, idx, lists, bufs, qk=qk)
+    with pytest.raises(ValueError, match="frame_shape"):
+        svg.svg_layer(q, q, q, 4, 64, 1, idx, lists, bufs,
+                      repeat=torch.ones(2, dtype=torch.int32))
+    with pytest.raises(ValueError, match="frame_shape"):
+        svg.svg_layer(q, q, q, 4, 64, 1, idx, lists, bufs,
+                      repeat=torch.ones(2, dtype=torch.int32), frame_shape=(8, 9))
