@@ -109,3 +109,18 @@ def test_traffic_tracks_kernel_sources(monkeypatch):
     monkeypatch.setattr(bench, "attn_sources_sha256", lambda: "0" * 64)
     assert bench.attn_traffic("cogvideox") is None
     assert bench.attn_traffic("wan480") is None
+
+
+def test_effective_flops_count_the_element_mask():
+    # the metric's work 4 d sum(kept pairs): kept pairs equal the number of
+    # (query, key) elements the oracle's block mask keeps, ragged tiles
+    # counted by their valid rows and columns
+    from oracle import svg_oracle as O
+    for name in ("cogvideox", "hunyuan720"):
+        wl = si.small(name)
+        for kind in (O.MODE_SPATIAL, O.MODE_TEMPORAL, O.MODE_DENSE):
+            ip, ix = O.geometric_block_lists(kind, wl.F, wl.P, wl.width, wl.N)
+            want = int(O.block_mask_from_lists(ip, ix, wl.N).sum())
+            assert bench.kept_pairs(ip, ix, wl.N) == want
+    ip, ix = O.geometric_block_lists(O.MODE_DENSE, 1, 300, 0, 300)
+    assert bench.kept_pairs(ip, ix, 300) == 300 * 300
