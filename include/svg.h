@@ -5,6 +5,8 @@
  * The library implements one attention layer of Sparse VideoGen-style sparse
  * 3D attention for video diffusion transformers:
  *
+ *   0. svg_qk_norm_rope         (optional) QK-Norm + RoPE of q and k, with
+ *                               their token-major copies in the same pass;
  *   1. svg_profile_heads        online profiling: per head, pick the spatial or
  *                               the temporal mask from a few sampled queries;
  *   2. svg_permute_token_major  frame-major -> token-major reordering of the
@@ -12,12 +14,16 @@
  *   3. svg_build_block_mask     per-query-block key-block lists (CSR) from the
  *                               spatial / temporal geometry, or
  *      svg_block_energy +
- *      svg_build_block_mask_calibrated   lists from cumulative-energy calibration;
+ *      svg_build_block_mask_calibrated   lists from cumulative-energy calibration
+ *                               (svg_epsilon_schedule, svg_lists_to_intervals,
+ *                               svg_lists_to_bitmap: schedule and encodings);
  *   4. svg_sparse_attn          block-sparse attention over 128x128 tiles that
- *                               walks only the kept key blocks;
+ *                               walks only the kept key blocks
+ *                               (svg_sparse_attn_fused: with the reordering of
+ *                               temporal heads folded in);
  *   5. svg_permute_frame_major  the inverse reordering of the output;
- *   6. svg_row_similarity, svg_anchor_lists, svg_row_broadcast
- *                               spatial-repetition heads (anchor rows only).
+ *   6. svg_row_similarity, svg_anchor_lists, svg_anchor_list_ids,
+ *      svg_row_broadcast        spatial-repetition heads (anchor rows only).
  *
  * Sources (cited by page title and section):
  *   [SVG]  Sparse VideoGen article, m.jxzklqfsx.com/article/815093.html
