@@ -124,3 +124,18 @@ def test_effective_flops_count_the_element_mask():
             assert bench.kept_pairs(ip, ix, wl.N) == want
     ip, ix = O.geometric_block_lists(O.MODE_DENSE, 1, 300, 0, 300)
     assert bench.kept_pairs(ip, ix, 300) == 300 * 300
+
+
+def test_clock_samples_summary():
+    # nvidia-smi rows: index, clocks.sm, clocks.max.sm, power.draw, active mask,
+    # hw_slowdown, hw_thermal_slowdown, sw_thermal_slowdown, sw_power_cap
+    lines = ["0, 1965, 1965, 612.3, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active\n",
+             "0, 1950, 1965, 998.1, 0x0000000000000004, Not Active, Not Active, Not Active, Active\n",
+             "0, 1890, 1965, 1001.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active\n",
+             "garbage line\n"]
+    got = bench.parse_clock_samples(lines)
+    assert got["sm_mhz"] == 1950 and got["sm_max_mhz"] == 1965 and got["samples"] == 3
+    assert got["reasons"] == ["sw_power_cap"]
+    hot = lines[:1] + ["0, 1200, 1965, 700, 0x8, Active, Not Active, Active, Not Active\n"]
+    assert bench.parse_clock_samples(hot)["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
+    assert bench.parse_clock_samples([])["reasons"] == ["no samples"]
