@@ -6,8 +6,11 @@ A step is one pass of the whole hot path over one layer's inputs:
     copies and write their output back frame-major (svg_sparse_attn_fused).
 The permutation kernel is also timed on its own beside the step, and the
 unfused layer (permute -> attention -> permute back) for comparison.
-Workload (default): the CogVideoX-shaped layer, B=1 H=48 N=17550 (13 frames x
-30x45 tokens) d=64 bf16, synthetic biased-Gaussian q/k/v, 64 sampled queries.
+Workload (default): the largest layer, HunyuanVideo-720p-shaped, B=1 H=24
+N=118800 (33 frames x 45x80 tokens) d=128 bf16, band |f - f'| <= 2, synthetic
+biased-Gaussian q/k/v, 64 sampled queries.  --config picks another layer;
+--config wan720 times the calibrated Wan 2.1 720p layer (per-head lists built
+from four calibration inputs, the build timed separately).
 
 Metric: effective TFLOPS of the layer = sum over heads of 4 * d * (query-key
 pairs inside kept 128x128 tiles, ragged tiles counted by their valid rows and
@@ -15,8 +18,11 @@ columns) / step time.  tokens/s = B * N / step time is reported beside it.
 
 Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
         python bench.py --impl reference ...    (the float64 CPU oracle)
-Multi-GPU (torchrun): every rank runs its own independent layer (a different
-input seed); no collective touches the data path (weak scaling).
+Multi-GPU (torchrun): by default the heads of one layer are split into
+contiguous ranges, one per rank (--shard heads; strong scaling: the whole
+layer's work over the slowest rank's time); --shard replicas runs an
+independent layer per rank instead (weak scaling).  No collective touches the
+data path either way.
 """
 from __future__ import annotations
 
@@ -75,8 +81,47 @@ def attn_traffic(workload):
 
 
 def rank_seed(wl, rank):
-    """Each rank runs its own independent layer (weak scaling)."""
+    """With --shard replicas each rank runs its own independent layer (weak
+    scaling) on this input seed."""
     return wl.seed + rank
+
+
+def shard_heads(H, world, rank):
+    """Contiguous head range of one rank when the heads of one layer are
+    split over `world` GPUs: the first H mod world ranks take one head more."""
+    base, extra = divmod(H, world)
+    start = rank * base + min(rank, extra)
+    return range(start, start + base + (1 if rank < extra else 0))
+
+
+def rank_heads(args, wl, rank, world):
+    """(heads, sharded, input seed) of this rank: a --heads range (one GPU,
+    small profiling captures), the rank's contiguous share of the layer's
+    heads (--shard heads), or the whole layer (one GPU, or --shard replicas
+    with an independent input per rank)."""
+    if args.heads is not None:
+        if world > 1:
+            raise SystemExit("--heads runs on one GPU")
+        a, b = (int(x) for x in args.heads.split(":"))
+        if not 0 <= a < b <= wl.H:
+            raise SystemExit(f"--heads {args.heads} outside 0:{wl.H}")
+        return range(a, b), False, wl.seed
+    if args.shard == "heads" and world > 1:
+        if wl.H < world:
+            raise SystemExit(f"{wl.H} heads cannot be split over {world} GPUs")
+        return shard_heads(wl.H, world, rank), True, wl.seed
+    return range(wl.H), False, rank_seed(wl, rank)
+
+
+def sum_over_ranks(values, world, device):
+    """Element-wise sum of per-rank values (every rank gets the result)."""
+    if world == 1:
+        return [float(x) for x in values]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x) for x in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return [float(x) for x in t.tolist()]
 
 
 def max_over_ranks(values, world, device):
@@ -90,12 +135,12 @@ def max_over_ranks(values, world, device):
     return [float(x) for x in t.tolist()]
 
 
-def aggregate(flops_per_rank, total_ms, steps, world, tokens_per_rank):
-    """Whole-job throughput: the work of all ranks over the slowest rank's
-    time per step.  Returns (TFLOPS, tokens/s, ms per step)."""
+def aggregate(job_flops, total_ms, steps, job_tokens):
+    """Whole-job throughput: the work of all ranks (job_flops, job_tokens per
+    step) over the slowest rank's time per step (total_ms over `steps`).
+    Returns (TFLOPS, tokens/s, ms per step)."""
     ms = total_ms / steps
-    return (flops_per_rank * world / (ms * 1e-3) / 1e12,
-            tokens_per_rank * world / (ms * 1e-3), ms)
+    return job_flops / (ms * 1e-3) / 1e12, job_tokens / (ms * 1e-3), ms
 
 
 def workload_config(wl):
@@ -187,9 +232,10 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     wl = si.WORKLOADS[args.config]
     if wl.kind != "profiled":
-        raise SystemExit(f"bench runs profiled layers; {wl.name} is {wl.kind}")
-    seed = rank_seed(wl, rank)
-    q, k, v, types = si.generate(wl, seed=seed)
+        raise SystemExit(f"run_ours times profiled layers; {wl.name} is {wl.kind}")
+    heads, sharded, seed = rank_heads(args, wl, rank, world)
+    q, k, v, types = si.generate(wl, seed=seed, heads=heads)
+    Hl = len(heads)
     idx = si.sample_queries(wl, seed=wl.seed)
     host = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in (q, k, v)]
     del q, k, v
@@ -357,7 +403,7 @@ def run_ours(args, rank, world, local_rank):
     ph, pw = wl.ph, wl.pw
     mid = torch.tensor([F // 2], dtype=torch.int32, device=dev)
     rs_ws = torch.empty(max(256, svg._lib.lib.svg_row_similarity_workspace_size(
-        svg._lib.SVG_BF16, wl.B, wl.H, ph, pw, 1)), dtype=torch.uint8, device=dev)
+        svg._lib.SVG_BF16, wl.B, Hl, ph, pw, 1)), dtype=torch.uint8, device=dev)
     sims = svg.svg_row_similarity(qd, kd, F, ph, pw, mid, workspace=rs_ws)
     rs_ms = timed(lambda: svg.svg_row_similarity(qd, kd, F, ph, pw, mid, out=sims,
                                                  workspace=rs_ws))
@@ -377,6 +423,10 @@ def run_ours(args, rank, world, local_rank):
     rep_attn_pairs_ms = timed(lambda: svg.svg_sparse_attn_fused(
         qd, kd, vd, F, P, ids, alists._replace(tile_order=None),
         layout=svg._lib.SVG_FUSE_OUTPUT, copies=(bufs.qp, bufs.kp, bufs.vp), out=bufs.o))
+
+    # the fixed-scratch profiling entry point on the same inputs, alone
+    noalloc_ms = timed(lambda: svg.svg_profile_heads_noalloc(
+        qd, kd, vd, F, P, w, idx_d, mse_out=bufs.mse, mode_out=bufs.mode))
 
     # end to end through the public API with host buffers
     out_host = torch.empty(qd.shape, dtype=torch.bfloat16).pin_memory()
@@ -403,28 +453,40 @@ def run_ours(args, rank, world, local_rank):
     e2e_ms = e0.elapsed_time(e1)
 
     (total_ms, e2e_ms, attn_avg, prof_avg, perm_avg, unf_avg, fwd_perm_avg, qk_ms, qk_layer_ms,
-     qk_then_layer_ms, rs_ms, rep_attn_ms, rep_layer_ms, rep_attn_pairs_ms) = max_over_ranks(
+     qk_then_layer_ms, rs_ms, rep_attn_ms, rep_layer_ms, rep_attn_pairs_ms,
+     noalloc_avg) = max_over_ranks(
         [total_ms, e2e_ms, attn_avg, prof_avg, perm_avg, unf_avg, fwd_perm_avg, qk_ms,
-         qk_layer_ms, qk_then_layer_ms, rs_ms, rep_attn_ms, rep_layer_ms, rep_attn_pairs_ms],
-        world, dev)
+         qk_layer_ms, qk_then_layer_ms, rs_ms, rep_attn_ms, rep_layer_ms, rep_attn_pairs_ms,
+         noalloc_ms], world, dev)
+    h2d = sum(h.numel() * 2 for h in host)
+    d2h = out_host.numel() * 2 + mode_host.numel() * 4
+    # the job's work per step: every rank's heads (one layer split over the
+    # ranks, or one layer per rank)
+    job_flops, job_h2d, job_d2h, n_spatial, n_temporal = sum_over_ranks(
+        [flops, h2d, d2h, int((modes == 0).sum()), int((modes == 1).sum())], world, dev)
+    job_tokens = wl.B * N * (1 if sharded else world)
     if rank != 0:
         return None
 
     peaks, src = load_peaks()
     peak_tf = float(peaks["bf16_tflops"])
-    value, tokens_s, step_ms_avg = aggregate(flops, total_ms, K, world, wl.B * N)
-    e2e_value, _, e2e_step_ms = aggregate(flops, e2e_ms, K, world, wl.B * N)
+    value, tokens_s, step_ms_avg = aggregate(job_flops, total_ms, K, job_tokens)
+    e2e_value, _, e2e_step_ms = aggregate(job_flops, e2e_ms, K, job_tokens)
+    # the attention kernel of the slowest rank against its own work
     attn_tf = flops / (attn_avg * 1e-3) / 1e12
     hbm_gbs = float(peaks["hbm_gbs"])
-    elems = wl.B * wl.H * N * d
+    elems = wl.B * Hl * N * d
     perm_bytes = 2 * elems * 2      # one tensor read and written once
     prof_bytes = 2 * elems * 2      # K and V streamed once
     # q, k read once; q, k written frame-major and token-major; cos, sin once
     qk_bytes = 6 * elems * 2 + 2 * N * (d // 2) * 4
-    h2d = sum(h.numel() * 2 for h in host)
-    d2h = out_host.numel() * 2 + mode_host.numel() * 4
     # profile partial, merge, finalize; 3 permutes; attention (output reordering fused)
     launches_per_step = 3 + 3 + 1
+    if sharded:
+        parallelism = (f"heads of one layer split over {world} GPUs "
+                       f"(contiguous ranges, rank 0 heads {heads.start}-{heads.stop - 1})")
+    else:
+        parallelism = f"independent layer per GPU x{world}" if world > 1 else "1 GPU"
     line = {
         "metric": METRIC,
         "value": round(value, 3),
@@ -434,16 +496,18 @@ def run_ours(args, rank, world, local_rank):
         "warmup": W,
         "ms_per_step": round(step_ms_avg, 5),
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": "strong" if sharded else "weak",
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded biased-Gaussian q/k/v, no model weights)",
         "config": {**workload_config(wl),
-                   "modes": {"spatial": int((modes == 0).sum()), "temporal": int((modes == 1).sum())},
+                   **({"heads_subset": f"{heads.start}:{heads.stop}"}
+                      if args.heads is not None else {}),
+                   "modes": {"spatial": int(n_spatial), "temporal": int(n_temporal)},
                    "kept_fraction": {"spatial": round(kept_frac[0], 5),
                                      "temporal": round(kept_frac[1], 5)},
                    "l2": "flushed (256 MB write) before every timed step",
-                   "parallelism": f"independent layer per GPU x{world}"},
+                   "parallelism": parallelism},
         "tokens_per_s": round(tokens_s, 1),
         "pct_of_bf16_peak": round(100 * value / world / peak_tf, 2),
         "attention_only": {"ms": round(attn_avg, 5), "effective_tflops": round(attn_tf, 3),
@@ -477,15 +541,188 @@ def run_ours(args, rank, world, local_rank):
             "layer_ms_spatial_heads_repeating": round(rep_layer_ms, 5),
             "note": "anchors k=5 per frame; every spatial head forced to repeat for timing"},
         "profile": {"ms": round(prof_avg, 5),
-                    "kv_gbs": round(prof_bytes / (prof_avg * 1e-3) / 1e9, 1)},
+                    "kv_gbs": round(prof_bytes / (prof_avg * 1e-3) / 1e9, 1),
+                    "share_of_step": round(prof_avg / step_ms_avg, 4),
+                    "noalloc_ms": round(noalloc_avg, 5),
+                    "note": "ms beside the side-stream copies (the step's schedule); "
+                            "noalloc_ms: the fixed-scratch entry point alone"},
         "roofline": {"kernel": "svg_sparse_attn_fused", "bound": "tensor",
                      "achieved": round(attn_tf, 3),
                      "peak": peak_tf, "unit": "TFLOP/s", "frac": round(attn_tf / peak_tf, 4),
                      "peak_source": f"{src} bf16 burst", "traffic": attn_traffic(wl.name)},
         "e2e": {"value": round(e2e_value, 3), "unit": "TFLOPS",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "h2d_bytes_per_step": int(job_h2d), "d2h_bytes_per_step": int(job_d2h),
                 "ms_per_step": round(e2e_step_ms, 5)},
         "gpu_launches": launches_per_step * K,
+        "clocks": clk,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_budget)
+    return line
+
+
+# ------------------------------------------------------- calibrated layer
+
+def run_calibrated(args, rank, world, local_rank):
+    """The calibrated Wan 2.1 720p layer ([CAL] 3.1): per-head key-block lists
+    built once from the block energies of the calibration inputs (timed
+    separately: energy per input, list build), then a step = block-sparse
+    attention of every head on its own list (list_id = h, frame-major) on
+    the timed input."""
+    import torch
+    import torch.distributed as dist
+
+    import sparse_attention_video_svg_b200 as svg
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = si.WORKLOADS[args.config]
+    heads, sharded, seed = rank_heads(args, wl, rank, world)
+    Hl = len(heads)
+    N, d = wl.N, wl.d
+    nb = svg.n_tiles(N)
+    stream = torch.cuda.current_stream()
+    tseed = wl.calib_seeds[0]
+    shift = seed - wl.seed  # replicas: every rank its own inputs
+
+    def ev():
+        return torch.cuda.Event(enable_timing=True)
+
+    # calibration: block energies of every calibration input, then the lists
+    E = torch.empty(len(wl.calib_seeds), Hl, nb, nb, dtype=torch.float32, device=dev)
+    ews = torch.empty(max(256, svg._lib.lib.svg_block_energy_workspace_size(1, Hl, N)),
+                      dtype=torch.uint8, device=dev)
+    energy_ms = []
+    for r, s in enumerate(wl.calib_seeds):
+        q, k, _, _ = si.generate(wl, seed=s + shift, types_seed=tseed, heads=heads)
+        qd, kd = (torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev) for x in (q, k))
+        del q, k
+        torch.cuda.synchronize()
+        e0, e1 = ev(), ev()
+        e0.record(stream)
+        svg.svg_block_energy(qd, kd, out=E[r], workspace=ews)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        energy_ms.append(e0.elapsed_time(e1))
+        del qd, kd
+    del ews
+    svg.svg_build_block_mask_calibrated(E, wl.eps, wl.rho)  # warm-up
+    torch.cuda.synchronize()
+    e0, e1 = ev(), ev()
+    e0.record(stream)
+    lists = svg.svg_build_block_mask_calibrated(E, wl.eps, wl.rho)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    build_ms = e0.elapsed_time(e1)
+    del E
+    ip = lists.indptr.cpu().numpy().reshape(Hl, nb + 1)
+    ix = lists.indices.cpu().numpy()
+    pairs = [kept_pairs(ip[h] - ip[h][0], ix[ip[h][0]:ip[h][-1]], N) for h in range(Hl)]
+    flops = float(sum(4 * d * p for p in pairs))
+
+    q, k, v, _ = si.generate(wl, seed=seed, types_seed=tseed, heads=heads)
+    host = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in (q, k, v)]
+    del q, k, v
+    qd, kd, vd = (h.to(dev) for h in host)
+    o = torch.empty_like(qd)
+    list_id = torch.arange(Hl, dtype=torch.int32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    K, W = args.steps, args.warmup
+
+    def step():
+        svg.svg_sparse_attn(qd, kd, vd, list_id, lists, out=o)
+
+    for _ in range(W):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    evs = [(ev(), ev()) for _ in range(K)]
+    for i in range(K):
+        flush.fill_(i & 0xff)
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    total_ms = float(sum(a.elapsed_time(b) for a, b in evs))
+
+    # end to end: q, k, v from pinned host memory, o back, every step
+    out_host = torch.empty(qd.shape, dtype=torch.bfloat16).pin_memory()
+    for _ in range(2):
+        for x, h in zip((qd, kd, vd), host):
+            x.copy_(h, non_blocking=True)
+        step()
+        out_host.copy_(o, non_blocking=True)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = ev(), ev()
+    e0.record(stream)
+    for _ in range(K):
+        for x, h in zip((qd, kd, vd), host):
+            x.copy_(h, non_blocking=True)
+        step()
+        out_host.copy_(o, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+
+    energy_avg = float(sum(energy_ms) / len(energy_ms))
+    total_ms, e2e_ms, energy_avg, build_ms = max_over_ranks(
+        [total_ms, e2e_ms, energy_avg, build_ms], world, dev)
+    h2d = sum(h.numel() * 2 for h in host)
+    d2h = out_host.numel() * 2
+    job_flops, job_h2d, job_d2h, job_pairs = sum_over_ranks(
+        [flops, h2d, d2h, float(sum(pairs))], world, dev)
+    job_tokens = wl.B * N * (1 if sharded else world)
+    if rank != 0:
+        return None
+    peaks, src = load_peaks()
+    peak_tf = float(peaks["bf16_tflops"])
+    value, tokens_s, ms = aggregate(job_flops, total_ms, K, job_tokens)
+    e2e_value, _, e2e_step_ms = aggregate(job_flops, e2e_ms, K, job_tokens)
+    attn_tf = flops / (total_ms / K * 1e-3) / 1e12
+    job_heads = wl.H if sharded else Hl * world
+    energy_flops = 2 * 2 * float(N) * N * d * Hl  # two dense Q K^T passes per head
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOPS", "n_gpus": world,
+        "steps": K, "warmup": W, "ms_per_step": round(ms, 5), "higher_is_better": True,
+        "scaling": "strong" if sharded else "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded biased-Gaussian q/k/v, no model weights)",
+        "config": {**workload_config(wl),
+                   **({"heads_subset": f"{heads.start}:{heads.stop}"}
+                      if args.heads is not None else {}),
+                   "lists": f"calibrated per head: eps {wl.eps}, rho {wl.rho}, inputs "
+                            f"{list(wl.calib_seeds)}, timed on seed {wl.seed}",
+                   "kept_fraction": round(job_pairs / (float(N) * N * job_heads), 5),
+                   "l2": "flushed (256 MB write) before every timed step",
+                   "parallelism": (f"heads of one layer split over {world} GPUs" if sharded else
+                                   f"independent layer per GPU x{world}" if world > 1 else
+                                   "1 GPU")},
+        "tokens_per_s": round(tokens_s, 1),
+        "pct_of_bf16_peak": round(100 * value / world / peak_tf, 2),
+        "attention_only": {"ms": round(total_ms / K, 5), "effective_tflops": round(attn_tf, 3),
+                           "kernel": "svg_sparse_attn (list_id = h)"},
+        "calibration": {"energy_ms_per_input": round(energy_avg, 3),
+                        "energy_tflops": round(energy_flops / (energy_avg * 1e-3) / 1e12, 1),
+                        "build_lists_ms": round(build_ms, 3),
+                        "inputs": len(wl.calib_seeds),
+                        "note": "offline, not in the step"},
+        "roofline": {"kernel": "svg_sparse_attn", "bound": "tensor", "achieved": round(attn_tf, 3),
+                     "peak": peak_tf, "unit": "TFLOP/s", "frac": round(attn_tf / peak_tf, 4),
+                     "peak_source": f"{src} bf16 burst", "traffic": attn_traffic(wl.name)},
+        "e2e": {"value": round(e2e_value, 3), "unit": "TFLOPS",
+                "h2d_bytes_per_step": int(job_h2d), "d2h_bytes_per_step": int(job_d2h),
+                "ms_per_step": round(e2e_step_ms, 5)},
+        "gpu_launches": 1 * K,
         "clocks": clk,
     }
     if not args.no_cpu_baseline and world == 1:
@@ -504,12 +741,61 @@ def oracle_threads():
         return os.cpu_count() or 1
 
 
+def cpu_baseline_calibrated(wl, budget_s=15.0):
+    """The float64 oracle on a bounded sample of the calibrated layer: for
+    query tiles of two heads, the energy rows of the tile on every
+    calibration input, the voted list row, then block-sparse attention of
+    the tile on the timed input.  The value counts the attention alone (the
+    calibration is offline); its time is reported beside it."""
+    from oracle import svg_oracle as O
+
+    heads = range(2)
+    tseed = wl.calib_seeds[0]
+    cal = [si.generate(wl, seed=s, types_seed=tseed, heads=heads)[:2] for s in wl.calib_seeds]
+    q, k, v, _ = si.generate(wl, seed=wl.seed, types_seed=tseed, heads=heads)
+    N = wl.N
+    nb = O.n_tiles(N)
+    order = np.random.default_rng(0).permutation(nb)
+    t_cal = t_att = 0.0
+    flops = 0.0
+    units = 0
+    t_start = time.perf_counter()
+    for h in heads:
+        qh, kh, vh = (si.as_float64(t[0, h]) for t in (q, k, v))
+        cal_h = [(si.as_float64(cq[0, h]), si.as_float64(ck[0, h])) for cq, ck in cal]
+        for i in order:
+            t0 = time.perf_counter()
+            Es = [O.block_energy(cq, ck, row_blocks=[int(i)]) for cq, ck in cal_h]
+            ip1, ix1 = O.calibrate_lists(Es, wl.eps, wl.rho)
+            t1 = time.perf_counter()
+            ip = np.zeros(nb + 1, np.int64)
+            ip[i + 1:] = len(ix1)
+            rows = O.tile_rows(int(i), N)
+            O.block_sparse_rows(qh, kh, vh, rows, ip, ix1)
+            t2 = time.perf_counter()
+            t_cal += t1 - t0
+            t_att += t2 - t1
+            flops += 4.0 * wl.d * len(rows) * sum(min(128, N - j * 128) for j in ix1)
+            units += 1
+            if t2 - t_start > budget_s:
+                break
+        if time.perf_counter() - t_start > budget_s:
+            break
+    return {"value": flops / t_att / 1e12, "unit": "TFLOPS", "cores": oracle_threads(),
+            "kind": "oracle",
+            "sample": f"{wl.name}: {units} query tiles of 2 heads: calibrated list rows "
+                      f"({len(wl.calib_seeds)} inputs, {t_cal:.1f} s, not in the value) and "
+                      f"block-sparse attention (float64 NumPy, {t_att:.1f} s)"}
+
+
 def cpu_baseline(wl, budget_s=15.0, seed=None):
     """The float64 oracle on a bounded sample of the same layer: profiling and
     block-sparse attention for as many (head, query tile) units as fit the
     budget, converted to the same effective-TFLOPS unit."""
     from oracle import svg_oracle as O
 
+    if wl.kind == "calibrated":
+        return cpu_baseline_calibrated(wl, budget_s)
     seed = wl.seed if seed is None else seed
     one = wl.scaled(wl.name, H=2)
     q, k, v, types = si.generate(one, seed=seed)
@@ -562,7 +848,9 @@ def run_reference(args, world=1):
         "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": round(1e3 * statistics.mean(wall), 3), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic (seeded biased-Gaussian q/k/v, no model weights)",
-        "config": {**workload_config(wl), "oracle": "rank 0 host cores only"},
+        "config": {**workload_config(wl),
+                   **({"heads_subset": f"{heads.start}:{heads.stop}"}
+                      if args.heads is not None else {}), "oracle": "rank 0 host cores only"},
         "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": vals[-1]["cores"],
                          "kind": "oracle", "sample": vals[-1]["sample"]},
         "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0,
@@ -575,7 +863,12 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", default="cogvideox", choices=[n for n in si.ORDER if n != "tiny"])
+    ap.add_argument("--config", default="hunyuan720",
+                    choices=[n for n in si.ORDER if n != "tiny"])
+    ap.add_argument("--heads", default=None, metavar="A:B",
+                    help="run only heads A..B-1 of the layer (small cases for ncu captures)")
+    ap.add_argument("--shard", default="heads", choices=["heads", "replicas"],
+                    help="multi-GPU: split one layer's heads (default) or one layer per GPU")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -597,7 +890,10 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
-    line = run_ours(args, rank, world, local_rank)
+    if si.WORKLOADS[args.config].kind == "calibrated":
+        line = run_calibrated(args, rank, world, local_rank)
+    else:
+        line = run_ours(args, rank, world, local_rank)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()

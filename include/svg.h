@@ -154,10 +154,12 @@ svg_status svg_profile_heads(const void* q, const void* k, const void* v, int dt
  *  No device memory is allocated or freed by this call.
  *  The first call on a device looks up the array's device address
  *  (cudaGetSymbolAddress); make that first call on each device before any
- *  stream capture.  Every call shares the one array and leaves its contents
- *  behind; nothing in it needs to start at zero.  Calls whose kernels
- *  overlap on the GPU (e.g. on two streams) race on the array: serialise
- *  them.
+ *  stream capture.  The address is kept for the life of the process, so a
+ *  cudaDeviceReset (or any teardown of the device's primary context) makes
+ *  it stale: do not call this entry point on a device after resetting it.
+ *  Every call shares the one array and leaves its contents behind; nothing
+ *  in it needs to start at zero.  Calls whose kernels overlap on the GPU
+ *  (e.g. on two streams) race on the array: serialise them.
  * ------------------------------------------------------------------------ */
 svg_status svg_profile_heads_noalloc(const void* q, const void* k, const void* v, int dtype,
                                      int B, int H, int N, int d,

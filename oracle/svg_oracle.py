@@ -300,19 +300,22 @@ def block_sparse_attention(q, k, v, indptr, indices, T: int = 128, scale=None):
 # O9: energy-threshold calibration with cross-input vote   ([CAL] 3.1)
 # ---------------------------------------------------------------------------
 
-def block_energy(q, k, T: int = 128, scale=None) -> np.ndarray:
+def block_energy(q, k, T: int = 128, scale=None, row_blocks=None) -> np.ndarray:
     """E[r, c] = sum_{i in block r, j in block c} p_ij / |block r|, p the dense
-    softmax of one head.  q, k [N, d] -> E [nB, nB]."""
+    softmax of one head.  q, k [N, d] -> E [nB, nB].  row_blocks (a sequence
+    of query-block indices) computes only those rows of E, in that order
+    (each row depends on its own query block alone)."""
     q = np.asarray(q, np.float64)
     N = q.shape[0]
     scale = softmax_scale(q.shape[1]) if scale is None else scale
     nb = n_tiles(N, T)
-    E = np.zeros((nb, nb))
-    for r in range(nb):
+    row_blocks = range(nb) if row_blocks is None else row_blocks
+    E = np.zeros((len(row_blocks), nb))
+    for out_r, r in enumerate(row_blocks):
         rows = tile_rows(r, N, T)
         p = attention_probs(q[rows], k, scale)
         for c in range(nb):
-            E[r, c] = p[:, c * T: min(N, (c + 1) * T)].sum() / len(rows)
+            E[out_r, c] = p[:, c * T: min(N, (c + 1) * T)].sum() / len(rows)
     return E
 
 

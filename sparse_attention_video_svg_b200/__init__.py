@@ -33,7 +33,8 @@ from ._lib import (SVG_BF16, SVG_FP32, SVG_MODE_DENSE, SVG_MODE_SPATIAL, SVG_MOD
 
 __all__ = [
     "SVG_MODE_SPATIAL", "SVG_MODE_TEMPORAL", "SVG_MODE_DENSE", "SVG_TILE", "SvgError",
-    "BlockLists", "svg_version", "svg_profile_heads", "svg_permute_token_major",
+    "BlockLists", "svg_version", "svg_profile_heads", "svg_profile_heads_noalloc",
+    "svg_permute_token_major",
     "svg_permute_frame_major", "svg_build_block_mask", "svg_block_energy",
     "svg_build_block_mask_calibrated", "svg_sparse_attn", "svg_sparse_attn_fused",
     "svg_epsilon_schedule", "svg_lists_to_intervals", "svg_lists_to_bitmap", "geometric_lists",
@@ -116,6 +117,23 @@ def svg_profile_heads(q, k, v, frames: int, tokens_per_frame: int, spatial_width
               frames, tokens_per_frame, spatial_width, sample_idx.data_ptr(), S,
               mse_out.data_ptr(), mode_out.data_ptr(), workspace.data_ptr(), workspace.numel(),
               _stream(stream))
+    return mse_out, mode_out
+
+
+def svg_profile_heads_noalloc(q, k, v, frames: int, tokens_per_frame: int, spatial_width: int,
+                              sample_idx: torch.Tensor, *, mse_out=None, mode_out=None,
+                              stream=None):
+    """svg_profile_heads with the library's fixed device scratch instead of a
+    workspace (for callers that cannot allocate); returns (mse, mode)."""
+    B, H, N, d = _check_qkv(q, k, v)
+    dev = q.device
+    if mse_out is None:
+        mse_out = torch.empty(B * H, 2, dtype=torch.float32, device=dev)
+    if mode_out is None:
+        mode_out = torch.empty(B * H, dtype=torch.int32, device=dev)
+    _lib.call("svg_profile_heads_noalloc", q.data_ptr(), k.data_ptr(), v.data_ptr(), _dt(q), B,
+              H, N, d, frames, tokens_per_frame, spatial_width, sample_idx.data_ptr(),
+              sample_idx.numel(), mse_out.data_ptr(), mode_out.data_ptr(), _stream(stream))
     return mse_out, mode_out
 
 

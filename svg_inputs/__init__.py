@@ -14,7 +14,7 @@ q/k/v are synthetic:
 
     u ~ N(0, 1)                        [H, F, d]      (one vector per frame)
     w ~ N(0, 1)                        [H, P, d]      (one vector per position)
-    z_q, z_k, z_v ~ N(0, 1)            [B, H, N, d]   (drawn after u, w, in that order)
+    z_q, z_k, z_v ~ N(0, 1)            [B, H, N, d]   (one stream per (tensor, b, h) slab)
     x[b,h,n] = z[b,h,n] + 2.0 * u[h, n // P]    for a spatial-type head
     x[b,h,n] = z[b,h,n] + 2.0 * w[h, n %  P]    for a temporal-type head
 
@@ -23,13 +23,17 @@ one frame (spatial-type heads) or of one spatial position (temporal-type
 heads).  Tokens are frame-major: n = f * P + s with P = ph * pw tokens per frame.
 QK-Norm weights and 3D rotary tables for the fused QK-Norm + RoPE step are
 synthetic inputs too (``qk_norm_weights``, ``rope_tables``).
-All draws use numpy's PCG64 ``default_rng(seed)`` in float32; bf16 workloads
-are rounded to bf16 with round-to-nearest-even and both sides consume the
-rounded values.
+All draws use numpy's PCG64 in float32: u and w come from ``default_rng(seed)``,
+each (N, d) slab of z from its own ``default_rng((seed, tensor, b, h))`` (tensor
+0, 1, 2 for q, k, v), so slabs are drawn in parallel threads and the result does
+not depend on the thread count.  bf16 workloads are rounded to bf16 with
+round-to-nearest-even and both sides consume the rounded values.
 """
 from __future__ import annotations
 
 import dataclasses
+import os
+from concurrent.futures import ThreadPoolExecutor
 from typing import Optional
 
 import numpy as np
@@ -154,8 +158,12 @@ def head_types(wl: Workload, seed: Optional[int] = None) -> np.ndarray:
     return t
 
 
+def _threads() -> int:
+    return max(1, min(32, os.cpu_count() or 1))
+
+
 def generate(wl: Workload, seed: Optional[int] = None,
-             types_seed: Optional[int] = None):
+             types_seed: Optional[int] = None, heads: Optional[range] = None):
     """Draw q, k, v for one workload.
 
     Returns ``(q, k, v, types)``.  For bf16 workloads q/k/v are uint16 bf16
@@ -163,9 +171,12 @@ def generate(wl: Workload, seed: Optional[int] = None,
     row-major.  ``types_seed`` fixes the head-type draw independently of the
     data seed (the calibrated workload keeps the types of its first input).
 
-    Draw order from default_rng(seed): u [H, F, d], w [H, P, d], then z_q,
-    z_k, z_v one (N, d) slab per (b, h) in row-major order, so that each slab
-    is biased and rounded as soon as it is drawn."""
+    u [H, F, d] and w [H, P, d] come from default_rng(seed) in that order; the
+    (N, d) slab of tensor t (0 = q, 1 = k, 2 = v) for (b, h) comes from
+    default_rng((seed, t, b, h)), is biased and rounded on its own, and the
+    slabs are filled by a thread pool.  ``heads`` (a range of head indices)
+    draws only those heads' slabs: the result equals the same slice of the
+    whole layer, and ``types`` stays the whole layer's."""
     seed = wl.seed if seed is None else seed
     tseed = seed if types_seed is None else types_seed
     B, H, N, d, F, P = wl.B, wl.H, wl.N, wl.d, wl.F, wl.P
@@ -176,19 +187,26 @@ def generate(wl: Workload, seed: Optional[int] = None,
     bf16 = wl.dtype == "bf16"
     out_dtype = np.uint16 if bf16 else np.float32
     two = np.float32(2.0)
-    outs = []
-    for _ in range(3):
-        x = np.empty((B, H, N, d), dtype=out_dtype)
-        for b in range(B):
-            for h in range(H):
-                z = rng.standard_normal((N, d), dtype=np.float32).reshape(F, P, d)
-                if types[h] == SPATIAL_TYPE:
-                    z += two * u[h][:, None, :]
-                else:
-                    z += two * wv[h][None, :, :]
-                z = z.reshape(N, d)
-                x[b, h] = to_bf16_bits(z) if bf16 else z
-        outs.append(x)
+    heads = range(H) if heads is None else heads
+    if len(heads) and (heads.start < 0 or heads.stop > H or heads.step != 1):
+        raise ValueError(f"heads {heads} outside 0..{H}")
+    outs = [np.empty((B, len(heads), N, d), dtype=out_dtype) for _ in range(3)]
+
+    def slab(job):
+        t, b, hl = job
+        h = heads[hl]
+        z = np.random.default_rng((seed, t, b, h)).standard_normal((N, d), dtype=np.float32)
+        z = z.reshape(F, P, d)
+        if types[h] == SPATIAL_TYPE:
+            z += two * u[h][:, None, :]
+        else:
+            z += two * wv[h][None, :, :]
+        z = z.reshape(N, d)
+        outs[t][b, hl] = to_bf16_bits(z) if bf16 else z
+
+    jobs = [(t, b, hl) for t in range(3) for b in range(B) for hl in range(len(heads))]
+    with ThreadPoolExecutor(max_workers=_threads()) as ex:
+        list(ex.map(slab, jobs))
     return outs[0], outs[1], outs[2], types
 
 

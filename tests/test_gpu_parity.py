@@ -493,6 +493,26 @@ def test_calibrated_lists_bit_exact_given_energies():
             np.testing.assert_array_equal(ix[ip[l][0]:ip[l][-1]], ox)
 
 
+@pytest.mark.parametrize("R,L,nq,nk", [(4, 5, 600, 600), (3, 2, 1100, 929), (4, 40, 64, 591)])
+def test_calibrated_lists_bit_exact_given_energies_large(R, L, nq, nk):
+    """Rows wider than 512 key blocks (the 1024-entry sort) and more rows
+    than one scan chunk (L * nQB > 1024, carried across chunks)."""
+    rng = np.random.default_rng(1000 + nk)
+    E = rng.dirichlet(np.ones(nk) * 0.05, size=(R, L, nq)).astype(np.float32)
+    E[0, 0, 1] = np.float32(1.0 / nk)            # all ties
+    for eps, rho in [(0.9, 0.5), (0.97, 0.75)]:
+        lists = svg.svg_build_block_mask_calibrated(torch.from_numpy(E).to(DEV), eps, rho)
+        ip = lists.indptr.cpu().numpy().reshape(L, nq + 1)
+        ix = lists.indices.cpu().numpy()
+        assert ip[0][0] == 0 and (np.diff(ip.reshape(-1)[:-1]) >= 0).all()
+        for l in sorted({0, L // 2, L - 1}):
+            op, ox = O.calibrate_lists([E[r, l].astype(np.float64) for r in range(R)], eps, rho)
+            np.testing.assert_array_equal(ip[l] - ip[l][0], op, err_msg=f"list {l} eps {eps}")
+            np.testing.assert_array_equal(ix[ip[l][0]:ip[l][-1]], ox)
+        # every list starts where the previous one ends (one shared indices array)
+        np.testing.assert_array_equal(ip[1:, 0], ip[:-1, -1])
+
+
 def cut_margin(e_row, eps):
     order = O.energy_order(e_row)
     cum = np.cumsum(np.asarray(e_row, np.float64)[order])
@@ -535,6 +555,71 @@ def test_calibration_end_to_end_small():
         hx = ix[ip[h][0]:ip[h][-1]]
         ref = O.block_sparse_attention(head64(q, 0, h), head64(k, 0, h), head64(v, 0, h), hp, hx)
         assert_close(o[0, h], ref, f"calibrated head {h}")
+
+
+def test_calibration_full_size_sampled():
+    """The calibrated Wan 2.1 720p layer at full size (B=1, H=40, N=75600,
+    d=128): GPU block energies of the four calibration inputs, the 40
+    per-head lists built from them, and attention on the timed input with
+    list_id = h.  The oracle computes energy rows of sampled query blocks
+    (float64, full N keys) for sampled heads; a list row is compared where
+    every input's cut margin exceeds 1e-3.  Attention is compared on sampled
+    query tiles of sampled heads, element by element, on the lists the GPU
+    built."""
+    wl = si.WORKLOADS["wan720"]
+    rng = np.random.default_rng(720)
+    heads = sorted(rng.choice(wl.H, 4, replace=False).tolist())
+    nb = svg.n_tiles(wl.N)
+    blocks = sorted(rng.choice(nb - 1, 3, replace=False).tolist()) + [nb - 1]  # + ragged tail
+    types_seed = wl.calib_seeds[0]
+    Es = []
+    ref_E = {h: [] for h in heads}
+    for s in wl.calib_seeds:
+        q, k, _, _ = si.generate(wl, seed=s, types_seed=types_seed)
+        qd, kd = to_device(q), to_device(k)
+        Es.append(svg.svg_block_energy(qd, kd))
+        del qd, kd
+        for h in heads:
+            ref_E[h].append(O.block_energy(head64(q, 0, h), head64(k, 0, h), row_blocks=blocks))
+        del q, k
+    E = torch.stack(Es).contiguous()  # [R, 40, 591, 591]
+    del Es
+    Eh = E.cpu().numpy()
+    for h in heads:  # the GPU energies of the sampled rows, against float64
+        for s in range(len(wl.calib_seeds)):
+            np.testing.assert_allclose(Eh[s, h][blocks], ref_E[h][s], rtol=2e-3, atol=2e-5)
+    lists = svg.svg_build_block_mask_calibrated(E, wl.eps, wl.rho)
+    del E
+    ip = lists.indptr.cpu().numpy().reshape(wl.H, nb + 1)
+    ix = lists.indices.cpu().numpy()
+    compared = 0
+    for h in heads:
+        op, ox = O.calibrate_lists(ref_E[h], wl.eps, wl.rho)
+        for n, r in enumerate(blocks):
+            if min(cut_margin(ref_E[h][s][n], wl.eps) for s in range(len(wl.calib_seeds))) <= 1e-3:
+                continue
+            compared += 1
+            np.testing.assert_array_equal(ix[ip[h][r]:ip[h][r + 1]], ox[op[n]:op[n + 1]],
+                                          err_msg=f"head {h} block {r}")
+    assert compared >= len(heads)
+    kept = (ip[:, -1] - ip[:, 0]).sum() / float(wl.H * nb * nb)
+    assert 0.0 < kept < 1.0
+    # attention on the timed input, every head on its own list
+    q, k, v, _ = si.generate(wl, seed=wl.seed, types_seed=types_seed)
+    qd, kd, vd = (to_device(x) for x in (q, k, v))
+    list_id = torch.arange(wl.H, dtype=torch.int32, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o = svg.svg_sparse_attn(qd, kd, vd, list_id, lists, status=status)
+    assert int(status.item()) == 0
+    for h in heads:
+        hp = ip[h] - ip[h][0]
+        hx = ix[ip[h][0]:ip[h][-1]]
+        qh, kh, vh = head64(q, 0, h), head64(k, 0, h), head64(v, 0, h)
+        for t in blocks:
+            rows = O.tile_rows(t, wl.N)
+            ref = O.block_sparse_rows(qh, kh, vh, rows, hp, hx)
+            got = to_float64(o[0, h, rows[0]:rows[-1] + 1])
+            assert_close(got, ref, f"calibrated head {h} tile {t}")
 
 
 # ------------------------------------------------ mask encodings (skip list, bitmap)

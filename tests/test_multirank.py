@@ -1,15 +1,19 @@
 """Multi-rank host logic of bench.py on CPU (gloo, world size 2).
 
-The layer shards by (batch, head) with no exchange step, so N GPUs run N
-independent layers (weak scaling); the only cross-rank operations are the
-barrier and the max-over-ranks of the step timings.  These tests run that
-logic as real gloo ranks and launch the reference arm through torchrun."""
+The layer shards by (batch, head) with no exchange step.  By default the heads
+of one layer are split into contiguous ranges, one per GPU (strong scaling);
+--shard replicas runs one independent layer per GPU (weak scaling).  The only
+cross-rank operations are the barrier, the max-over-ranks of the step timings
+and the sum of the ranks' work.  These tests run that logic as real gloo
+ranks, check that the head partition reassembles the one-rank layer, and
+launch the reference arm through torchrun."""
 import json
 import os
 import socket
 import subprocess
 import sys
 
+import numpy as np
 import pytest
 import torch.multiprocessing as mp
 
@@ -38,10 +42,11 @@ def _rank_main(rank, world, port, results):
         # per-rank timings that differ in every slot
         mine = [10.0 + rank, 5.0 - rank, 1.0 + 0.5 * rank]
         got = bench.max_over_ranks(mine, world, torch.device("cpu"))
+        work = bench.sum_over_ranks([1.0e12 * (rank + 1), 3.0], world, torch.device("cpu"))
         wl = si.WORKLOADS["cogvideox"]
-        value, tok, ms = bench.aggregate(2.0e12, got[0], 4, world, wl.B * wl.N)
+        value, tok, ms = bench.aggregate(work[0], got[0], 4, world * wl.B * wl.N)
         dist.barrier()
-        results[rank] = {"max": got, "value": value, "tokens": tok, "ms": ms,
+        results[rank] = {"max": got, "sum": work, "value": value, "tokens": tok, "ms": ms,
                          "seed": bench.rank_seed(wl, rank)}
     finally:
         dist.destroy_process_group()
@@ -55,9 +60,10 @@ def test_max_over_ranks_and_aggregate_gloo():
                        join=True, start_method="spawn")
     r0, r1 = results[0], results[1]
     assert r0["max"] == r1["max"] == [11.0, 5.0, 1.5]
+    assert r0["sum"] == r1["sum"] == [3.0e12, 6.0]
     # whole-job value: both ranks' work over the slowest rank's step time
     assert r0["ms"] == pytest.approx(11.0 / 4)
-    assert r0["value"] == pytest.approx(2 * 2.0e12 / (11.0 / 4 * 1e-3) / 1e12)
+    assert r0["value"] == pytest.approx(3.0e12 / (11.0 / 4 * 1e-3) / 1e12)
     assert r0["tokens"] == pytest.approx(2 * 17550 / (11.0 / 4 * 1e-3))
     assert r0["value"] == r1["value"]
     # independent inputs per rank
@@ -66,8 +72,68 @@ def test_max_over_ranks_and_aggregate_gloo():
 
 def test_single_rank_passthrough():
     assert bench.max_over_ranks([3, 2.5], 1, None) == [3.0, 2.5]
-    v, t, ms = bench.aggregate(1.0e12, 20.0, 10, 1, 100)
+    assert bench.sum_over_ranks([3, 2.5], 1, None) == [3.0, 2.5]
+    v, t, ms = bench.aggregate(1.0e12, 20.0, 10, 100)
     assert ms == 2.0 and v == pytest.approx(500.0) and t == pytest.approx(5.0e4)
+
+
+def test_head_shards_partition_the_layer():
+    # every head on exactly one rank, contiguous ranges in rank order, sizes
+    # within one of each other (H not divisible by the rank count included)
+    for H in (1, 2, 3, 7, 24, 40, 48):
+        for world in range(1, min(H, 8) + 1):
+            shards = [bench.shard_heads(H, world, r) for r in range(world)]
+            assert [h for s in shards for h in s] == list(range(H)), (H, world)
+            sizes = [len(s) for s in shards]
+            assert max(sizes) - min(sizes) <= 1 and min(sizes) >= 1
+            assert sizes == sorted(sizes, reverse=True)
+    assert bench.shard_heads(24, 5, 0) == range(0, 5) and bench.shard_heads(24, 5, 4) == range(20, 24)
+
+
+def _shard_layer_main(rank, world, port, results):
+    """One rank of a head-sharded layer: draw only this rank's heads, run the
+    oracle layer on them, and gather (heads, o, mode, mse) on every rank."""
+    import datetime
+
+    import torch.distributed as dist
+    from oracle import svg_oracle as O
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=120))
+    try:
+        wl = si.small("hunyuan720").scaled("shard-test", H=3)
+        heads = bench.shard_heads(wl.H, world, rank)
+        q, k, v, _ = si.generate(wl, seed=wl.seed, heads=heads)
+        idx = si.sample_queries(wl)
+        o, mode, mse = O.svg_layer(*(si.as_float64(t) for t in (q, k, v)), idx, wl.F, wl.P,
+                                   wl.width)
+        got = [None] * world
+        dist.all_gather_object(got, (heads.start, heads.stop, o, mode, mse))
+        if rank == 0:
+            results["parts"] = got
+    finally:
+        dist.destroy_process_group()
+
+
+def test_head_sharded_layer_reassembles_gloo():
+    """World size 2 over a 3-head layer (uneven split): the ranks' outputs,
+    modes and errors, put back in head order, equal the one-rank layer."""
+    from oracle import svg_oracle as O
+    world = 2
+    mgr = mp.get_context("spawn").Manager()
+    results = mgr.dict()
+    mp.start_processes(_shard_layer_main, args=(world, _free_port(), results), nprocs=world,
+                       join=True, start_method="spawn")
+    parts = results["parts"]
+    assert [(p[0], p[1]) for p in parts] == [(0, 2), (2, 3)]
+    wl = si.small("hunyuan720").scaled("shard-test", H=3)
+    q, k, v, _ = si.generate(wl)
+    o, mode, mse = O.svg_layer(*(si.as_float64(t) for t in (q, k, v)), si.sample_queries(wl),
+                               wl.F, wl.P, wl.width)
+    np.testing.assert_array_equal(np.concatenate([p[2] for p in parts], axis=1), o)
+    np.testing.assert_array_equal(np.concatenate([p[3] for p in parts]), mode)
+    np.testing.assert_array_equal(np.concatenate([p[4] for p in parts]), mse)
+    assert set(mode.tolist()) == {0, 1}  # both kinds of heads occur
 
 
 def test_rank_inputs_differ():
@@ -95,7 +161,7 @@ def test_reference_arm_under_torchrun_prints_once():
                 "cpu_baseline", "e2e", "impl"):
         assert key in line, key
     assert line["impl"] == "reference" and line["n_gpus"] == 2
-    assert line["config"]["workload"] == "cogvideox"
+    assert line["config"]["workload"] == "hunyuan720"
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
     assert line["value"] > 0

@@ -413,6 +413,9 @@ class TestCalibration:
         counts = np.array([64, 64, 64, 8])[:, None]
         np.testing.assert_allclose(E, sums / counts, atol=1e-13)
         np.testing.assert_allclose(E.sum(1), 1.0, atol=1e-13)
+        # a subset of query blocks, in the order asked for
+        Er = O.block_energy(q, k, T, row_blocks=[3, 0])
+        np.testing.assert_allclose(Er, (sums / counts)[[3, 0]], atol=1e-13)
 
     def test_energy_uniform_for_zero_queries(self):
         N, T = 150, 64

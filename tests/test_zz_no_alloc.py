@@ -54,6 +54,18 @@ def test_noalloc_matches_workspace_entry_point(wl):
     mse_ref, mode_ref = svg.svg_profile_heads(qd, kd, vd, wl.F, wl.P, wl.width, idx_d)
     mse_ref = mse_ref.cpu().numpy().astype(np.float64)
     mode_ref = mode_ref.cpu().numpy()
+    if wl.name == "tiny":
+        # the small case also straight against the float64 oracle
+        from oracle import svg_oracle as O
+        mse_o, mode_o = O.profile_heads(*(si.as_float64(x) for x in (q, k, v)),
+                                        si.sample_queries(wl), wl.F, wl.P, wl.width)
+        mse, mode = _run_noalloc(qd, kd, vd, wl, idx_d)
+        for i in range(len(mode_o)):
+            for c in range(2):
+                assert abs(mse[i, c] - mse_o[i, c]) <= 0.02 * mse_o[i, c] + 2e-5, (i, mse[i], mse_o[i])
+            margin = abs(mse_o[i, 0] - mse_o[i, 1]) / max(mse_o[i].max(), 1e-30)
+            if margin > MODE_MARGIN:
+                assert mode[i] == mode_o[i], i
     for call in range(2):
         mse, mode = _run_noalloc(qd, kd, vd, wl, idx_d)
         for i in range(len(mode_ref)):
