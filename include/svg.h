@@ -103,6 +103,18 @@ const char* svg_version(void);
 /* Text of the last error returned on the calling host thread ("" if none). */
 const char* svg_last_error(void);
 
+/* Bounded device waits.  Every mbarrier wait of the tcgen05 attention kernel
+ * polls at most `polls` times (default 1 << 22, which no working pipeline
+ * comes near) before it gives up: the kernel then sets SVG_DEVICE_TIMEOUT in
+ * the call's device status word, lets its copies and tensor-core operations
+ * in flight finish, frees its tensor memory and returns, so the CUDA context
+ * stays usable.  This setting exists to test that path and to diagnose
+ * stalls; it is process-wide, applies to launches made after the call, and
+ * 0 restores the default.  The pages have no counterpart to it.
+ * svg_get_wait_limit returns the current value. */
+svg_status svg_set_wait_limit(uint32_t polls);
+uint32_t svg_get_wait_limit(void);
+
 /* --------------------------------------------------------------------------
  * 1. Online head profiling
  *    [SVG] section "動態自適應的稀疏策略", steps 1-3: sample a few query
@@ -361,7 +373,11 @@ svg_status svg_lists_to_bitmap(int n_rows, int n_cols, const int32_t* indptr,
  *               the profiling output mode_out is a valid list_id.
  *  indptr       device int32 [n_lists][n_qblocks + 1], absolute offsets into
  *               `indices`; n_qblocks must equal nB.
- *  indices      device int32, key-block indices in [0, nB), ascending per row.
+ *  indices      device int32, key-block indices in [0, nB), strictly
+ *               ascending per row (a row is a set of key blocks).  An entry
+ *               outside [0, nB), or not above the row's previous used entry
+ *               (a repeat or a descending entry), is skipped and sets
+ *               SVG_DEVICE_BAD_INDEX; no key block is attended twice.
  *  scale        softmax scale; 0 selects 1/sqrt(d).
  *  device_status  optional device int32 (may be NULL), see SVG_DEVICE_*.
  * Arithmetic (bf16): Q.K^T on bf16 tensor cores with fp32 accumulation, fp32

@@ -32,6 +32,8 @@ _f = C.c_float
 SIGNATURES = {
     "svg_version": (C.c_char_p, []),
     "svg_last_error": (C.c_char_p, []),
+    "svg_set_wait_limit": (_i, [C.c_uint32]),
+    "svg_get_wait_limit": (C.c_uint32, []),
     "svg_profile_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
     "svg_profile_heads": (_i, [_p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _p, _i, _p, _p, _p, _sz,
                                _p]),

@@ -39,6 +39,9 @@ struct AttnArgs {
   // 0 .. n_qblocks-1 per list); null = index order.  Results never depend
   // on it.
   const int32_t* tile_order;
+  // Polls of one mbarrier wait before the tcgen05 kernel gives up with
+  // SVG_DEVICE_TIMEOUT (svg_set_wait_limit).
+  uint32_t spin_limit;
 };
 
 __device__ __forceinline__ bool reads_copies(const AttnArgs& a, int bh);

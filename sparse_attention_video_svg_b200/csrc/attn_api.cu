@@ -52,7 +52,8 @@ svg_status sparse_attn_impl(const char* who, const void* q, const void* k, const
   if (!(scale >= 0.f) || isinf(scale)) return fail(SVG_ERR_INVALID_ARG, "%s: bad scale", who);
   AttnArgs a{q, k, v, o, dtype, B, H, N, d, list_id, n_lists, n_qblocks, indptr, indices,
              scale == 0.f ? 1.f / sqrtf(static_cast<float>(d)) : scale, device_status,
-             order, frames, tokens_per_frame, layout, q_tm, k_tm, v_tm, tile_order};
+             order, frames, tokens_per_frame, layout, q_tm, k_tm, v_tm, tile_order,
+             wait_limit()};
   cudaStream_t s = as_stream(stream);
   if (dtype == SVG_FP32) return d == 64 ? launch_attn_fp32<64>(a, s) : launch_attn_fp32<128>(a, s);
   return d == 64 ? launch_attn_sm100<64>(a, s) : launch_attn_sm100<128>(a, s);

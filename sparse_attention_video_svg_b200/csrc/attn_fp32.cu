@@ -62,12 +62,16 @@ __global__ void __launch_bounds__(256) attn_fp32(AttnArgs a) {
       qv[e] = q[rq * D + lane + 32 * e];
       acc[e] = 0.f;
     }
+    int last = -1;
     for (int t = 0; t < lst.len; ++t) {
       const int j = lst.idx[t];
-      if (j < 0 || j >= nb) {
+      // rows must be strictly ascending: an out-of-range, repeated or
+      // descending entry is skipped, so no key block is attended twice
+      if (j < 0 || j >= nb || j <= last) {
         set_status(a.status, SVG_DEVICE_BAD_INDEX);
         continue;
       }
+      last = j;
       for (int c = j * SVG_TILE; c < min(N, (j + 1) * SVG_TILE); ++c) {
         const long long rc = row(c);
         float dot = 0.f;

@@ -58,7 +58,6 @@ constexpr int kThreads = 384;
 constexpr int kBox = 16384;           // one 128-row x 128-byte TMA box
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;  // lazy-rescale threshold (factor 256)
-constexpr uint32_t kSpinLimit = 1u << 22;
 constexpr uint32_t kDrainLimit = 1u << 20;
 constexpr int kLaunchRegs = 168;      // 65536 / 384, rounded down to a multiple of 8
 
@@ -70,11 +69,21 @@ struct Cfg {
   // K/V ring entries; even, so K tiles always sit in even and V tiles in odd
   // entries
   static constexpr int kSlots = D == 64 ? 8 : 4;
-  static constexpr int kSteps = kSlots / 2;        // merged-walk steps in flight
+  static constexpr int kSteps = kSlots / 2;        // merged-walk steps in the ring
+  // Step records in flight.  K and V entries are claimed one at a time, so
+  // the producer may run up to kSteps + 1 steps ahead of the slowest reader
+  // of a record (the converter): kSteps + 2 records are live at most.
+  static constexpr int kInfo = 8;
+  static_assert(kInfo >= kSteps + 2, "step records");
   static constexpr bool kSepP = D == 64;           // P_t in TMEM columns of its own
+  // d = 128: one MMA issuer for both members (warp 1), which fixes the
+  // order on the tensor core, and two V converter warps (2, 3); d = 64: one
+  // issuer per member (warps 1, 2) and one converter (warp 3)
+  static constexpr bool kOneIssuer = D == 128;
+  static constexpr int kConvWarps = kOneIssuer ? 2 : 1;
   static constexpr int kOffQ = 0;                  // [member][depth]
   static constexpr int kOffKV = 2 * kQDepth * kTile;
-  static constexpr int kOffInfo = kOffKV + kSlots * kTile;  // uint32 [kSteps]
+  static constexpr int kOffInfo = kOffKV + kSlots * kTile;  // uint32 [kInfo]
   static constexpr int kOffBar = kOffInfo + 64;
   static constexpr int kBars = 4 * kQDepth + 3 * kSlots + 5 * 2;
   static constexpr int kSmem = kOffBar + kBars * 8 + 16 + 1024;  // + alignment slack
@@ -87,8 +96,8 @@ struct Cfg {
   // Register split of the 384 x 168 launch registers: warpgroup 0
   // (producer, MMA issuers, converter) drops to kRegsLow, the two softmax
   // warpgroups rise to kRegsHigh (the split with the fewest spills ptxas reports).
-  static constexpr int kRegsLow = 80;
-  static constexpr int kRegsHigh = 208;
+  static constexpr int kRegsLow = D == 128 ? 72 : 88;
+  static constexpr int kRegsHigh = D == 128 ? 216 : 208;
   static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kLaunchRegs, "register split");
   static constexpr uint32_t kIdescQK = idesc_bf16(128, 128, false);
   static constexpr uint32_t kIdescPV = idesc_f16(128, D, true);
@@ -144,18 +153,24 @@ __device__ __forceinline__ void member_list(const AttnArgs& a, int bh, int qt, i
   end = e;
 }
 
-__device__ __forceinline__ void skip_invalid(const AttnArgs& a, int nb, int& p, int e,
+// A list entry is used when it is a valid key block above the member's last
+// used one: rows must be strictly ascending, and an out-of-range, repeated or
+// descending entry is skipped (and reported), so a key block is never
+// attended twice.  The softmax warps apply the same rule to the same list.
+__device__ __forceinline__ bool usable(int j, int last, int nb) { return valid_tile(j, nb) && j > last; }
+
+__device__ __forceinline__ void skip_invalid(const AttnArgs& a, int nb, int& p, int e, int last,
                                              bool report) {
-  while (p < e && !valid_tile(a.indices[p], nb)) {
+  while (p < e && !usable(a.indices[p], last, nb)) {
     if (report) set_status(a.status, SVG_DEVICE_BAD_INDEX);
     ++p;
   }
 }
 
 // Next key block of the merged walk over both members' lists, whose heads
-// are valid (or exhausted).  mask bit t: member t keeps block j.  Every entry
-// of either list is visited exactly once, in whatever order the lists come;
-// equal heads are shared.  Afterwards both heads are again valid or
+// are usable (or exhausted).  mask bit t: member t keeps block j.  Every
+// usable entry of either list is visited exactly once, in ascending order;
+// equal heads are shared.  Afterwards both heads are again usable or
 // exhausted.
 __device__ __forceinline__ bool merge_next(const AttnArgs& a, int nb, int (&p)[2],
                                            const int (&e)[2], int& j, int& mask, bool report) {
@@ -169,17 +184,21 @@ __device__ __forceinline__ bool merge_next(const AttnArgs& a, int nb, int (&p)[2
   for (int t = 0; t < 2; ++t)
     if (mask >> t & 1) {
       ++p[t];
-      skip_invalid(a, nb, p[t], e[t], report);
+      skip_invalid(a, nb, p[t], e[t], j, report);
     }
   return true;
 }
 
 // Bounded wait on an mbarrier phase; false if it timed out or another role
-// aborted.
+// aborted (checked every 256 polls).  SW (a launch whose svg_set_wait_limit
+// differs from the default) reads the poll limit from the shared word after
+// the CTA's abort flag; otherwise the limit is the compile-time default.
+template <bool SW>
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                          int32_t* status) {
   const uint32_t addr = smem_u32(bar);
-  for (uint32_t i = 0; i < kSpinLimit; ++i) {
+  const uint32_t limit = SW ? static_cast<uint32_t>(abort_flag[1]) : kDefaultWaitLimit;
+  for (uint32_t i = 0; i < limit; ++i) {
     if (mbar_try_wait(addr, parity)) return true;
     if ((i & 255u) == 255u && *abort_flag) return false;
   }
@@ -197,7 +216,7 @@ __device__ __forceinline__ void drain_bar(uint64_t* bar, uint32_t parity) {
 }
 
 // Softmax and epilogue of member t (warps 4 + 4t .. 7 + 4t).
-template <int D>
+template <int D, bool SW>
 __device__ __forceinline__ void softmax_member(const AttnArgs& a, const Bars& B,
                                                volatile int* abort_flag, uint32_t tmem,
                                                int n_items, int n_pairs, int nb) {
@@ -222,10 +241,12 @@ __device__ __forceinline__ void softmax_member(const AttnArgs& a, const Bars& B,
     member_list(a, bh, qt, nb, beg, end, false);
     float m_used = -INFINITY, l = 0.f;
     bool first = true;
+    int last = -1;
     for (int e = beg; e < end; ++e) {
       const int j = a.indices[e];
-      if (!valid_tile(j, nb)) continue;
-      if (!(ok = wait_bar(&B.s_full[t], g & 1, abort_flag, a.status))) break;
+      if (!usable(j, last, nb)) continue;
+      last = j;
+      if (!(ok = wait_bar<SW>(&B.s_full[t], g & 1, abort_flag, a.status))) break;
       tc_fence_after();
       float s[128];
       {
@@ -295,7 +316,7 @@ __device__ __forceinline__ void softmax_member(const AttnArgs& a, const Bars& B,
         // P_t and O_t are free once the previous P.V of this member is done
         // (waited for only now, so that P.V overlaps the exponentials)
         if (g > 0) {
-          if (!(ok = wait_bar(&B.o_done[t], (g - 1) & 1, abort_flag, a.status))) break;
+          if (!(ok = wait_bar<SW>(&B.o_done[t], (g - 1) & 1, abort_flag, a.status))) break;
           tc_fence_after();
         }
       }
@@ -329,7 +350,7 @@ __device__ __forceinline__ void softmax_member(const AttnArgs& a, const Bars& B,
     const bool empty = first;
     float inv = 0.f;
     if (!empty) {
-      if (!(ok = wait_bar(&B.o_done[t], (g - 1) & 1, abort_flag, a.status))) break;
+      if (!(ok = wait_bar<SW>(&B.o_done[t], (g - 1) & 1, abort_flag, a.status))) break;
       tc_fence_after();
       inv = l > 0.f ? 1.f / l : 0.f;
     }
@@ -408,7 +429,7 @@ __device__ __forceinline__ void gather_rows(unsigned char* dst, const __nv_bfloa
 // adds the phase's regular arrival, so the barrier completes when the rows
 // have landed.  The consumers fence the async proxy after their wait, as the
 // tensor core reads what the generic proxy wrote.
-template <int D>
+template <int D, bool SW>
 __device__ __forceinline__ void producer(const AttnArgs& a, const Maps& maps, const Bars& B,
                                          unsigned char* smem, volatile uint32_t* step_info,
                                          volatile int* abort_flag, int n_items, int n_pairs,
@@ -422,7 +443,7 @@ __device__ __forceinline__ void producer(const AttnArgs& a, const Maps& maps, co
   bool ok = true;
   auto leader_wait = [&](uint64_t* bar, uint32_t parity) -> bool {
     int r = 1;
-    if (leader) r = wait_bar(bar, parity, abort_flag, a.status) ? 1 : 0;
+    if (leader) r = wait_bar<SW>(bar, parity, abort_flag, a.status) ? 1 : 0;
     return __shfl_sync(0xffffffffu, r, 0) != 0;
   };
   // gathered tile: lanes' copies, then the barrier takes them over
@@ -432,10 +453,24 @@ __device__ __forceinline__ void producer(const AttnArgs& a, const Maps& maps, co
     __syncwarp();
     if (leader) mbar_arrive(bar);
   };
-  auto claim = [&]() -> bool {  // the K and V entries of the step at ring index L are free
-    return leader_wait(&B.kv_empty[L % S], ((L / S) & 1) ^ 1) &&
-           leader_wait(&B.kv_empty[(L + 1) % S], (((L + 1) / S) & 1) ^ 1);
+  // Ring entry l is free (its previous occupant released).  With one MMA
+  // issuer the K and V entries of a step are claimed one at a time: a K tile
+  // is released after the two Q K^T of its step, a V tile only after the two
+  // P.V, which that thread issues while serving the next step, so the next K
+  // load does not wait for the last P.V.  With an issuer per member both
+  // entries are claimed before the K copy: a member that skips a step
+  // releases the step's V entry at once, and were the next K tile loaded
+  // first it could pass the reuse of that entry and release it a second
+  // time before the other member's P.V has read it.
+  auto claim = [&](uint32_t l) -> bool {
+    return leader_wait(&B.kv_empty[l % S], ((l / S) & 1) ^ 1);
   };
+  // claims made before the copy of entry L + kv of a step
+  auto claim_step = [&](int kv) -> bool {
+    if (C::kOneIssuer) return claim(L + kv);
+    return kv == 1 || (claim(L) && claim(L + 1));
+  };
+  uint32_t issued = 0;  // ring entries whose copies were issued
   for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
     const int bh = item / n_pairs, qt0 = 2 * (item - bh * n_pairs);
     const bool tm = gathers_input(a, bh);
@@ -450,7 +485,7 @@ __device__ __forceinline__ void producer(const AttnArgs& a, const Maps& maps, co
       qtile[t] = query_tile(a, bh, qt0 + t, nb);
       if (qtile[t] < 0 && qt0 + t < nb && leader) set_status(a.status, SVG_DEVICE_BAD_INDEX);
       member_list(a, bh, qtile[t], nb, p[t], e[t], leader);
-      skip_invalid(a, nb, p[t], e[t], leader);
+      skip_invalid(a, nb, p[t], e[t], -1, leader);
     }
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
@@ -478,9 +513,10 @@ __device__ __forceinline__ void producer(const AttnArgs& a, const Maps& maps, co
                             (m & 2u) * (p[1] >= e[1] ? 1u : 0u);
       const uint32_t info = m | ((m & ~seen) << 2) | (last << 4) | (tm ? kStepGathered : 0u);
       seen |= m;
-      if (!(ok = claim())) break;
-      if (leader) step_info[(L / 2) % C::kSteps] = info;  // released by the step's arrives
       for (int kv = 0; kv < 2; ++kv) {
+        if (!(ok = claim_step(kv))) break;
+        // the record is read after the step's K entry is full
+        if (kv == 0 && leader) step_info[(L / 2) % C::kInfo] = info;
         const uint32_t slot = (L + kv) % S;
         unsigned char* dst = smem + C::kOffKV + slot * C::kTile;
         const void* src = kv == 0 ? a.k : a.v;
@@ -495,24 +531,26 @@ __device__ __forceinline__ void producer(const AttnArgs& a, const Maps& maps, co
           gather_into(dst, static_cast<const __nv_bfloat16*>(src) + head, j * 128,
                       &B.kv_full[slot]);
         }
+        issued = L + kv + 1;
       }
       L += 2;
     }
   }
   // end record in the next step's entries; plain arrives complete their
   // phases
-  if (ok && (ok = claim())) {
+  for (int kv = 0; kv < 2 && ok; ++kv) {
+    if (!(ok = claim_step(kv))) break;
     if (leader) {
-      step_info[(L / 2) % C::kSteps] = kStepEnd;
-      mbar_arrive(&B.kv_full[L % S]);
-      mbar_arrive(&B.kv_full[(L + 1) % S]);
+      if (kv == 0) step_info[(L / 2) % C::kInfo] = kStepEnd;
+      mbar_arrive(&B.kv_full[(L + kv) % S]);
     }
   }
   if (!ok) {
     // let the copies already issued land before the CTA can exit
     cp_async_wait<0>();
     if (leader) {
-      for (uint32_t l = L > S ? L - S : 0; l < L; ++l) drain_bar(&B.kv_full[l % S], (l / S) & 1);
+      for (uint32_t l = issued > S ? issued - S : 0; l < issued; ++l)
+        drain_bar(&B.kv_full[l % S], (l / S) & 1);
       for (int t = 0; t < 2; ++t)
         for (uint32_t c = cq[t] > QD ? cq[t] - QD : 0; c < cq[t]; ++c)
           drain_bar(&B.q_full[t * QD + c % QD], (c / QD) & 1);
@@ -520,7 +558,153 @@ __device__ __forceinline__ void producer(const AttnArgs& a, const Maps& maps, co
   }
 }
 
-template <int D>
+// MMA issuer (one thread).  With kOneIssuer it serves both members in a
+// fixed order per step: member 0's pending P.V, member 0's Q K^T, member 1's
+// pending P.V, member 1's Q K^T.  The tensor core runs its instructions in
+// issue order, so member 1's scores land one P.V + Q K^T after member 0's and
+// the two softmax warpgroups take turns on the exponential unit instead of
+// sharing it.  Otherwise each member has an issuer thread of its own.  The
+// thread serves members t0 .. t1.
+template <int D, int t0, int t1, bool SW>
+__device__ __forceinline__ void issuer(const Bars& B, unsigned char* smem,
+                                       volatile uint32_t* step_info, volatile int* abort_flag,
+                                       uint32_t tmem, int32_t* status) {
+  using C = Cfg<D>;
+  constexpr int QD = C::kQDepth, S = C::kSlots;
+  uint32_t t_s[2], t_p[2], t_o[2];
+  uint64_t dq[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    t_s[t] = tmem + C::kColS + 128 * t;
+    t_p[t] = tmem + C::kColP + C::kPStride * t;
+    t_o[t] = tmem + C::kColO + C::kOStride * t;
+    // descriptor of the member's first Q buffer; a buffer at byte offset x
+    // adds x >> 4 (the start-address field)
+    dq[t] = sdesc_sw128(smem_u32(smem + C::kOffQ + t * QD * C::kTile), 16, 1024);
+  }
+  const uint64_t dk = sdesc_sw128(smem_u32(smem + C::kOffKV), 16, 1024);
+  const uint64_t dv = sdesc_sw128(smem_u32(smem + C::kOffKV), kBox, 1024);
+  uint32_t L = 0, cq[2] = {0, 0}, nq[2] = {0, 0}, np[2] = {0, 0}, pend_lv[2] = {0, 0};
+  bool ok = true, pend[2] = {false, false}, pend_first[2] = {false, false};
+  auto issue_pv = [&](int t) -> bool {
+    if (!wait_bar<SW>(&B.p_ready[t], np[t] & 1, abort_flag, status)) return false;
+    const uint32_t slot = pend_lv[t] % S;
+    if (!wait_bar<SW>(&B.v_ready[slot], (pend_lv[t] / S) & 1, abort_flag, status)) return false;
+    tc_fence_after();
+    const uint64_t d0 = dv + ((slot * C::kTile) >> 4);
+    mma_ts_k128(t_o[t], t_p[t], d0, C::kIdescPV, pend_first[t] ? 0u : 1u);
+    tc_commit(&B.o_done[t]);
+    tc_commit(&B.kv_empty[slot]);
+    ++np[t];
+    pend[t] = false;
+    return true;
+  };
+  while (ok) {
+    const uint32_t kslot = L % S;
+    if (!(ok = wait_bar<SW>(&B.kv_full[kslot], (L / S) & 1, abort_flag, status))) break;
+    const uint32_t info = step_info[(L / 2) % C::kInfo];
+    // gathered tiles were written through the generic proxy
+    if (info & kStepGathered) fence_proxy_async_smem();
+    if (info & kStepEnd) break;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {  // unrolled: the per-member state stays in registers
+      if (t < t0 || t > t1 || !ok) continue;
+      if (!(info >> t & 1u)) {
+        // this member skips the block: its pending P.V goes now (otherwise
+        // that V entry could stay held past the point where the producer
+        // needs it again), then its share of both entries is released
+        if (pend[t] && !(ok = issue_pv(t))) continue;
+        tc_commit(&B.kv_empty[kslot]);
+        tc_commit(&B.kv_empty[kslot + 1]);
+        continue;
+      }
+      if constexpr (!C::kSepP) {
+        // P_t lives in S_t: the previous P.V goes first (tensor-core order)
+        if (pend[t] && !(ok = issue_pv(t))) continue;
+      } else if (nq[t] > 0) {
+        if (!(ok = wait_bar<SW>(&B.s_free[t], (nq[t] - 1) & 1, abort_flag, status))) continue;
+      }
+      const uint32_t qs = cq[t] % QD;
+      if (info >> (2 + t) & 1u) {  // first block of the item: a new Q tile
+        if (!(ok = wait_bar<SW>(&B.q_full[t * QD + qs], (cq[t] / QD) & 1, abort_flag, status)))
+          continue;
+        if (info & kStepGathered) fence_proxy_async_smem();
+      }
+      tc_fence_after();
+      const uint64_t q0 = dq[t] + ((qs * C::kTile) >> 4), k0 = dk + ((kslot * C::kTile) >> 4);
+      if constexpr (D == 64)
+        mma_ss_k64(t_s[t], q0, k0, C::kIdescQK);
+      else
+        mma_ss_k128(t_s[t], q0, k0, C::kIdescQK, kBox >> 4);
+      tc_commit(&B.s_full[t]);
+      tc_commit(&B.kv_empty[kslot]);
+      if (info >> (4 + t) & 1u) {  // last block of the item: its Q buffer is free
+        tc_commit(&B.q_empty[t * QD + qs]);
+        ++cq[t];
+      }
+      ++nq[t];
+      if constexpr (C::kSepP) {
+        if (pend[t] && !(ok = issue_pv(t))) continue;
+      }
+      pend[t] = true;
+      pend_first[t] = (info >> (2 + t)) & 1u;
+      pend_lv[t] = L + 1;
+    }
+    L += 2;
+  }
+#pragma unroll
+  for (int t = 0; t < 2; ++t)
+    if (t >= t0 && t <= t1 && ok && pend[t]) ok = issue_pv(t);
+  // every MMA issued by this thread completes before TMEM is released
+  tc_commit(&B.drain[t0]);
+  drain_bar(&B.drain[t0], 0);
+}
+
+// Converts every V tile in place from bf16 to fp16, in ring order; `part` of
+// C::kConvWarps warps (each takes every kConvWarps-th 16-byte piece, and
+// each arrives once on the tile's v_ready).  bf16 -> fp16 is exact for
+// |v| <= 65504 (fp16 subnormals keep the absolute error below 2^-25);
+// larger values become inf and are reported as SVG_DEVICE_RANGE.  The check
+// is on the bf16 bits: a magnitude field of 0x4780 (65536) or more, inf and
+// NaN included, carries into bit 15 of its half once 0x3880 is added, and the
+// 15-bit fields cannot carry into each other.
+template <int D, bool SW>
+__device__ __forceinline__ void converter(const AttnArgs& a, const Bars& B, unsigned char* smem,
+                                          volatile uint32_t* step_info, volatile int* abort_flag,
+                                          int part) {
+  using C = Cfg<D>;
+  constexpr int S = C::kSlots;
+  const int lane = threadIdx.x & 31;
+  uint32_t L = 0, over = 0;
+  bool ok = true;
+  while (ok) {
+    const uint32_t slot = (L + 1) % S;
+    if (!(ok = wait_bar<SW>(&B.kv_full[slot], ((L + 1) / S) & 1, abort_flag, a.status))) break;
+    if (step_info[(L / 2) % C::kInfo] & kStepEnd) break;
+    uint4* tile = reinterpret_cast<uint4*>(smem + C::kOffKV + slot * C::kTile);
+#pragma unroll 4
+    for (int c = part * 32 + lane; c < C::kTile / 16; c += 32 * C::kConvWarps) {
+      uint4 v = tile[c];
+      uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xffff0000u);
+        over |= (w[i] & 0x7fff7fffu) + 0x38803880u;
+        const __half2 h = __floats2half2_rn(lo, hi);
+        w[i] = *reinterpret_cast<const uint32_t*>(&h);
+      }
+      tile[c] = v;
+    }
+    fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&B.v_ready[slot]);
+    L += 2;
+  }
+  if (__any_sync(0xffffffffu, (over & 0x80008000u) != 0u) && lane == 0)
+    set_status(a.status, SVG_DEVICE_RANGE);
+}
+
+template <int D, bool SW>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_sm100_kernel(const __grid_constant__ Maps maps, const AttnArgs a) {
   using C = Cfg<D>;
@@ -541,6 +725,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   B.o_done = B.p_ready + 2;
   B.drain = B.o_done + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(B.drain + 2);
+  // abort flag, then the poll limit of every wait
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile uint32_t* step_info = reinterpret_cast<volatile uint32_t*>(smem + C::kOffInfo);
 
@@ -557,7 +742,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < S; ++i) {
       mbar_init(&B.kv_full[i], 1);
       mbar_init(&B.kv_empty[i], 2);
-      mbar_init(&B.v_ready[i], 1);
+      mbar_init(&B.v_ready[i], C::kConvWarps);
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&B.s_full[t], 1);
@@ -566,7 +751,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&B.o_done[t], 1);
       mbar_init(&B.drain[t], 1);
     }
-    *abort_flag = 0;
+    abort_flag[0] = 0;
+    abort_flag[1] = static_cast<int>(min(a.spin_limit, 0x7fffffffu));
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
@@ -591,129 +777,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     reg_dealloc<C::kRegsLow>();
     // ------------------------------------------------------------ producer
-    producer<D>(a, maps, B, smem, step_info, abort_flag, n_items, n_pairs, nb);
-  } else if (warp == 1 || warp == 2) {
+    producer<D, SW>(a, maps, B, smem, step_info, abort_flag, n_items, n_pairs, nb);
+  } else if (warp == 1 || (warp == 2 && !C::kOneIssuer)) {
     reg_dealloc<C::kRegsLow>();
     // ------------------------------------------------------------ MMA issuers
     if (lane == 0) {
-      const int t = warp - 1;  // member
-      const uint32_t t_s = tmem + C::kColS + 128 * t;
-      const uint32_t t_p = tmem + C::kColP + C::kPStride * t;
-      const uint32_t t_o = tmem + C::kColO + C::kOStride * t;
-      // descriptors of the first Q buffer and of ring entry 0; a buffer at
-      // byte offset x adds x >> 4 (the start-address field)
-      const uint64_t dq = sdesc_sw128(smem_u32(smem + C::kOffQ + t * QD * C::kTile), 16, 1024);
-      const uint64_t dk = sdesc_sw128(smem_u32(smem + C::kOffKV), 16, 1024);
-      const uint64_t dv = sdesc_sw128(smem_u32(smem + C::kOffKV), kBox, 1024);
-      uint32_t L = 0, cq = 0, nq = 0, np = 0;
-      bool ok = true, pend = false, pend_first = false;
-      uint32_t pend_lv = 0;
-      auto issue_pv = [&]() -> bool {
-        if (!wait_bar(&B.p_ready[t], np & 1, abort_flag, a.status)) return false;
-        const uint32_t slot = pend_lv % S;
-        if (!wait_bar(&B.v_ready[slot], (pend_lv / S) & 1, abort_flag, a.status)) return false;
-        tc_fence_after();
-        const uint64_t d0 = dv + ((slot * C::kTile) >> 4);
-        mma_ts_k128(t_o, t_p, d0, C::kIdescPV, pend_first ? 0u : 1u);
-        tc_commit(&B.o_done[t]);
-        tc_commit(&B.kv_empty[slot]);
-        ++np;
-        pend = false;
-        return true;
-      };
-      while (ok) {
-        const uint32_t kslot = L % S;
-        if (!(ok = wait_bar(&B.kv_full[kslot], (L / S) & 1, abort_flag, a.status))) break;
-        const uint32_t info = step_info[(L / 2) % C::kSteps];
-        // gathered tiles were written through the generic proxy
-        if (info & kStepGathered) fence_proxy_async_smem();
-        if (info & kStepEnd) break;
-        if (!(info >> t & 1u)) {
-          // this member skips the block: its pending P.V goes now (otherwise
-          // that V entry could stay held past the point where the producer
-          // needs it again), then its share of both entries is released
-          if (pend && !(ok = issue_pv())) break;
-          tc_commit(&B.kv_empty[kslot]);
-          tc_commit(&B.kv_empty[kslot + 1]);
-          L += 2;
-          continue;
-        }
-        if constexpr (!C::kSepP) {
-          // P_t lives in S_t: the previous P.V goes first (tensor-core order)
-          if (pend && !(ok = issue_pv())) break;
-        } else if (nq > 0) {
-          if (!(ok = wait_bar(&B.s_free[t], (nq - 1) & 1, abort_flag, a.status))) break;
-        }
-        const uint32_t qs = cq % QD;
-        if (info >> (2 + t) & 1u) {  // first block of the item: a new Q tile
-          if (!(ok = wait_bar(&B.q_full[t * QD + qs], (cq / QD) & 1, abort_flag, a.status))) break;
-          if (info & kStepGathered) fence_proxy_async_smem();
-        }
-        tc_fence_after();
-        const uint64_t q0 = dq + ((qs * C::kTile) >> 4), k0 = dk + ((kslot * C::kTile) >> 4);
-        if constexpr (D == 64)
-          mma_ss_k64(t_s, q0, k0, C::kIdescQK);
+      if constexpr (C::kOneIssuer) {
+        issuer<D, 0, 1, SW>(B, smem, step_info, abort_flag, tmem, a.status);
+      } else {
+        if (warp == 1)
+          issuer<D, 0, 0, SW>(B, smem, step_info, abort_flag, tmem, a.status);
         else
-          mma_ss_k128(t_s, q0, k0, C::kIdescQK, kBox >> 4);
-        tc_commit(&B.s_full[t]);
-        tc_commit(&B.kv_empty[kslot]);
-        if (info >> (4 + t) & 1u) {  // last block of the item: its Q buffer is free
-          tc_commit(&B.q_empty[t * QD + qs]);
-          ++cq;
-        }
-        ++nq;
-        if constexpr (C::kSepP) {
-          if (pend && !(ok = issue_pv())) break;
-        }
-        pend = true;
-        pend_first = (info >> (2 + t)) & 1u;
-        pend_lv = L + 1;
-        L += 2;
+          issuer<D, 1, 1, SW>(B, smem, step_info, abort_flag, tmem, a.status);
       }
-      if (ok && pend) ok = issue_pv();
-      // every MMA issued by this thread completes before TMEM is released
-      tc_commit(&B.drain[t]);
-      drain_bar(&B.drain[t], 0);
     }
-  } else if (warp == 3) {
+  } else if (warp <= 3) {
     reg_dealloc<C::kRegsLow>();
     // ------------------------------------------------------------ V to fp16
-    // Converts every V tile in place, in ring order.  bf16 -> fp16 is exact
-    // for |v| <= 65504 (fp16 subnormals keep the absolute error below
-    // 2^-25); larger values become inf and are reported as SVG_DEVICE_RANGE.
-    // The check is on the bf16 bits: a magnitude field of 0x4780 (65536) or
-    // more, inf and NaN included, carries into bit 15 of its half once
-    // 0x3880 is added, and the 15-bit fields cannot carry into each other.
-    uint32_t L = 0, over = 0;
-    bool ok = true;
-    while (ok) {
-      const uint32_t slot = (L + 1) % S;
-      if (!(ok = wait_bar(&B.kv_full[slot], ((L + 1) / S) & 1, abort_flag, a.status))) break;
-      if (step_info[(L / 2) % C::kSteps] & kStepEnd) break;
-      uint4* tile = reinterpret_cast<uint4*>(smem + C::kOffKV + slot * C::kTile);
-#pragma unroll 4
-      for (int c = lane; c < C::kTile / 16; c += 32) {
-        uint4 v = tile[c];
-        uint32_t* w = reinterpret_cast<uint32_t*>(&v);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xffff0000u);
-          over |= (w[i] & 0x7fff7fffu) + 0x38803880u;
-          const __half2 h = __floats2half2_rn(lo, hi);
-          w[i] = *reinterpret_cast<const uint32_t*>(&h);
-        }
-        tile[c] = v;
-      }
-      fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&B.v_ready[slot]);
-      L += 2;
-    }
-    if (__any_sync(0xffffffffu, (over & 0x80008000u) != 0u) && lane == 0)
-      set_status(a.status, SVG_DEVICE_RANGE);
+    converter<D, SW>(a, B, smem, step_info, abort_flag, warp - (4 - C::kConvWarps));
   } else {
     reg_alloc<C::kRegsHigh>();
-    softmax_member<D>(a, B, abort_flag, tmem, n_items, n_pairs, nb);
+    softmax_member<D, SW>(a, B, abort_flag, tmem, n_items, n_pairs, nb);
   }
   tc_fence_before();
   __syncthreads();
@@ -766,12 +850,16 @@ svg_status launch_attn_sm100(const AttnArgs& a, cudaStream_t s) {
        (!make_map(&maps.qt, a.q_tm, BH, a.N, D) || !make_map(&maps.kt, a.k_tm, BH, a.N, D) ||
         !make_map(&maps.vt, a.v_tm, BH, a.N, D))))
     return fail(SVG_ERR_CUDA, "sparse_attn: cannot encode TMA descriptors");
-  if (cudaFuncSetAttribute(attn_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           C::kSmem) != cudaSuccess)
+  // a launch with a poll limit other than the default runs the instantiation
+  // that reads it (the same code otherwise)
+  const bool sw = a.spin_limit != kDefaultWaitLimit;
+  auto kernel = sw ? attn_sm100_kernel<D, true> : attn_sm100_kernel<D, false>;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem) !=
+      cudaSuccess)
     return fail(SVG_ERR_CUDA, "sparse_attn: cannot reserve %d bytes of shared memory", C::kSmem);
   const long long items = static_cast<long long>(BH) * ((n_tiles(a.N) + 1) / 2);
   const int grid = static_cast<int>(items < sm_count() ? items : sm_count());
-  attn_sm100_kernel<D><<<grid, kThreads, C::kSmem, s>>>(maps, a);
+  kernel<<<grid, kThreads, C::kSmem, s>>>(maps, a);
   return check_launch("sparse_attn sm100");
 }
 

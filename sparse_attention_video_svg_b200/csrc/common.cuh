@@ -30,6 +30,11 @@ inline int elt_bytes(int dtype) { return dtype == SVG_FP32 ? 4 : 2; }
 // Number of SMs of the current device (cached per device).
 int sm_count();
 
+// Polls of one bounded device wait before a kernel gives up
+// (svg_set_wait_limit; kDefaultWaitLimit unless changed).
+constexpr uint32_t kDefaultWaitLimit = 1u << 22;
+uint32_t wait_limit();
+
 // ---------------------------------------------------------------- device side
 
 __device__ __forceinline__ void set_status(int32_t* status, int bits) {

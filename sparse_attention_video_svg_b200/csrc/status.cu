@@ -3,6 +3,7 @@
 #include <stdarg.h>
 #include <stdio.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -42,8 +43,20 @@ int sm_count() {
   return cache[dev];
 }
 
+static std::atomic<uint32_t> g_wait_limit{kDefaultWaitLimit};
+
+uint32_t wait_limit() { return g_wait_limit.load(std::memory_order_relaxed); }
+
 }  // namespace svg
 
 extern "C" const char* svg_last_error(void) { return svg::g_last_error; }
+
+extern "C" svg_status svg_set_wait_limit(uint32_t polls) {
+  svg::clear_error();
+  svg::g_wait_limit.store(polls == 0 ? svg::kDefaultWaitLimit : polls, std::memory_order_relaxed);
+  return SVG_OK;
+}
+
+extern "C" uint32_t svg_get_wait_limit(void) { return svg::wait_limit(); }
 
 extern "C" const char* svg_version(void) { return "svg_b200 0.1 sm_100a"; }

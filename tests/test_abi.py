@@ -46,6 +46,17 @@ def test_version():
     assert L.svg_version().decode().startswith("svg_b200")
 
 
+def test_wait_limit_setting_round_trip():
+    default = L.svg_get_wait_limit()
+    assert default == 1 << 22
+    try:
+        assert L.svg_set_wait_limit(7) == _lib.SVG_OK
+        assert L.svg_get_wait_limit() == 7
+    finally:
+        assert L.svg_set_wait_limit(0) == _lib.SVG_OK  # 0 restores the default
+    assert L.svg_get_wait_limit() == default
+
+
 def test_workspace_sizes():
     assert L.svg_profile_workspace_size(1, 48, 17550, 64, 64) > 0
     assert L.svg_profile_workspace_size(1, 48, 17550, 64, 64) % 256 == 0

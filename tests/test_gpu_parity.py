@@ -250,6 +250,72 @@ def test_sparse_attn_empty_and_invalid_lists():
         assert_close(o[0, h], ref, f"head {h}")
 
 
+@pytest.mark.parametrize("name", ["wan480", "cogvideox", "tiny"])
+def test_sparse_attn_repeated_and_descending_entries(name):
+    """A row is a set of key blocks: an entry that repeats or falls below the
+    row's previous used entry is skipped and flagged (SVG_DEVICE_BAD_INDEX),
+    so no block is attended twice.  Checked against the oracle on the rows'
+    strictly ascending parts, for both members of a work item."""
+    wl = si.small(name)
+    (q, k, v), (qd, kd, vd), _ = workload_tensors(wl)
+    N, nb = wl.N, svg.n_tiles(wl.N)
+    rows = [[0, 0, 2], [2, 1, 2, nb - 1], [1, 1, 1], [nb - 1, 0]] + \
+        [[i, i] for i in range(4, nb)]
+    rows = rows[:nb]
+    ip = np.cumsum([0] + [len(r) for r in rows]).astype(np.int32)
+    ix = np.array([j for r in rows for j in r], dtype=np.int32)
+    lists = svg.BlockLists(torch.from_numpy(ip).to(DEV), torch.from_numpy(ix).to(DEV), 1, nb)
+    list_id = torch.zeros(wl.B * wl.H, dtype=torch.int32, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o = to_float64(svg.svg_sparse_attn(qd, kd, vd, list_id, lists, status=status))
+    assert status.item() & svg._lib.SVG_DEVICE_BAD_INDEX
+
+    def used(r):
+        out, last = [], -1
+        for j in r:
+            if 0 <= j < nb and j > last:
+                out.append(j)
+                last = j
+        return out
+    clean = [used(r) for r in rows]
+    if nb >= 4:
+        assert clean[:4] == [[0, 2], [2, nb - 1], [1], [nb - 1]]
+    okp = np.cumsum([0] + [len(r) for r in clean]).astype(np.int32)
+    okx = np.array([j for r in clean for j in r], dtype=np.int32)
+    for h in range(wl.H):
+        ref = O.block_sparse_attention(head64(q, 0, h), head64(k, 0, h), head64(v, 0, h), okp, okx)
+        assert_close(o[0, h], ref, f"{name} head {h}", bf16=wl.dtype == "bf16")
+
+
+@pytest.mark.parametrize("name", ["wan480", "cogvideox"])
+def test_wait_timeout_returns_and_context_survives(name):
+    """With the poll limit of the pipeline waits cut to one, a wait runs out
+    at once: the call returns, the device status word carries
+    SVG_DEVICE_TIMEOUT, and the next call (default limit) is again bit-exact
+    with the first, so the kernel drained its copies and MMAs, freed its
+    tensor memory and left the context usable.  No fault, no trap."""
+    wl = si.small(name)
+    (q, k, v), (qd, kd, vd), types = workload_tensors(wl)
+    lists = svg.geometric_lists(wl.F, wl.P, wl.width, wl.N)
+    list_id = torch.full((wl.B * wl.H,), O.MODE_DENSE, dtype=torch.int32, device=DEV)
+    ref = bits(svg.svg_sparse_attn(qd, kd, vd, list_id, lists))
+    lib = svg._lib.lib
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    try:
+        assert lib.svg_set_wait_limit(1) == svg._lib.SVG_OK
+        svg.svg_sparse_attn(qd, kd, vd, list_id, lists, status=status)
+        torch.cuda.synchronize()
+    finally:
+        lib.svg_set_wait_limit(0)
+    assert status.item() & svg._lib.SVG_DEVICE_TIMEOUT
+    assert lib.svg_get_wait_limit() == 1 << 22
+    status.zero_()
+    again = svg.svg_sparse_attn(qd, kd, vd, list_id, lists, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    np.testing.assert_array_equal(bits(again), ref)
+
+
 @pytest.mark.parametrize("N,d", [(100, 64), (128, 128), (129, 64), (383, 128)])
 def test_sparse_attn_ragged_dense(N, d):
     rng = np.random.default_rng(N + d)
@@ -570,7 +636,7 @@ def test_calibration_full_size_sampled():
     rng = np.random.default_rng(720)
     heads = sorted(rng.choice(wl.H, 4, replace=False).tolist())
     nb = svg.n_tiles(wl.N)
-    blocks = sorted(rng.choice(nb - 1, 3, replace=False).tolist()) + [nb - 1]  # + ragged tail
+    blocks = sorted(rng.choice(nb - 1, 5, replace=False).tolist()) + [nb - 1]  # + ragged tail
     types_seed = wl.calib_seeds[0]
     Es = []
     ref_E = {h: [] for h in heads}
@@ -592,16 +658,26 @@ def test_calibration_full_size_sampled():
     del E
     ip = lists.indptr.cpu().numpy().reshape(wl.H, nb + 1)
     ix = lists.indices.cpu().numpy()
+    R = len(wl.calib_seeds)
     compared = 0
     for h in heads:
+        # the builder at full size (1024-entry sorts, 23640 rows over many
+        # scan chunks) is bit-exact given the energies it was handed ...
+        Eg = [Eh[s, h][blocks].astype(np.float64) for s in range(R)]
+        gp, gx = O.calibrate_lists(Eg, wl.eps, wl.rho)
+        # ... and end to end it equals the float64 pipeline on every row whose
+        # per-input eps-cuts come out the same from the GPU's fp32 energies
+        # as from the oracle's (near-ties of 591 small energies can flip)
         op, ox = O.calibrate_lists(ref_E[h], wl.eps, wl.rho)
         for n, r in enumerate(blocks):
-            if min(cut_margin(ref_E[h][s][n], wl.eps) for s in range(len(wl.calib_seeds))) <= 1e-3:
-                continue
-            compared += 1
-            np.testing.assert_array_equal(ix[ip[h][r]:ip[h][r + 1]], ox[op[n]:op[n + 1]],
-                                          err_msg=f"head {h} block {r}")
-    assert compared >= len(heads)
+            got = ix[ip[h][r]:ip[h][r + 1]]
+            np.testing.assert_array_equal(got, gx[gp[n]:gp[n + 1]], err_msg=f"head {h} block {r}")
+            if all(O.minimal_energy_set(Eg[s][n], wl.eps) ==
+                   O.minimal_energy_set(ref_E[h][s][n], wl.eps) for s in range(R)):
+                compared += 1
+                np.testing.assert_array_equal(got, ox[op[n]:op[n + 1]],
+                                              err_msg=f"head {h} block {r}")
+    assert compared >= 1
     kept = (ip[:, -1] - ip[:, 0]).sum() / float(wl.H * nb * nb)
     assert 0.0 < kept < 1.0
     # attention on the timed input, every head on its own list
