@@ -284,6 +284,7 @@ def run_ours(args, rank, world, local_rank):
         side.wait_event(s0)
         for x, y in ((qd, bufs.qp), (kd, bufs.kp), (vd, bufs.vp)):
             svg.svg_permute_token_major(x, F, P, None, out=y, stream=side)
+        svg.svg_v_exponents(vd, out=bufs.vexp, stream=side)
         copied = torch.cuda.Event()
         copied.record(side)
         svg.svg_profile_heads(qd, kd, vd, F, P, w, idx_d, mse_out=bufs.mse, mode_out=bufs.mode,
@@ -293,7 +294,8 @@ def run_ours(args, rank, world, local_rank):
         a0.record(stream)
         svg.svg_sparse_attn_fused(qd, kd, vd, F, P, bufs.mode, lists,
                                   layout=svg._lib.SVG_FUSE_OUTPUT,
-                                  copies=(bufs.qp, bufs.kp, bufs.vp), out=bufs.o)
+                                  copies=(bufs.qp, bufs.kp, bufs.vp), out=bufs.o,
+                                  v_exp=bufs.vexp)
         s1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
@@ -480,8 +482,9 @@ def run_ours(args, rank, world, local_rank):
     prof_bytes = 2 * elems * 2      # K and V streamed once
     # q, k read once; q, k written frame-major and token-major; cos, sin once
     qk_bytes = 6 * elems * 2 + 2 * N * (d // 2) * 4
-    # profile partial, merge, finalize; 3 permutes; attention (output reordering fused)
-    launches_per_step = 3 + 3 + 1
+    # profile partial, merge, finalize; 3 permutes; V exponents (max, finalize);
+    # attention (output reordering fused)
+    launches_per_step = 3 + 3 + 2 + 1
     if sharded:
         parallelism = (f"heads of one layer split over {world} GPUs "
                        f"(contiguous ranges, rank 0 heads {heads.start}-{heads.stop - 1})")
@@ -626,11 +629,14 @@ def run_calibrated(args, rank, world, local_rank):
     qd, kd, vd = (h.to(dev) for h in host)
     o = torch.empty_like(qd)
     list_id = torch.arange(Hl, dtype=torch.int32, device=dev)
+    vexp = torch.empty(wl.B * Hl, dtype=torch.int32, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     K, W = args.steps, args.warmup
 
     def step():
-        svg.svg_sparse_attn(qd, kd, vd, list_id, lists, out=o)
+        # the per-head V exponents (one read of v), then every head on its list
+        svg.svg_v_exponents(vd, out=vexp)
+        svg.svg_sparse_attn(qd, kd, vd, list_id, lists, out=o, v_exp=vexp)
 
     for _ in range(W):
         step()
@@ -710,7 +716,7 @@ def run_calibrated(args, rank, world, local_rank):
         "tokens_per_s": round(tokens_s, 1),
         "pct_of_bf16_peak": round(100 * value / world / peak_tf, 2),
         "attention_only": {"ms": round(total_ms / K, 5), "effective_tflops": round(attn_tf, 3),
-                           "kernel": "svg_sparse_attn (list_id = h)"},
+                           "kernel": "svg_v_exponents + svg_sparse_attn (list_id = h)"},
         "calibration": {"energy_ms_per_input": round(energy_avg, 3),
                         "energy_tflops": round(energy_flops / (energy_avg * 1e-3) / 1e12, 1),
                         "build_lists_ms": round(build_ms, 3),
@@ -722,7 +728,7 @@ def run_calibrated(args, rank, world, local_rank):
         "e2e": {"value": round(e2e_value, 3), "unit": "TFLOPS",
                 "h2d_bytes_per_step": int(job_h2d), "d2h_bytes_per_step": int(job_d2h),
                 "ms_per_step": round(e2e_step_ms, 5)},
-        "gpu_launches": 1 * K,
+        "gpu_launches": 3 * K,   # V exponents (max, finalize), attention
         "clocks": clk,
     }
     if not args.no_cpu_baseline and world == 1:

@@ -85,7 +85,7 @@ typedef enum {
 #define SVG_DEVICE_BAD_INDEX 0x2     /* a key-block index outside [0, nB)   */
 #define SVG_DEVICE_TIMEOUT 0x4       /* a bounded pipeline wait gave up      */
 #define SVG_DEVICE_CAPACITY 0x8      /* a list did not fit the given buffer */
-#define SVG_DEVICE_RANGE 0x10        /* a bf16 V value is outside the fp16 range, inf or NaN */
+#define SVG_DEVICE_RANGE 0x10        /* a V value stayed outside the fp16 range (see 4a) */
 
 #define SVG_TILE 128
 
@@ -380,19 +380,38 @@ svg_status svg_lists_to_bitmap(int n_rows, int n_cols, const int32_t* indptr,
  *               SVG_DEVICE_BAD_INDEX; no key block is attended twice.
  *  scale        softmax scale; 0 selects 1/sqrt(d).
  *  device_status  optional device int32 (may be NULL), see SVG_DEVICE_*.
+ *  v_exp        optional device int32 [B*H] from svg_v_exponents (may be
+ *               NULL: every exponent 0).  Head (b, h) converts v * 2^-e to
+ *               fp16 and multiplies its output by 2^e, exactly (powers of
+ *               two), so any finite bf16 V gives the right result.
  * Arithmetic (bf16): Q.K^T on bf16 tensor cores with fp32 accumulation, fp32
  * online softmax; P.V on fp16 tensor cores (P in [0, 256] with an 11-bit
  * significand; V converted from bf16 to fp16 on chip, exact for
- * |v| <= 65504 -- a larger, infinite or NaN value in a visited key block
- * sets SVG_DEVICE_RANGE; larger values become inf) with
- * fp32 accumulation; output rounded to nearest bf16.  fp32 inputs use fp32
- * arithmetic throughout.
+ * |v| * 2^-e <= 65504) with fp32 accumulation; output rounded to nearest
+ * bf16.  A visited V value that stays beyond the fp16 range (no v_exp given,
+ * or an inf / NaN) becomes inf and sets SVG_DEVICE_RANGE.  fp32 inputs use
+ * fp32 arithmetic throughout and ignore v_exp.
  * ------------------------------------------------------------------------ */
 svg_status svg_sparse_attn(const void* q, const void* k, const void* v, void* o, int dtype,
                            int B, int H, int N, int d,
                            const int32_t* list_id, int n_lists, int n_qblocks,
                            const int32_t* indptr, const int32_t* indices,
-                           float scale, int32_t* device_status, void* stream);
+                           float scale, int32_t* device_status, const int32_t* v_exp,
+                           void* stream);
+
+/* --------------------------------------------------------------------------
+ * 4a. V exponents for the fp16 P.V product
+ *    The pages have no counterpart: it keeps the tensor-core arithmetic of
+ *    section 4 exact in range for every finite bf16 V.  For every (b, h):
+ *        exps[b*H + h] = the smallest e >= 0 with max |v[b,h]| * 2^-e <= 65504
+ *    (0 when the head already fits fp16; 255 when it holds inf or NaN).  One
+ *    read of v.  bf16 only.
+ *
+ *  v      device bf16 [B, H, N, d], 16-byte aligned.
+ *  exps   device int32 [B*H] (written; zeroed by this call first).
+ * ------------------------------------------------------------------------ */
+svg_status svg_v_exponents(const void* v, int dtype, int B, int H, int N, int d, int32_t* exps,
+                           void* stream);
 
 /* --------------------------------------------------------------------------
  * 4b. Block-sparse attention with the layout transformation fused in
@@ -442,7 +461,7 @@ svg_status svg_sparse_attn_fused(const void* q, const void* k, const void* v,
                                  int tokens_per_frame, const int32_t* mode, int layout,
                                  int n_lists, int n_qblocks, const int32_t* indptr,
                                  const int32_t* indices, const int32_t* tile_order, float scale,
-                                 int32_t* device_status, void* stream);
+                                 int32_t* device_status, const int32_t* v_exp, void* stream);
 
 /* --------------------------------------------------------------------------
  * 6. Spatial-repetition heads

@@ -37,6 +37,7 @@ __all__ = [
     "svg_permute_token_major",
     "svg_permute_frame_major", "svg_build_block_mask", "svg_block_energy",
     "svg_build_block_mask_calibrated", "svg_sparse_attn", "svg_sparse_attn_fused",
+    "svg_v_exponents",
     "svg_epsilon_schedule", "svg_lists_to_intervals", "svg_lists_to_bitmap", "geometric_lists",
     "QKTransform", "svg_qk_norm_rope", "svg_row_similarity", "svg_anchor_lists",
     "svg_anchor_list_ids", "svg_row_broadcast", "svg_repeat_attention", "svg_layer",
@@ -224,21 +225,32 @@ def svg_build_block_mask_calibrated(energy: torch.Tensor, eps: float, rho: float
 
 
 def svg_sparse_attn(q, k, v, list_id: torch.Tensor, lists: BlockLists, *, scale: float = 0.0,
-                    out=None, status=None, stream=None):
-    """Block-sparse attention over 128x128 tiles; returns o [B, H, N, d]."""
+                    v_exp=None, out=None, status=None, stream=None):
+    """Block-sparse attention over 128x128 tiles; returns o [B, H, N, d].
+    v_exp: optional int32 [B*H] from svg_v_exponents (V scaled into the fp16
+    range of the P.V product)."""
     B, H, N, d = _check_qkv(q, k, v)
     if out is None:
         out = torch.empty_like(q)
     _lib.call("svg_sparse_attn", q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), _dt(q),
               B, H, N, d, list_id.data_ptr(), lists.n_lists, lists.n_qblocks,
               lists.indptr.data_ptr(), lists.indices.data_ptr(), float(scale), _ptr(status),
-              _stream(stream))
+              _ptr(v_exp), _stream(stream))
+    return out
+
+
+def svg_v_exponents(v, *, out=None, stream=None):
+    """Per-head exponents e (int32 [B*H]) with max|v| * 2^-e <= 65504."""
+    B, H, N, d = _check_qkv(v)
+    if out is None:
+        out = torch.empty(B * H, dtype=torch.int32, device=v.device)
+    _lib.call("svg_v_exponents", v.data_ptr(), _dt(v), B, H, N, d, out.data_ptr(), _stream(stream))
     return out
 
 
 def svg_sparse_attn_fused(q, k, v, frames: int, tokens_per_frame: int, mode: torch.Tensor,
                           lists: BlockLists, *, layout: int = 3, copies=None, scale: float = 0.0,
-                          out=None, status=None, stream=None):
+                          v_exp=None, out=None, status=None, stream=None):
     """Block-sparse attention with the token-major reordering of temporal
     heads fused in: layout bit 1 (SVG_FUSE_INPUT) gathers q, k, v from
     frame-major memory, bit 2 (SVG_FUSE_OUTPUT) writes o frame-major.
@@ -252,7 +264,7 @@ def svg_sparse_attn_fused(q, k, v, frames: int, tokens_per_frame: int, mode: tor
               out.data_ptr(), _dt(q), B, H, N, d, frames, tokens_per_frame, mode.data_ptr(),
               int(layout), lists.n_lists, lists.n_qblocks, lists.indptr.data_ptr(),
               lists.indices.data_ptr(), _ptr(lists.tile_order), float(scale), _ptr(status),
-              _stream(stream))
+              _ptr(v_exp), _stream(stream))
     return out
 
 
@@ -442,6 +454,8 @@ class LayerBuffers:
         if not layout & _lib.SVG_FUSE_OUTPUT:  # token-major output
             self.op = torch.empty_like(q)
         self.o = torch.empty_like(q)
+        # per-head V exponents (svg_v_exponents) for the fp16 P.V product
+        self.vexp = torch.empty(B * H, dtype=torch.int32, device=dev)
         self.mse = torch.empty(B * H, 2, dtype=torch.float32, device=dev)
         self.mode = torch.empty(B * H, dtype=torch.int32, device=dev)
         self.ws = _scratch(_lib.lib.svg_profile_workspace_size(B, H, N, d, S), dev)
@@ -467,6 +481,8 @@ def svg_layer(q, k, v, frames: int, tokens_per_frame: int, spatial_width: int,
     svg_row_similarity > 0.87) with frame_shape = (rows, cols): those heads,
     unless profiled temporal, compute only the query tiles holding anchor
     rows and take the anchors' outputs on the other rows.
+    Every bf16 layer also computes the per-head V exponents
+    (svg_v_exponents), so any finite V stays exact in the fp16 P.V product.
     Returns (o, mode, mse)."""
     if bufs is None:
         bufs = LayerBuffers(q, sample_idx.numel(), layout, qk=qk is not None)
@@ -512,6 +528,8 @@ def svg_layer(q, k, v, frames: int, tokens_per_frame: int, spatial_width: int,
             ((q, bufs.qp), (k, bufs.kp), (v, bufs.vp))
         for x, y in side_work:
             svg_permute_token_major(x, F, P, None, out=y, stream=bufs.side)
+        if v.dtype == torch.bfloat16:
+            svg_v_exponents(v, out=bufs.vexp, stream=bufs.side)
         copied = torch.cuda.Event()
         copied.record(bufs.side)
         if qk is not None:
@@ -526,7 +544,8 @@ def svg_layer(q, k, v, frames: int, tokens_per_frame: int, spatial_width: int,
         out = bufs.o if layout & _lib.SVG_FUSE_OUTPUT else bufs.op
         use_lists, ids = select_lists(main)
         svg_sparse_attn_fused(q, k, v, F, P, ids, use_lists, layout=layout,
-                              copies=(bufs.qp, bufs.kp, bufs.vp), out=out, stream=main)
+                              copies=(bufs.qp, bufs.kp, bufs.vp), out=out, stream=main,
+                              v_exp=bufs.vexp if v.dtype == torch.bfloat16 else None)
         if not layout & _lib.SVG_FUSE_OUTPUT:
             svg_permute_frame_major(bufs.op, F, P, bufs.mode, out=bufs.o, stream=main)
         broadcast(ids, main)
@@ -543,12 +562,15 @@ def svg_layer(q, k, v, frames: int, tokens_per_frame: int, spatial_width: int,
             svg_permute_token_major(x, F, P, bufs.mode, out=y, stream=stream)
         ins = (bufs.qp, bufs.kp, bufs.vp)
     use_lists, ids = select_lists(stream)
+    vexp = None
+    if v.dtype == torch.bfloat16:
+        vexp = svg_v_exponents(v, out=bufs.vexp, stream=stream)
     if layout & _lib.SVG_FUSE_OUTPUT:
         svg_sparse_attn_fused(*ins, F, P, ids, use_lists, layout=layout, out=bufs.o,
-                              stream=stream)
+                              stream=stream, v_exp=vexp)
     else:
         svg_sparse_attn_fused(*ins, F, P, ids, use_lists, layout=layout, out=bufs.op,
-                              stream=stream)
+                              stream=stream, v_exp=vexp)
         svg_permute_frame_major(bufs.op, F, P, bufs.mode, out=bufs.o, stream=stream)
     broadcast(ids, stream)
     return bufs.o, bufs.mode, bufs.mse

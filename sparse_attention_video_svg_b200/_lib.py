@@ -47,12 +47,14 @@ SIGNATURES = {
     "svg_calibrated_workspace_size": (_sz, [_i, _i, _i]),
     "svg_build_block_mask_calibrated": (_i, [_p, _i, _i, _i, _i, _d, _d, _p, _p, _i64, _p, _p, _p,
                                              _sz, _p]),
-    "svg_sparse_attn": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _i, _p, _i, _i, _p, _p, _f, _p, _p]),
+    "svg_sparse_attn": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _i, _p, _i, _i, _p, _p, _f, _p, _p,
+                             _p]),
     "svg_epsilon_schedule": (_i, [_i, C.c_double, C.c_double, _p]),
     "svg_lists_to_intervals": (_i, [_i, _i, _p, _p, _p, _p, _p, C.c_int64, _p, _p, _p]),
     "svg_lists_to_bitmap": (_i, [_i, _i, _p, _p, _p, _p, _p]),
     "svg_sparse_attn_fused": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p,
-                                   _i, _i, _i, _p, _p, _p, _f, _p, _p]),
+                                   _i, _i, _i, _p, _p, _p, _f, _p, _p, _p]),
+    "svg_v_exponents": (_i, [_p, _i, _i, _i, _i, _i, _p, _p]),
     "svg_qk_norm_rope": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _p, _p, _f,
                               _p, _p, _p]),
     "svg_row_similarity_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),

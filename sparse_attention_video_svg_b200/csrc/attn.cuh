@@ -39,6 +39,10 @@ struct AttnArgs {
   // 0 .. n_qblocks-1 per list); null = index order.  Results never depend
   // on it.
   const int32_t* tile_order;
+  // Optional per-(b, h) V exponents from svg_v_exponents: the tcgen05 kernel
+  // converts v * 2^-e to fp16 and multiplies the head's output by 2^e (a
+  // value of 255 marks inf / NaN: converted unscaled).  Null: e = 0.
+  const int32_t* v_exp;
   // Polls of one mbarrier wait before the tcgen05 kernel gives up with
   // SVG_DEVICE_TIMEOUT (svg_set_wait_limit).
   uint32_t spin_limit;

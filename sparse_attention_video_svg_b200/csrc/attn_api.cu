@@ -13,7 +13,7 @@ svg_status sparse_attn_impl(const char* who, const void* q, const void* k, const
                             const int32_t* indices, float scale, int32_t* device_status,
                             const int32_t* order, int frames, int tokens_per_frame, int layout,
                             const void* q_tm, const void* k_tm, const void* v_tm,
-                            const int32_t* tile_order, void* stream) {
+                            const int32_t* tile_order, const int32_t* v_exp, void* stream) {
   clear_error();
   if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || list_id == nullptr ||
       indptr == nullptr || indices == nullptr)
@@ -52,7 +52,7 @@ svg_status sparse_attn_impl(const char* who, const void* q, const void* k, const
   if (!(scale >= 0.f) || isinf(scale)) return fail(SVG_ERR_INVALID_ARG, "%s: bad scale", who);
   AttnArgs a{q, k, v, o, dtype, B, H, N, d, list_id, n_lists, n_qblocks, indptr, indices,
              scale == 0.f ? 1.f / sqrtf(static_cast<float>(d)) : scale, device_status,
-             order, frames, tokens_per_frame, layout, q_tm, k_tm, v_tm, tile_order,
+             order, frames, tokens_per_frame, layout, q_tm, k_tm, v_tm, tile_order, v_exp,
              wait_limit()};
   cudaStream_t s = as_stream(stream);
   if (dtype == SVG_FP32) return d == 64 ? launch_attn_fp32<64>(a, s) : launch_attn_fp32<128>(a, s);
@@ -65,10 +65,11 @@ extern "C" svg_status svg_sparse_attn(const void* q, const void* k, const void* 
                                       int dtype, int B, int H, int N, int d,
                                       const int32_t* list_id, int n_lists, int n_qblocks,
                                       const int32_t* indptr, const int32_t* indices, float scale,
-                                      int32_t* device_status, void* stream) {
+                                      int32_t* device_status, const int32_t* v_exp,
+                                      void* stream) {
   return sparse_attn_impl("sparse_attn", q, k, v, o, dtype, B, H, N, d, list_id, n_lists,
                           n_qblocks, indptr, indices, scale, device_status, nullptr, 0, 0, 0,
-                          nullptr, nullptr, nullptr, nullptr, stream);
+                          nullptr, nullptr, nullptr, nullptr, v_exp, stream);
 }
 
 extern "C" svg_status svg_sparse_attn_fused(const void* q, const void* k, const void* v,
@@ -78,8 +79,9 @@ extern "C" svg_status svg_sparse_attn_fused(const void* q, const void* k, const 
                                             const int32_t* mode, int layout, int n_lists,
                                             int n_qblocks, const int32_t* indptr,
                                             const int32_t* indices, const int32_t* tile_order,
-                                            float scale, int32_t* device_status, void* stream) {
+                                            float scale, int32_t* device_status,
+                                            const int32_t* v_exp, void* stream) {
   return sparse_attn_impl("sparse_attn_fused", q, k, v, o, dtype, B, H, N, d, mode, n_lists,
                           n_qblocks, indptr, indices, scale, device_status, mode, frames,
-                          tokens_per_frame, layout, q_tm, k_tm, v_tm, tile_order, stream);
+                          tokens_per_frame, layout, q_tm, k_tm, v_tm, tile_order, v_exp, stream);
 }

@@ -131,6 +131,17 @@ __device__ __forceinline__ bool valid_tile(int j, int nb) { return j >= 0 && j <
 // of the item, bits 4-5 the last; bit 6 marks the end (no tile loaded).
 constexpr uint32_t kStepEnd = 1u << 6;
 constexpr uint32_t kStepGathered = 1u << 7;  // Q / K / V of this step came through cp.async
+// bits 8-15: the head's V exponent e (v * 2^-e is converted; 0 = unscaled)
+constexpr int kStepExpShift = 8;
+
+// The V exponent the kernel applies to head bh: svg_v_exponents' value when
+// it is a usable scale (1 .. 126), else 0 (no exponents given, a head that
+// already fits fp16, or 255 for inf / NaN, which no scale fixes).
+__device__ __forceinline__ uint32_t v_exponent(const AttnArgs& a, int bh) {
+  if (a.v_exp == nullptr) return 0;
+  const int e = a.v_exp[bh];
+  return (e > 0 && e < 127) ? static_cast<uint32_t>(e) : 0u;
+}
 
 // Entries [beg, end) of `indices` for query tile qt of head bh; empty for a
 // tile past the end or a bad list.
@@ -352,7 +363,10 @@ __device__ __forceinline__ void softmax_member(const AttnArgs& a, const Bars& B,
     if (!empty) {
       if (!(ok = wait_bar<SW>(&B.o_done[t], (g - 1) & 1, abort_flag, a.status))) break;
       tc_fence_after();
+      // 1 / l, times 2^e for a head whose V was converted as v * 2^-e
       inv = l > 0.f ? 1.f / l : 0.f;
+      const uint32_t e = v_exponent(a, bh);
+      if (e) inv *= __uint_as_float((127u + e) << 23);
     }
     const int n = qt * 128 + row;
     // token-major heads over frame-major memory write row n back to its frame-major place
@@ -475,6 +489,7 @@ __device__ __forceinline__ void producer(const AttnArgs& a, const Maps& maps, co
     const int bh = item / n_pairs, qt0 = 2 * (item - bh * n_pairs);
     const bool tm = gathers_input(a, bh);
     const bool cp = reads_copies(a, bh);
+    const uint32_t vexp = v_exponent(a, bh);
     const CUtensorMap* mq = cp ? &maps.qt : &maps.q;
     const CUtensorMap* mk = cp ? &maps.kt : &maps.k;
     const CUtensorMap* mv = cp ? &maps.vt : &maps.v;
@@ -511,7 +526,8 @@ __device__ __forceinline__ void producer(const AttnArgs& a, const Maps& maps, co
       const uint32_t m = static_cast<uint32_t>(mask);
       const uint32_t last = (m & 1u) * (p[0] >= e[0] ? 1u : 0u) |
                             (m & 2u) * (p[1] >= e[1] ? 1u : 0u);
-      const uint32_t info = m | ((m & ~seen) << 2) | (last << 4) | (tm ? kStepGathered : 0u);
+      const uint32_t info = m | ((m & ~seen) << 2) | (last << 4) | (tm ? kStepGathered : 0u) |
+                            (vexp << kStepExpShift);
       seen |= m;
       for (int kv = 0; kv < 2; ++kv) {
         if (!(ok = claim_step(kv))) break;
@@ -563,8 +579,8 @@ __device__ __forceinline__ void producer(const AttnArgs& a, const Maps& maps, co
 // pending P.V, member 1's Q K^T.  The tensor core runs its instructions in
 // issue order, so member 1's scores land one P.V + Q K^T after member 0's and
 // the two softmax warpgroups take turns on the exponential unit instead of
-// sharing it.  Otherwise each member has an issuer thread of its own.  The
-// thread serves members t0 .. t1.
+// sharing it.  (Without kOneIssuer each member has an issuer thread of its
+// own, issuer_member.)  The thread serves members t0 .. t1.
 template <int D, int t0, int t1, bool SW>
 __device__ __forceinline__ void issuer(const Bars& B, unsigned char* smem,
                                        volatile uint32_t* step_info, volatile int* abort_flag,
@@ -660,6 +676,87 @@ __device__ __forceinline__ void issuer(const Bars& B, unsigned char* smem,
   drain_bar(&B.drain[t0], 0);
 }
 
+// MMA issuer of one member (two-issuer mode): the same steps as `issuer`
+// for member t alone.  One copy of this code serves both issuer warps (t is a
+// runtime value), which keeps the kernel's instruction footprint small.
+template <int D, bool SW>
+__device__ __forceinline__ void issuer_member(const Bars& B, unsigned char* smem,
+                                              volatile uint32_t* step_info,
+                                              volatile int* abort_flag, uint32_t tmem,
+                                              int32_t* status, int t) {
+  using C = Cfg<D>;
+  constexpr int QD = C::kQDepth, S = C::kSlots;
+  const uint32_t t_s = tmem + C::kColS + 128 * t;
+  const uint32_t t_p = tmem + C::kColP + C::kPStride * t;
+  const uint32_t t_o = tmem + C::kColO + C::kOStride * t;
+  // descriptors of the member's first Q buffer and of ring entry 0; a buffer
+  // at byte offset x adds x >> 4 (the start-address field)
+  const uint64_t dq = sdesc_sw128(smem_u32(smem + C::kOffQ + t * QD * C::kTile), 16, 1024);
+  const uint64_t dk = sdesc_sw128(smem_u32(smem + C::kOffKV), 16, 1024);
+  const uint64_t dv = sdesc_sw128(smem_u32(smem + C::kOffKV), kBox, 1024);
+  uint32_t L = 0, cq = 0, nq = 0, np = 0, pend_lv = 0;
+  bool ok = true, pend = false, pend_first = false;
+  auto issue_pv = [&]() -> bool {
+    if (!wait_bar<SW>(&B.p_ready[t], np & 1, abort_flag, status)) return false;
+    const uint32_t slot = pend_lv % S;
+    if (!wait_bar<SW>(&B.v_ready[slot], (pend_lv / S) & 1, abort_flag, status)) return false;
+    tc_fence_after();
+    mma_ts_k128(t_o, t_p, dv + ((slot * C::kTile) >> 4), C::kIdescPV, pend_first ? 0u : 1u);
+    tc_commit(&B.o_done[t]);
+    tc_commit(&B.kv_empty[slot]);
+    ++np;
+    pend = false;
+    return true;
+  };
+  while (ok) {
+    const uint32_t kslot = L % S;
+    if (!(ok = wait_bar<SW>(&B.kv_full[kslot], (L / S) & 1, abort_flag, status))) break;
+    const uint32_t info = step_info[(L / 2) % C::kInfo];
+    if (info & kStepGathered) fence_proxy_async_smem();
+    if (info & kStepEnd) break;
+    if (!(info >> t & 1u)) {  // skipped block: as in `issuer`
+      if (pend && !(ok = issue_pv())) break;
+      tc_commit(&B.kv_empty[kslot]);
+      tc_commit(&B.kv_empty[kslot + 1]);
+      L += 2;
+      continue;
+    }
+    if constexpr (!C::kSepP) {
+      if (pend && !(ok = issue_pv())) break;
+    } else if (nq > 0) {
+      if (!(ok = wait_bar<SW>(&B.s_free[t], (nq - 1) & 1, abort_flag, status))) break;
+    }
+    const uint32_t qs = cq % QD;
+    if (info >> (2 + t) & 1u) {
+      if (!(ok = wait_bar<SW>(&B.q_full[t * QD + qs], (cq / QD) & 1, abort_flag, status))) break;
+      if (info & kStepGathered) fence_proxy_async_smem();
+    }
+    tc_fence_after();
+    const uint64_t q0 = dq + ((qs * C::kTile) >> 4), k0 = dk + ((kslot * C::kTile) >> 4);
+    if constexpr (D == 64)
+      mma_ss_k64(t_s, q0, k0, C::kIdescQK);
+    else
+      mma_ss_k128(t_s, q0, k0, C::kIdescQK, kBox >> 4);
+    tc_commit(&B.s_full[t]);
+    tc_commit(&B.kv_empty[kslot]);
+    if (info >> (4 + t) & 1u) {
+      tc_commit(&B.q_empty[t * QD + qs]);
+      ++cq;
+    }
+    ++nq;
+    if constexpr (C::kSepP) {
+      if (pend && !(ok = issue_pv())) break;
+    }
+    pend = true;
+    pend_first = (info >> (2 + t)) & 1u;
+    pend_lv = L + 1;
+    L += 2;
+  }
+  if (ok && pend) ok = issue_pv();
+  tc_commit(&B.drain[t]);
+  drain_bar(&B.drain[t], 0);
+}
+
 // Converts every V tile in place from bf16 to fp16, in ring order; `part` of
 // C::kConvWarps warps (each takes every kConvWarps-th 16-byte piece, and
 // each arrives once on the tile's v_ready).  bf16 -> fp16 is exact for
@@ -680,20 +777,39 @@ __device__ __forceinline__ void converter(const AttnArgs& a, const Bars& B, unsi
   while (ok) {
     const uint32_t slot = (L + 1) % S;
     if (!(ok = wait_bar<SW>(&B.kv_full[slot], ((L + 1) / S) & 1, abort_flag, a.status))) break;
-    if (step_info[(L / 2) % C::kInfo] & kStepEnd) break;
+    const uint32_t info = step_info[(L / 2) % C::kInfo];
+    if (info & kStepEnd) break;
     uint4* tile = reinterpret_cast<uint4*>(smem + C::kOffKV + slot * C::kTile);
+    const uint32_t e = (info >> kStepExpShift) & 0xffu;
+    if (e == 0) {
 #pragma unroll 4
-    for (int c = part * 32 + lane; c < C::kTile / 16; c += 32 * C::kConvWarps) {
-      uint4 v = tile[c];
-      uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+      for (int c = part * 32 + lane; c < C::kTile / 16; c += 32 * C::kConvWarps) {
+        uint4 v = tile[c];
+        uint32_t* w = reinterpret_cast<uint32_t*>(&v);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xffff0000u);
-        over |= (w[i] & 0x7fff7fffu) + 0x38803880u;
-        const __half2 h = __floats2half2_rn(lo, hi);
-        w[i] = *reinterpret_cast<const uint32_t*>(&h);
+        for (int i = 0; i < 4; ++i) {
+          const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xffff0000u);
+          over |= (w[i] & 0x7fff7fffu) + 0x38803880u;
+          const __half2 h = __floats2half2_rn(lo, hi);
+          w[i] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+        tile[c] = v;
       }
-      tile[c] = v;
+    } else {
+      // v * 2^-e (exact), which the head's exponent brings into fp16 range
+      const float sc = __uint_as_float((127u - e) << 23);
+#pragma unroll 4
+      for (int c = part * 32 + lane; c < C::kTile / 16; c += 32 * C::kConvWarps) {
+        uint4 v = tile[c];
+        uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const __half2 h = __floats2half2_rn(__uint_as_float(w[i] << 16) * sc,
+                                              __uint_as_float(w[i] & 0xffff0000u) * sc);
+          w[i] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+        tile[c] = v;
+      }
     }
     fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
     __syncwarp();
@@ -782,14 +898,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     reg_dealloc<C::kRegsLow>();
     // ------------------------------------------------------------ MMA issuers
     if (lane == 0) {
-      if constexpr (C::kOneIssuer) {
+      if constexpr (C::kOneIssuer)
         issuer<D, 0, 1, SW>(B, smem, step_info, abort_flag, tmem, a.status);
-      } else {
-        if (warp == 1)
-          issuer<D, 0, 0, SW>(B, smem, step_info, abort_flag, tmem, a.status);
-        else
-          issuer<D, 1, 1, SW>(B, smem, step_info, abort_flag, tmem, a.status);
-      }
+      else
+        issuer_member<D, SW>(B, smem, step_info, abort_flag, tmem, a.status, warp - 1);
     }
   } else if (warp <= 3) {
     reg_dealloc<C::kRegsLow>();

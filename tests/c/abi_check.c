@@ -39,7 +39,7 @@ int main(void) {
 
   /* d = 96 is not supported: rejected before launch, with a message */
   svg_status st = svg_sparse_attn(fake, fake, fake, fake2, SVG_BF16, 1, 2, 256, 96, fake, 3, 2,
-                                  fake, fake, 0.f, NULL, NULL);
+                                  fake, fake, 0.f, NULL, NULL, NULL);
   CHECK(st == SVG_ERR_INVALID_ARG && strstr(svg_last_error(), "d=96") != NULL, "d=96 rejected");
   /* a successful host-only call clears the error text */
   CHECK(svg_epsilon_schedule(1, 0.9, 0.9, eps) == SVG_OK && svg_last_error()[0] == '\0',

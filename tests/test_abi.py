@@ -79,7 +79,7 @@ INVALID = _lib.SVG_ERR_INVALID_ARG
 class TestHostValidation:
     def test_sparse_attn(self):
         base = [FAKE, FAKE2, FAKE3, FAKE4 * 4, 0, 1, 2, 256, 64, FAKE, 3, 2, FAKE, FAKE, 0.0, None,
-                None]
+                None, None]
         expect(_lib.SVG_OK if False else INVALID, "svg_sparse_attn",
                *(base[:8] + [96] + base[9:]), match="d=96")
         expect(INVALID, "svg_sparse_attn", *(base[:11] + [3] + base[12:]), match="n_qblocks")
@@ -91,9 +91,9 @@ class TestHostValidation:
 
     def test_sparse_attn_fused(self):
         # q k v q_tm k_tm v_tm o dtype B H N d F P mode layout n_lists n_qblocks indptr
-        # indices tile_order scale status stream
+        # indices tile_order scale status v_exp stream
         base = [FAKE, FAKE2, FAKE3, None, None, None, FAKE4 * 4, 0, 1, 2, 256, 64, 4, 64, FAKE,
-                3, 3, 2, FAKE, FAKE, None, 0.0, None, None]
+                3, 3, 2, FAKE, FAKE, None, 0.0, None, None, None]
         expect(INVALID, "svg_sparse_attn_fused", *(base[:12] + [5] + base[13:]), match="frames")
         expect(INVALID, "svg_sparse_attn_fused", *(base[:11] + [96] + base[12:]), match="d=96")
         expect(INVALID, "svg_sparse_attn_fused", *(base[:14] + [None] + base[15:]), match="null")

@@ -463,6 +463,75 @@ def test_sparse_attn_v_range_flag(value, flagged):
         assert (err <= bound).all(), f"v = {value}: worst excess {(err - bound).max():.4g}"
 
 
+def _v_exponents_ref(vbits):
+    """Oracle-free reference of svg_v_exponents from the bf16 bits: the
+    smallest e >= 0 with max|v| * 2^-e <= 65504 (255 for inf / NaN)."""
+    B, H = vbits.shape[:2]
+    out = np.zeros(B * H, np.int64)
+    for b in range(B):
+        for h in range(H):
+            m = int((vbits[b, h].astype(np.uint32) & 0x7fff).max())
+            if m >= 0x7f80:
+                out[b * H + h] = 255
+                continue
+            mx = float(si.bf16_bits_to_f32(np.array([m], np.uint16))[0])
+            e = 0
+            while mx * 2.0 ** -e > 65504.0:
+                e += 1
+            out[b * H + h] = e
+    return out
+
+
+@pytest.mark.parametrize("name", ["wan480", "cogvideox"])
+def test_v_exponents_scale_v_into_fp16_range(name):
+    """V beyond the fp16 range gives the correct output when the call takes
+    svg_v_exponents' per-head exponents: head 0 holds one outlier (checked
+    against the oracle), head 1 is the whole head times 2^20 (its output is
+    exactly 2^20 times the unscaled head's, bit for bit), head 2 an inf
+    (exponent 255, flagged), head 3 is untouched (exponent 0, bits equal to
+    the call without exponents)."""
+    wl = si.small(name)
+    (q, k, v), (qd, kd, vd), _ = workload_tensors(wl)
+    lists = svg.geometric_lists(wl.F, wl.P, wl.width, wl.N)
+    dense = torch.full((wl.B * wl.H,), O.MODE_DENSE, dtype=torch.int32, device=DEV)
+    plain = svg.svg_sparse_attn(qd, kd, vd, dense, lists)
+    v2 = vd.clone()
+    v2[0, 0, 7, 3] = 3.0e5
+    v2[0, 1] = vd[0, 1] * 2.0 ** 20
+    v2[0, 2, 9, 1] = float("inf")
+    vbits = v2.view(torch.int16).cpu().numpy().view(np.uint16)
+    exps = svg.svg_v_exponents(v2)
+    np.testing.assert_array_equal(exps.cpu().numpy(), _v_exponents_ref(vbits))
+    assert exps[0].item() > 0 and exps[1].item() > 0 and exps[2].item() == 255
+    assert exps[3].item() == 0
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o = svg.svg_sparse_attn(qd, kd, v2, dense, lists, v_exp=exps, status=status)
+    torch.cuda.synchronize()
+    assert status.item() & svg._lib.SVG_DEVICE_RANGE  # head 2's inf
+    # head 0: the outlier, against the oracle (as in the range-flag test)
+    vh = head64(v, 0, 0)
+    vh[7, 3] = float(v2[0, 0, 7, 3].item())
+    ip, ix = O.geometric_block_lists(O.MODE_DENSE, wl.F, wl.P, wl.width, wl.N)
+    want = O.block_sparse_rows(head64(q, 0, 0), head64(k, 0, 0), vh, np.arange(wl.N), ip, ix)
+    got = to_float64(o[0, 0])
+    bound = np.maximum(MAX_ABS, half_ulp_bf16(want) + 1e-3 + 2.0 ** -11 * np.abs(want))
+    assert (np.abs(got - want) <= bound).all()
+    # head 1: 2^20 times the unscaled head (the scaled head converts v * 2^12
+    # to fp16, exact, so the products only move by a power of two; a value
+    # below the fp16 normal range may keep more bits there than unscaled,
+    # hence one bf16 ulp of slack)
+    g1, w1 = to_float64(o[0, 1]), to_float64(plain[0, 1]) * 2.0 ** 20
+    assert (np.abs(g1 - w1) <= 2 * half_ulp_bf16(w1)).all()
+    assert (g1 == w1).mean() > 0.999
+    # head 3: the same bits as without exponents
+    np.testing.assert_array_equal(bits(o[0, 3]), bits(plain[0, 3]))
+    # without exponents head 1 overflows fp16: flagged
+    status.zero_()
+    svg.svg_sparse_attn(qd, kd, v2, dense, lists, status=status)
+    torch.cuda.synchronize()
+    assert status.item() & svg._lib.SVG_DEVICE_RANGE
+
+
 # ---------------------------------------------------------------- the layer
 
 @pytest.mark.parametrize("wl", SMALL, ids=lambda w: w.name)
