@@ -43,8 +43,6 @@
 #include <cudaTypedefs.h>
 #include <limits.h>
 
-#include <mutex>
-
 #include "attn.cuh"
 #include "common.cuh"
 #include "sm100.cuh"
@@ -319,7 +317,9 @@ __device__ __forceinline__ void softmax_member(const AttnArgs& a, const Bars& B,
           p1 = fast_exp2(t1);
           const __half2 h = __floats2half2_rn(p0, p1);
           ph[c][i] = *reinterpret_cast<const uint32_t*>(&h);
-          // the row sum uses the fp16-rounded weights the MMA sees
+          // the row sum uses the fp16-rounded weights the MMA sees (an fp32
+          // sum of the unrounded weights is faster, but leaves the output off
+          // by up to ~2e-4 of |o|, beyond the bf16 tolerance at |o| >= 8)
           add_f16x2_to_f32(lx, ly, ph[c][i]);
         }
       }
@@ -906,7 +906,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp <= 3) {
     reg_dealloc<C::kRegsLow>();
     // ------------------------------------------------------------ V to fp16
-    converter<D, SW>(a, B, smem, step_info, abort_flag, warp - (4 - C::kConvWarps));
+    // (the converter warps are the last kConvWarps of warpgroup 0)
+    if (warp >= 4 - C::kConvWarps)
+      converter<D, SW>(a, B, smem, step_info, abort_flag, warp - (4 - C::kConvWarps));
   } else {
     reg_alloc<C::kRegsHigh>();
     softmax_member<D, SW>(a, B, abort_flag, tmem, n_items, n_pairs, nb);
@@ -919,36 +921,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ------------------------------------------------------------ host side
 
-PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
-// [B*H][N][d] bf16 viewed as a 3-D tensor (d, N, B*H); box 64 x 128 x 1,
-// 128-byte swizzle.  Rows beyond N are zero-filled on load.
-bool make_map(CUtensorMap* m, const void* base, int BH, int N, int d) {
-  auto enc = get_encode();
-  if (enc == nullptr) return false;
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
-                        static_cast<cuuint64_t>(BH)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
-  cuuint32_t box[3] = {64, 128, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-         CUDA_SUCCESS;
-}
-
 }  // namespace
 
 template <int D>
@@ -956,11 +928,11 @@ svg_status launch_attn_sm100(const AttnArgs& a, cudaStream_t s) {
   using C = Cfg<D>;
   Maps maps = {};
   const int BH = a.B * a.H;
-  if (!make_map(&maps.q, a.q, BH, a.N, D) || !make_map(&maps.k, a.k, BH, a.N, D) ||
-      !make_map(&maps.v, a.v, BH, a.N, D) ||
-      (a.q_tm != nullptr &&
-       (!make_map(&maps.qt, a.q_tm, BH, a.N, D) || !make_map(&maps.kt, a.k_tm, BH, a.N, D) ||
-        !make_map(&maps.vt, a.v_tm, BH, a.N, D))))
+  if (!make_tma_map_3d(&maps.q, a.q, BH, a.N, D) || !make_tma_map_3d(&maps.k, a.k, BH, a.N, D) ||
+      !make_tma_map_3d(&maps.v, a.v, BH, a.N, D) ||
+      (a.q_tm != nullptr && (!make_tma_map_3d(&maps.qt, a.q_tm, BH, a.N, D) ||
+                             !make_tma_map_3d(&maps.kt, a.k_tm, BH, a.N, D) ||
+                             !make_tma_map_3d(&maps.vt, a.v_tm, BH, a.N, D))))
     return fail(SVG_ERR_CUDA, "sparse_attn: cannot encode TMA descriptors");
   // a launch with a poll limit other than the default runs the instantiation
   // that reads it (the same code otherwise)

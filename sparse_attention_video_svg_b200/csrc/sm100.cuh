@@ -9,6 +9,11 @@
 #include "common.cuh"
 
 namespace svg {
+
+// Host: TMA map of a [BH][N][d] bf16 tensor viewed as (d, N, BH), box
+// 64 x 128 x 1 with 128-byte swizzle; rows past N are zero-filled on load.
+bool make_tma_map_3d(CUtensorMap* m, const void* base, int BH, int N, int d);
+
 namespace sm100 {
 
 // ------------------------------------------------------------------ mbarrier
@@ -47,18 +52,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // the phase also needs its regular arrivals).
 __device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
   asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];\n" ::"r"(smem_u32(bar)) : "memory");
-}
-
-// Non-blocking test of an mbarrier phase.
-__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-      " selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
 }
 
 // ------------------------------------------------------------------ TMA
