@@ -8,16 +8,16 @@
 // the squared difference; an exact tie keeps SPATIAL.
 //
 // Work split (one layer, all heads, one launch each):
-//   partial  grid (chunks, B*H): the keys of a head are cut into `chunks`
-//            contiguous ranges.  A CTA of 4 warps streams one range through
-//            a cp.async ring (4 stages of 64 keys at d = 64, 3 at d = 128);
-//            each warp owns 16 of the 64 sampled rows and keeps two
-//            online-softmax states (max, sum, o) for them: dense and under
-//            the spatial mask (each row's band of frames is one contiguous
-//            key range, tested with two compares; the spatial update is
-//            skipped for stages outside the warp's bands).  Both updates
-//            share one Q K^T per stage.  bf16: mma.sync tensor-core products;
-//            fp32: SIMT (one launch per mask, grid z).
+//   partial  the keys of a head are cut into `chunks` contiguous ranges (a
+//            multiple of 128 keys each); a unit is one (range, head).  bf16:
+//            a persistent tcgen05 kernel, one CTA per SM looping over units,
+//            the 64 sampled rows as one M = 128 tile, K and V streamed by TMA
+//            through rings of their own, S = Q K^T and both P.V products on
+//            the tensor core with TMEM accumulators, and two online-softmax
+//            states per row (dense, and under the spatial mask: each row's
+//            band of frames is one contiguous key range, tested with two
+//            compares) sharing one Q K^T per tile.  fp32: SIMT, one launch
+//            per mask (grid z).
 //   merge    grid (B*H, 16), one warp per sampled row: the chunk weights
 //            exp2(m_c - M) / L, the merged dense and spatial outputs, the
 //            temporal output (a row sees only the F keys of its position,
@@ -28,14 +28,13 @@
 #include <float.h>
 
 #include "common.cuh"
-#include "mma_frag.cuh"
+#include "sm100.cuh"
 
 namespace svg {
 namespace {
 
 constexpr int kRows = 64;          // sampled rows per head (S padded to 64)
-constexpr int kKeys = 64;          // keys per shared-memory stage
-constexpr int kThreads = 128;      // bf16 partial: 4 warps, 16 rows each
+constexpr int kTileKeys = 128;     // keys per tile of the tcgen05 path; ranges are multiples
 constexpr int kTargetCtas = 888;   // partial-grid size the chunking aims for (6 x 148)
 constexpr int kMaxChunks = 32;     // merge holds one chunk weight per lane
 constexpr float kLog2e = 1.4426950408889634f;
@@ -45,16 +44,16 @@ __device__ __forceinline__ int clamp_index(int n, int N) { return n < 0 ? 0 : (n
 
 struct ProfileShape {
   int chunks;     // key ranges per head
-  int chunk_len;  // keys per range (multiple of kKeys)
+  int chunk_len;  // keys per range (multiple of kTileKeys)
 };
 
 ProfileShape shape_for(int N, long long chunks) {
-  const long long max_chunks = (N + 4 * kKeys - 1) / (4 * kKeys);  // >= 4 stages per range
+  const long long max_chunks = (N + 4 * kTileKeys - 1) / (4 * kTileKeys);  // >= 4 tiles per range
   if (chunks > max_chunks) chunks = max_chunks;
   if (chunks > kMaxChunks) chunks = kMaxChunks;
   if (chunks < 1) chunks = 1;
   long long len = (N + chunks - 1) / chunks;
-  len = (len + kKeys - 1) / kKeys * kKeys;
+  len = (len + kTileKeys - 1) / kTileKeys * kTileKeys;
   chunks = (N + len - 1) / len;
   return {static_cast<int>(chunks), static_cast<int>(len)};
 }
@@ -83,190 +82,6 @@ size_t errors_bytes(int B, int H) {
 size_t partial_bytes(int B, int H, int N, int d) {
   ProfileShape ps = profile_shape(B, H, N);
   return states_bytes(B, H, ps.chunks, d) + errors_bytes(B, H);
-}
-
-// --------------------------------------------------------------- bf16 partial
-
-template <int D>
-constexpr int stages_for() {
-  return D == 64 ? 4 : 3;  // cp.async ring depth (shared memory: 3 or 2 CTAs per SM)
-}
-template <int D>
-constexpr size_t partial_smem() {
-  return static_cast<size_t>(kRows) * D * 2 + 2 * static_cast<size_t>(stages_for<D>()) * kKeys * D * 2;
-}
-
-// One stage's online-softmax update of a warp's 16 rows: s holds the scores
-// (scale * log2 e applied below), keys outside [lo[h], hi[h]) are masked for
-// the thread's row h; P is rounded to bf16 and the row sum adds the rounded
-// values.
-template <int D>
-__device__ __forceinline__ void stage_update(float (&m)[2], float (&l)[2], float (&o)[D / 8][4],
-                                             float (&s)[kKeys / 8][4], const int (&lo)[2],
-                                             const int (&hi)[2], int key0, float scale_log2,
-                                             uint32_t vtile) {
-  const int t4 = threadIdx.x & 3;
-  float mx[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-  for (int n = 0; n < kKeys / 8; ++n)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int key = key0 + 8 * n + 2 * t4 + (e & 1);
-      const int h = e >> 1;
-      s[n][e] = (key >= lo[h] && key < hi[h]) ? s[n][e] * scale_log2 : -INFINITY;
-      mx[h] = fmaxf(mx[h], s[n][e]);
-    }
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
-    mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
-    const float mn = fmaxf(m[h], mx[h]);
-    const float base = mn == -INFINITY ? 0.f : mn;
-    const float alpha = fast_exp2(m[h] - base);  // exp2(-inf) = 0 on the first update
-    m[h] = mn;
-    l[h] *= alpha;
-#pragma unroll
-    for (int n = 0; n < D / 8; ++n) {
-      o[n][2 * h] *= alpha;
-      o[n][2 * h + 1] *= alpha;
-    }
-#pragma unroll
-    for (int n = 0; n < kKeys / 8; ++n) {
-      s[n][2 * h] = round_bf16(fast_exp2(s[n][2 * h] - base));
-      s[n][2 * h + 1] = round_bf16(fast_exp2(s[n][2 * h + 1] - base));
-      l[h] += s[n][2 * h] + s[n][2 * h + 1];
-    }
-  }
-  pv_frags<D, kKeys>(o, s, vtile, 0);
-}
-
-template <int D>
-__device__ __forceinline__ void store_state(float* base, int row0, const float (&m)[2],
-                                            float (&l)[2], const float (&o)[D / 8][4]) {
-  const int lane = threadIdx.x & 31, g = lane >> 2, t4 = lane & 3;
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    l[h] += __shfl_xor_sync(0xffffffffu, l[h], 1);
-    l[h] += __shfl_xor_sync(0xffffffffu, l[h], 2);
-  }
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    float* row = base + (row0 + g + 8 * h) * state_floats<D>();
-    if (t4 == 0) {
-      row[0] = m[h];
-      row[1] = l[h];
-    }
-#pragma unroll
-    for (int n = 0; n < D / 8; ++n) {
-      row[2 + 8 * n + 2 * t4] = o[n][2 * h];
-      row[2 + 8 * n + 2 * t4 + 1] = o[n][2 * h + 1];
-    }
-  }
-}
-
-template <int D>
-__global__ void __launch_bounds__(kThreads, D == 64 ? 3 : 2) profile_partial_bf16(
-    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-    const __nv_bfloat16* __restrict__ v, const int32_t* __restrict__ idx, int S, int N, int P,
-    int width, float scale_log2, int chunks, int chunk_len, float* __restrict__ ws) {
-  constexpr int ST = stages_for<D>();
-  constexpr int TILE = kKeys * D * 2;  // bytes of one K or V stage
-  extern __shared__ __align__(128) unsigned char smem[];
-  unsigned char* sQ = smem;
-  unsigned char* sK = smem + kRows * D * 2;
-  unsigned char* sV = sK + ST * TILE;
-
-  const int chunk = blockIdx.x, bh = blockIdx.y;
-  const long long head = static_cast<long long>(bh) * N * D;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row0 = warp * 16;
-  const int g = lane >> 2;
-  const int key_begin = chunk * chunk_len;
-  const int key_end = min(N, key_begin + chunk_len);
-  const int n_stages = (key_end - key_begin + kKeys - 1) / kKeys;
-
-  // gather the sampled query rows (padding rows are zero)
-  for (int t = threadIdx.x; t < kRows * (D / 8); t += kThreads) {
-    const int r = t / (D / 8), c = t % (D / 8);
-    const bool ok = r < S;
-    const int n = ok ? clamp_index(idx[r], N) : 0;
-    cp_async16(sQ + swz(r, c, 2 * D), q + head + static_cast<long long>(n) * D + c * 8, ok);
-  }
-  // the keys each of this thread's two rows may see, clipped to the chunk:
-  // every key of the chunk (dense) and the row's band of frames (spatial)
-  int dlo[2], dhi[2], slo[2], shi[2];
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int r = row0 + g + 8 * h;
-    dlo[h] = slo[h] = key_begin;
-    dhi[h] = shi[h] = key_end;
-    if (r >= S) {
-      dhi[h] = shi[h] = key_begin;  // padding row: no keys
-    } else {
-      const int f = clamp_index(idx[r], N) / P;
-      slo[h] = max(key_begin, max(0, f - width) * P);
-      shi[h] = min(key_end, static_cast<int>(min(static_cast<long long>(N),
-                                                 static_cast<long long>(f + width + 1) * P)));
-    }
-  }
-  int wlo = min(slo[0], slo[1]), whi = max(shi[0], shi[1]);
-#pragma unroll
-  for (int o2 = 4; o2 < 32; o2 <<= 1) {
-    wlo = min(wlo, __shfl_xor_sync(0xffffffffu, wlo, o2));
-    whi = max(whi, __shfl_xor_sync(0xffffffffu, whi, o2));
-  }
-
-#pragma unroll
-  for (int st = 0; st < ST - 1; ++st) {
-    if (st < n_stages) {
-      load_tile_async<D, kKeys, kThreads>(sK + st * TILE, k + head, key_begin + st * kKeys, key_end);
-      load_tile_async<D, kKeys, kThreads>(sV + st * TILE, v + head, key_begin + st * kKeys, key_end);
-    }
-    cp_async_commit();
-  }
-
-  float md[2] = {-INFINITY, -INFINITY}, ld[2] = {0.f, 0.f};
-  float ms[2] = {-INFINITY, -INFINITY}, ls[2] = {0.f, 0.f};
-  float od[D / 8][4], os[D / 8][4];
-#pragma unroll
-  for (int n = 0; n < D / 8; ++n)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) od[n][e] = os[n][e] = 0.f;
-  uint32_t qa[D / 16][4];
-
-  for (int st = 0; st < n_stages; ++st) {
-    cp_async_wait<ST - 2>();
-    __syncthreads();  // stage st landed; the buffer refilled below is free
-    {
-      const int ns = st + ST - 1;
-      if (ns < n_stages) {
-        const int b = ns % ST;
-        load_tile_async<D, kKeys, kThreads>(sK + b * TILE, k + head, key_begin + ns * kKeys, key_end);
-        load_tile_async<D, kKeys, kThreads>(sV + b * TILE, v + head, key_begin + ns * kKeys, key_end);
-      }
-      cp_async_commit();
-    }
-    if (st == 0) load_a_frags<D>(qa, smem_u32(sQ), row0);
-    const int key0 = key_begin + st * kKeys;
-    const int b = st % ST;
-    float s[kKeys / 8][4];
-    qk_frags<D, kKeys>(s, qa, smem_u32(sK + b * TILE), 0);
-    if (key0 < whi && key0 + kKeys > wlo) {  // some row of this warp has band keys here
-      float sp[kKeys / 8][4];
-#pragma unroll
-      for (int n = 0; n < kKeys / 8; ++n)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) sp[n][e] = s[n][e];
-      stage_update<D>(ms, ls, os, sp, slo, shi, key0, scale_log2, smem_u32(sV + b * TILE));
-    }
-    stage_update<D>(md, ld, od, s, dlo, dhi, key0, scale_log2, smem_u32(sV + b * TILE));
-  }
-
-  // per-row partial states -> workspace [bh][variant][chunk][row][m, l, o[D]]
-  const long long stride = static_cast<long long>(chunks) * kRows * state_floats<D>();
-  float* base = ws + (static_cast<long long>(bh) * 2 * chunks + chunk) * kRows * state_floats<D>();
-  store_state<D>(base, row0, md, ld, od);
-  store_state<D>(base + stride, row0, ms, ls, os);
 }
 
 // --------------------------------------------------------------- fp32 partial
@@ -323,6 +138,533 @@ __global__ void __launch_bounds__(256) profile_partial_fp32(
 #pragma unroll
     for (int e = 0; e < E; ++e) row[2 + lane + 32 * e] = acc[e];
   }
+}
+
+// --------------------------------------------------------------- tcgen05 partial (bf16)
+//
+// Persistent, one CTA per SM, looping over work units (key range c, head bh).
+// The 64 sampled rows fill rows 0-63 of a 128-row M tile (rows 64-127 are
+// zero and never read back).  Seven warps:
+//   warps 0, 4  softmax of rows 0-31, warps 1, 5 of rows 32-63 (TMEM lanes
+//               0-63 belong to warps 0 and 1 modulo 4); of the two warps of a
+//               row group, one takes key columns 0-63 of every tile and the
+//               other 64-127, and their row maxima and sums meet in shared
+//               memory (an mbarrier per row group, bounded waits).  Per 128-key tile: the dense and the spatial
+//               online-softmax states of the row, with lazy rescaling (an
+//               output is rescaled only when its running max grows by more
+//               than 2^8);
+//   warp 2      K loader: gathers the unit's sampled Q rows (cp.async, into
+//               the 128-byte-swizzled K-major layout), then streams the K
+//               tiles of the range through a ring (TMA);
+//   warp 6      V loader: the V tiles through a ring of their own, so that a
+//               K entry is refilled as soon as its Q K^T is done while a V
+//               entry waits for its P.V;
+//   warp 3      MMA issuer (one thread): S_j = Q K_j^T into one of two TMEM
+//               score buffers, then O_d += P_d,j-1 V_j-1 and O_s += P_s,j-1
+//               V_j-1 with both P from TMEM (bf16, written over the scores
+//               they came from) and V from shared memory.
+// The scores of tile j are computed while the softmax works on tile j-1.
+// Every wait is bounded; a CTA that gives up writes NaN into the states of
+// its unit (so the head's errors come out NaN) and drains.
+
+constexpr int kTcThreads = 224;
+
+template <int D>
+struct TcCfg {
+  static constexpr int kTile = 128 * D * 2;         // a 128-row Q / K / V tile
+  static constexpr int kBox = 16384;                // 128 rows x 128 bytes
+  static constexpr int kBoxes = D / 64;
+  static constexpr int kStages = D == 64 ? 6 : 3;   // K ring and V ring entries each
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kTile;               // [stage]
+  static constexpr int kOffV = kOffK + kStages * kTile;
+  static constexpr int kOffBar = kOffV + kStages * kTile;
+  // q_full, q_empty, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2],
+  // p_ready[2], o_done, drain, xchg[2]
+  static constexpr int kBars = 2 + 4 * kStages + 2 + 2 + 2 + 2;
+  static constexpr int kOffX = kOffBar + kBars * 8 + 16;  // float [2][2][32][2] exchange
+  static constexpr int kSmem = kOffX + 1024 + 1024;  // + the base's 1024-byte alignment
+  static constexpr uint32_t kColS = 0;               // S_b at 128 b; P_d in its columns 0-63, P_s 64-127
+  static constexpr uint32_t kColOd = 256;
+  static constexpr uint32_t kColOs = 256 + D;
+  static constexpr uint32_t kIdescQK = sm100::idesc_bf16(128, 128, false);
+  static constexpr uint32_t kIdescPV = sm100::idesc_bf16(128, D, true);
+  static_assert(kSmem <= 227 * 1024, "shared memory budget");
+};
+
+constexpr uint32_t kTcSpin = 1u << 22;
+constexpr uint32_t kTcDrain = 1u << 20;
+
+__device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  const uint32_t addr = smem_u32(bar);
+  for (uint32_t i = 0; i < kTcSpin; ++i) {
+    if (sm100::mbar_try_wait(addr, parity)) return true;
+    if ((i & 255u) == 255u && *abort_flag) return false;
+  }
+  *abort_flag = 1;
+  return false;
+}
+// The same wait taken by a whole warp: every lane leaves with the same answer,
+// so a timeout cannot split the warp across the warp-wide instructions after it.
+__device__ __forceinline__ bool tc_wait_warp(uint64_t* bar, uint32_t parity,
+                                             volatile int* abort_flag) {
+  return __all_sync(0xffffffffu, tc_wait(bar, parity, abort_flag)) != 0;
+}
+__device__ __forceinline__ void tc_drain(uint64_t* bar, uint32_t parity) {
+  const uint32_t addr = smem_u32(bar);
+  for (uint32_t i = 0; i < kTcDrain; ++i)
+    if (sm100::mbar_try_wait(addr, parity)) return;
+}
+
+struct TcUnit {
+  int bh, chunk, key_begin, key_end, tiles;
+};
+__device__ __forceinline__ TcUnit tc_unit(int u, int chunks, int chunk_len, int N) {
+  TcUnit w;
+  w.bh = u / chunks;
+  w.chunk = u - w.bh * chunks;
+  w.key_begin = w.chunk * chunk_len;
+  w.key_end = min(N, w.key_begin + chunk_len);
+  w.tiles = w.key_end > w.key_begin ? (w.key_end - w.key_begin + kTileKeys - 1) / kTileKeys : 0;
+  return w;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kTcThreads, 1) profile_partial_tc(
+    const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
+    const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ idx, int S, int N, int P,
+    int width, float scale_log2, int chunks, int chunk_len, int n_units,
+    float* __restrict__ ws) {
+  using C = TcCfg<D>;
+  using namespace sm100;
+  constexpr int ST = C::kStages;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* q_full = bars;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* k_full = bars + 2;
+  uint64_t* k_empty = k_full + ST;
+  uint64_t* v_full = k_empty + ST;
+  uint64_t* v_empty = v_full + ST;
+  uint64_t* s_full = v_empty + ST;
+  uint64_t* p_ready = s_full + 2;
+  uint64_t* o_done = p_ready + 2;
+  uint64_t* drain = o_done + 1;
+  uint64_t* xchg = drain + 1;  // [2]: the two softmax warps of a row group meet here
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xchg + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // rows 64-127 of the Q tile stay zero
+  for (int i = threadIdx.x; i < C::kTile / 16; i += kTcThreads) {
+    const int box = i / (C::kBox / 16), row = (i % (C::kBox / 16)) / 8;
+    if (row >= kRows) reinterpret_cast<uint4*>(smem + C::kOffQ)[box * (C::kBox / 16) + (i % (C::kBox / 16))] = make_uint4(0, 0, 0, 0);
+  }
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int i = 0; i < ST; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&p_ready[b], 4);
+    }
+    mbar_init(o_done, 1);
+    mbar_init(drain, 1);
+    mbar_init(&xchg[0], 2);
+    mbar_init(&xchg[1], 2);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 3) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  fence_proxy_async_smem();  // the zeroed rows, for the tensor core
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 2) {
+    // ------------------------------------------------------------------ loader
+    if (lane == 0) {
+      prefetch_tmap(&mk);
+      prefetch_tmap(&mv);
+    }
+    constexpr int CH = D / 8;  // 16-byte chunks per row
+    uint32_t gt = 0, nu = 0;  // tiles and units loaded
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const TcUnit w = tc_unit(u, chunks, chunk_len, N);
+      if (w.tiles == 0) continue;
+      int r_ok = 1;
+      if (lane == 0) r_ok = tc_wait(q_empty, (nu & 1) ^ 1, abort_flag) ? 1 : 0;
+      if (!(ok = __shfl_sync(0xffffffffu, r_ok, 0) != 0)) break;
+      ++nu;
+      const __nv_bfloat16* qh = q + static_cast<long long>(w.bh) * N * D;
+      for (int t = lane; t < kRows * CH; t += 32) {
+        const int r = t / CH, c = t % CH;
+        const bool valid = r < S;
+        const int n = valid ? clamp_index(idx[r], N) : 0;
+        cp_async16(smem + C::kOffQ + (c >> 3) * C::kBox + r * 128 + (((c & 7) ^ (r & 7)) << 4),
+                   qh + static_cast<long long>(n) * D + c * 8, valid);
+      }
+      cp_async_mbar_arrive(q_full);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(q_full);
+      for (int j = 0; j < w.tiles; ++j) {
+        const uint32_t st = gt % ST;
+        int r_ok = 1;  // lane 0 waits and copies; the warp learns the outcome
+        if (lane == 0) {
+          if (tc_wait(&k_empty[st], ((gt / ST) & 1) ^ 1, abort_flag)) {
+            mbar_arrive_expect_tx(&k_full[st], C::kTile);
+            const int key0 = w.key_begin + j * kTileKeys;
+            for (int bx = 0; bx < C::kBoxes; ++bx)
+              tma_load_3d(smem + C::kOffK + st * C::kTile + bx * C::kBox, &mk, &k_full[st],
+                          64 * bx, key0, w.bh);
+          } else {
+            r_ok = 0;
+          }
+        }
+        if (!(ok = __shfl_sync(0xffffffffu, r_ok, 0) != 0)) break;
+        ++gt;
+      }
+    }
+    cp_async_wait<0>();
+    if (!ok && lane == 0) {  // copies in flight land before the CTA can exit
+      for (uint32_t l = gt > ST ? gt - ST : 0; l < gt; ++l) tc_drain(&k_full[l % ST], (l / ST) & 1);
+      if (nu > 0) tc_drain(q_full, (nu - 1) & 1);
+    }
+  } else if (warp == 6) {
+    // ------------------------------------------------------------------ V loader
+    if (lane == 0) {
+      uint32_t gt = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        const TcUnit w = tc_unit(u, chunks, chunk_len, N);
+        for (int j = 0; j < w.tiles; ++j) {
+          const uint32_t st = gt % ST;
+          if (!(ok = tc_wait(&v_empty[st], ((gt / ST) & 1) ^ 1, abort_flag))) break;
+          mbar_arrive_expect_tx(&v_full[st], C::kTile);
+          for (int bx = 0; bx < C::kBoxes; ++bx)
+            tma_load_3d(smem + C::kOffV + st * C::kTile + bx * C::kBox, &mv, &v_full[st], 64 * bx,
+                        w.key_begin + j * kTileKeys, w.bh);
+          ++gt;
+        }
+      }
+      if (!ok)  // copies in flight land before the CTA can exit
+        for (uint32_t l = gt > ST ? gt - ST : 0; l < gt; ++l) tc_drain(&v_full[l % ST], (l / ST) & 1);
+    }
+  } else if (warp == 3) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint64_t dq = sdesc_sw128(smem_u32(smem + C::kOffQ), 16, 1024);
+      const uint64_t dk = sdesc_sw128(smem_u32(smem + C::kOffK), 16, 1024);
+      const uint64_t dv = sdesc_sw128(smem_u32(smem + C::kOffV), C::kBox, 1024);
+      uint32_t gt = 0, nu = 0;
+      bool ok = true;
+      auto issue_pv = [&](uint32_t g, bool first) -> bool {
+        const uint32_t b = g & 1, st = g % ST;
+        if (!tc_wait(&p_ready[b], (g >> 1) & 1, abort_flag)) return false;
+        if (!tc_wait(&v_full[st], (g / ST) & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint64_t v0 = dv + ((st * C::kTile) >> 4);
+        const uint32_t sb = tmem + C::kColS + 128 * b;
+        mma_ts_k128(tmem + C::kColOd, sb, v0, C::kIdescPV, first ? 0u : 1u);
+        mma_ts_k128(tmem + C::kColOs, sb + 64, v0, C::kIdescPV, first ? 0u : 1u);
+        tc_commit(o_done);
+        tc_commit(&v_empty[st]);
+        return true;
+      };
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        const TcUnit w = tc_unit(u, chunks, chunk_len, N);
+        if (w.tiles == 0) continue;
+        if (!(ok = tc_wait(q_full, nu & 1, abort_flag))) break;
+        fence_proxy_async_smem();  // Q came through cp.async (generic proxy)
+        tc_fence_after();
+        for (int j = 0; j < w.tiles; ++j, ++gt) {
+          const uint32_t st = gt % ST, b = gt & 1;
+          if (!(ok = tc_wait(&k_full[st], (gt / ST) & 1, abort_flag))) break;
+          tc_fence_after();
+          const uint64_t k0 = dk + ((st * C::kTile) >> 4);
+          if constexpr (D == 64)
+            mma_ss_k64(tmem + C::kColS + 128 * b, dq, k0, C::kIdescQK);
+          else
+            mma_ss_k128(tmem + C::kColS + 128 * b, dq, k0, C::kIdescQK, C::kBox >> 4);
+          tc_commit(&s_full[b]);
+          tc_commit(&k_empty[st]);
+          if (j == w.tiles - 1) tc_commit(q_empty);  // the unit's last Q K^T
+          if (j > 0 && !(ok = issue_pv(gt - 1, j == 1))) break;
+        }
+        if (!ok) break;
+        if (!(ok = issue_pv(gt - 1, w.tiles == 1))) break;
+        ++nu;
+      }
+      tc_commit(drain);  // every MMA completes before TMEM is released
+      tc_drain(drain, 0);
+    }
+  } else if (warp == 0 || warp == 1 || warp == 4 || warp == 5) {
+    // ------------------------------------------------------------------ softmax
+    // Two warps per row group: warp q (q = 0, 1) and warp q + 4 share TMEM
+    // lanes 32 q .. 32 q + 31 (rows) and take key columns 0-63 and 64-127 of
+    // every tile; their row maxima meet in shared memory.
+    const int quarter = warp & 3, half = warp >> 2;
+    const int r = quarter * 32 + lane;  // sampled row = TMEM lane
+    uint64_t* xb_bar = &xchg[quarter];
+    uint32_t xph = 0;  // exchange phases completed
+    // both warps of the row group reach this point (bounded wait)
+    auto meet = [&]() -> bool {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(xb_bar);
+      const bool met = tc_wait_warp(xb_bar, xph & 1, abort_flag);
+      ++xph;
+      return met;
+    };
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    // this warp's half of each output (for rescaling and the epilogue)
+    const uint32_t t_od = tmem + lane_off + C::kColOd + half * (D / 2);
+    const uint32_t t_os = tmem + lane_off + C::kColOs + half * (D / 2);
+    // [quarter][half][lane][2]: the two warps' partial maxima / sums
+    volatile float* xb = reinterpret_cast<volatile float*>(smem + C::kOffX);
+    volatile float* mine = xb + ((quarter * 2 + half) * 32 + lane) * 2;
+    volatile float* other = xb + ((quarter * 2 + (half ^ 1)) * 32 + lane) * 2;
+    uint32_t gt = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const TcUnit w = tc_unit(u, chunks, chunk_len, N);
+      if (w.tiles == 0) continue;
+      // this row's keys in the range: all of them (dense), its band of frames (spatial)
+      int dhi = w.key_end, slo = w.key_begin, shi = w.key_begin;
+      if (r < S) {
+        const int f = clamp_index(idx[r], N) / P;
+        slo = max(w.key_begin, max(0, f - width) * P);
+        shi = static_cast<int>(min(static_cast<long long>(w.key_end),
+                                   static_cast<long long>(f + width + 1) * P));
+      } else {
+        dhi = w.key_begin;
+      }
+      float md = -INFINITY, ms = -INFINITY;
+      float ld0 = 0.f, ld1 = 0.f, ls0 = 0.f, ls1 = 0.f;  // this half's row sums
+      for (int j = 0; j < w.tiles; ++j, ++gt) {
+        const uint32_t b = gt & 1;
+        const uint32_t t_s = tmem + lane_off + C::kColS + 128 * b;
+        if (!(ok = tc_wait_warp(&s_full[b], (gt >> 1) & 1, abort_flag))) break;
+        tc_fence_after();
+        float s[64];
+        {
+          uint32_t rr[2][32];
+          tmem_ld32(t_s + 64 * half, rr[0]);
+          tmem_ld32(t_s + 64 * half + 32, rr[1]);
+          tmem_wait_ld();
+          reg_fence32(rr[0]);
+          reg_fence32(rr[1]);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            s[i] = __uint_as_float(rr[0][i]) * scale_log2;
+            s[32 + i] = __uint_as_float(rr[1][i]) * scale_log2;
+          }
+        }
+        // this half's columns of the tile: keys c0 .. c0 + 63
+        const int c0 = w.key_begin + j * kTileKeys + 64 * half;
+        const int nd = max(0, min(64, dhi - c0));                        // dense [0, nd)
+        const int s0 = max(0, slo - c0), s1 = max(s0, min(64, shi - c0));  // band [s0, s1)
+        const bool dfull = nd == 64, sfull = s0 == 0 && s1 == 64, sempty = s1 <= s0;
+        float mxd, mxs;
+        if (dfull) {
+          float m4[4] = {s[0], s[1], s[2], s[3]};
+#pragma unroll
+          for (int i = 4; i < 60; i += 8)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) m4[c] = sm100::max3(m4[c], s[i + c], s[i + 4 + c]);
+          mxd = sm100::max3(sm100::max3(m4[0], s[60], s[61]), sm100::max3(m4[1], s[62], s[63]),
+                            fmaxf(m4[2], m4[3]));
+        } else {
+          mxd = -INFINITY;
+#pragma unroll
+          for (int i = 0; i < 64; ++i) mxd = i < nd ? fmaxf(mxd, s[i]) : mxd;
+        }
+        if (sfull && dfull) {
+          mxs = mxd;
+        } else if (sempty) {
+          mxs = -INFINITY;
+        } else {
+          mxs = -INFINITY;
+#pragma unroll
+          for (int i = 0; i < 64; ++i) mxs = (i >= s0 && i < s1) ? fmaxf(mxs, s[i]) : mxs;
+        }
+        mine[0] = mxd;
+        mine[1] = mxs;
+        if (!(ok = meet())) break;
+        mxd = fmaxf(mxd, other[0]);
+        mxs = fmaxf(mxs, other[1]);
+        if (!(ok = meet())) break;  // the buffer may be written again
+        // lazy rescaling: a running max moves only when it grows by more than
+        // 2^8 (both warps of the row group decide alike)
+        float ad = 1.f, as = 1.f;
+        bool rd = false, rs = false;
+        if (mxd > md + 8.f) {
+          if (md != -INFINITY) {
+            ad = exp2f(md - mxd);
+            rd = true;
+          }
+          md = mxd;
+        }
+        if (mxs > ms + 8.f) {
+          if (ms != -INFINITY) {
+            as = exp2f(ms - mxs);
+            rs = true;
+          }
+          ms = mxs;
+        }
+        ld0 *= ad;
+        ld1 *= ad;
+        ls0 *= as;
+        ls1 *= as;
+        // the outputs may be rescaled once the previous tile's P.V finished
+        // (these scores imply the P.V two tiles back did, so the barrier is
+        // at most one phase ahead of this wait); each warp its half
+        if (__any_sync(0xffffffffu, rd || rs)) {
+          if (!(ok = tc_wait_warp(o_done, (gt - 1) & 1, abort_flag))) break;
+          tc_fence_after();
+          uint32_t rr[32];
+#pragma unroll
+          for (int ch = 0; ch < D / 64; ++ch) {
+            tmem_ld32(t_od + 32 * ch, rr);
+            tmem_wait_ld();
+            reg_fence32(rr);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * ad);
+            tmem_st32(t_od + 32 * ch, rr);
+            tmem_ld32(t_os + 32 * ch, rr);
+            tmem_wait_ld();
+            reg_fence32(rr);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * as);
+            tmem_st32(t_os + 32 * ch, rr);
+          }
+        }
+        // weights as bf16 pairs: P_d over the scores' columns 0-63, P_s over
+        // 64-127 (the scores are in registers); the row sums add the rounded
+        // weights the tensor core sees
+        uint32_t pd[2][16];
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int k = 32 * c + 2 * i;
+            float d0, d1;
+            if (dfull) {
+              d0 = fast_exp2(s[k] - md);
+              d1 = fast_exp2(s[k + 1] - md);
+            } else {
+              d0 = k < nd ? fast_exp2(s[k] - md) : 0.f;
+              d1 = k + 1 < nd ? fast_exp2(s[k + 1] - md) : 0.f;
+            }
+            pd[c][i] = pack_bf16x2(d0, d1);
+            ld0 += __uint_as_float(pd[c][i] << 16);
+            ld1 += __uint_as_float(pd[c][i] & 0xffff0000u);
+          }
+        // (tcgen05.st and wait::st are warp-wide: the lanes meet before each,
+        // and the row-dependent choice below only selects register values)
+        __syncwarp();
+        tmem_st16(t_s + 32 * half, pd[0]);
+        tmem_st16(t_s + 32 * half + 16, pd[1]);
+        tmem_wait_st();  // pd's registers are free again
+        if (!(sfull && dfull && ms == md)) {
+          // (otherwise the whole half is in the band and both states share
+          // their max: the spatial weights are the dense ones)
+#pragma unroll
+          for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int k = 32 * c + 2 * i;
+              float e0 = 0.f, e1 = 0.f;
+              if (!sempty) {
+                e0 = (k >= s0 && k < s1) ? fast_exp2(s[k] - ms) : 0.f;
+                e1 = (k + 1 >= s0 && k + 1 < s1) ? fast_exp2(s[k + 1] - ms) : 0.f;
+              }
+              pd[c][i] = pack_bf16x2(e0, e1);
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            ls0 += __uint_as_float(pd[c][i] << 16);
+            ls1 += __uint_as_float(pd[c][i] & 0xffff0000u);
+          }
+        __syncwarp();
+        tmem_st16(t_s + 64 + 32 * half, pd[0]);
+        tmem_st16(t_s + 64 + 32 * half + 16, pd[1]);
+        tmem_wait_st();
+        // before the unit's last weights are released, the P.V before them
+        // has finished: o_done then stands at most one phase past what the
+        // epilogue waits for (two would alias its parity)
+        if (j == w.tiles - 1 && gt > 0 && !(ok = tc_wait_warp(o_done, (gt - 1) & 1, abort_flag))) break;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_ready[b]);
+      }
+      if (!ok) break;
+      // the unit's states: [bh][variant][chunk][row][m, l, o[D]].  o_done
+      // completes one phase per tile's P.V; the one before the last has
+      // finished, so a single wait finds the last.
+      mine[0] = ld0 + ld1;
+      mine[1] = ls0 + ls1;
+      if (!(ok = meet())) break;
+      const float ld = ld0 + ld1 + other[0], ls = ls0 + ls1 + other[1];
+      if (!(ok = meet())) break;
+      if (!(ok = tc_wait_warp(o_done, (gt - 1) & 1, abort_flag))) break;
+      tc_fence_after();
+      const long long vstride = static_cast<long long>(chunks) * kRows * state_floats<D>();
+      float* rd_ = ws + (static_cast<long long>(w.bh) * 2 * chunks + w.chunk) * kRows * state_floats<D>() +
+                   static_cast<long long>(r) * state_floats<D>();
+      float* rs_ = rd_ + vstride;
+      if (half == 0) {
+        rd_[0] = md;
+        rd_[1] = ld;
+        rs_[0] = ms;
+        rs_[1] = ls;
+      }
+      uint32_t rr[32];
+#pragma unroll
+      for (int ch = 0; ch < D / 64; ++ch) {
+        const int col = half * (D / 2) + 32 * ch;
+        tmem_ld32(t_od + 32 * ch, rr);
+        tmem_wait_ld();
+        reg_fence32(rr);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) rd_[2 + col + i] = __uint_as_float(rr[i]);
+        tmem_ld32(t_os + 32 * ch, rr);
+        tmem_wait_ld();
+        reg_fence32(rr);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) rs_[2 + col + i] = __uint_as_float(rr[i]);
+      }
+      // (the next unit's first P.V overwrites O only after this warp's next
+      // p_ready, which follows these reads in program order)
+    }
+    if (!ok) {
+      // a wait gave up: this CTA's results are not to be trusted
+      for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+        const TcUnit w = tc_unit(u, chunks, chunk_len, N);
+        float* rd_ = ws + (static_cast<long long>(w.bh) * 2 * chunks + w.chunk) * kRows * state_floats<D>() +
+                     static_cast<long long>(r) * state_floats<D>();
+        rd_[0] = __int_as_float(0x7fc00000);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 3) tmem_dealloc(tmem, 512);
 }
 
 // --------------------------------------------------------------- combine
@@ -485,14 +827,18 @@ svg_status launch_profile_shaped(const void* q, const void* k, const void* v, in
   const float scale_log2 = kLog2e / sqrtf(static_cast<float>(D));
   float* errs = ws + states_bytes(B, H, ps.chunks, D) / sizeof(float);
   if (dtype == SVG_BF16) {
-    const size_t smem = partial_smem<D>();
-    if (cudaFuncSetAttribute(profile_partial_bf16<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
+    using C = TcCfg<D>;
+    CUtensorMap mk, mv;
+    if (!make_tma_map_3d(&mk, k, B * H, N, D) || !make_tma_map_3d(&mv, v, B * H, N, D))
+      return fail(SVG_ERR_CUDA, "%s: cannot encode TMA descriptors", who);
+    if (cudaFuncSetAttribute(profile_partial_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kSmem) != cudaSuccess)
       return fail(SVG_ERR_CUDA, "%s: cannot reserve shared memory", who);
-    profile_partial_bf16<D><<<dim3(ps.chunks, B * H), kThreads, smem, s>>>(
-        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-        static_cast<const __nv_bfloat16*>(v), idx, S, N, P, width, scale_log2, ps.chunks,
-        ps.chunk_len, ws);
+    const int units = ps.chunks * B * H;
+    const int grid = units < sm_count() ? units : sm_count();
+    profile_partial_tc<D><<<grid, kTcThreads, C::kSmem, s>>>(
+        mk, mv, static_cast<const __nv_bfloat16*>(q), idx, S, N, P, width, scale_log2, ps.chunks,
+        ps.chunk_len, units, ws);
     if (svg_status st = check_launch(who)) return st;
     profile_merge<D, __nv_bfloat16><<<dim3(B * H, kRows / kMergeRows), 32 * kMergeRows, 0, s>>>(
         static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
