@@ -202,6 +202,18 @@ svg_status svg_permute_frame_major(const void* x, void* y, int dtype,
                                    int frames, int tokens_per_frame,
                                    const int32_t* mode, void* stream);
 
+/*  svg_permute_temporal_heads: the token-major reordering of
+ *  svg_permute_token_major for the heads whose mode is SVG_MODE_TEMPORAL
+ *  only; every other head of y is left as it is (not written).  This is the
+ *  copy svg_sparse_attn_fused reads for temporal heads (q_tm, k_tm, v_tm),
+ *  made after profiling at the cost of the temporal heads alone.  mode is
+ *  required (NULL: SVG_ERR_INVALID_ARG); other arguments and errors as for
+ *  svg_permute_token_major.  Bit-exact. */
+svg_status svg_permute_temporal_heads(const void* x, void* y, int dtype,
+                                      int B, int H, int N, int d,
+                                      int frames, int tokens_per_frame,
+                                      const int32_t* mode, void* stream);
+
 /* --------------------------------------------------------------------------
  * 2b. QK-Norm + RoPE of q and k, with optional token-major copies
  *    [SVG] section "Layout Transformation + Kernel 加速": next to the

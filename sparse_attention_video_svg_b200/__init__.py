@@ -34,7 +34,7 @@ from ._lib import (SVG_BF16, SVG_FP32, SVG_MODE_DENSE, SVG_MODE_SPATIAL, SVG_MOD
 __all__ = [
     "SVG_MODE_SPATIAL", "SVG_MODE_TEMPORAL", "SVG_MODE_DENSE", "SVG_TILE", "SvgError",
     "BlockLists", "svg_version", "svg_profile_heads", "svg_profile_heads_noalloc",
-    "svg_permute_token_major",
+    "svg_permute_token_major", "svg_permute_temporal_heads",
     "svg_permute_frame_major", "svg_build_block_mask", "svg_block_energy",
     "svg_build_block_mask_calibrated", "svg_sparse_attn", "svg_sparse_attn_fused",
     "svg_v_exponents",
@@ -151,6 +151,15 @@ def svg_permute_token_major(x, frames: int, tokens_per_frame: int, mode=None, ou
                             stream=None):
     """y[b,h,s*F+f] = x[b,h,f*P+s] for TEMPORAL heads (all heads if mode is None)."""
     return _permute("svg_permute_token_major", x, frames, tokens_per_frame, mode, out, stream)
+
+
+def svg_permute_temporal_heads(x, frames: int, tokens_per_frame: int, mode, out=None,
+                               stream=None):
+    """svg_permute_token_major for TEMPORAL heads only; the other heads of
+    `out` are not written (the copy the fused attention reads)."""
+    if mode is None:
+        raise ValueError("svg_permute_temporal_heads needs the modes")
+    return _permute("svg_permute_temporal_heads", x, frames, tokens_per_frame, mode, out, stream)
 
 
 def svg_permute_frame_major(x, frames: int, tokens_per_frame: int, mode=None, out=None,
@@ -472,11 +481,14 @@ def svg_layer(q, k, v, frames: int, tokens_per_frame: int, spatial_width: int,
     (svg_sparse_attn_fused); the other side runs as permutation kernels.
     The default fuses only the output side: on B200 the permutation kernel
     moves q, k, v faster than row gathers inside the attention kernel.  With
-    overlap (input side not fused), the token-major copies of every head are
-    made on a side stream while the heads are profiled.
+    overlap (input side not fused), the V exponents are computed on a side
+    stream while the heads are profiled, and the token-major copies of the
+    temporal heads alone follow the profiling (svg_permute_temporal_heads):
+    the profiling kernel occupies every SM, so copies of every head beside it
+    cost more than the copies the modes call for after it.
     qk applies QK-Norm + RoPE to q and k first (svg_qk_norm_rope); with
     overlap that pass also writes the token-major copies of q and k, and only
-    v is permuted on the side stream.
+    v is copied after the profiling.
     repeat (int32 [B*H], nonzero = spatially repeating head, e.g. from
     svg_row_similarity > 0.87) with frame_shape = (rows, cols): those heads,
     unless profiled temporal, compute only the query tiles holding anchor
@@ -513,8 +525,8 @@ def svg_layer(q, k, v, frames: int, tokens_per_frame: int, spatial_width: int,
             svg_row_broadcast(bufs.o, F, frame_shape[0], frame_shape[1], ids, lists.n_lists,
                               anchors=anchors, stream=st)
     if overlap and not layout & _lib.SVG_FUSE_INPUT:
-        # token-major copies of every head on a side stream, concurrent with
-        # the (latency-bound) profiling; temporal heads read the copies
+        # V exponents on a side stream beside the profiling; then token-major
+        # copies of the temporal heads, which the attention reads for them
         if stream is None:
             main = torch.cuda.current_stream()
         elif hasattr(stream, "wait_event"):
@@ -524,23 +536,22 @@ def svg_layer(q, k, v, frames: int, tokens_per_frame: int, spatial_width: int,
         ready = torch.cuda.Event()
         ready.record(main)
         bufs.side.wait_event(ready)
-        side_work = ((v, bufs.vp),) if qk is not None else \
-            ((q, bufs.qp), (k, bufs.kp), (v, bufs.vp))
-        for x, y in side_work:
-            svg_permute_token_major(x, F, P, None, out=y, stream=bufs.side)
         if v.dtype == torch.bfloat16:
             svg_v_exponents(v, out=bufs.vexp, stream=bufs.side)
-        copied = torch.cuda.Event()
-        copied.record(bufs.side)
+        side_done = torch.cuda.Event()
+        side_done.record(bufs.side)
         if qk is not None:
             svg_qk_norm_rope(q, k, qk, out=(bufs.qn, bufs.kn), tm_out=(bufs.qp, bufs.kp),
                              frames=F, tokens_per_frame=P, stream=main)
             q, k = bufs.qn, bufs.kn
         svg_profile_heads(q, k, v, F, P, spatial_width, sample_idx, mse_out=bufs.mse,
                           mode_out=bufs.mode, workspace=bufs.ws, stream=main)
-        main.wait_event(copied)
-        for t in (bufs.qp, bufs.kp, bufs.vp):
-            t.record_stream(main)
+        copy_work = ((v, bufs.vp),) if qk is not None else \
+            ((q, bufs.qp), (k, bufs.kp), (v, bufs.vp))
+        for x, y in copy_work:
+            svg_permute_temporal_heads(x, F, P, bufs.mode, out=y, stream=main)
+        main.wait_event(side_done)
+        bufs.vexp.record_stream(bufs.side)
         out = bufs.o if layout & _lib.SVG_FUSE_OUTPUT else bufs.op
         use_lists, ids = select_lists(main)
         svg_sparse_attn_fused(q, k, v, F, P, ids, use_lists, layout=layout,

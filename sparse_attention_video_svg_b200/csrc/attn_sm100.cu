@@ -14,19 +14,27 @@
 // Warp roles (384 threads, three warpgroups):
 //   warp 0      TMA producer: each member's Q tile, then K and V of every
 //               step into a ring, with a step record (which members keep the
-//               block, item boundaries) in shared memory;
-//   warps 1, 2  MMA issuers of members 0 and 1 (one thread each):
+//               block, item boundaries, the head's V exponent) in shared
+//               memory;
+//   d = 64:  warps 1, 2 MMA issuers of members 0 and 1 (one thread each),
+//               warp 3 the V converter;
+//   d = 128: warp 1 the one MMA issuer of both members (order on the tensor
+//               core: P.V of member 0, Q K^T of member 0, P.V of member 1,
+//               Q K^T of member 1), warps 2 and 3 the V converters (half a
+//               tile each);
 //               S_t = Q_t K^T into TMEM (bf16 operands) and O_t += P_t V
 //               (fp16 operands, P_t read from TMEM, V from smem).  A K/V ring
-//               entry is released when both issuers have passed it;
-//   warp 3      converts each V tile in shared memory from bf16 to fp16;
+//               entry is released when every issuer has passed it;
+//   converters  each V tile in shared memory from bf16 to fp16, scaled by
+//               2^-e with the head's V exponent e (0 unless |v| > 65504 occurs
+//               in the head), so any finite bf16 V is exact in fp16;
 //   warps 4-7   softmax of member 0, warps 8-11 of member 1: one thread per
 //               query row holds the tile's 128 scores, fp32 online softmax
 //               with lazy rescaling (O is rescaled only when the running max
 //               grows by more than 2^8); the weights go to TMEM as fp16
 //               (11 significant bits) and the row sums add the same rounded
-//               values (mixed-precision adds).  The epilogue writes O / l as
-//               bf16 from registers.
+//               values (mixed-precision adds).  The epilogue writes
+//               O * 2^e / l as bf16 from registers.
 // Every exponential runs on the MUFU (ex2.approx): FMA-pipe work in the
 // softmax warps measurably slows the issue of the tensor-core instructions,
 // so the softmax keeps its FMA-pipe share small.  Each tile's MMAs are

@@ -21,9 +21,10 @@ constexpr int kUnroll = 4;  // 16-byte chunks per thread, all loads issued befor
 template <bool kToTokenMajor>
 __global__ void __launch_bounds__(kThreads) permute_rows_kernel(
     const int4* __restrict__ x, int4* __restrict__ y, int N, int chunk_log2, int F, int P,
-    const int32_t* __restrict__ mode) {
+    const int32_t* __restrict__ mode, bool only_temporal) {
   const int bh = blockIdx.y;
   const bool permute = (mode == nullptr) || (mode[bh] == SVG_MODE_TEMPORAL);
+  if (only_temporal && !permute) return;  // this head of y is left as it is
   const long long head_chunks = static_cast<long long>(N) << chunk_log2;
   const int4* xh = x + head_chunks * bh;
   int4* yh = y + head_chunks * bh;
@@ -60,8 +61,11 @@ __global__ void __launch_bounds__(kThreads) permute_rows_kernel(
 }
 
 svg_status permute_impl(bool to_token_major, const void* x, void* y, int dtype, int B, int H,
-                        int N, int d, int F, int P, const int32_t* mode, void* stream) {
+                        int N, int d, int F, int P, const int32_t* mode, void* stream,
+                        bool only_temporal = false) {
   clear_error();
+  if (only_temporal && mode == nullptr)
+    return fail(SVG_ERR_INVALID_ARG, "permute_temporal_heads: mode is required");
   if (x == nullptr || y == nullptr) return fail(SVG_ERR_INVALID_ARG, "permute: null tensor");
   if (dtype != SVG_BF16 && dtype != SVG_FP32)
     return fail(SVG_ERR_INVALID_ARG, "permute: bad dtype %d", dtype);
@@ -89,10 +93,10 @@ svg_status permute_impl(bool to_token_major, const void* x, void* y, int dtype, 
   auto* ys = static_cast<int4*>(y);
   if (to_token_major)
     permute_rows_kernel<true><<<grid, kThreads, 0, as_stream(stream)>>>(xs, ys, N, chunk_log2, F,
-                                                                        P, mode);
+                                                                        P, mode, only_temporal);
   else
     permute_rows_kernel<false><<<grid, kThreads, 0, as_stream(stream)>>>(xs, ys, N, chunk_log2,
-                                                                         F, P, mode);
+                                                                         F, P, mode, false);
   return check_launch("permute");
 }
 
@@ -110,4 +114,11 @@ extern "C" svg_status svg_permute_frame_major(const void* x, void* y, int dtype,
                                               const int32_t* mode, void* stream) {
   return svg::permute_impl(false, x, y, dtype, B, H, N, d, frames, tokens_per_frame, mode,
                            stream);
+}
+
+extern "C" svg_status svg_permute_temporal_heads(const void* x, void* y, int dtype, int B, int H,
+                                                 int N, int d, int frames, int tokens_per_frame,
+                                                 const int32_t* mode, void* stream) {
+  return svg::permute_impl(true, x, y, dtype, B, H, N, d, frames, tokens_per_frame, mode, stream,
+                           true);
 }

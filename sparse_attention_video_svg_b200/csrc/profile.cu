@@ -26,6 +26,7 @@
 // The pass reads K and V once per head and costs a few percent of the
 // attention it configures.
 #include <float.h>
+#include <limits.h>
 
 #include "common.cuh"
 #include "sm100.cuh"
@@ -35,7 +36,8 @@ namespace {
 
 constexpr int kRows = 64;          // sampled rows per head (S padded to 64)
 constexpr int kTileKeys = 128;     // keys per tile of the tcgen05 path; ranges are multiples
-constexpr int kTargetCtas = 888;   // partial-grid size the chunking aims for (6 x 148)
+constexpr int kSms = 148;          // persistent CTAs the chunking plans for (B200)
+constexpr int kUnitTiles = 2;      // fixed cost of a unit (Q gather, fill, epilogue) in tiles
 constexpr int kMaxChunks = 32;     // merge holds one chunk weight per lane
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -58,9 +60,24 @@ ProfileShape shape_for(int N, long long chunks) {
   return {static_cast<int>(chunks), static_cast<int>(len)};
 }
 
+// The key-range count whose busiest CTA does the least: units of one
+// (range, head) go round-robin to kSms persistent CTAs, so the critical path
+// is ceil(units / kSms) units of (tiles per range + kUnitTiles) tiles each.
+// Ties go to fewer ranges (less merge work).
 ProfileShape profile_shape(int B, int H, int N) {
   const long long bh = static_cast<long long>(B) * H;
-  return shape_for(N, (kTargetCtas + bh - 1) / bh);
+  ProfileShape best = shape_for(N, 1);
+  long long best_cost = -1;
+  for (int c = 1; c <= kMaxChunks; ++c) {
+    const ProfileShape ps = shape_for(N, c);
+    const long long rounds = (bh * ps.chunks + kSms - 1) / kSms;
+    const long long cost = rounds * (ps.chunk_len / kTileKeys + kUnitTiles);
+    if (best_cost < 0 || cost < best_cost) {
+      best = ps;
+      best_cost = cost;
+    }
+  }
+  return best;
 }
 
 // floats per partial state row: m, l, o[D]
@@ -143,29 +160,32 @@ __global__ void __launch_bounds__(256) profile_partial_fp32(
 // --------------------------------------------------------------- tcgen05 partial (bf16)
 //
 // Persistent, one CTA per SM, looping over work units (key range c, head bh).
-// The 64 sampled rows fill rows 0-63 of a 128-row M tile (rows 64-127 are
-// zero and never read back).  Seven warps:
-//   warps 0, 4  softmax of rows 0-31, warps 1, 5 of rows 32-63 (TMEM lanes
-//               0-63 belong to warps 0 and 1 modulo 4); of the two warps of a
-//               row group, one takes key columns 0-63 of every tile and the
-//               other 64-127, and their row maxima and sums meet in shared
-//               memory (an mbarrier per row group, bounded waits).  Per 128-key tile: the dense and the spatial
-//               online-softmax states of the row, with lazy rescaling (an
-//               output is rescaled only when its running max grows by more
-//               than 2^8);
-//   warp 2      K loader: gathers the unit's sampled Q rows (cp.async, into
-//               the 128-byte-swizzled K-major layout), then streams the K
-//               tiles of the range through a ring (TMA);
+// The M = 128 tile holds the 64 sampled rows twice: rows 0-63 for the dense
+// state, rows 64-127 (the same queries) for the state under the spatial mask.
+// One Q K^T gives both copies of the scores, and one P.V (P of the dense
+// state in TMEM lanes 0-63, of the spatial state in lanes 64-127) gives both
+// outputs.  Seven warps:
+//   warps 0-3   softmax: warp w owns TMEM lanes 32 w .. 32 w + 31, i.e.
+//               sampled rows 32 (w & 1) + lane of state w >> 1 (0 dense,
+//               1 spatial), and works through every 128-key tile of the unit
+//               for them (fp32 online softmax with lazy rescaling: an output
+//               is rescaled only when its running max grows by more than 2^8;
+//               the weights go to TMEM as bf16 over the scores they came
+//               from, and the row sums add the same rounded values).  A
+//               spatial warp whose rows have no band key in a tile writes
+//               zero weights without touching the scores;
+//   warp 4      K loader: gathers the unit's sampled Q rows (cp.async, into
+//               both halves of the 128-byte-swizzled K-major Q tile), then
+//               streams the K tiles of the range through a ring (TMA);
+//   warp 5      MMA issuer (one thread): S_j = Q K_j^T into one of two TMEM
+//               score buffers, then O += P_j-1 V_j-1 with P from TMEM and V
+//               from shared memory;
 //   warp 6      V loader: the V tiles through a ring of their own, so that a
 //               K entry is refilled as soon as its Q K^T is done while a V
-//               entry waits for its P.V;
-//   warp 3      MMA issuer (one thread): S_j = Q K_j^T into one of two TMEM
-//               score buffers, then O_d += P_d,j-1 V_j-1 and O_s += P_s,j-1
-//               V_j-1 with both P from TMEM (bf16, written over the scores
-//               they came from) and V from shared memory.
+//               entry waits for its P.V.
 // The scores of tile j are computed while the softmax works on tile j-1.
 // Every wait is bounded; a CTA that gives up writes NaN into the states of
-// its unit (so the head's errors come out NaN) and drains.
+// its units (so the head's errors come out NaN) and drains.
 
 constexpr int kTcThreads = 224;
 
@@ -180,13 +200,11 @@ struct TcCfg {
   static constexpr int kOffV = kOffK + kStages * kTile;
   static constexpr int kOffBar = kOffV + kStages * kTile;
   // q_full, q_empty, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2],
-  // p_ready[2], o_done, drain, xchg[2]
-  static constexpr int kBars = 2 + 4 * kStages + 2 + 2 + 2 + 2;
-  static constexpr int kOffX = kOffBar + kBars * 8 + 16;  // float [2][2][32][2] exchange
-  static constexpr int kSmem = kOffX + 1024 + 1024;  // + the base's 1024-byte alignment
-  static constexpr uint32_t kColS = 0;               // S_b at 128 b; P_d in its columns 0-63, P_s 64-127
-  static constexpr uint32_t kColOd = 256;
-  static constexpr uint32_t kColOs = 256 + D;
+  // p_ready[2], o_done, drain
+  static constexpr int kBars = 2 + 4 * kStages + 2 + 2 + 2;
+  static constexpr int kSmem = kOffBar + kBars * 8 + 16 + 1024;  // + the base's 1024-byte alignment
+  static constexpr uint32_t kColS = 0;  // S_b at 128 b; P_b (bf16) over its columns 0-63
+  static constexpr uint32_t kColO = 256;
   static constexpr uint32_t kIdescQK = sm100::idesc_bf16(128, 128, false);
   static constexpr uint32_t kIdescPV = sm100::idesc_bf16(128, D, true);
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
@@ -194,12 +212,28 @@ struct TcCfg {
 
 constexpr uint32_t kTcSpin = 1u << 22;
 constexpr uint32_t kTcDrain = 1u << 20;
+constexpr unsigned kNapIssue = 32;   // ns between polls of the MMA issuer
+constexpr unsigned kNapLoad = 128;   // ns between polls of the loaders
 
 __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   const uint32_t addr = smem_u32(bar);
   for (uint32_t i = 0; i < kTcSpin; ++i) {
     if (sm100::mbar_try_wait(addr, parity)) return true;
     if ((i & 255u) == 255u && *abort_flag) return false;
+  }
+  *abort_flag = 1;
+  return false;
+}
+// The helper warps (loaders, issuer) share their SM sub-partitions with the
+// softmax warps: between polls they sleep for `ns` nanoseconds instead of
+// taking issue slots.  Bounded like tc_wait.
+__device__ __forceinline__ bool tc_wait_nap(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                            unsigned ns) {
+  const uint32_t addr = smem_u32(bar);
+  for (uint32_t i = 0; i < kTcSpin; ++i) {
+    if (sm100::mbar_try_wait(addr, parity)) return true;
+    if ((i & 255u) == 255u && *abort_flag) return false;
+    __nanosleep(ns);
   }
   *abort_flag = 1;
   return false;
@@ -229,6 +263,16 @@ __device__ __forceinline__ TcUnit tc_unit(int u, int chunks, int chunk_len, int 
   return w;
 }
 
+// The state row [m, l, o[D]] of sampled row r, variant (0 dense, 1 spatial),
+// of unit w in the workspace [bh][variant][chunk][row].
+template <int D>
+__device__ __forceinline__ float* tc_state_row(float* ws, const TcUnit& w, int variant, int r,
+                                               int chunks) {
+  return ws + ((static_cast<long long>(w.bh) * 2 + variant) * chunks + w.chunk) * kRows *
+                  state_floats<D>() +
+         static_cast<long long>(r) * state_floats<D>();
+}
+
 template <int D>
 __global__ void __launch_bounds__(kTcThreads, 1) profile_partial_tc(
     const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
@@ -252,16 +296,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) profile_partial_tc(
   uint64_t* p_ready = s_full + 2;
   uint64_t* o_done = p_ready + 2;
   uint64_t* drain = o_done + 1;
-  uint64_t* xchg = drain + 1;  // [2]: the two softmax warps of a row group meet here
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xchg + 2);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // rows 64-127 of the Q tile stay zero
-  for (int i = threadIdx.x; i < C::kTile / 16; i += kTcThreads) {
-    const int box = i / (C::kBox / 16), row = (i % (C::kBox / 16)) / 8;
-    if (row >= kRows) reinterpret_cast<uint4*>(smem + C::kOffQ)[box * (C::kBox / 16) + (i % (C::kBox / 16))] = make_uint4(0, 0, 0, 0);
-  }
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
@@ -277,23 +315,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) profile_partial_tc(
     }
     mbar_init(o_done, 1);
     mbar_init(drain, 1);
-    mbar_init(&xchg[0], 2);
-    mbar_init(&xchg[1], 2);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 3) {
+  if (warp == 5) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
-  fence_proxy_async_smem();  // the zeroed rows, for the tensor core
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 2) {
-    // ------------------------------------------------------------------ loader
+  if (warp == 4) {
+    // ------------------------------------------------------------------ K loader
     if (lane == 0) {
       prefetch_tmap(&mk);
       prefetch_tmap(&mv);
@@ -305,16 +340,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) profile_partial_tc(
       const TcUnit w = tc_unit(u, chunks, chunk_len, N);
       if (w.tiles == 0) continue;
       int r_ok = 1;
-      if (lane == 0) r_ok = tc_wait(q_empty, (nu & 1) ^ 1, abort_flag) ? 1 : 0;
+      if (lane == 0) r_ok = tc_wait_nap(q_empty, (nu & 1) ^ 1, abort_flag, kNapLoad) ? 1 : 0;
       if (!(ok = __shfl_sync(0xffffffffu, r_ok, 0) != 0)) break;
       ++nu;
+      // sampled row r into tile rows r and r + 64 (same swizzle phase: r & 7)
       const __nv_bfloat16* qh = q + static_cast<long long>(w.bh) * N * D;
       for (int t = lane; t < kRows * CH; t += 32) {
         const int r = t / CH, c = t % CH;
         const bool valid = r < S;
         const int n = valid ? clamp_index(idx[r], N) : 0;
-        cp_async16(smem + C::kOffQ + (c >> 3) * C::kBox + r * 128 + (((c & 7) ^ (r & 7)) << 4),
-                   qh + static_cast<long long>(n) * D + c * 8, valid);
+        const __nv_bfloat16* src = qh + static_cast<long long>(n) * D + c * 8;
+        unsigned char* dst = smem + C::kOffQ + (c >> 3) * C::kBox + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+        cp_async16(dst, src, valid);
+        cp_async16(dst + kRows * 128, src, valid);
       }
       cp_async_mbar_arrive(q_full);
       __syncwarp();
@@ -323,7 +361,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) profile_partial_tc(
         const uint32_t st = gt % ST;
         int r_ok = 1;  // lane 0 waits and copies; the warp learns the outcome
         if (lane == 0) {
-          if (tc_wait(&k_empty[st], ((gt / ST) & 1) ^ 1, abort_flag)) {
+          if (tc_wait_nap(&k_empty[st], ((gt / ST) & 1) ^ 1, abort_flag, kNapLoad)) {
             mbar_arrive_expect_tx(&k_full[st], C::kTile);
             const int key0 = w.key_begin + j * kTileKeys;
             for (int bx = 0; bx < C::kBoxes; ++bx)
@@ -351,7 +389,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) profile_partial_tc(
         const TcUnit w = tc_unit(u, chunks, chunk_len, N);
         for (int j = 0; j < w.tiles; ++j) {
           const uint32_t st = gt % ST;
-          if (!(ok = tc_wait(&v_empty[st], ((gt / ST) & 1) ^ 1, abort_flag))) break;
+          if (!(ok = tc_wait_nap(&v_empty[st], ((gt / ST) & 1) ^ 1, abort_flag, kNapLoad))) break;
           mbar_arrive_expect_tx(&v_full[st], C::kTile);
           for (int bx = 0; bx < C::kBoxes; ++bx)
             tma_load_3d(smem + C::kOffV + st * C::kTile + bx * C::kBox, &mv, &v_full[st], 64 * bx,
@@ -362,7 +400,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) profile_partial_tc(
       if (!ok)  // copies in flight land before the CTA can exit
         for (uint32_t l = gt > ST ? gt - ST : 0; l < gt; ++l) tc_drain(&v_full[l % ST], (l / ST) & 1);
     }
-  } else if (warp == 3) {
+  } else if (warp == 5) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint64_t dq = sdesc_sw128(smem_u32(smem + C::kOffQ), 16, 1024);
@@ -372,13 +410,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) profile_partial_tc(
       bool ok = true;
       auto issue_pv = [&](uint32_t g, bool first) -> bool {
         const uint32_t b = g & 1, st = g % ST;
-        if (!tc_wait(&p_ready[b], (g >> 1) & 1, abort_flag)) return false;
-        if (!tc_wait(&v_full[st], (g / ST) & 1, abort_flag)) return false;
+        if (!tc_wait_nap(&p_ready[b], (g >> 1) & 1, abort_flag, kNapIssue)) return false;
+        if (!tc_wait_nap(&v_full[st], (g / ST) & 1, abort_flag, kNapIssue)) return false;
         tc_fence_after();
-        const uint64_t v0 = dv + ((st * C::kTile) >> 4);
-        const uint32_t sb = tmem + C::kColS + 128 * b;
-        mma_ts_k128(tmem + C::kColOd, sb, v0, C::kIdescPV, first ? 0u : 1u);
-        mma_ts_k128(tmem + C::kColOs, sb + 64, v0, C::kIdescPV, first ? 0u : 1u);
+        mma_ts_k128(tmem + C::kColO, tmem + C::kColS + 128 * b, dv + ((st * C::kTile) >> 4),
+                    C::kIdescPV, first ? 0u : 1u);
         tc_commit(o_done);
         tc_commit(&v_empty[st]);
         return true;
@@ -386,12 +422,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) profile_partial_tc(
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
         const TcUnit w = tc_unit(u, chunks, chunk_len, N);
         if (w.tiles == 0) continue;
-        if (!(ok = tc_wait(q_full, nu & 1, abort_flag))) break;
+        if (!(ok = tc_wait_nap(q_full, nu & 1, abort_flag, kNapIssue))) break;
         fence_proxy_async_smem();  // Q came through cp.async (generic proxy)
         tc_fence_after();
         for (int j = 0; j < w.tiles; ++j, ++gt) {
           const uint32_t st = gt % ST, b = gt & 1;
-          if (!(ok = tc_wait(&k_full[st], (gt / ST) & 1, abort_flag))) break;
+          if (!(ok = tc_wait_nap(&k_full[st], (gt / ST) & 1, abort_flag, kNapIssue))) break;
           tc_fence_after();
           const uint64_t k0 = dk + ((st * C::kTile) >> 4);
           if constexpr (D == 64)
@@ -410,261 +446,163 @@ __global__ void __launch_bounds__(kTcThreads, 1) profile_partial_tc(
       tc_commit(drain);  // every MMA completes before TMEM is released
       tc_drain(drain, 0);
     }
-  } else if (warp == 0 || warp == 1 || warp == 4 || warp == 5) {
+  } else {
     // ------------------------------------------------------------------ softmax
-    // Two warps per row group: warp q (q = 0, 1) and warp q + 4 share TMEM
-    // lanes 32 q .. 32 q + 31 (rows) and take key columns 0-63 and 64-127 of
-    // every tile; their row maxima meet in shared memory.
-    const int quarter = warp & 3, half = warp >> 2;
-    const int r = quarter * 32 + lane;  // sampled row = TMEM lane
-    uint64_t* xb_bar = &xchg[quarter];
-    uint32_t xph = 0;  // exchange phases completed
-    // both warps of the row group reach this point (bounded wait)
-    auto meet = [&]() -> bool {
-      __syncwarp();
-      if (lane == 0) mbar_arrive(xb_bar);
-      const bool met = tc_wait_warp(xb_bar, xph & 1, abort_flag);
-      ++xph;
-      return met;
-    };
-    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    // this warp's half of each output (for rescaling and the epilogue)
-    const uint32_t t_od = tmem + lane_off + C::kColOd + half * (D / 2);
-    const uint32_t t_os = tmem + lane_off + C::kColOs + half * (D / 2);
-    // [quarter][half][lane][2]: the two warps' partial maxima / sums
-    volatile float* xb = reinterpret_cast<volatile float*>(smem + C::kOffX);
-    volatile float* mine = xb + ((quarter * 2 + half) * 32 + lane) * 2;
-    volatile float* other = xb + ((quarter * 2 + (half ^ 1)) * 32 + lane) * 2;
+    const int variant = warp >> 1;          // 0 dense, 1 spatial
+    const int r = (warp & 1) * 32 + lane;   // sampled row
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t t_o = tmem + lane_off + C::kColO;
+    const int f = r < S ? clamp_index(idx[r], N) / P : 0;
     uint32_t gt = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       const TcUnit w = tc_unit(u, chunks, chunk_len, N);
       if (w.tiles == 0) continue;
-      // this row's keys in the range: all of them (dense), its band of frames (spatial)
-      int dhi = w.key_end, slo = w.key_begin, shi = w.key_begin;
+      // this row's keys in the range: [lo, hi), all of them (dense) or its
+      // band of frames (spatial); empty for padding rows
+      int lo = w.key_begin, hi = w.key_begin;
       if (r < S) {
-        const int f = clamp_index(idx[r], N) / P;
-        slo = max(w.key_begin, max(0, f - width) * P);
-        shi = static_cast<int>(min(static_cast<long long>(w.key_end),
-                                   static_cast<long long>(f + width + 1) * P));
-      } else {
-        dhi = w.key_begin;
+        if (variant == 0) {
+          hi = w.key_end;
+        } else {
+          lo = max(w.key_begin, max(0, f - width) * P);
+          hi = static_cast<int>(min(static_cast<long long>(w.key_end),
+                                    static_cast<long long>(f + width + 1) * P));
+        }
       }
-      float md = -INFINITY, ms = -INFINITY;
-      float ld0 = 0.f, ld1 = 0.f, ls0 = 0.f, ls1 = 0.f;  // this half's row sums
+      // the warp's keys: tiles outside [wlo, whi) need no scores
+      const int wlo = __reduce_min_sync(0xffffffffu, lo < hi ? lo : INT_MAX);
+      const int whi = __reduce_max_sync(0xffffffffu, lo < hi ? hi : INT_MIN);
+      float m = -INFINITY, lx = 0.f, ly = 0.f;
       for (int j = 0; j < w.tiles; ++j, ++gt) {
         const uint32_t b = gt & 1;
         const uint32_t t_s = tmem + lane_off + C::kColS + 128 * b;
         if (!(ok = tc_wait_warp(&s_full[b], (gt >> 1) & 1, abort_flag))) break;
         tc_fence_after();
-        float s[64];
-        {
-          uint32_t rr[2][32];
-          tmem_ld32(t_s + 64 * half, rr[0]);
-          tmem_ld32(t_s + 64 * half + 32, rr[1]);
-          tmem_wait_ld();
-          reg_fence32(rr[0]);
-          reg_fence32(rr[1]);
+        const int c0 = w.key_begin + j * kTileKeys;
+        uint32_t p[4][16];
+        if (c0 < whi && c0 + kTileKeys > wlo) {  // warp-uniform
+          float s[128];
+          {
+            uint32_t rr[4][32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            s[i] = __uint_as_float(rr[0][i]) * scale_log2;
-            s[32 + i] = __uint_as_float(rr[1][i]) * scale_log2;
+            for (int c = 0; c < 4; ++c) tmem_ld32(t_s + 32 * c, rr[c]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              reg_fence32(rr[c]);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(rr[c][i]) * scale_log2;
+            }
           }
-        }
-        // this half's columns of the tile: keys c0 .. c0 + 63
-        const int c0 = w.key_begin + j * kTileKeys + 64 * half;
-        const int nd = max(0, min(64, dhi - c0));                        // dense [0, nd)
-        const int s0 = max(0, slo - c0), s1 = max(s0, min(64, shi - c0));  // band [s0, s1)
-        const bool dfull = nd == 64, sfull = s0 == 0 && s1 == 64, sempty = s1 <= s0;
-        float mxd, mxs;
-        if (dfull) {
+          // keys outside this row's [lo, hi) score -inf (a warp-uniform pass,
+          // taken only where some row of the warp is cut inside the tile)
+          const int a0 = max(0, lo - c0), a1 = max(a0, min(kTileKeys, hi - c0));
+          if (__any_sync(0xffffffffu, a0 != 0 || a1 != kTileKeys)) {
+#pragma unroll
+            for (int i = 0; i < kTileKeys; ++i) s[i] = (i >= a0 && i < a1) ? s[i] : -INFINITY;
+          }
           float m4[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-          for (int i = 4; i < 60; i += 8)
+          for (int i = 4; i < 124; i += 8)
 #pragma unroll
             for (int c = 0; c < 4; ++c) m4[c] = sm100::max3(m4[c], s[i + c], s[i + 4 + c]);
-          mxd = sm100::max3(sm100::max3(m4[0], s[60], s[61]), sm100::max3(m4[1], s[62], s[63]),
-                            fmaxf(m4[2], m4[3]));
-        } else {
-          mxd = -INFINITY;
-#pragma unroll
-          for (int i = 0; i < 64; ++i) mxd = i < nd ? fmaxf(mxd, s[i]) : mxd;
-        }
-        if (sfull && dfull) {
-          mxs = mxd;
-        } else if (sempty) {
-          mxs = -INFINITY;
-        } else {
-          mxs = -INFINITY;
-#pragma unroll
-          for (int i = 0; i < 64; ++i) mxs = (i >= s0 && i < s1) ? fmaxf(mxs, s[i]) : mxs;
-        }
-        mine[0] = mxd;
-        mine[1] = mxs;
-        if (!(ok = meet())) break;
-        mxd = fmaxf(mxd, other[0]);
-        mxs = fmaxf(mxs, other[1]);
-        if (!(ok = meet())) break;  // the buffer may be written again
-        // lazy rescaling: a running max moves only when it grows by more than
-        // 2^8 (both warps of the row group decide alike)
-        float ad = 1.f, as = 1.f;
-        bool rd = false, rs = false;
-        if (mxd > md + 8.f) {
-          if (md != -INFINITY) {
-            ad = exp2f(md - mxd);
-            rd = true;
-          }
-          md = mxd;
-        }
-        if (mxs > ms + 8.f) {
-          if (ms != -INFINITY) {
-            as = exp2f(ms - mxs);
-            rs = true;
-          }
-          ms = mxs;
-        }
-        ld0 *= ad;
-        ld1 *= ad;
-        ls0 *= as;
-        ls1 *= as;
-        // the outputs may be rescaled once the previous tile's P.V finished
-        // (these scores imply the P.V two tiles back did, so the barrier is
-        // at most one phase ahead of this wait); each warp its half
-        if (__any_sync(0xffffffffu, rd || rs)) {
-          if (!(ok = tc_wait_warp(o_done, (gt - 1) & 1, abort_flag))) break;
-          tc_fence_after();
-          uint32_t rr[32];
-#pragma unroll
-          for (int ch = 0; ch < D / 64; ++ch) {
-            tmem_ld32(t_od + 32 * ch, rr);
-            tmem_wait_ld();
-            reg_fence32(rr);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * ad);
-            tmem_st32(t_od + 32 * ch, rr);
-            tmem_ld32(t_os + 32 * ch, rr);
-            tmem_wait_ld();
-            reg_fence32(rr);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * as);
-            tmem_st32(t_os + 32 * ch, rr);
-          }
-        }
-        // weights as bf16 pairs: P_d over the scores' columns 0-63, P_s over
-        // 64-127 (the scores are in registers); the row sums add the rounded
-        // weights the tensor core sees
-        uint32_t pd[2][16];
-#pragma unroll
-        for (int c = 0; c < 2; ++c)
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int k = 32 * c + 2 * i;
-            float d0, d1;
-            if (dfull) {
-              d0 = fast_exp2(s[k] - md);
-              d1 = fast_exp2(s[k + 1] - md);
-            } else {
-              d0 = k < nd ? fast_exp2(s[k] - md) : 0.f;
-              d1 = k + 1 < nd ? fast_exp2(s[k + 1] - md) : 0.f;
+          const float mx = sm100::max3(sm100::max3(m4[0], s[124], s[125]),
+                                       sm100::max3(m4[1], s[126], s[127]), fmaxf(m4[2], m4[3]));
+          // lazy rescaling: the running max moves only when it grows by more
+          // than 2^8
+          float alpha = 1.f;
+          bool need = false;
+          if (mx > m + 8.f) {
+            if (m != -INFINITY) {
+              alpha = exp2f(m - mx);
+              need = true;
             }
-            pd[c][i] = pack_bf16x2(d0, d1);
-            ld0 += __uint_as_float(pd[c][i] << 16);
-            ld1 += __uint_as_float(pd[c][i] & 0xffff0000u);
+            m = mx;
           }
-        // (tcgen05.st and wait::st are warp-wide: the lanes meet before each,
-        // and the row-dependent choice below only selects register values)
-        __syncwarp();
-        tmem_st16(t_s + 32 * half, pd[0]);
-        tmem_st16(t_s + 32 * half + 16, pd[1]);
-        tmem_wait_st();  // pd's registers are free again
-        if (!(sfull && dfull && ms == md)) {
-          // (otherwise the whole half is in the band and both states share
-          // their max: the spatial weights are the dense ones)
+          lx *= alpha;
+          ly *= alpha;
+          // O may be rescaled once the previous tile's P.V finished (these
+          // scores imply the P.V two tiles back did, so the barrier is at
+          // most one phase ahead of this wait)
+          if (__any_sync(0xffffffffu, need)) {
+            if (!(ok = tc_wait_warp(o_done, (gt - 1) & 1, abort_flag))) break;
+            tc_fence_after();
+            uint32_t rr[32];
 #pragma unroll
-          for (int c = 0; c < 2; ++c)
+            for (int ch = 0; ch < D / 32; ++ch) {
+              tmem_ld32(t_o + 32 * ch, rr);
+              tmem_wait_ld();
+              reg_fence32(rr);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
+              tmem_st32(t_o + 32 * ch, rr);
+            }
+          }
+          // weights as bf16 pairs (a row with no key yet subtracts 0: its
+          // scores are all -inf and their weights 0); the row sums add the
+          // rounded weights the tensor core sees
+          const float neg = m == -INFINITY ? 0.f : -m;
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const int k = 32 * c + 2 * i;
-              float e0 = 0.f, e1 = 0.f;
-              if (!sempty) {
-                e0 = (k >= s0 && k < s1) ? fast_exp2(s[k] - ms) : 0.f;
-                e1 = (k + 1 >= s0 && k + 1 < s1) ? fast_exp2(s[k + 1] - ms) : 0.f;
-              }
-              pd[c][i] = pack_bf16x2(e0, e1);
+              p[c][i] = pack_bf16x2(fast_exp2(s[k] + neg), fast_exp2(s[k + 1] + neg));
+              lx += __uint_as_float(p[c][i] << 16);
+              ly += __uint_as_float(p[c][i] & 0xffff0000u);
             }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int i = 0; i < 16; ++i) p[c][i] = 0u;
         }
-#pragma unroll
-        for (int c = 0; c < 2; ++c)
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            ls0 += __uint_as_float(pd[c][i] << 16);
-            ls1 += __uint_as_float(pd[c][i] & 0xffff0000u);
-          }
+        // (tcgen05.st and wait::st are warp-wide: the lanes meet first)
         __syncwarp();
-        tmem_st16(t_s + 64 + 32 * half, pd[0]);
-        tmem_st16(t_s + 64 + 32 * half + 16, pd[1]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_st16(t_s + 16 * c, p[c]);
         tmem_wait_st();
         // before the unit's last weights are released, the P.V before them
         // has finished: o_done then stands at most one phase past what the
         // epilogue waits for (two would alias its parity)
-        if (j == w.tiles - 1 && gt > 0 && !(ok = tc_wait_warp(o_done, (gt - 1) & 1, abort_flag))) break;
+        if (j == w.tiles - 1 && gt > 0 && !(ok = tc_wait_warp(o_done, (gt - 1) & 1, abort_flag)))
+          break;
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_ready[b]);
       }
       if (!ok) break;
-      // the unit's states: [bh][variant][chunk][row][m, l, o[D]].  o_done
-      // completes one phase per tile's P.V; the one before the last has
-      // finished, so a single wait finds the last.
-      mine[0] = ld0 + ld1;
-      mine[1] = ls0 + ls1;
-      if (!(ok = meet())) break;
-      const float ld = ld0 + ld1 + other[0], ls = ls0 + ls1 + other[1];
-      if (!(ok = meet())) break;
+      // the unit's state rows; o_done completes one phase per tile's P.V and
+      // the one before the last has finished, so a single wait finds the last
       if (!(ok = tc_wait_warp(o_done, (gt - 1) & 1, abort_flag))) break;
       tc_fence_after();
-      const long long vstride = static_cast<long long>(chunks) * kRows * state_floats<D>();
-      float* rd_ = ws + (static_cast<long long>(w.bh) * 2 * chunks + w.chunk) * kRows * state_floats<D>() +
-                   static_cast<long long>(r) * state_floats<D>();
-      float* rs_ = rd_ + vstride;
-      if (half == 0) {
-        rd_[0] = md;
-        rd_[1] = ld;
-        rs_[0] = ms;
-        rs_[1] = ls;
-      }
+      float* row = tc_state_row<D>(ws, w, variant, r, chunks);
+      row[0] = m;
+      row[1] = lx + ly;
       uint32_t rr[32];
 #pragma unroll
-      for (int ch = 0; ch < D / 64; ++ch) {
-        const int col = half * (D / 2) + 32 * ch;
-        tmem_ld32(t_od + 32 * ch, rr);
+      for (int ch = 0; ch < D / 32; ++ch) {
+        tmem_ld32(t_o + 32 * ch, rr);
         tmem_wait_ld();
         reg_fence32(rr);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) rd_[2 + col + i] = __uint_as_float(rr[i]);
-        tmem_ld32(t_os + 32 * ch, rr);
-        tmem_wait_ld();
-        reg_fence32(rr);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) rs_[2 + col + i] = __uint_as_float(rr[i]);
+        for (int i = 0; i < 32; ++i) row[2 + 32 * ch + i] = __uint_as_float(rr[i]);
       }
       // (the next unit's first P.V overwrites O only after this warp's next
       // p_ready, which follows these reads in program order)
     }
     if (!ok) {
       // a wait gave up: this CTA's results are not to be trusted
-      for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
-        const TcUnit w = tc_unit(u, chunks, chunk_len, N);
-        float* rd_ = ws + (static_cast<long long>(w.bh) * 2 * chunks + w.chunk) * kRows * state_floats<D>() +
-                     static_cast<long long>(r) * state_floats<D>();
-        rd_[0] = __int_as_float(0x7fc00000);
-      }
+      for (int u = blockIdx.x; u < n_units; u += gridDim.x)
+        tc_state_row<D>(ws, tc_unit(u, chunks, chunk_len, N), variant, r, chunks)[0] =
+            __int_as_float(0x7fc00000);
     }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 3) tmem_dealloc(tmem, 512);
+  if (warp == 5) tmem_dealloc(tmem, 512);
 }
 
 // --------------------------------------------------------------- combine

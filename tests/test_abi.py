@@ -160,6 +160,10 @@ class TestHostValidation:
         expect(INVALID, "svg_permute_token_major", *(args[:7] + [5] + args[8:]), match="!= N")
         expect(INVALID, "svg_permute_frame_major", *([FAKE, FAKE + 64] + args[2:]), match="overlap")
         expect(INVALID, "svg_permute_token_major", *(args[:6] + [32] + args[7:]), match="d=32")
+        # the temporal-only copy needs the modes, and checks shapes like the others
+        expect(INVALID, "svg_permute_temporal_heads", *args, match="mode is required")
+        expect(INVALID, "svg_permute_temporal_heads", *(args[:7] + [5] + args[8:9] + [FAKE] + args[10:]),
+               match="!= N")
 
     def test_profile(self):
         ws = L.svg_profile_workspace_size(1, 2, 256, 64, 16)

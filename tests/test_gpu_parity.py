@@ -91,6 +91,28 @@ def bits_t(t):
     return t.view(torch.int16) if t.dtype == torch.bfloat16 else t.view(torch.int32)
 
 
+@pytest.mark.parametrize("wl", SMALL, ids=lambda w: w.name)
+def test_permute_temporal_heads_bit_exact(wl):
+    """Temporal heads: the token-major rows; every other head of the output
+    keeps what was there (a sentinel pattern), untouched."""
+    (q, _, _), (qd, _, _), types = workload_tensors(wl)
+    mode = torch.from_numpy(types).to(DEV)
+    F, P = wl.F, wl.P
+    y = torch.empty_like(qd)
+    bits_t(y).fill_(0x5a5a)
+    sentinel = bits(y).copy()
+    svg.svg_permute_temporal_heads(qd, F, P, mode, out=y)
+    yb = bits(y)
+    for b in range(wl.B):
+        for h in range(wl.H):
+            if types[h] == si.TEMPORAL_TYPE:
+                want = O.permute_token_major(q[b, h], F, P)
+                np.testing.assert_array_equal(yb[b, h], want.view(yb.dtype))
+            else:
+                np.testing.assert_array_equal(yb[b, h], sentinel[b, h])
+    assert (types == si.TEMPORAL_TYPE).any() and (types != si.TEMPORAL_TYPE).any()
+
+
 @pytest.mark.parametrize("F,P,d,dt", [(1, 77, 64, "bf16"), (77, 1, 128, "bf16"), (3, 5, 128, "fp32"),
                                       (9, 13, 64, "fp32")])
 def test_permute_edge_shapes(F, P, d, dt):
