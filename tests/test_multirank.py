@@ -169,12 +169,17 @@ def test_reference_arm_under_torchrun_prints_once():
 
 def test_traffic_tracks_kernel_sources(monkeypatch):
     """DRAM traffic is reported only for the kernel sources it was measured on."""
-    rec = bench.ATTN_TRAFFIC["cogvideox"]
+    rec = bench.ATTN_TRAFFIC["hunyuan720"]
     monkeypatch.setattr(bench, "attn_sources_sha256", lambda: rec["sha256"])
-    assert bench.attn_traffic("cogvideox") == rec["bytes"]
-    monkeypatch.setattr(bench, "attn_sources_sha256", lambda: "0" * 64)
-    assert bench.attn_traffic("cogvideox") is None
+    assert bench.attn_traffic("hunyuan720") == rec["bytes"]
     assert bench.attn_traffic("wan480") is None
+    monkeypatch.setattr(bench, "attn_sources_sha256", lambda: "0" * 64)
+    assert bench.attn_traffic("hunyuan720") is None
+
+
+def test_recorded_traffic_matches_the_sources():
+    """The recorded capture belongs to the attention sources in the tree."""
+    assert bench.attn_traffic("hunyuan720") == bench.ATTN_TRAFFIC["hunyuan720"]["bytes"]
 
 
 def test_effective_flops_count_the_element_mask():
