@@ -37,7 +37,7 @@ __all__ = [
     "svg_permute_token_major", "svg_permute_temporal_heads",
     "svg_permute_frame_major", "svg_build_block_mask", "svg_block_energy",
     "svg_build_block_mask_calibrated", "svg_sparse_attn", "svg_sparse_attn_fused",
-    "svg_v_exponents",
+    "svg_v_exponents", "svg_layer_from_host", "HostLayerBuffers",
     "svg_epsilon_schedule", "svg_lists_to_intervals", "svg_lists_to_bitmap", "geometric_lists",
     "QKTransform", "svg_qk_norm_rope", "svg_row_similarity", "svg_anchor_lists",
     "svg_anchor_list_ids", "svg_row_broadcast", "svg_repeat_attention", "svg_layer",
@@ -457,8 +457,7 @@ class LayerBuffers:
             self.qp = torch.empty_like(q)
             self.kp = torch.empty_like(q)
             self.vp = torch.empty_like(q)
-            # the copies of every head are made on this stream while the
-            # heads are profiled
+            # the V exponents run on this stream beside the profiling
             self.side = torch.cuda.Stream(device=dev) if dev.type == "cuda" else None
         if not layout & _lib.SVG_FUSE_OUTPUT:  # token-major output
             self.op = torch.empty_like(q)
@@ -585,3 +584,78 @@ def svg_layer(q, k, v, frames: int, tokens_per_frame: int, spatial_width: int,
         svg_permute_frame_major(bufs.op, F, P, bufs.mode, out=bufs.o, stream=stream)
     broadcast(ids, stream)
     return bufs.o, bufs.mode, bufs.mse
+
+
+class HostLayerBuffers:
+    """Device slots for svg_layer_from_host: two chunks of `heads` heads each
+    (inputs and LayerBuffers), and the copy streams."""
+
+    def __init__(self, heads: int, N: int, d: int, S: int, device=None):
+        dev = torch.device(device) if device is not None else torch.device("cuda")
+        self.heads = heads
+        self.slots = []
+        for _ in range(2):
+            x = torch.empty(3, 1, heads, N, d, dtype=torch.bfloat16, device=dev)
+            slot = {"q": x[0], "k": x[1], "v": x[2], "bufs": LayerBuffers(x[0], S),
+                    "loaded": torch.cuda.Event(), "computed": torch.cuda.Event(),
+                    "unloaded": torch.cuda.Event(), "used": False}
+            self.slots.append(slot)
+        self.h2d = torch.cuda.Stream(device=dev)
+        self.d2h = torch.cuda.Stream(device=dev)
+
+
+def svg_layer_from_host(q, k, v, frames: int, tokens_per_frame: int, spatial_width: int,
+                        sample_idx: torch.Tensor, lists: BlockLists, *, out=None, mode_out=None,
+                        heads_per_chunk: int = 4, buffers: Optional[HostLayerBuffers] = None,
+                        stream=None):
+    """svg_layer for q, k, v in pinned host memory ([B, H, N, d] bf16): the
+    B*H heads go through the GPU in chunks of `heads_per_chunk` (a divisor of
+    B*H) on two device slots, so that the copy of chunk c + 1 to the device
+    and of chunk c - 1 back to the host run while chunk c is computed (heads
+    are independent in every step of the layer).  Returns (out, mode_out):
+    pinned host [B, H, N, d] bf16 and [B*H] int32, complete once `stream`
+    (default: the current stream) has passed this call."""
+    B, H, N, d = q.shape
+    BH = B * H
+    for x in (q, k, v):
+        if x.device.type != "cpu" or not x.is_pinned() or x.dtype != torch.bfloat16 \
+                or not x.is_contiguous() or x.shape != q.shape:
+            raise ValueError("svg_layer_from_host takes contiguous pinned host bf16 [B, H, N, d]")
+    if heads_per_chunk <= 0 or BH % heads_per_chunk:
+        raise ValueError(f"heads_per_chunk must divide B*H = {BH}")
+    hc = heads_per_chunk
+    dev = sample_idx.device
+    if buffers is None or buffers.heads != hc or buffers.slots[0]["q"].shape[2:] != (N, d):
+        buffers = HostLayerBuffers(hc, N, d, sample_idx.numel(), dev)
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+    if mode_out is None:
+        mode_out = torch.empty(BH, dtype=torch.int32).pin_memory()
+    main = torch.cuda.current_stream(dev) if stream is None else stream
+    qf, kf, vf, of = (x.view(BH, N, d) for x in (q, k, v, out))
+    for c in range(BH // hc):
+        slot = buffers.slots[c % 2]
+        lo, hi = c * hc, (c + 1) * hc
+        # inputs of chunk c once chunk c - 2 has been computed from this slot
+        if slot["used"]:
+            buffers.h2d.wait_event(slot["computed"])
+        with torch.cuda.stream(buffers.h2d):
+            for src, dst in ((qf, slot["q"]), (kf, slot["k"]), (vf, slot["v"])):
+                dst[0].copy_(src[lo:hi], non_blocking=True)
+        slot["loaded"].record(buffers.h2d)
+        main.wait_event(slot["loaded"])
+        if slot["used"]:  # the slot's output has gone back to the host
+            main.wait_event(slot["unloaded"])
+        o, mode, _ = svg_layer(slot["q"], slot["k"], slot["v"], frames, tokens_per_frame,
+                               spatial_width, sample_idx, lists, slot["bufs"], stream=main)
+        slot["computed"].record(main)
+        buffers.d2h.wait_event(slot["computed"])
+        with torch.cuda.stream(buffers.d2h):
+            of[lo:hi].copy_(o[0], non_blocking=True)
+            mode_out[lo:hi].copy_(mode, non_blocking=True)
+        slot["unloaded"].record(buffers.d2h)
+        slot["used"] = True
+    for slot in buffers.slots:
+        if slot["used"]:
+            main.wait_event(slot["unloaded"])
+    return out, mode_out

@@ -592,6 +592,36 @@ def test_layer_small_layouts_agree(wl):
         np.testing.assert_array_equal(o, outs[0][0])
 
 
+@pytest.mark.parametrize("wl", [w for w in SMALL if w.dtype == "bf16" and w.kind == "profiled"],
+                         ids=lambda w: w.name)
+def test_layer_from_host_matches_device_layer(wl):
+    """The host-streamed layer (chunks of heads through two device slots, copies
+    overlapped with compute) gives the device layer's bits, for one chunk per
+    head, two heads per chunk and all heads in one chunk; repeated calls reuse
+    the slots."""
+    (q, k, v), (qd, kd, vd), _ = workload_tensors(wl)
+    idx = torch.from_numpy(si.sample_queries(wl)).to(DEV)
+    lists = svg.geometric_lists(wl.F, wl.P, wl.width, wl.N)
+    o_ref, m_ref, _ = svg.svg_layer(qd, kd, vd, wl.F, wl.P, wl.width, idx, lists)
+    torch.cuda.synchronize()
+    o_ref, m_ref = bits(o_ref), m_ref.cpu().numpy()
+    host = [x.cpu().pin_memory() for x in (qd, kd, vd)]
+    BH = wl.B * wl.H
+    for hc in (1, 2, BH):
+        if BH % hc:
+            continue
+        bufs = svg.HostLayerBuffers(hc, wl.N, wl.d, idx.numel())
+        for call in range(3):  # own buffers, then the same slots twice
+            out, mode = svg.svg_layer_from_host(*host, wl.F, wl.P, wl.width, idx, lists,
+                                                heads_per_chunk=hc,
+                                                buffers=None if call == 0 else bufs)
+            torch.cuda.synchronize()
+            np.testing.assert_array_equal(mode.numpy(), m_ref)
+            np.testing.assert_array_equal(bits(out), o_ref)
+    with pytest.raises(ValueError):
+        svg.svg_layer_from_host(*host, wl.F, wl.P, wl.width, idx, lists, heads_per_chunk=BH + 1)
+
+
 def test_layer_full_size_cogvideox_sampled(full_inputs):
     name = "cogvideox"
     wl = si.WORKLOADS[name]

@@ -177,6 +177,12 @@ def test_traffic_tracks_kernel_sources(monkeypatch):
     assert bench.attn_traffic("hunyuan720") is None
 
 
+def test_host_chunk_divides_the_heads():
+    for bh, want in ((24, 4), (40, 4), (48, 4), (7, 1), (6, 3), (3, 3), (1, 1), (12, 4)):
+        assert bench.host_chunk(bh) == want
+        assert bh % bench.host_chunk(bh) == 0
+
+
 def test_recorded_traffic_matches_the_sources():
     """The recorded capture belongs to the attention sources in the tree."""
     assert bench.attn_traffic("hunyuan720") == bench.ATTN_TRAFFIC["hunyuan720"]["bytes"]
