@@ -492,13 +492,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) profile_partial_tc(
             for (int c = 0; c < 4; ++c) {
               reg_fence32(rr[c]);
 #pragma unroll
-              for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(rr[c][i]) * scale_log2;
+              for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(rr[c][i]);
             }
           }
-          // keys outside this row's [lo, hi) score -inf (a warp-uniform pass,
-          // taken only where some row of the warp is cut inside the tile)
+          // the raw scores s; the scale (> 0) enters the max afterwards and
+          // the exponent through one fused multiply-add.  This row's keys in
+          // the tile are the columns [a0, a1): a row with none takes no part
+          // (max -inf, weights 0); a warp-uniform -inf pass over the other
+          // columns runs only where some row is cut inside the tile
           const int a0 = max(0, lo - c0), a1 = max(a0, min(kTileKeys, hi - c0));
-          if (__any_sync(0xffffffffu, a0 != 0 || a1 != kTileKeys)) {
+          const bool none = a1 <= a0;
+          if (__any_sync(0xffffffffu, !none && (a0 != 0 || a1 != kTileKeys))) {
 #pragma unroll
             for (int i = 0; i < kTileKeys; ++i) s[i] = (i >= a0 && i < a1) ? s[i] : -INFINITY;
           }
@@ -507,8 +511,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) profile_partial_tc(
           for (int i = 4; i < 124; i += 8)
 #pragma unroll
             for (int c = 0; c < 4; ++c) m4[c] = sm100::max3(m4[c], s[i + c], s[i + 4 + c]);
-          const float mx = sm100::max3(sm100::max3(m4[0], s[124], s[125]),
-                                       sm100::max3(m4[1], s[126], s[127]), fmaxf(m4[2], m4[3]));
+          const float mx = none ? -INFINITY
+                                : sm100::max3(sm100::max3(m4[0], s[124], s[125]),
+                                              sm100::max3(m4[1], s[126], s[127]),
+                                              fmaxf(m4[2], m4[3])) * scale_log2;
           // lazy rescaling: the running max moves only when it grows by more
           // than 2^8
           float alpha = 1.f;
@@ -539,16 +545,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) profile_partial_tc(
               tmem_st32(t_o + 32 * ch, rr);
             }
           }
-          // weights as bf16 pairs (a row with no key yet subtracts 0: its
-          // scores are all -inf and their weights 0); the row sums add the
-          // rounded weights the tensor core sees
-          const float neg = m == -INFINITY ? 0.f : -m;
+          // weights as bf16 pairs, exp2(s * scale - m); a row with no key in
+          // the tile, or none yet, takes -inf as the offset (weights 0); the
+          // row sums add the rounded weights the tensor core sees
+          const float neg = (none || m == -INFINITY) ? -INFINITY : -m;
 #pragma unroll
           for (int c = 0; c < 4; ++c)
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const int k = 32 * c + 2 * i;
-              p[c][i] = pack_bf16x2(fast_exp2(s[k] + neg), fast_exp2(s[k + 1] + neg));
+              float t0, t1;
+              sm100::fma2(t0, t1, s[k], s[k + 1], scale_log2, scale_log2, neg, neg);
+              p[c][i] = pack_bf16x2(fast_exp2(t0), fast_exp2(t1));
               lx += __uint_as_float(p[c][i] << 16);
               ly += __uint_as_float(p[c][i] & 0xffff0000u);
             }
