@@ -174,6 +174,32 @@ def test_profile_small(wl):
     np.testing.assert_array_equal(mode.cpu().numpy(), types)
 
 
+# bf16 profiling shapes at the edges of the tiled pass: padded sample rows
+# (S < 64), a single frame, a band wider than the clip (spatial = dense), a
+# ragged last tile, keys of a single tile, B > 1, and both head dims
+PROFILE_EDGES = [
+    si.WORKLOADS["hunyuan720"].scaled("edge-s5", H=2, F=6, ph=5, pw=7, S=5),          # N = 210
+    si.WORKLOADS["cogvideox"].scaled("edge-one-frame", H=3, F=1, ph=9, pw=15, S=64),  # N = 135
+    si.WORKLOADS["wan480"].scaled("edge-wide-band", H=2, F=3, ph=6, pw=10, width=5),  # N = 180
+    si.WORKLOADS["wan480"].scaled("edge-one-tile", H=2, F=4, ph=4, pw=7, S=17),       # N = 112
+    si.WORKLOADS["cogvideox"].scaled("edge-b2", B=2, H=2, F=5, ph=7, pw=9, S=33),     # N = 315
+]
+
+
+@pytest.mark.parametrize("wl", PROFILE_EDGES, ids=lambda w: w.name)
+def test_profile_edges(wl):
+    (q, k, v), (qd, kd, vd), _ = workload_tensors(wl)
+    idx = si.sample_queries(wl)
+    mse, mode = svg.svg_profile_heads(qd, kd, vd, wl.F, wl.P, wl.width,
+                                      torch.from_numpy(idx).to(DEV))
+    mse_ref, mode_ref = O.profile_heads(si.as_float64(q), si.as_float64(k), si.as_float64(v), idx,
+                                        wl.F, wl.P, wl.width)
+    check_profile(mse.cpu().numpy(), mode.cpu().numpy(), mse_ref, mode_ref, wl.name)
+    if wl.width >= wl.F - 1:
+        # every key in the band: the spatial output is the dense one
+        assert np.all(mse.cpu().numpy()[:, 0] <= 1e-6)
+
+
 @pytest.fixture(scope="module")
 def full_inputs():
     cache = {}
