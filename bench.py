@@ -631,6 +631,26 @@ def run_calibrated(args, rank, world, local_rank):
     ix = lists.indices.cpu().numpy()
     pairs = [kept_pairs(ip[h] - ip[h][0], ix[ip[h][0]:ip[h][-1]], N) for h in range(Hl)]
     flops = float(sum(4 * d * p for p in pairs))
+    # the pairing order of the query tiles (once per list set, like the lists)
+    svg.svg_pair_query_tiles(lists)  # warm-up
+    torch.cuda.synchronize()
+    e0, e1 = ev(), ev()
+    e0.record(stream)
+    lists = svg.svg_pair_query_tiles(lists)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    pairing_ms = e0.elapsed_time(e1)
+    # merged-walk steps of the work items with and without the order (a
+    # key block kept by both tiles of an item is one step)
+    order = lists.tile_order.cpu().numpy().reshape(Hl, nb)
+    rows = [[set(ix[ip[h][i]:ip[h][i + 1]].tolist()) for i in range(nb)] for h in range(Hl)]
+
+    def steps_of(seq):
+        return sum(len(rows[h][seq[h][i]] | (rows[h][seq[h][i + 1]] if i + 1 < nb else set()))
+                   for h in range(Hl) for i in range(0, nb, 2))
+    steps_index = steps_of([list(range(nb))] * Hl)
+    steps_paired = steps_of(order.tolist())
+    del rows
 
     q, k, v, _ = si.generate(wl, seed=seed, types_seed=tseed, heads=heads)
     host = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in (q, k, v)]
@@ -643,9 +663,11 @@ def run_calibrated(args, rank, world, local_rank):
     K, W = args.steps, args.warmup
 
     def step():
-        # the per-head V exponents (one read of v), then every head on its list
+        # the per-head V exponents (one read of v), then every head on its
+        # list, query tiles paired by the order
         svg.svg_v_exponents(vd, out=vexp)
-        svg.svg_sparse_attn(qd, kd, vd, list_id, lists, out=o, v_exp=vexp)
+        svg.svg_sparse_attn_fused(qd, kd, vd, wl.F, wl.P, list_id, lists, layout=0, out=o,
+                                  v_exp=vexp)
 
     for _ in range(W):
         step()
@@ -725,13 +747,18 @@ def run_calibrated(args, rank, world, local_rank):
         "tokens_per_s": round(tokens_s, 1),
         "pct_of_bf16_peak": round(100 * value / world / peak_tf, 2),
         "attention_only": {"ms": round(total_ms / K, 5), "effective_tflops": round(attn_tf, 3),
-                           "kernel": "svg_v_exponents + svg_sparse_attn (list_id = h)"},
+                           "kernel": "svg_v_exponents + svg_sparse_attn_fused (list_id = h, "
+                                     "tiles paired by svg_pair_query_tiles)"},
         "calibration": {"energy_ms_per_input": round(energy_avg, 3),
                         "energy_tflops": round(energy_flops / (energy_avg * 1e-3) / 1e12, 1),
                         "build_lists_ms": round(build_ms, 3),
+                        "pairing_ms": round(pairing_ms, 3),
+                        "item_steps": {"index_pairs": int(steps_index),
+                                       "paired_order": int(steps_paired)},
                         "inputs": len(wl.calib_seeds),
                         "note": "offline, not in the step"},
-        "roofline": {"kernel": "svg_sparse_attn", "bound": "tensor", "achieved": round(attn_tf, 3),
+        "roofline": {"kernel": "svg_sparse_attn_fused", "bound": "tensor",
+                     "achieved": round(attn_tf, 3),
                      "peak": peak_tf, "unit": "TFLOP/s", "frac": round(attn_tf / peak_tf, 4),
                      "peak_source": f"{src} bf16 burst", "traffic": attn_traffic(wl.name)},
         "e2e": {"value": round(e2e_value, 3), "unit": "TFLOPS",

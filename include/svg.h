@@ -476,6 +476,41 @@ svg_status svg_sparse_attn_fused(const void* q, const void* k, const void* v,
                                  int32_t* device_status, const int32_t* v_exp, void* stream);
 
 /* --------------------------------------------------------------------------
+ * 4c. Pairing order of query tiles
+ *    [CAL] sections 2.2 and 3.3: attention on 128 x 128 tiles through
+ *    per-query-block lists of kept key blocks.  svg_sparse_attn_fused runs
+ *    two query tiles of a head as one work item and loads a key block kept
+ *    by both once; tile_order says which tiles go together.  This pass
+ *    computes, per list, an order in which consecutive pairs share many key
+ *    blocks: greedily, the smallest unpaired query tile takes the unpaired
+ *    tile whose row has the most key blocks in common with its own (ties:
+ *    the smaller index).  A scheduling choice only (results do not depend on
+ *    it); meant for lists that are built once and used many times (the
+ *    calibrated lists).
+ *
+ *  indptr       device int32 [n_lists][n_qblocks + 1], absolute offsets into
+ *               indices (as for svg_sparse_attn).
+ *  indices      device int32 key-block indices; an index outside
+ *               [0, n_kblocks) or a bad row range is skipped and sets
+ *               SVG_DEVICE_BAD_INDEX in device_status (may be NULL).
+ *  tile_order   device int32 [n_lists][n_qblocks], written: each row a
+ *               permutation of 0 .. n_qblocks-1, paired as (2i, 2i + 1).
+ *  workspace    device, 4-byte aligned, at least
+ *               svg_pair_query_tiles_workspace_size(n_lists, n_qblocks,
+ *               n_kblocks) bytes (the rows as bitmaps).
+ *  Errors: SVG_ERR_INVALID_ARG for null pointers, non-positive sizes, more
+ *  than 65535 lists, a short or misaligned workspace, or rows too many for
+ *  the pass's shared memory (n_qblocks + (n_kblocks + 31) / 32 * 4 bytes
+ *  beyond 48 KB).
+ * ------------------------------------------------------------------------ */
+size_t svg_pair_query_tiles_workspace_size(int n_lists, int n_qblocks, int n_kblocks);
+
+svg_status svg_pair_query_tiles(const int32_t* indptr, const int32_t* indices, int n_lists,
+                                int n_qblocks, int n_kblocks, int32_t* tile_order,
+                                int32_t* device_status, void* workspace, size_t workspace_bytes,
+                                void* stream);
+
+/* --------------------------------------------------------------------------
  * 6. Spatial-repetition heads
  *    [CAL] section 3.2: in some heads the image rows of a frame attend almost
  *    alike.  They are found by the mean cosine similarity of the rows'

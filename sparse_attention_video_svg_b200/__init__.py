@@ -37,7 +37,7 @@ __all__ = [
     "svg_permute_token_major", "svg_permute_temporal_heads",
     "svg_permute_frame_major", "svg_build_block_mask", "svg_block_energy",
     "svg_build_block_mask_calibrated", "svg_sparse_attn", "svg_sparse_attn_fused",
-    "svg_v_exponents", "svg_layer_from_host", "HostLayerBuffers",
+    "svg_v_exponents", "svg_pair_query_tiles", "svg_layer_from_host", "HostLayerBuffers",
     "svg_epsilon_schedule", "svg_lists_to_intervals", "svg_lists_to_bitmap", "geometric_lists",
     "QKTransform", "svg_qk_norm_rope", "svg_row_similarity", "svg_anchor_lists",
     "svg_anchor_list_ids", "svg_row_broadcast", "svg_repeat_attention", "svg_layer",
@@ -275,6 +275,23 @@ def svg_sparse_attn_fused(q, k, v, frames: int, tokens_per_frame: int, mode: tor
               lists.indices.data_ptr(), _ptr(lists.tile_order), float(scale), _ptr(status),
               _ptr(v_exp), _stream(stream))
     return out
+
+
+def svg_pair_query_tiles(lists: BlockLists, n_kblocks: Optional[int] = None, *, status=None,
+                         stream=None) -> BlockLists:
+    """The lists with a pairing order of their query tiles (tile_order): per
+    list, consecutive pairs share many key blocks (greedy, on the GPU).  For
+    lists built once and used for many steps; the attention results do not
+    depend on it.  n_kblocks defaults to n_qblocks (square lists)."""
+    nk = lists.n_qblocks if n_kblocks is None else int(n_kblocks)
+    dev = lists.indptr.device
+    ws = _scratch(_lib.lib.svg_pair_query_tiles_workspace_size(lists.n_lists, lists.n_qblocks, nk),
+                  dev)
+    order = torch.empty(lists.n_lists * lists.n_qblocks, dtype=torch.int32, device=dev)
+    _lib.call("svg_pair_query_tiles", lists.indptr.data_ptr(), lists.indices.data_ptr(),
+              lists.n_lists, lists.n_qblocks, nk, order.data_ptr(), _ptr(status), ws.data_ptr(),
+              ws.numel(), _stream(stream))
+    return lists._replace(tile_order=order)
 
 
 class QKTransform(NamedTuple):

@@ -42,6 +42,8 @@ SIGNATURES = {
     "svg_permute_token_major": (_i, [_p, _p, _i, _i, _i, _i, _i, _i, _i, _p, _p]),
     "svg_permute_frame_major": (_i, [_p, _p, _i, _i, _i, _i, _i, _i, _i, _p, _p]),
     "svg_permute_temporal_heads": (_i, [_p, _p, _i, _i, _i, _i, _i, _i, _i, _p, _p]),
+    "svg_pair_query_tiles_workspace_size": (_sz, [_i, _i, _i]),
+    "svg_pair_query_tiles": (_i, [_p, _p, _i, _i, _i, _p, _p, _p, _sz, _p]),
     "svg_build_block_mask": (_i, [_i, _i, _i, _i, _i, _p, _p, _i64, _i64, _p, _p, _p]),
     "svg_block_energy_workspace_size": (_sz, [_i, _i, _i]),
     "svg_block_energy": (_i, [_p, _p, _i, _i, _i, _i, _i, _p, _p, _sz, _p]),

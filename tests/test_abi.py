@@ -155,6 +155,19 @@ class TestHostValidation:
         expect(INVALID, f, *(base[:11] + [0] + base[12:]), match="n_lists")
         expect(INVALID, f, *([FAKE + 8] + base[1:]), match="aligned")
 
+    def test_pair_query_tiles(self):
+        f = "svg_pair_query_tiles"
+        ws = L.svg_pair_query_tiles_workspace_size(2, 5, 5)
+        assert ws == 2 * 5 * 1 * 4 and L.svg_pair_query_tiles_workspace_size(0, 5, 5) == 0
+        # indptr indices lists rows blocks order status ws ws_bytes stream
+        base = [FAKE, FAKE2, 2, 5, 5, FAKE3, None, FAKE4, ws, None]
+        expect(INVALID, f, *([None] + base[1:]), match="null")
+        expect(INVALID, f, *(base[:3] + [0] + base[4:]), match="bad sizes")
+        expect(INVALID, f, *(base[:8] + [ws - 4] + base[9:]), match="workspace")
+        expect(INVALID, f, *(base[:3] + [60000, 10 ** 6] + base[5:8]
+                             + [L.svg_pair_query_tiles_workspace_size(2, 60000, 10 ** 6)] + base[9:]),
+               match="limit")
+
     def test_permute(self):
         args = [FAKE, FAKE4 * 4, 0, 1, 2, 12, 64, 3, 4, None, None]
         expect(INVALID, "svg_permute_token_major", *(args[:7] + [5] + args[8:]), match="!= N")

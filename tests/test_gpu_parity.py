@@ -1160,6 +1160,86 @@ def test_tile_order_changes_no_result():
     assert status.item() & svg._lib.SVG_DEVICE_BAD_INDEX
 
 
+def _greedy_pairing(rows, nq):
+    """The pairing rule restated: the smallest unpaired tile takes the unpaired
+    tile with the most key blocks in common (ties: the smaller index)."""
+    taken = [False] * nq
+    order = []
+    for a in range(nq):
+        if taken[a]:
+            continue
+        taken[a] = True
+        order.append(a)
+        best, best_c = -1, -1
+        for c in range(nq):
+            if not taken[c]:
+                ov = len(rows[a] & rows[c])
+                if ov > best:
+                    best, best_c = ov, c
+        if best_c >= 0:
+            taken[best_c] = True
+            order.append(best_c)
+    return order
+
+
+def test_pair_query_tiles_on_calibrated_lists():
+    """svg_pair_query_tiles: each row a permutation equal to the greedy rule,
+    more shared key blocks per work item than index pairs on the heads that
+    attend along time, and attention results bit-identical with the order."""
+    wl = si.small("wan720")
+    types_seed = wl.calib_seeds[0]
+    E = []
+    for s in wl.calib_seeds:
+        (_, _, _), (qd, kd, _), _ = workload_tensors(wl, seed=s, types_seed=types_seed)
+        E.append(svg.svg_block_energy(qd, kd))
+    lists = svg.svg_build_block_mask_calibrated(torch.stack(E).contiguous(), wl.eps, wl.rho)
+    nq = svg.n_tiles(wl.N)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    paired = svg.svg_pair_query_tiles(lists, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    order = paired.tile_order.cpu().numpy().reshape(wl.H, nq)
+    ip = lists.indptr.cpu().numpy().reshape(wl.H, nq + 1)
+    ix = lists.indices.cpu().numpy()
+    shared_idx = shared_paired = 0
+    for h in range(wl.H):
+        assert sorted(order[h].tolist()) == list(range(nq))
+        rows = [set(ix[ip[h][r]:ip[h][r + 1]].tolist()) for r in range(nq)]
+        assert order[h].tolist() == _greedy_pairing(rows, nq)
+        for i in range(0, nq - 1, 2):
+            shared_idx += len(rows[i] & rows[i + 1])
+            shared_paired += len(rows[order[h][i]] & rows[order[h][i + 1]])
+    assert shared_paired >= shared_idx
+    (_, _, _), (qd, kd, vd), _ = workload_tensors(wl, seed=wl.seed, types_seed=types_seed)
+    list_id = torch.arange(wl.H, dtype=torch.int32, device=DEV)
+    a = svg.svg_sparse_attn(qd, kd, vd, list_id, lists)
+    b = svg.svg_sparse_attn_fused(qd, kd, vd, wl.F, wl.P, list_id, paired, layout=0)
+    np.testing.assert_array_equal(bits(a), bits(b))
+
+
+def test_pair_query_tiles_edges():
+    """One tile; an odd count; empty rows; a row set shared by far-apart tiles;
+    an out-of-range index is skipped and flagged."""
+    def run(rows, nk):
+        nq = len(rows)
+        indptr = np.zeros(nq + 1, np.int32)
+        indptr[1:] = np.cumsum([len(r) for r in rows])
+        flat = [c for r in rows for c in r] or [0]
+        lists = svg.BlockLists(torch.from_numpy(indptr).to(DEV),
+                               torch.tensor(flat, dtype=torch.int32, device=DEV), 1, nq)
+        status = torch.zeros(1, dtype=torch.int32, device=DEV)
+        out = svg.svg_pair_query_tiles(lists, nk, status=status)
+        torch.cuda.synchronize()
+        return out.tile_order.cpu().numpy().tolist(), status.item()
+    assert run([[0, 1]], 2) == ([0], 0)
+    assert run([[0], [1], [2]], 3) == ([0, 1, 2], 0)
+    assert run([[], [], [], []], 1) == ([0, 1, 2, 3], 0)
+    # tile 0 and tile 3 keep the same blocks, as do 1 and 2
+    assert run([[0, 5, 9], [2, 3], [2, 3], [0, 5, 9]], 10) == ([0, 3, 1, 2], 0)
+    order, st = run([[0, 40], [1], [0]], 8)
+    assert sorted(order) == [0, 1, 2] and st & svg._lib.SVG_DEVICE_BAD_INDEX
+
+
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 def test_row_broadcast_bit_exact(dtype):
     wl = si.small("hunyuan720")
