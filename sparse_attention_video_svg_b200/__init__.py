@@ -38,6 +38,7 @@ __all__ = [
     "svg_permute_frame_major", "svg_build_block_mask", "svg_block_energy",
     "svg_build_block_mask_calibrated", "svg_sparse_attn", "svg_sparse_attn_fused",
     "svg_v_exponents", "svg_pair_query_tiles", "svg_layer_from_host", "HostLayerBuffers",
+    "svg_attention_from_host",
     "svg_epsilon_schedule", "svg_lists_to_intervals", "svg_lists_to_bitmap", "geometric_lists",
     "QKTransform", "svg_qk_norm_rope", "svg_row_similarity", "svg_anchor_lists",
     "svg_anchor_list_ids", "svg_row_broadcast", "svg_repeat_attention", "svg_layer",
@@ -676,3 +677,59 @@ def svg_layer_from_host(q, k, v, frames: int, tokens_per_frame: int, spatial_wid
         if slot["used"]:
             main.wait_event(slot["unloaded"])
     return out, mode_out
+
+
+def svg_attention_from_host(q, k, v, list_id: torch.Tensor, lists: BlockLists, *, out=None,
+                            heads_per_chunk: int = 4, buffers: Optional[HostLayerBuffers] = None,
+                            stream=None):
+    """Block-sparse attention (V exponents, then every head on its list:
+    svg_v_exponents + svg_sparse_attn_fused with the lists' tile order) for
+    q, k, v in pinned host memory ([B, H, N, d] bf16), streamed like
+    svg_layer_from_host: chunks of `heads_per_chunk` heads (a divisor of B*H)
+    through two device slots, the copies in and out overlapping the compute.
+    list_id: device int32 [B*H].  Returns out (pinned host), complete once
+    `stream` (default: the current stream) has passed this call."""
+    B, H, N, d = q.shape
+    BH = B * H
+    for x in (q, k, v):
+        if x.device.type != "cpu" or not x.is_pinned() or x.dtype != torch.bfloat16 \
+                or not x.is_contiguous() or x.shape != q.shape:
+            raise ValueError("svg_attention_from_host takes contiguous pinned host bf16 [B, H, N, d]")
+    if heads_per_chunk <= 0 or BH % heads_per_chunk:
+        raise ValueError(f"heads_per_chunk must divide B*H = {BH}")
+    if list_id.numel() != BH or list_id.dtype != torch.int32:
+        raise ValueError("list_id must be int32 [B*H]")
+    hc = heads_per_chunk
+    dev = list_id.device
+    if buffers is None or buffers.heads != hc or buffers.slots[0]["q"].shape[2:] != (N, d):
+        buffers = HostLayerBuffers(hc, N, d, 1, dev)
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+    main = torch.cuda.current_stream(dev) if stream is None else stream
+    qf, kf, vf, of = (x.view(BH, N, d) for x in (q, k, v, out))
+    for c in range(BH // hc):
+        slot = buffers.slots[c % 2]
+        lo, hi = c * hc, (c + 1) * hc
+        if slot["used"]:
+            buffers.h2d.wait_event(slot["computed"])
+        with torch.cuda.stream(buffers.h2d):
+            for src, dst in ((qf, slot["q"]), (kf, slot["k"]), (vf, slot["v"])):
+                dst[0].copy_(src[lo:hi], non_blocking=True)
+        slot["loaded"].record(buffers.h2d)
+        main.wait_event(slot["loaded"])
+        if slot["used"]:
+            main.wait_event(slot["unloaded"])
+        bufs = slot["bufs"]
+        vexp = svg_v_exponents(slot["v"], out=bufs.vexp, stream=main)
+        o = svg_sparse_attn_fused(slot["q"], slot["k"], slot["v"], 1, N, list_id[lo:hi], lists,
+                                  layout=0, out=bufs.o, v_exp=vexp, stream=main)
+        slot["computed"].record(main)
+        buffers.d2h.wait_event(slot["computed"])
+        with torch.cuda.stream(buffers.d2h):
+            of[lo:hi].copy_(o[0], non_blocking=True)
+        slot["unloaded"].record(buffers.d2h)
+        slot["used"] = True
+    for slot in buffers.slots:
+        if slot["used"]:
+            main.wait_event(slot["unloaded"])
+    return out

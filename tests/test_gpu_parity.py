@@ -1217,6 +1217,23 @@ def test_pair_query_tiles_on_calibrated_lists():
     np.testing.assert_array_equal(bits(a), bits(b))
 
 
+def test_attention_from_host_matches_device_call():
+    """The host-streamed attention (chunks of heads, copies overlapped) gives
+    the device call's bits, with and without a pairing order."""
+    wl = si.small("wan720")
+    (_, _, _), (qd, kd, vd), _ = workload_tensors(wl)
+    lists = svg.geometric_lists(wl.F, wl.P, wl.width, wl.N)
+    list_id = torch.tensor([h % 3 for h in range(wl.H)], dtype=torch.int32, device=DEV)
+    vexp = svg.svg_v_exponents(vd)
+    ref = bits(svg.svg_sparse_attn(qd, kd, vd, list_id, lists, v_exp=vexp))
+    host = [x.cpu().pin_memory() for x in (qd, kd, vd)]
+    for ls in (lists, svg.svg_pair_query_tiles(lists)):
+        for hc in (1, 2, wl.H):
+            out = svg.svg_attention_from_host(*host, list_id, ls, heads_per_chunk=hc)
+            torch.cuda.synchronize()
+            np.testing.assert_array_equal(bits(out), ref)
+
+
 def test_pair_query_tiles_edges():
     """One tile; an odd count; empty rows; a row set shared by far-apart tiles;
     an out-of-range index is skipped and flagged."""
