@@ -55,15 +55,18 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-# DRAM bytes (read + write) of one attention launch on the HunyuanVideo
-# 720p-shaped layer, from an ncu capture of the kernel built from the sources
-# whose sha256 is recorded here: a 4-head slice of the layer (heads 2-5, two
-# spatial and two temporal; 370402048 + 101969152 bytes), scaled by the head
-# count (24 / 4), since each head's q, k, v are read and its o written once.
-# Reported only while the sources still match.
+# DRAM bytes (read + write) of one attention launch, from ncu captures of the
+# kernel built from the sources whose sha256 is recorded here: a 4-head slice
+# of each layer, scaled by the head count, since each head's q, k, v are read
+# and its o written once.  HunyuanVideo 720p: heads 2-5 (two spatial, two
+# temporal), 370402048 + 101969152 bytes, x 24 / 4.  Wan 2.1 720p with the
+# calibrated lists and the pairing order: heads 14-17 (two of each type),
+# 243936000 + 59193600 bytes, x 40 / 4.  Reported only while the sources
+# still match.
 ATTN_SOURCES = ("attn_sm100.cu", "sm100.cuh", "attn.cuh", "common.cuh")
-ATTN_TRAFFIC = {"hunyuan720": {"sha256": "3e36e93d3b8ea8d5059f4b6b6643b86a3d2c97b441c1e4d23108dc558d01b64e",
-                               "bytes": (370402048 + 101969152) * 24 // 4}}
+_ATTN_SHA = "3e36e93d3b8ea8d5059f4b6b6643b86a3d2c97b441c1e4d23108dc558d01b64e"
+ATTN_TRAFFIC = {"hunyuan720": {"sha256": _ATTN_SHA, "bytes": (370402048 + 101969152) * 24 // 4},
+                "wan720": {"sha256": _ATTN_SHA, "bytes": (243936000 + 59193600) * 40 // 4}}
 
 
 def attn_sources_sha256():

@@ -185,7 +185,8 @@ def test_host_chunk_divides_the_heads():
 
 def test_recorded_traffic_matches_the_sources():
     """The recorded capture belongs to the attention sources in the tree."""
-    assert bench.attn_traffic("hunyuan720") == bench.ATTN_TRAFFIC["hunyuan720"]["bytes"]
+    for name in ("hunyuan720", "wan720"):
+        assert bench.attn_traffic(name) == bench.ATTN_TRAFFIC[name]["bytes"]
 
 
 def test_effective_flops_count_the_element_mask():
