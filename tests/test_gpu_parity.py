@@ -34,6 +34,21 @@ def head64(x, b, h):
     return si.as_float64(x[b, h])
 
 
+def tile_rows_kept_keys(q, k, v, t, N, indptr, indices):
+    """The oracle's block-sparse rows of query tile t (O8), with the softmax
+    taken over the kept key columns only: the columns of the tile's kept key
+    tiles are gathered and the oracle's masked attention runs on them with
+    every gathered key kept -- the same restricted softmax, without scoring
+    the N - |kept| masked keys (thousands of tiles at full size)."""
+    rows = O.tile_rows(int(t), N)
+    cols = np.concatenate([np.arange(j * 128, min(N, (j + 1) * 128))
+                           for j in indices[indptr[t]:indptr[t + 1]]] or [np.zeros(0, np.int64)])
+    if cols.size == 0:
+        return rows, np.zeros((len(rows), q.shape[1]))
+    mask = np.ones((len(rows), cols.size), dtype=bool)
+    return rows, O.masked_attention(q[rows], k[cols], v[cols], mask)
+
+
 # --------------------------------------------------------------------- lists
 
 def gpu_list(kind, F, P, w, N):
@@ -648,6 +663,37 @@ def test_layer_from_host_matches_device_layer(wl):
         svg.svg_layer_from_host(*host, wl.F, wl.P, wl.width, idx, lists, heads_per_chunk=BH + 1)
 
 
+def test_layer_full_size_hunyuan_every_head(full_inputs):
+    """The HunyuanVideo 720p layer (B=1, H=24, N=118800, d=128, band 2) as the
+    bench runs it (profiling, token-major copies of the temporal heads,
+    attention writing frame-major rows): the modes, and 64 query tiles of
+    every head (the ragged tail among them) against the oracle."""
+    name = "hunyuan720"
+    wl = si.WORKLOADS[name]
+    (q, k, v), (qd, kd, vd), types = full_inputs(name)
+    idx = si.sample_queries(wl)
+    lists = svg.geometric_lists(wl.F, wl.P, wl.width, wl.N)
+    o, mode, _ = svg.svg_layer(qd, kd, vd, wl.F, wl.P, wl.width, torch.from_numpy(idx).to(DEV),
+                               lists)
+    mode = mode.cpu().numpy()
+    np.testing.assert_array_equal(mode, types)
+    src = O.token_major_source(wl.F, wl.P)
+    rng = np.random.default_rng(118800)
+    nb = svg.n_tiles(wl.N)
+    geo = {md: O.geometric_block_lists(md, wl.F, wl.P, wl.width, wl.N) for md in (0, 1)}
+    for h in range(wl.H):
+        md = int(mode[h])
+        ip, ix = geo[md]
+        qh, kh, vh = head64(q, 0, h), head64(k, 0, h), head64(v, 0, h)
+        if md == O.MODE_TEMPORAL:
+            qh, kh, vh = (O.permute_token_major(t, wl.F, wl.P) for t in (qh, kh, vh))
+        for t in np.r_[rng.choice(nb - 1, size=63, replace=False), nb - 1]:
+            rows, ref = tile_rows_kept_keys(qh, kh, vh, int(t), wl.N, ip, ix)
+            out_rows = src[rows] if md == O.MODE_TEMPORAL else rows
+            got = to_float64(o[0, h][torch.from_numpy(out_rows).to(DEV)])
+            assert_close(got, ref, f"layer head {h} tile {t}")
+
+
 def test_layer_full_size_cogvideox_sampled(full_inputs):
     name = "cogvideox"
     wl = si.WORKLOADS[name]
@@ -827,20 +873,24 @@ def test_calibration_full_size_sampled():
     assert compared >= 1
     kept = (ip[:, -1] - ip[:, 0]).sum() / float(wl.H * nb * nb)
     assert 0.0 < kept < 1.0
-    # attention on the timed input, every head on its own list
+    # attention on the timed input as the bench runs it (V exponents, every
+    # head on its own list, query tiles paired by svg_pair_query_tiles): 64
+    # query tiles of every head, the ragged tail among them
     q, k, v, _ = si.generate(wl, seed=wl.seed, types_seed=types_seed)
     qd, kd, vd = (to_device(x) for x in (q, k, v))
     list_id = torch.arange(wl.H, dtype=torch.int32, device=DEV)
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
-    o = svg.svg_sparse_attn(qd, kd, vd, list_id, lists, status=status)
+    paired = svg.svg_pair_query_tiles(lists, status=status)
+    o = svg.svg_sparse_attn_fused(qd, kd, vd, wl.F, wl.P, list_id, paired, layout=0,
+                                  v_exp=svg.svg_v_exponents(vd), status=status)
     assert int(status.item()) == 0
-    for h in heads:
+    del qd, kd, vd
+    for h in range(wl.H):
         hp = ip[h] - ip[h][0]
         hx = ix[ip[h][0]:ip[h][-1]]
         qh, kh, vh = head64(q, 0, h), head64(k, 0, h), head64(v, 0, h)
-        for t in blocks:
-            rows = O.tile_rows(t, wl.N)
-            ref = O.block_sparse_rows(qh, kh, vh, rows, hp, hx)
+        for t in np.r_[rng.choice(nb - 1, size=63, replace=False), nb - 1]:
+            rows, ref = tile_rows_kept_keys(qh, kh, vh, int(t), wl.N, hp, hx)
             got = to_float64(o[0, h, rows[0]:rows[-1] + 1])
             assert_close(got, ref, f"calibrated head {h} tile {t}")
 
