@@ -10,7 +10,9 @@
  *   1. svg_profile_heads        online profiling: per head, pick the spatial or
  *                               the temporal mask from a few sampled queries;
  *   2. svg_permute_token_major  frame-major -> token-major reordering of the
- *                               heads that run temporal;
+ *                               heads that run temporal
+ *                               (svg_permute_temporal_heads: those heads only,
+ *                               the copy the fused attention reads);
  *   3. svg_build_block_mask     per-query-block key-block lists (CSR) from the
  *                               spatial / temporal geometry, or
  *      svg_block_energy +
@@ -20,7 +22,10 @@
  *   4. svg_sparse_attn          block-sparse attention over 128x128 tiles that
  *                               walks only the kept key blocks
  *                               (svg_sparse_attn_fused: with the reordering of
- *                               temporal heads folded in);
+ *                               temporal heads folded in; svg_v_exponents:
+ *                               per-head V scale for its fp16 P.V;
+ *                               svg_pair_query_tiles: a pairing order of the
+ *                               query tiles for lists used many times);
  *   5. svg_permute_frame_major  the inverse reordering of the output;
  *   6. svg_row_similarity, svg_anchor_lists, svg_anchor_list_ids,
  *      svg_row_broadcast        spatial-repetition heads (anchor rows only).
