@@ -52,6 +52,17 @@ int main(void) {
         "RoPE without tables rejected");
   st = svg_row_broadcast(fake, SVG_BF16, 1, 2, 256, 64, 4, 4, 15, 5, fake2, 3, NULL);
   CHECK(st == SVG_ERR_INVALID_ARG, "frame shape that does not tile N rejected");
+  /* the temporal-heads copy needs the modes */
+  st = svg_permute_temporal_heads(fake, fake2, SVG_BF16, 1, 2, 12, 64, 3, 4, NULL, NULL);
+  CHECK(st == SVG_ERR_INVALID_ARG && strstr(svg_last_error(), "mode is required") != NULL,
+        "temporal-heads copy without modes rejected");
+  /* pairing order: one bitmap word per 32 key blocks, per row and list */
+  CHECK(svg_pair_query_tiles_workspace_size(2, 5, 33) == 2 * 5 * 2 * sizeof(uint32_t),
+        "pairing workspace size");
+  CHECK(svg_pair_query_tiles_workspace_size(0, 5, 33) == 0, "pairing workspace of no lists");
+  st = svg_pair_query_tiles(fake, fake2, 2, 5, 33, fake, NULL, fake2, 4, NULL);
+  CHECK(st == SVG_ERR_INVALID_ARG && strstr(svg_last_error(), "workspace") != NULL,
+        "short pairing workspace rejected");
 
   if (failures == 0) printf("c abi ok: %s\n", svg_version());
   return failures == 0 ? 0 : 1;
